@@ -1,0 +1,271 @@
+/*
+ * pnmix.h -- C ABI of the PN-Mix mixed-precision KV-cache library for B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * The method is PN-Mix ("PN-Mix: Pair-Norm Guided Mixed-Precision Key Cache
+ * Quantization for Efficient Long-Output LLM Inference", abstract): RoPE
+ * channel pairs whose query pair-norm x key pair-norm product is large carry
+ * most of the attention-logit error under low-bit key quantization, so those
+ * pairs get more bits.  The salient pairs are chosen once at prefill and kept
+ * for the whole decode.  Values are quantized per token (the per-token value
+ * scheme of "MixKVQ: Query-Aware Mixed-Precision KV Cache Quantization for
+ * Long-Context Reasoning", abstract and "Innovation" list; the KIVI-style
+ * per-channel-key / per-token-value split recorded in the PM-KVQ review,
+ * "key_machinery").
+ *
+ * The five calls of the path, in call order:
+ *   pnmix_select_pairs    -- prefill: score the 64 RoPE pairs per KV head, keep the top k
+ *   pnmix_quantize_keys   -- prefill: per-channel 32-token groups, salient pairs at b_hi bits
+ *   pnmix_quantize_values -- prefill: per-token 32-channel groups at b_v bits
+ *   pnmix_append          -- decode: write one new K/V row, quantize every full 32-token group
+ *   pnmix_decode_attention-- decode: split-K attention over the packed cache + bf16 residual
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers unless a comment says otherwise.
+ *    bf16 tensors are passed as `const uint16_t*` holding the raw bf16 bits.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call only enqueues work on that stream; no call synchronises, allocates
+ *    or frees device memory.  The caller owns every buffer.
+ *  - Arguments are validated on the host before anything is enqueued.  A call
+ *    that returns anything but PNMIX_OK has enqueued nothing, except
+ *    PNMIX_ERR_CUDA, which reports a launch error from the CUDA runtime.
+ *  - Conditions only the device can see (a full cache on append, a bounded wait
+ *    that ran out) set bits in the cache's device error word; read it with
+ *    pnmix_read_error.  No kernel traps or asserts.
+ *  - head_dim is 128; rows of K, V and Q are 128 contiguous bf16 values.
+ *
+ * Numerical contract
+ * ------------------
+ * Quantization (codes, fp16 scales and zero points, packing, pair indices) is
+ * computed in IEEE fp32 round-to-nearest-even in the op order below, with no
+ * FMA contraction, and is bit-exact with the reference definition:
+ *   pair p in [0,64) is channels (p, p+64) (half-split RoPE pairing);
+ *   key norm     K_p = sqrt(max_t (k_{t,p}^2 + k_{t,p+64}^2)) over all L prefill tokens;
+ *   query norm   Q_p = (sum over heads h of the group, then tokens of the window,
+ *                       of sqrt(q_{h,t,p}^2 + q_{h,t,p+64}^2)) / (G * W');
+ *   score        s_p = Q_p * K_p, top k by (s desc, p asc);
+ *   quantizer    mn, mx over the group; s16 = fp16(fl(mx - mn) / (2^b - 1));
+ *                z16 = fp16(mn); code = clamp(rint((x - z) / s), 0, 2^b - 1)
+ *                with s, z the fp32 values of s16, z16; all codes 0 when s16 == 0.
+ * Attention is  out_h = sum_t softmax_t(q_h . k^_t * scale) v^_t  over every
+ * cached token, with k^ = code*s + z for packed tokens and the bf16 value for
+ * residual tokens; it is accumulated in fp32 and returned in fp32.
+ *
+ * Packed cache layout (the contract the oracle and the kernels share)
+ * ------------------------------------------------------------------
+ * The cache of one sequence b and KV head h is a run of fixed-size GROUP
+ * RECORDS, one per 32 tokens, followed (logically) by a bf16 residual window of
+ * the newest len % 32 tokens.  Group g of (b, h) lives at
+ *     records + ((b * n_kv_heads + h) * (capacity_tokens / 32) + g) * record_bytes.
+ *
+ * Key positions.  Within (b, h) the 128 key channels are put in POSITION order:
+ * first the 2k salient channels {p, p+64 : p salient} ascending, then the other
+ * channels ascending.  perm[j] is the channel at position j.  Positions
+ * [0, 2k) use b_hi bits, positions [2k, 128) use b_lo bits.  Position slice
+ * sigma = j / 16 (8 slices; 2k is a multiple of 16).
+ *
+ * Lane coordinates.  Everything below is indexed by a 32-lane coordinate
+ * L = 4*gq + tq (gq = L >> 2 in [0,8), tq = L & 3 in [0,4)), the fragment
+ * ownership of a 16x8x16 matrix-multiply-accumulate tile.
+ *
+ * Record, in this order (all offsets are multiples of 128 bytes):
+ *  1. Key codes, KC = 128 * (WH + WL) bytes, WH = (2k/16) * b_hi / 2,
+ *     WL = ((128-2k)/16) * b_lo / 2 words per lane.
+ *     A key SLOT is (slice sigma, c in {0,1}, u in {0..3}); it names the two
+ *     positions P0 = 16*sigma + 2*tq + 8*c and P1 = P0 + 1 of token
+ *     tau = gq + 8*u.  Within the hi block (slices [0, 2k/16)) the lane-local
+ *     slot number is n = (sigma*8 + c*4 + u); within the lo block it is
+ *     n = ((sigma - 2k/16)*8 + c*4 + u).  With m = 16 / b slots per 32-bit word,
+ *     the slot sits in lane-local word n / m (counted from 0 for the hi block and
+ *     from WH for the lo block), at position r = n % m: the code of (tau, P0) at
+ *     bits [b*r, b*r + b) and the code of (tau, P1) at bits [16 + b*r, 16 + b*r + b).
+ *     Lane-local word w of lane L is stored at byte offset (w * 32 + L) * 4.
+ *  2. Key scales, 128 fp16 (256 B): the scale of position
+ *     j = 16*sigma + 8*e + 2*tq + v  (e, v in {0,1}) is fp16 element
+ *     ((tq * 8 + sigma) * 2 + e) * 2 + v.
+ *  3. Key zero points, 128 fp16 (256 B), same order as 2.
+ *  4. Value codes, 1024 B, b_v = 2 bits.  A value SLOT is (m in {0..7},
+ *     r in {0,1}, p in {0..3}); it names channel 16*m + gq + 8*r and the token
+ *     pair (2*tq + 8*p, 2*tq + 8*p + 1).  The slot is word m of lane L at
+ *     position q = r*4 + p: the code of the first token at bits [2q, 2q+2), of the
+ *     second at bits [16 + 2q, 16 + 2q + 2).  Word m of lane L is stored at
+ *     byte offset ((m >> 2) * 32 + L) * 16 + (m & 3) * 4.
+ *  5. Value scales, 64 fp16x2 (256 B): element (tp * 4 + jg) is the pair
+ *     (scale of token 2*tp, scale of token 2*tp+1) of channel group jg
+ *     (channels [32*jg, 32*jg + 32)), tp in [0,16).
+ *  6. Value zero points, 256 B, same order as 5.
+ * record_bytes = KC + 2048 (3200 B at b_hi=4, b_lo=2, k=8, i.e. 100 B/token).
+ *
+ * Other regions of the cache (all carved out of one caller-owned buffer by
+ * pnmix_cache_init): residual K and V bf16 [B][Hkv][32][128] (slot = token % 32),
+ * len int32 [B], pair_idx uint8 [B][Hkv][64] (first k entries, ascending),
+ * pair_mask uint64 [B][Hkv] (bit p set iff pair p is salient), perm uint8
+ * [B][Hkv][128], pair_scores fp32 [B][Hkv][64] (s_p of the last
+ * pnmix_select_pairs), scratch and the error word.
+ */
+#ifndef PNMIX_H
+#define PNMIX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PNMIX_OK = 0,
+  PNMIX_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shapes */
+  PNMIX_ERR_UNSUPPORTED = 2,  /* a configuration outside the supported set below */
+  PNMIX_ERR_CAPACITY = 3,     /* the request does not fit the cache or the workspace */
+  PNMIX_ERR_CUDA = 4,         /* the CUDA runtime reported an error for a launch */
+  PNMIX_ERR_ALIGNMENT = 5,    /* a pointer is not aligned as required */
+  PNMIX_ERR_DEVICE = 6        /* pnmix_read_error found a non-zero device error word */
+} pnmix_status;
+
+/* Device error word bits (pnmix_read_error). */
+#define PNMIX_DEVERR_APPEND_FULL 0x1u  /* pnmix_append found len == capacity_tokens */
+
+/*
+ * Method parameters.  Supported set:
+ *   head_dim 128; group_tokens 32; residual_tokens 32; value_group 32; value_bits 2;
+ *   (key_bits_hi, key_bits_lo) in {(4,2), (2,1)};
+ *   n_salient_pairs k in {0, 8, 16, 32, 64} with WH and WL (see the layout) whole
+ *     numbers, i.e. every k for (4,2) and k in {0, 16, 32, 64} for (2,1);
+ *   G = n_q_heads / n_kv_heads in [1, 8];
+ *   saliency_window W in [1, 1024].
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ */
+typedef struct {
+  int32_t head_dim;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t group_tokens;
+  int32_t residual_tokens;
+  int32_t key_bits_hi;
+  int32_t key_bits_lo;
+  int32_t n_salient_pairs;
+  int32_t value_bits;
+  int32_t value_group;
+  int32_t saliency_window;
+  float softmax_scale;
+} pnmix_config;
+
+/* Device pointers into one caller-owned buffer; filled by pnmix_cache_init. */
+typedef struct {
+  int32_t batch;
+  int32_t capacity_tokens;   /* multiple of 32 */
+  int32_t n_kv_heads;
+  int32_t record_bytes;
+  uint8_t* records;          /* [B][Hkv][capacity/32][record_bytes] */
+  uint16_t* k_resid;         /* bf16 [B][Hkv][32][128] */
+  uint16_t* v_resid;         /* bf16 [B][Hkv][32][128] */
+  int32_t* len;              /* [B] tokens held (packed + residual) */
+  uint8_t* pair_idx;         /* [B][Hkv][64] */
+  uint64_t* pair_mask;       /* [B][Hkv] */
+  uint8_t* perm;             /* [B][Hkv][128] */
+  float* pair_scores;        /* [B][Hkv][64] */
+  uint32_t* scratch;         /* library-internal counters; zero between calls */
+  uint32_t* error;           /* device error word */
+  void* base;
+  size_t total_bytes;
+} pnmix_cache;
+
+/* Bytes of one group record (layout item list above); 0 if unsupported. */
+size_t pnmix_record_bytes(const pnmix_config* cfg);
+
+/*
+ * Bytes a cache of `batch` sequences and `capacity_tokens` tokens each needs.
+ * capacity_tokens must be a positive multiple of 32.  Host-only.
+ */
+pnmix_status pnmix_cache_bytes(const pnmix_config* cfg, int batch, int capacity_tokens,
+                               size_t* total_bytes);
+
+/*
+ * Carve the regions of a cache out of `device_base` (>= pnmix_cache_bytes bytes,
+ * 256-byte aligned) and fill *out.  Host-only: touches no device memory.  The
+ * buffer must be zero-filled before the first pnmix call that uses it
+ * (pnmix_cache_reset does that).
+ */
+pnmix_status pnmix_cache_init(const pnmix_config* cfg, int batch, int capacity_tokens,
+                              void* device_base, size_t bytes, pnmix_cache* out);
+
+/* Zero the whole cache buffer on `stream` (lengths 0, no salient pairs, no error). */
+pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream);
+
+/*
+ * Prefill step 1 (PN-Mix abstract: salient pairs are picked once at prefill from
+ * the query-key pair-norm product).  For every (b, kv head h):
+ *   K_p from the first L rows of k, Q_p from the n_window rows of q_window of the
+ *   G query heads h*G .. h*G+G-1, s_p = Q_p * K_p; the k = n_salient_pairs pairs
+ *   with the largest s_p (ties to the lower p) become salient.
+ * q_window: bf16 [B][Hq][n_window][128] -- the LAST n_window prefill queries, after RoPE.
+ * k:        bf16 [B][Hkv][ld_tokens][128], rows [0, L) used, after RoPE.
+ * n_window must equal min(L, saliency_window); 1 <= L <= ld_tokens.
+ * Writes pair_idx, pair_mask, perm and pair_scores of every (b, h).
+ */
+pnmix_status pnmix_select_pairs(const pnmix_config* cfg, const uint16_t* q_window, int n_window,
+                                const uint16_t* k, int L, int ld_tokens, pnmix_cache* cache,
+                                void* stream);
+
+/*
+ * Prefill step 2 (mixed-precision per-channel keys; PN-Mix abstract).  Quantizes
+ * tokens [0, 32*floor(L/32)) of k into the key part of group records 0..,
+ * copies the last L % 32 rows into the K residual and sets len[b] = L.
+ * Uses the salient set written by pnmix_select_pairs.  L <= capacity_tokens.
+ */
+pnmix_status pnmix_quantize_keys(const pnmix_config* cfg, const uint16_t* k, int L, int ld_tokens,
+                                 pnmix_cache* cache, void* stream);
+
+/*
+ * Prefill step 3 (per-token values; MixKVQ abstract).  Same token split as
+ * pnmix_quantize_keys, into the value part of the records and the V residual;
+ * sets len[b] = L.
+ */
+pnmix_status pnmix_quantize_values(const pnmix_config* cfg, const uint16_t* v, int L, int ld_tokens,
+                                   pnmix_cache* cache, void* stream);
+
+/*
+ * Decode step 1 (streaming append; PN-Mix abstract: the prefill choice of
+ * salient pairs is reused for the whole decode).  k_new, v_new: bf16 [B][Hkv][128].
+ * For every b: the row goes to residual slot len[b] % 32; when that slot is 31
+ * the 32 residual rows are quantized into group record len[b] / 32 with the
+ * prefill's salient pairs; then len[b] += 1.  A sequence whose len[b] equals
+ * capacity_tokens is left unchanged and PNMIX_DEVERR_APPEND_FULL is raised.
+ */
+pnmix_status pnmix_append(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
+                          pnmix_cache* cache, void* stream);
+
+/*
+ * Workspace bytes pnmix_decode_attention needs for `batch` sequences whose
+ * lengths are at most max_context.  The workspace must be zero-filled before its
+ * first use; every call leaves it ready for the next one.
+ */
+size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context);
+
+/*
+ * Decode step 2 (attention over the quantized cache).  q: bf16 [B][Hq][128]
+ * (after RoPE); out: fp32 [B][Hq][128].  Attends over all len[b] cached tokens
+ * (the query's own K/V must have been appended first if it is to be included).
+ * max_context is an upper bound on len[b] used to size the split-K grid; the
+ * result does not depend on it.  A sequence with len[b] == 0 gets zeros.
+ */
+pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
+                                    const pnmix_cache* cache, int max_context, float* out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronously read (and, if clear != 0, zero) the device error word.  Host pointer out. */
+pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error);
+
+/* Static string for a status code. */
+const char* pnmix_status_string(pnmix_status status);
+
+/* Library version, e.g. "pnmix 0.1". */
+const char* pnmix_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PNMIX_H */

@@ -1,0 +1,324 @@
+"""Reference oracle of the PN-Mix KV-cache path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library in
+``decode_attention_prefill_b200``) never imports it and fails loudly when its
+own extension is missing.
+
+The arithmetic lives in ``pnmix_oracle.c`` (plain single-threaded C, compiled
+here with gcc on first use); this module only marshals numpy arrays and loops
+over (sequence, KV head) units.  It shares no code with the CUDA library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pnmix_oracle.c")
+_LIB = os.path.join(_HERE, "libpnmix_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-fexcess-precision=standard", "-mno-fma"]
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+
+
+def build(force: bool = False) -> str:
+    """Compile pnmix_oracle.c into libpnmix_oracle.so next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags.c_contiguous, "oracle arrays must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            vp, i, d, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float
+            sig = {
+                "orc_f32_from_bf16": (f, [ctypes.c_uint16]),
+                "orc_f32_from_f16": (f, [ctypes.c_uint16]),
+                "orc_f16_from_f32": (ctypes.c_uint16, [f]),
+                "orc_pair_scores": (None, [i, i, i, vp, vp, vp, vp, vp]),
+                "orc_topk": (None, [vp, i, vp, vp]),
+                "orc_position_order": (i, [ctypes.c_uint64, vp]),
+                "orc_minmax_quant": (None, [vp, i, i, vp, vp, vp]),
+                "orc_key_group": (None, [vp, vp, i, i, i, vp, vp, vp]),
+                "orc_value_token": (None, [vp, i, vp, vp, vp]),
+                "orc_record_bytes": (ctypes.c_long, [i, i, i]),
+                "orc_pack_record": (i, [i, i, i, vp, vp, vp, vp, vp, vp, vp]),
+                "orc_unpack_record": (i, [i, i, i, vp, vp, vp, vp, vp, vp, vp]),
+                "orc_make_record": (i, [i, i, i, i, vp, vp, vp, vp]),
+                "orc_prefill_unit": (i, [i, i, i, i, vp, i, vp, vp, vp, vp, vp]),
+                "orc_append_unit": (i, [i, i, i, i, vp, i, vp, vp, vp, vp, vp]),
+                "orc_attention_core": (None, [i, vp, vp, vp, ctypes.c_long, d, vp]),
+                "orc_attend_unit": (i, [i, vp, d, i, i, i, vp, vp, i, vp, vp, i, vp, vp, vp]),
+                "orc_exact_attention": (None, [i, vp, vp, vp, ctypes.c_long, d, vp]),
+                "orc_key_code_bits": (d, [i, i, i]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- formats
+
+def f16_from_f32(x: float) -> int:
+    return int(lib().orc_f16_from_f32(float(np.float32(x))))
+
+
+def f32_from_f16(h: int) -> float:
+    return float(lib().orc_f32_from_f16(int(h)))
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+# ---------------------------------------------------------------- step 1
+
+def pair_scores(qwin: np.ndarray, k: np.ndarray):
+    """qwin bf16 [G][W][128], k bf16 [L][128] -> (scores, key norms, query norms), fp32 [64]."""
+    qwin = np.ascontiguousarray(qwin, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    G, W, _ = qwin.shape
+    L = k.shape[0]
+    s = np.zeros(64, np.float32)
+    kn = np.zeros(64, np.float32)
+    qn = np.zeros(64, np.float32)
+    lib().orc_pair_scores(G, W, L, _p(qwin), _p(k), _p(s), _p(kn), _p(qn))
+    return s, kn, qn
+
+
+def topk(scores: np.ndarray, k: int):
+    """-> (idx uint8 [k] ascending, mask int)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float32)
+    idx = np.zeros(max(k, 1), np.uint8)
+    mask = np.zeros(1, np.uint64)
+    lib().orc_topk(_p(scores), k, _p(idx), _p(mask))
+    return idx[:k].copy(), int(mask[0])
+
+
+def position_order(mask: int):
+    perm = np.zeros(128, np.uint8)
+    nhi = lib().orc_position_order(ctypes.c_uint64(mask), _p(perm))
+    return perm, nhi
+
+
+def select_unit(qwin: np.ndarray, k: np.ndarray, n_salient: int):
+    """Full step 1 of one (b, KV head): scores, idx, mask, perm."""
+    s, _, _ = pair_scores(qwin, k)
+    idx, mask = topk(s, n_salient)
+    perm, _ = position_order(mask)
+    return s, idx, mask, perm
+
+
+# ---------------------------------------------------------------- quantizer
+
+def minmax_quant(x: np.ndarray, bits: int):
+    """x fp32 [n] -> (codes uint8 [n], s16 bits, z16 bits)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.zeros(x.shape[0], np.uint8)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    lib().orc_minmax_quant(_p(x), x.shape[0], bits, _p(s), _p(z), _p(codes))
+    return codes, int(s[0]), int(z[0])
+
+
+def key_group(rows: np.ndarray, perm: np.ndarray, nhi: int, bhi: int, blo: int):
+    rows = np.ascontiguousarray(rows, dtype=np.uint16)
+    perm = np.ascontiguousarray(perm, dtype=np.uint8)
+    codes = np.zeros((32, 128), np.uint8)
+    s = np.zeros(128, np.uint16)
+    z = np.zeros(128, np.uint16)
+    lib().orc_key_group(_p(rows), _p(perm), nhi, bhi, blo, _p(codes), _p(s), _p(z))
+    return codes, s, z
+
+
+def value_token(row: np.ndarray, bits: int = 2):
+    row = np.ascontiguousarray(row, dtype=np.uint16)
+    codes = np.zeros(128, np.uint8)
+    s = np.zeros(4, np.uint16)
+    z = np.zeros(4, np.uint16)
+    lib().orc_value_token(_p(row), bits, _p(codes), _p(s), _p(z))
+    return codes, s, z
+
+
+# ---------------------------------------------------------------- layout
+
+def record_bytes(k: int, bhi: int, blo: int) -> int:
+    return int(lib().orc_record_bytes(k, bhi, blo))
+
+
+def key_code_bits(k: int, bhi: int, blo: int) -> float:
+    return float(lib().orc_key_code_bits(k, bhi, blo))
+
+
+def pack_record(k, bhi, blo, kcodes, ks, kz, vcodes, vs, vz) -> np.ndarray:
+    R = record_bytes(k, bhi, blo)
+    rec = np.zeros(R, np.uint8)
+    arrs = [np.ascontiguousarray(a, dtype=t) for a, t in
+            ((kcodes, np.uint8), (ks, np.uint16), (kz, np.uint16), (vcodes, np.uint8),
+             (vs, np.uint16), (vz, np.uint16))]
+    rc = lib().orc_pack_record(k, bhi, blo, *[_p(a) for a in arrs], _p(rec))
+    if rc:
+        raise ValueError("unsupported record parameters")
+    return rec
+
+
+def unpack_record(k, bhi, blo, rec):
+    rec = np.ascontiguousarray(rec, dtype=np.uint8)
+    kc = np.zeros((32, 128), np.uint8)
+    ks = np.zeros(128, np.uint16)
+    kz = np.zeros(128, np.uint16)
+    vc = np.zeros((32, 128), np.uint8)
+    vs = np.zeros((32, 4), np.uint16)
+    vz = np.zeros((32, 4), np.uint16)
+    rc = lib().orc_unpack_record(k, bhi, blo, _p(rec), _p(kc), _p(ks), _p(kz), _p(vc), _p(vs),
+                                 _p(vz))
+    if rc:
+        raise ValueError("unsupported record parameters")
+    return kc, ks, kz, vc, vs, vz
+
+
+# ---------------------------------------------------------------- whole caches
+
+class Cache:
+    """Host image of the cache regions the tests compare with the device."""
+
+    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2):
+        self.batch, self.n_kv, self.capacity = batch, n_kv, capacity
+        self.k, self.bhi, self.blo, self.bv = k, bhi, blo, bv
+        self.R = record_bytes(k, bhi, blo)
+        if not self.R:
+            raise ValueError("unsupported bit point")
+        self.records = np.zeros((batch, n_kv, capacity // 32, self.R), np.uint8)
+        self.resid_k = np.zeros((batch, n_kv, 32, 128), np.uint16)
+        self.resid_v = np.zeros((batch, n_kv, 32, 128), np.uint16)
+        self.len = np.zeros(batch, np.int32)
+        self.idx = np.zeros((batch, n_kv, 64), np.uint8)
+        self.mask = np.zeros((batch, n_kv), np.uint64)
+        self.perm = np.zeros((batch, n_kv, 128), np.uint8)
+        self.scores = np.zeros((batch, n_kv, 64), np.float32)
+
+    def select(self, qwin: np.ndarray, kin: np.ndarray, L: int, units=None):
+        """qwin bf16 [B][Hq][W][128]; kin bf16 [B][Hkv][>=L][128]."""
+        G = qwin.shape[1] // self.n_kv
+        for b, h in units or [(b, h) for b in range(self.batch) for h in range(self.n_kv)]:
+            s, idx, mask, perm = select_unit(qwin[b, h * G:(h + 1) * G], kin[b, h, :L], self.k)
+            self.scores[b, h] = s
+            self.idx[b, h, :self.k] = idx
+            self.mask[b, h] = mask
+            self.perm[b, h] = perm
+
+    def prefill(self, kin: np.ndarray, vin: np.ndarray, L: int, units=None):
+        """Quantize tokens [0, L) of kin / vin (bf16 [B][Hkv][>=L][128])."""
+        for b, h in units or [(b, h) for b in range(self.batch) for h in range(self.n_kv)]:
+            kk = np.ascontiguousarray(kin[b, h, :L])
+            vv = np.ascontiguousarray(vin[b, h, :L])
+            rec = self.records[b, h]
+            rk = self.resid_k[b, h]
+            rv = self.resid_v[b, h]
+            rc = lib().orc_prefill_unit(self.k, self.bhi, self.blo, self.bv,
+                                        _p(self.perm[b, h]), L, _p(kk), _p(vv), _p(rec), _p(rk),
+                                        _p(rv))
+            assert rc == 0
+        self.len[:] = L
+
+    def append(self, knew: np.ndarray, vnew: np.ndarray):
+        """knew, vnew bf16 [B][Hkv][128]."""
+        for b in range(self.batch):
+            n = int(self.len[b])
+            if n >= self.capacity:
+                continue
+            for h in range(self.n_kv):
+                lib().orc_append_unit(self.k, self.bhi, self.blo, self.bv, _p(self.perm[b, h]), n,
+                                      _p(np.ascontiguousarray(knew[b, h])),
+                                      _p(np.ascontiguousarray(vnew[b, h])), _p(self.records[b, h]),
+                                      _p(self.resid_k[b, h]), _p(self.resid_v[b, h]))
+            self.len[b] = n + 1
+
+    def attend_unit(self, q: np.ndarray, b: int, h: int, scale: float | None = None) -> np.ndarray:
+        """q bf16 [G][128] of KV head h of sequence b -> fp64 [G][128]."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        G = q.shape[0]
+        n = int(self.len[b])
+        out = np.zeros((G, 128), np.float64)
+        rc = lib().orc_attend_unit(G, _p(q), scale if scale else 1.0 / np.sqrt(128.0), self.k,
+                                   self.bhi, self.blo, _p(self.perm[b, h]),
+                                   _p(self.records[b, h]), n // 32, _p(self.resid_k[b, h]),
+                                   _p(self.resid_v[b, h]), n % 32, None, None, _p(out))
+        assert rc == 0
+        return out
+
+    def attend(self, q: np.ndarray, heads=None) -> np.ndarray:
+        """q bf16 [B][Hq][128] -> fp64 [B][Hq][128] (only the listed (b, kv head) units)."""
+        B, Hq, _ = q.shape
+        G = Hq // self.n_kv
+        out = np.full((B, Hq, 128), np.nan)
+        for b, h in heads or [(b, h) for b in range(B) for h in range(self.n_kv)]:
+            out[b, h * G:(h + 1) * G] = self.attend_unit(q[b, h * G:(h + 1) * G], b, h)
+        return out
+
+
+def attend_passthrough(q: np.ndarray, kin: np.ndarray, vin: np.ndarray, n_groups: int,
+                       resid_k: np.ndarray, resid_v: np.ndarray, n_resid: int,
+                       scale: float | None = None) -> np.ndarray:
+    """The 16-bit setting of orc_attend_unit: dequantized values are the bf16 inputs."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    G = q.shape[0]
+    out = np.zeros((G, 128), np.float64)
+    dummy = np.zeros(128, np.uint8)
+    rc = lib().orc_attend_unit(G, _p(q), scale if scale else 1.0 / np.sqrt(128.0), 0, 16, 16,
+                               _p(np.arange(128, dtype=np.uint8)), _p(dummy), n_groups,
+                               _p(np.ascontiguousarray(resid_k, dtype=np.uint16)),
+                               _p(np.ascontiguousarray(resid_v, dtype=np.uint16)), n_resid,
+                               _p(np.ascontiguousarray(kin, dtype=np.uint16)),
+                               _p(np.ascontiguousarray(vin, dtype=np.uint16)), _p(out))
+    assert rc == 0
+    return out
+
+
+def exact_attention(q: np.ndarray, kin: np.ndarray, vin: np.ndarray,
+                    scale: float | None = None) -> np.ndarray:
+    """Plain softmax attention of q bf16 [G][128] over bf16 kin/vin [n][128], fp64."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    kin = np.ascontiguousarray(kin, dtype=np.uint16)
+    vin = np.ascontiguousarray(vin, dtype=np.uint16)
+    out = np.zeros((q.shape[0], 128), np.float64)
+    lib().orc_exact_attention(q.shape[0], _p(q), _p(kin), _p(vin), kin.shape[0],
+                              scale if scale else 1.0 / np.sqrt(128.0), _p(out))
+    return out
+
+
+def attention_core(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, scale: float) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    khat = np.ascontiguousarray(khat, dtype=np.float64)
+    vhat = np.ascontiguousarray(vhat, dtype=np.float64)
+    out = np.zeros((q.shape[0], 128), np.float64)
+    lib().orc_attention_core(q.shape[0], _p(q), _p(khat), _p(vhat), khat.shape[0], scale, _p(out))
+    return out
