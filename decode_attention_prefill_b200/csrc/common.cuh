@@ -1,0 +1,159 @@
+// common.cuh -- device-side helpers shared by the pnmix kernels (not by the oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pnmix.h"
+
+namespace pnmix {
+
+constexpr int kHeadDim = 128;
+constexpr int kGroup = 32;      // tokens per key group / value records
+constexpr int kMaxG = 8;        // query heads per KV head
+
+// Geometry derived from a validated pnmix_config (host computes, kernels read by value).
+struct Geometry {
+  int B, Hq, Hkv, G;
+  int k;          // salient pairs
+  int nhi;        // salient positions = 2k
+  int nhs;        // hi slices = nhi / 16
+  int bhi, blo, bv;
+  int wh, wl;     // key-code words per lane, hi / lo block
+  int kc_bytes;   // key-code bytes per record = 128 * (wh + wl)
+  int record_bytes;
+  int capacity;   // tokens per sequence
+  int gcap;       // records per (b, h) = capacity / 32
+  float scale;    // softmax scale
+};
+
+// Record part offsets.
+__host__ __device__ __forceinline__ int rec_kscale(const Geometry& g) { return g.kc_bytes; }
+__host__ __device__ __forceinline__ int rec_kzero(const Geometry& g) { return g.kc_bytes + 256; }
+__host__ __device__ __forceinline__ int rec_vcode(const Geometry& g) { return g.kc_bytes + 512; }
+__host__ __device__ __forceinline__ int rec_vscale(const Geometry& g) { return g.kc_bytes + 1536; }
+__host__ __device__ __forceinline__ int rec_vzero(const Geometry& g) { return g.kc_bytes + 1792; }
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// fp16 element index of key position j in the scale / zero arrays.
+__host__ __device__ __forceinline__ int kscale_index(int j) {
+  int sigma = j >> 4, e = (j >> 3) & 1, tq = (j >> 1) & 3, v = j & 1;
+  return ((tq * 8 + sigma) * 2 + e) * 2 + v;
+}
+
+// fp16 element index of the value scale of (token t, channel group jg).
+__host__ __device__ __forceinline__ int vscale_index(int t, int jg) {
+  return ((t >> 1) * 4 + jg) * 2 + (t & 1);
+}
+
+// Byte offset (inside the value-code area) of value word m of lane L.
+__host__ __device__ __forceinline__ int vword_offset(int m, int L) {
+  return ((m >> 2) * 32 + L) * 16 + (m & 3) * 4;
+}
+
+// Location of the key code of (token tau, position j): byte offset of its 32-bit
+// word in the record and its bit.  Follows the slot definition of pnmix.h.
+__device__ __forceinline__ void key_code_loc(const Geometry& g, int tau, int j, int& byte_off,
+                                             int& bit, int& bits) {
+  int sigma = j >> 4, rem = j & 15;
+  int c = rem >> 3, tq = (rem & 7) >> 1, half = rem & 1;
+  int gq = tau & 7, u = tau >> 3;
+  bool hi = sigma < g.nhs;
+  bits = hi ? g.bhi : g.blo;
+  int m = 16 / bits;
+  int n = (hi ? sigma : sigma - g.nhs) * 8 + c * 4 + u;
+  int w = (hi ? 0 : g.wh) + n / m;
+  int L = gq * 4 + tq;
+  byte_off = (w * 32 + L) * 4;
+  bit = 16 * half + bits * (n % m);
+}
+
+// Location of the value code of (token t, channel ch).
+__device__ __forceinline__ void value_code_loc(int t, int ch, int& byte_off, int& bit) {
+  int tq = (t & 7) >> 1, p = t >> 3, second = t & 1;
+  int m = ch >> 4, rem = ch & 15, r = rem >> 3, gq = rem & 7;
+  int q = r * 4 + p;
+  byte_off = vword_offset(m, gq * 4 + tq);
+  bit = 16 * second + 2 * q;
+}
+
+// The min-max quantizer parameters, bit-exact with the reference definition:
+// s16 = fp16(fl(mx - mn) / (2^b - 1)), z16 = fp16(mn).
+struct QParams {
+  float s, z;
+  uint16_t s16, z16;
+};
+
+__device__ __forceinline__ QParams quant_params(float mn, float mx, int bits) {
+  float levels = static_cast<float>((1 << bits) - 1);
+  float range = __fsub_rn(mx, mn);
+  float s32 = __fdiv_rn(range, levels);
+  __half hs = __float2half_rn(s32);
+  __half hz = __float2half_rn(mn);
+  QParams q;
+  q.s16 = __half_as_ushort(hs);
+  q.z16 = __half_as_ushort(hz);
+  q.s = __half2float(hs);
+  q.z = __half2float(hz);
+  return q;
+}
+
+// code = clamp(rint(fl(fl(x - z) / s)), 0, 2^b - 1); 0 when s == 0.
+__device__ __forceinline__ uint32_t quant_code(float x, const QParams& q, int bits) {
+  if (q.s == 0.0f) return 0u;
+  float d = __fsub_rn(x, q.z);
+  float r = rintf(__fdiv_rn(d, q.s));
+  float levels = static_cast<float>((1 << bits) - 1);
+  r = fminf(fmaxf(r, 0.0f), levels);
+  return static_cast<uint32_t>(r);
+}
+
+// Squared pair norm fl(fl(a*a) + fl(b*b)).
+__device__ __forceinline__ float pair_norm2(float a, float b) {
+  return __fadd_rn(__fmul_rn(a, a), __fmul_rn(b, b));
+}
+
+// Pointer helpers.
+__device__ __forceinline__ size_t unit_index(const Geometry& g, int b, int h) {
+  return static_cast<size_t>(b) * g.Hkv + h;
+}
+__device__ __forceinline__ uint8_t* record_ptr(const Geometry& g, uint8_t* records, int b, int h,
+                                               int grp) {
+  return records + (unit_index(g, b, h) * g.gcap + grp) * static_cast<size_t>(g.record_bytes);
+}
+
+// Scratch regions inside pnmix_cache::scratch.
+__host__ __device__ __forceinline__ size_t scratch_kmax_offset() { return 0; }
+__host__ __device__ __forceinline__ size_t scratch_select_ticket_offset(int B, int Hkv) {
+  return static_cast<size_t>(B) * Hkv * 64;
+}
+__host__ __device__ __forceinline__ size_t scratch_append_ticket_offset(int B, int Hkv) {
+  return static_cast<size_t>(B) * Hkv * 65;
+}
+__host__ __device__ __forceinline__ size_t scratch_words(int B, int Hkv) {
+  return static_cast<size_t>(B) * Hkv * 65 + B;
+}
+
+// Launchers (one translation unit each).
+cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int n_window,
+                                const uint16_t* k, int L, int ld, const pnmix_cache& c,
+                                cudaStream_t s);
+cudaError_t launch_quantize_keys(const Geometry& g, const uint16_t* k, int L, int ld,
+                                 const pnmix_cache& c, cudaStream_t s);
+cudaError_t launch_quantize_values(const Geometry& g, const uint16_t* v, int L, int ld,
+                                   const pnmix_cache& c, cudaStream_t s);
+cudaError_t launch_append(const Geometry& g, const uint16_t* k_new, const uint16_t* v_new,
+                          const pnmix_cache& c, cudaStream_t s);
+
+// Decode: split count for a batch / context bound, and the workspace it needs.
+int decode_splits(const Geometry& g, int max_context);
+size_t decode_workspace_bytes(const Geometry& g, int max_context);
+cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c,
+                          int max_context, float* out, void* ws, cudaStream_t s);
+
+}  // namespace pnmix

@@ -1,0 +1,282 @@
+// pnmix.cu -- the C ABI of include/pnmix.h: host-side validation, the cache layout and
+// the launches.  No entry point allocates, frees or synchronises (except
+// pnmix_read_error, which is a synchronous read by definition).
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "decode_common.cuh"
+
+namespace pnmix {
+
+static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capacity, Geometry* g) {
+  if (!cfg || !g) return PNMIX_ERR_INVALID_ARG;
+  if (cfg->n_q_heads <= 0 || cfg->n_kv_heads <= 0 || batch < 0 || capacity < 0)
+    return PNMIX_ERR_INVALID_ARG;
+  if (cfg->n_q_heads % cfg->n_kv_heads) return PNMIX_ERR_INVALID_ARG;
+  if (cfg->head_dim != 128 || cfg->group_tokens != 32 || cfg->residual_tokens != 32 ||
+      cfg->value_group != 32 || cfg->value_bits != 2)
+    return PNMIX_ERR_UNSUPPORTED;
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
+  if (G < 1 || G > kMaxG) return PNMIX_ERR_UNSUPPORTED;
+  const bool bits_ok = (cfg->key_bits_hi == 4 && cfg->key_bits_lo == 2) ||
+                       (cfg->key_bits_hi == 2 && cfg->key_bits_lo == 1);
+  if (!bits_ok) return PNMIX_ERR_UNSUPPORTED;
+  const int k = cfg->n_salient_pairs;
+  if (k != 0 && k != 8 && k != 16 && k != 32 && k != 64) return PNMIX_ERR_UNSUPPORTED;
+  const int nhs = 2 * k / 16;
+  if ((nhs * cfg->key_bits_hi) % 2 || ((8 - nhs) * cfg->key_bits_lo) % 2) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->saliency_window < 1 || cfg->saliency_window > 1024) return PNMIX_ERR_UNSUPPORTED;
+  g->B = batch;
+  g->Hq = cfg->n_q_heads;
+  g->Hkv = cfg->n_kv_heads;
+  g->G = G;
+  g->k = k;
+  g->nhi = 2 * k;
+  g->nhs = nhs;
+  g->bhi = cfg->key_bits_hi;
+  g->blo = cfg->key_bits_lo;
+  g->bv = cfg->value_bits;
+  g->wh = nhs * g->bhi / 2;
+  g->wl = (8 - nhs) * g->blo / 2;
+  g->kc_bytes = 128 * (g->wh + g->wl);
+  g->record_bytes = g->kc_bytes + 2048;
+  g->capacity = capacity;
+  g->gcap = capacity / kGroup;
+  g->scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale : 1.0f / sqrtf(128.0f);
+  return PNMIX_OK;
+}
+
+struct Layout {
+  size_t records, k_resid, v_resid, len, pair_idx, pair_mask, perm, pair_scores, scratch, error, total;
+};
+
+static Layout cache_layout(const Geometry& g) {
+  Layout L;
+  const size_t units = static_cast<size_t>(g.B) * g.Hkv;
+  size_t off = 0;
+  L.records = off;
+  off = align256(off + units * g.gcap * static_cast<size_t>(g.record_bytes));
+  L.k_resid = off;
+  off = align256(off + units * kGroup * kHeadDim * 2);
+  L.v_resid = off;
+  off = align256(off + units * kGroup * kHeadDim * 2);
+  L.len = off;
+  off = align256(off + static_cast<size_t>(g.B) * 4);
+  L.pair_idx = off;
+  off = align256(off + units * 64);
+  L.pair_mask = off;
+  off = align256(off + units * 8);
+  L.perm = off;
+  off = align256(off + units * 128);
+  L.pair_scores = off;
+  off = align256(off + units * 64 * 4);
+  L.scratch = off;
+  off = align256(off + scratch_words(g.B, g.Hkv) * 4);
+  L.error = off;
+  off = align256(off + 4);
+  L.total = off;
+  return L;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static pnmix_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PNMIX_OK : PNMIX_ERR_CUDA; }
+
+static pnmix_status check_cache(const Geometry& g, const pnmix_cache* c) {
+  if (!c || !c->base || !c->records) return PNMIX_ERR_INVALID_ARG;
+  if (c->batch != g.B || c->n_kv_heads != g.Hkv || c->record_bytes != g.record_bytes)
+    return PNMIX_ERR_INVALID_ARG;
+  return PNMIX_OK;
+}
+
+int decode_splits(const Geometry& g, int max_context) {
+  const int units = g.B * g.Hkv;
+  const int groups = max_context > 0 ? (max_context + kGroup - 1) / kGroup : 1;
+  int S = (4 * 148 + units - 1) / units;
+  if (S > groups) S = groups;
+  if (S > 256) S = 256;
+  if (S < 1) S = 1;
+  return S;
+}
+
+size_t decode_workspace_bytes(const Geometry& g, int max_context) {
+  const int S = decode_splits(g, max_context);
+  const int units = g.B * g.Hkv;
+  return decode_partial_bytes(units, S, g.G) + align256(sizeof(uint32_t) * units);
+}
+
+cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int max_context,
+                          float* out, void* ws, cudaStream_t s) {
+  const int S = decode_splits(g, max_context);
+  const int units = g.B * g.Hkv;
+  DecodeWs w;
+  w.part = static_cast<float*>(ws);
+  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(units, S, g.G));
+  return launch_decode_simt(g, q, c, S, out, w, s);
+}
+
+}  // namespace pnmix
+
+using namespace pnmix;
+
+extern "C" {
+
+size_t pnmix_record_bytes(const pnmix_config* cfg) {
+  Geometry g;
+  if (make_geometry(cfg, 1, 32, &g) != PNMIX_OK) return 0;
+  return static_cast<size_t>(g.record_bytes);
+}
+
+pnmix_status pnmix_cache_bytes(const pnmix_config* cfg, int batch, int capacity_tokens,
+                               size_t* total_bytes) {
+  if (!total_bytes || batch <= 0 || capacity_tokens <= 0 || capacity_tokens % kGroup)
+    return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  pnmix_status st = make_geometry(cfg, batch, capacity_tokens, &g);
+  if (st != PNMIX_OK) return st;
+  *total_bytes = cache_layout(g).total;
+  return PNMIX_OK;
+}
+
+pnmix_status pnmix_cache_init(const pnmix_config* cfg, int batch, int capacity_tokens,
+                              void* device_base, size_t bytes, pnmix_cache* out) {
+  if (!out || !device_base) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(device_base, 256)) return PNMIX_ERR_ALIGNMENT;
+  size_t need = 0;
+  pnmix_status st = pnmix_cache_bytes(cfg, batch, capacity_tokens, &need);
+  if (st != PNMIX_OK) return st;
+  if (bytes < need) return PNMIX_ERR_CAPACITY;
+  Geometry g;
+  make_geometry(cfg, batch, capacity_tokens, &g);
+  Layout L = cache_layout(g);
+  char* base = static_cast<char*>(device_base);
+  memset(out, 0, sizeof(*out));
+  out->batch = batch;
+  out->capacity_tokens = capacity_tokens;
+  out->n_kv_heads = g.Hkv;
+  out->record_bytes = g.record_bytes;
+  out->records = reinterpret_cast<uint8_t*>(base + L.records);
+  out->k_resid = reinterpret_cast<uint16_t*>(base + L.k_resid);
+  out->v_resid = reinterpret_cast<uint16_t*>(base + L.v_resid);
+  out->len = reinterpret_cast<int32_t*>(base + L.len);
+  out->pair_idx = reinterpret_cast<uint8_t*>(base + L.pair_idx);
+  out->pair_mask = reinterpret_cast<uint64_t*>(base + L.pair_mask);
+  out->perm = reinterpret_cast<uint8_t*>(base + L.perm);
+  out->pair_scores = reinterpret_cast<float*>(base + L.pair_scores);
+  out->scratch = reinterpret_cast<uint32_t*>(base + L.scratch);
+  out->error = reinterpret_cast<uint32_t*>(base + L.error);
+  out->base = device_base;
+  out->total_bytes = L.total;
+  return PNMIX_OK;
+}
+
+pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream) {
+  if (!cache || !cache->base) return PNMIX_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(cache->base, 0, cache->total_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_select_pairs(const pnmix_config* cfg, const uint16_t* q_window, int n_window,
+                                const uint16_t* k, int L, int ld_tokens, pnmix_cache* cache,
+                                void* stream) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, &g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
+  if (!q_window || !k || L < 1 || ld_tokens < L) return PNMIX_ERR_INVALID_ARG;
+  const int want_w = L < cfg->saliency_window ? L : cfg->saliency_window;
+  if (n_window != want_w) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(q_window, 16) || !aligned(k, 16)) return PNMIX_ERR_ALIGNMENT;
+  return cuda_status(launch_select_pairs(g, q_window, n_window, k, L, ld_tokens, *cache,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+static pnmix_status check_prefill(const pnmix_config* cfg, const uint16_t* x, int L, int ld,
+                                  const pnmix_cache* cache, Geometry* g) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(*g, cache)) != PNMIX_OK) return st;
+  if (!x || L < 0 || ld < L || ld < 1) return PNMIX_ERR_INVALID_ARG;
+  if (L > cache->capacity_tokens) return PNMIX_ERR_CAPACITY;
+  if (!aligned(x, 16)) return PNMIX_ERR_ALIGNMENT;
+  return PNMIX_OK;
+}
+
+pnmix_status pnmix_quantize_keys(const pnmix_config* cfg, const uint16_t* k, int L, int ld_tokens,
+                                 pnmix_cache* cache, void* stream) {
+  Geometry g;
+  pnmix_status st = check_prefill(cfg, k, L, ld_tokens, cache, &g);
+  if (st != PNMIX_OK) return st;
+  return cuda_status(launch_quantize_keys(g, k, L, ld_tokens, *cache, static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_quantize_values(const pnmix_config* cfg, const uint16_t* v, int L, int ld_tokens,
+                                   pnmix_cache* cache, void* stream) {
+  Geometry g;
+  pnmix_status st = check_prefill(cfg, v, L, ld_tokens, cache, &g);
+  if (st != PNMIX_OK) return st;
+  return cuda_status(launch_quantize_values(g, v, L, ld_tokens, *cache, static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_append(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
+                          pnmix_cache* cache, void* stream) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, &g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
+  if (!k_new || !v_new) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return PNMIX_ERR_ALIGNMENT;
+  return cuda_status(launch_append(g, k_new, v_new, *cache, static_cast<cudaStream_t>(stream)));
+}
+
+size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context) {
+  Geometry g;
+  if (batch <= 0 || make_geometry(cfg, batch, 32, &g) != PNMIX_OK) return 0;
+  return decode_workspace_bytes(g, max_context);
+}
+
+pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
+                                    const pnmix_cache* cache, int max_context, float* out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, &g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
+  if (!q || !out || !workspace || max_context < 0) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
+  return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error) {
+  if (!cache || !cache->error || !host_error) return PNMIX_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemcpy(host_error, cache->error, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return PNMIX_ERR_CUDA;
+  if (clear) {
+    e = cudaMemset(cache->error, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return PNMIX_ERR_CUDA;
+  }
+  return *host_error ? PNMIX_ERR_DEVICE : PNMIX_OK;
+}
+
+const char* pnmix_status_string(pnmix_status status) {
+  switch (status) {
+    case PNMIX_OK: return "ok";
+    case PNMIX_ERR_INVALID_ARG: return "invalid argument";
+    case PNMIX_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PNMIX_ERR_CAPACITY: return "capacity exceeded";
+    case PNMIX_ERR_CUDA: return "CUDA runtime error";
+    case PNMIX_ERR_ALIGNMENT: return "misaligned pointer";
+    case PNMIX_ERR_DEVICE: return "device error word set";
+  }
+  return "unknown status";
+}
+
+const char* pnmix_version(void) { return "pnmix 0.1"; }
+
+}  // extern "C"

@@ -111,6 +111,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define PNMIX_API __attribute__((visibility("default")))
+#else
+#define PNMIX_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -174,13 +180,13 @@ typedef struct {
 } pnmix_cache;
 
 /* Bytes of one group record (layout item list above); 0 if unsupported. */
-size_t pnmix_record_bytes(const pnmix_config* cfg);
+PNMIX_API size_t pnmix_record_bytes(const pnmix_config* cfg);
 
 /*
  * Bytes a cache of `batch` sequences and `capacity_tokens` tokens each needs.
  * capacity_tokens must be a positive multiple of 32.  Host-only.
  */
-pnmix_status pnmix_cache_bytes(const pnmix_config* cfg, int batch, int capacity_tokens,
+PNMIX_API pnmix_status pnmix_cache_bytes(const pnmix_config* cfg, int batch, int capacity_tokens,
                                size_t* total_bytes);
 
 /*
@@ -189,11 +195,11 @@ pnmix_status pnmix_cache_bytes(const pnmix_config* cfg, int batch, int capacity_
  * buffer must be zero-filled before the first pnmix call that uses it
  * (pnmix_cache_reset does that).
  */
-pnmix_status pnmix_cache_init(const pnmix_config* cfg, int batch, int capacity_tokens,
+PNMIX_API pnmix_status pnmix_cache_init(const pnmix_config* cfg, int batch, int capacity_tokens,
                               void* device_base, size_t bytes, pnmix_cache* out);
 
 /* Zero the whole cache buffer on `stream` (lengths 0, no salient pairs, no error). */
-pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream);
+PNMIX_API pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream);
 
 /*
  * Prefill step 1 (PN-Mix abstract: salient pairs are picked once at prefill from
@@ -206,7 +212,7 @@ pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream);
  * n_window must equal min(L, saliency_window); 1 <= L <= ld_tokens.
  * Writes pair_idx, pair_mask, perm and pair_scores of every (b, h).
  */
-pnmix_status pnmix_select_pairs(const pnmix_config* cfg, const uint16_t* q_window, int n_window,
+PNMIX_API pnmix_status pnmix_select_pairs(const pnmix_config* cfg, const uint16_t* q_window, int n_window,
                                 const uint16_t* k, int L, int ld_tokens, pnmix_cache* cache,
                                 void* stream);
 
@@ -216,7 +222,7 @@ pnmix_status pnmix_select_pairs(const pnmix_config* cfg, const uint16_t* q_windo
  * copies the last L % 32 rows into the K residual and sets len[b] = L.
  * Uses the salient set written by pnmix_select_pairs.  L <= capacity_tokens.
  */
-pnmix_status pnmix_quantize_keys(const pnmix_config* cfg, const uint16_t* k, int L, int ld_tokens,
+PNMIX_API pnmix_status pnmix_quantize_keys(const pnmix_config* cfg, const uint16_t* k, int L, int ld_tokens,
                                  pnmix_cache* cache, void* stream);
 
 /*
@@ -224,7 +230,7 @@ pnmix_status pnmix_quantize_keys(const pnmix_config* cfg, const uint16_t* k, int
  * pnmix_quantize_keys, into the value part of the records and the V residual;
  * sets len[b] = L.
  */
-pnmix_status pnmix_quantize_values(const pnmix_config* cfg, const uint16_t* v, int L, int ld_tokens,
+PNMIX_API pnmix_status pnmix_quantize_values(const pnmix_config* cfg, const uint16_t* v, int L, int ld_tokens,
                                    pnmix_cache* cache, void* stream);
 
 /*
@@ -235,7 +241,7 @@ pnmix_status pnmix_quantize_values(const pnmix_config* cfg, const uint16_t* v, i
  * prefill's salient pairs; then len[b] += 1.  A sequence whose len[b] equals
  * capacity_tokens is left unchanged and PNMIX_DEVERR_APPEND_FULL is raised.
  */
-pnmix_status pnmix_append(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
+PNMIX_API pnmix_status pnmix_append(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
                           pnmix_cache* cache, void* stream);
 
 /*
@@ -243,7 +249,7 @@ pnmix_status pnmix_append(const pnmix_config* cfg, const uint16_t* k_new, const 
  * lengths are at most max_context.  The workspace must be zero-filled before its
  * first use; every call leaves it ready for the next one.
  */
-size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context);
+PNMIX_API size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context);
 
 /*
  * Decode step 2 (attention over the quantized cache).  q: bf16 [B][Hq][128]
@@ -252,18 +258,18 @@ size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context
  * max_context is an upper bound on len[b] used to size the split-K grid; the
  * result does not depend on it.  A sequence with len[b] == 0 gets zeros.
  */
-pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
+PNMIX_API pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
                                     const pnmix_cache* cache, int max_context, float* out,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronously read (and, if clear != 0, zero) the device error word.  Host pointer out. */
-pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error);
+PNMIX_API pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error);
 
 /* Static string for a status code. */
-const char* pnmix_status_string(pnmix_status status);
+PNMIX_API const char* pnmix_status_string(pnmix_status status);
 
 /* Library version, e.g. "pnmix 0.1". */
-const char* pnmix_version(void);
+PNMIX_API const char* pnmix_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,112 @@
+"""The C ABI on the host: every declared symbol is exported and host-side
+validation answers without a GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import decode_attention_prefill_b200 as pm
+import oracle
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pnmix.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"PNMIX_API\s+[\w\s\*]+?\b(pnmix_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared()
+    assert len(names) >= 13
+    lib = ctypes.CDLL(pm.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(pm.EXPORTED)
+
+
+def test_version_and_status_strings():
+    assert pm.version().startswith("pnmix")
+    assert pm._lib.pnmix_status_string(0) == b"ok"
+    assert pm._lib.pnmix_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("k,bhi,blo", [(0, 4, 2), (8, 4, 2), (16, 4, 2), (32, 4, 2), (64, 4, 2),
+                                       (0, 2, 1), (16, 2, 1), (32, 2, 1), (64, 2, 1)])
+def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
+    cfg = pm.Config.make(32, 8, bhi, blo, k)
+    assert pm.record_bytes(cfg) == oracle.record_bytes(k, bhi, blo) > 0
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(n_salient_pairs=4), pm.ERR_UNSUPPORTED),
+    (dict(n_salient_pairs=8, key_bits_hi=2, key_bits_lo=1), pm.ERR_UNSUPPORTED),
+    (dict(key_bits_hi=8), pm.ERR_UNSUPPORTED),
+    (dict(head_dim=64), pm.ERR_UNSUPPORTED),
+    (dict(n_q_heads=36, n_kv_heads=4), pm.ERR_UNSUPPORTED),   # G = 9
+    (dict(n_q_heads=30, n_kv_heads=4), pm.ERR_INVALID_ARG),   # not a multiple
+    (dict(value_bits=4), pm.ERR_UNSUPPORTED),
+    (dict(saliency_window=0), pm.ERR_UNSUPPORTED),
+])
+def test_config_validation(change, status):
+    cfg = pm.Config.make(32, 8)
+    for k, v in change.items():
+        setattr(cfg, k, v)
+    out = ctypes.c_size_t(0)
+    assert pm._lib.pnmix_cache_bytes(ctypes.byref(cfg), 2, 64, ctypes.byref(out)) == status
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_cache_init_carves_aligned_regions_without_touching_memory():
+    cfg = pm.Config.make(32, 8)
+    nbytes = pm.cache_bytes(cfg, 4, 1024)
+    c = pm.Cache()
+    fake = 1 << 40   # never dereferenced: cache_init is host-only
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), 4, 1024, ctypes.c_void_p(fake), nbytes,
+                                    ctypes.byref(c)) == pm.OK
+    ptrs = [c.records, c.k_resid, c.v_resid, c.len, c.pair_idx, c.pair_mask, c.perm, c.pair_scores,
+            c.scratch, c.error]
+    assert all(p % 256 == 0 for p in ptrs) and ptrs == sorted(ptrs)
+    assert c.k_resid - c.records >= 4 * 8 * 32 * 3200
+    assert c.total_bytes == nbytes
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), 4, 1024, ctypes.c_void_p(fake + 16), nbytes,
+                                    ctypes.byref(c)) == pm.ERR_ALIGNMENT
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), 4, 1024, ctypes.c_void_p(fake), nbytes - 1,
+                                    ctypes.byref(c)) == pm.ERR_CAPACITY
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), 4, 1000, ctypes.c_void_p(fake), nbytes,
+                                    ctypes.byref(c)) == pm.ERR_INVALID_ARG
+
+
+def _fake_cache(cfg, B=2, cap=256):
+    c = pm.Cache()
+    nbytes = pm.cache_bytes(cfg, B, cap)
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), B, cap, ctypes.c_void_p(1 << 40), nbytes,
+                                    ctypes.byref(c)) == pm.OK
+    return c
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_entry_points_reject_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2)
+    c = _fake_cache(cfg)
+    P = ctypes.c_void_p(1 << 41)
+    odd = ctypes.c_void_p((1 << 41) + 2)
+    L = pm._lib
+    # window must be min(L, W)
+    assert L.pnmix_select_pairs(ctypes.byref(cfg), P, 63, P, 100, 128, ctypes.byref(c), None) == pm.ERR_INVALID_ARG
+    assert L.pnmix_select_pairs(ctypes.byref(cfg), P, 64, P, 100, 99, ctypes.byref(c), None) == pm.ERR_INVALID_ARG
+    assert L.pnmix_select_pairs(ctypes.byref(cfg), odd, 64, P, 100, 128, ctypes.byref(c), None) == pm.ERR_ALIGNMENT
+    assert L.pnmix_select_pairs(ctypes.byref(cfg), None, 64, P, 100, 128, ctypes.byref(c), None) == pm.ERR_INVALID_ARG
+    assert L.pnmix_quantize_keys(ctypes.byref(cfg), P, 257, 300, ctypes.byref(c), None) == pm.ERR_CAPACITY
+    assert L.pnmix_quantize_values(ctypes.byref(cfg), odd, 10, 10, ctypes.byref(c), None) == pm.ERR_ALIGNMENT
+    assert L.pnmix_append(ctypes.byref(cfg), P, None, ctypes.byref(c), None) == pm.ERR_INVALID_ARG
+    ws = pm.workspace_bytes(cfg, 2, 256)
+    assert ws > 0
+    assert L.pnmix_decode_attention(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, P, ws - 1, None) == pm.ERR_CAPACITY
+    assert L.pnmix_decode_attention(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, odd, ws, None) == pm.ERR_ALIGNMENT
+    other = pm.Config.make(8, 2, n_salient_pairs=16)   # record size differs from the cache's
+    assert L.pnmix_decode_attention(ctypes.byref(other), P, ctypes.byref(c), 256, P, P, ws, None) == pm.ERR_INVALID_ARG

@@ -1,0 +1,117 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the
+same seeded inputs.  Bit-exact for pair indices, masks, scores, codes, scales,
+zero points, packed records, residual rows and lengths; attention within
+max-abs 2e-3 and relative L2 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_harness import Case, assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_workload_end_to_end():
+    c = Case(1, 1, 1, 512)
+    c.prefill()
+    got, want = c.attend(c.query(512))
+    assert_close(got, want)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", [
+    (1, 1, 1, 1, 8, 4, 2),
+    (1, 4, 1, 31, 8, 4, 2),
+    (2, 8, 2, 32, 8, 4, 2),
+    (2, 8, 2, 33, 0, 4, 2),
+    (1, 7, 1, 517, 16, 4, 2),
+    (3, 8, 1, 100, 64, 4, 2),
+    (2, 16, 2, 200, 16, 2, 1),
+    (1, 28, 4, 96, 32, 2, 1),
+    (2, 4, 4, 300, 32, 4, 2),
+    (1, 8, 1, 64, 0, 2, 1),
+    (4, 32, 8, 1000, 8, 4, 2),
+])
+def test_prefill_and_decode_shapes(B, Hq, Hkv, L, k, bhi, blo):
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + k)
+    c.prefill()
+    got, want = c.attend(c.query(L))
+    assert_close(got, want)
+
+
+def test_append_stream_crosses_flush_boundaries():
+    c = Case(2, 8, 2, 40, extra_tokens=110, seed=3)
+    c.prefill()
+    for t in range(40, 150):
+        c.append(t)
+        if t in (40, 62, 63, 64, 95, 149):
+            got, want = c.attend(c.query(t))
+            assert_close(got, want)
+    c.check_state()
+
+
+def test_append_beyond_capacity_sets_the_error_word_and_changes_nothing():
+    c = Case(1, 4, 1, 64, capacity=64)
+    c.prefill()
+    assert c.cache.read_error() == 0
+    before = c.cache.records().clone()
+    c.cache.append(to_dev(c.kin[:, :, 0].copy()), to_dev(c.vin[:, :, 0].copy()))
+    torch.cuda.synchronize()
+    assert c.cache.read_error() == 0x1
+    assert c.cache.read_error() == 0          # cleared by the read
+    assert int(c.cache.lengths()[0]) == 64
+    assert torch.equal(before, c.cache.records())
+
+
+def test_empty_cache_attends_to_nothing():
+    import decode_attention_prefill_b200 as pm
+    cfg = pm.Config.make(8, 2)
+    cache = pm.PNMixCache(cfg, 2, 64)
+    q = torch.randn(2, 8, 128, device="cuda").to(torch.bfloat16)
+    out = cache.attend(q)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out) == 0
+
+
+def test_decode_is_repeatable_and_leaves_the_workspace_ready():
+    c = Case(2, 8, 2, 300, seed=11)
+    c.prefill()
+    q = c.query(300)
+    a, want = c.attend(q)
+    b, _ = c.attend(q)
+    np.testing.assert_array_equal(a, b)
+    assert_close(a, want)
+
+
+def test_split_count_does_not_change_the_result_beyond_rounding():
+    c = Case(1, 4, 1, 2000, seed=12)
+    c.prefill()
+    q = to_dev(c.query(2000))
+    outs = []
+    for mc in (32, 500, 2000, 8192):
+        import decode_attention_prefill_b200 as pm
+        ws = torch.zeros(pm.workspace_bytes(c.cfg, 1, mc), dtype=torch.uint8, device="cuda")
+        out = torch.empty(1, 4, 128, dtype=torch.float32, device="cuda")
+        pm.pnmix_decode_attention(c.cfg, q, c.cache, out, workspace=ws, max_context=mc)
+        outs.append(out.cpu().numpy())
+    want = c.ocache.attend(c.query(2000))
+    for o in outs:
+        assert_close(o, want)
+
+
+@pytest.mark.slow
+def test_llama3_8b_decode_step_full_size():
+    """Batch 8, 32/8 heads, context 8192: every record and every head."""
+    c = Case(8, 32, 8, 8192, seed=0)
+    c.prefill()
+    got, want = c.attend(c.query(8192))
+    assert_close(got, want)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("k,bhi,blo", [(0, 4, 2), (8, 4, 2), (16, 4, 2), (32, 4, 2), (16, 2, 1), (32, 2, 1)])
+def test_sweep_128k_bit_points(k, bhi, blo):
+    """Batch 2, 28/4 heads (GQA 7), context 131072, at each bit point."""
+    c = Case(2, 28, 4, 131072, k, bhi, blo, seed=0)
+    c.prefill()
+    got, want = c.attend(c.query(131072))
+    assert_close(got, want)

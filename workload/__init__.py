@@ -57,6 +57,12 @@ def _load():
                                     ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                     ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                     ctypes.c_void_p, ctypes.c_int]
+            lib.wl_fill_block.restype = ctypes.c_int
+            lib.wl_fill_block.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_int64, ctypes.c_double,
+                                          ctypes.c_double, ctypes.c_double, ctypes.c_void_p,
+                                          ctypes.c_int]
             lib.wl_outlier_pairs.restype = None
             lib.wl_outlier_pairs.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_void_p]
@@ -98,6 +104,19 @@ def rows(seed: int, tensor: int, batch: int, heads: int, t0: int, n: int, *, gro
     if rc != 0:
         raise ValueError("wl_fill rejected its arguments")
     return out
+
+
+def unit_rows(seed: int, tensor: int, b: int, head0: int, heads: int, t0: int, n: int, *,
+              group: int = 1, threads: int | None = None) -> np.ndarray:
+    """Rows of batch row b, heads head0 .. head0+heads-1: uint16 [heads][n][128]."""
+    lib = _load()
+    out = np.empty((1, heads, n, 128), dtype=np.uint16)
+    rc = lib.wl_fill_block(seed, tensor, b, 1, head0, heads, group, t0, n, n, THETA,
+                           KEY_OUTLIER_SCALE, QUERY_OUTLIER_SCALE, out.ctypes.data,
+                           threads or default_threads())
+    if rc != 0:
+        raise ValueError("wl_fill_block rejected its arguments")
+    return out[0]
 
 
 def outlier_pairs(seed: int, query: bool, b: int, kv_head: int) -> list[int]:

@@ -172,6 +172,7 @@ void wl_row_double(uint64_t seed, int tensor, int G, double theta, double key_sc
 
 typedef struct {
   wl_params P;
+  int b0, h0;      /* first batch row and head of the block */
   int B, H, n;
   int64_t t0;
   int64_t ld;      /* rows between consecutive heads in out */
@@ -185,19 +186,20 @@ static void* wl_worker(void* arg) {
     int64_t bh = r / J->n;
     int64_t t = r % J->n;
     int b = (int)(bh / J->H), h = (int)(bh % J->H);
-    wl_one_row(&J->P, b, h, J->t0 + t, J->out + (bh * J->ld + t) * 128);
+    wl_one_row(&J->P, J->b0 + b, J->h0 + h, J->t0 + t, J->out + (bh * J->ld + t) * 128);
   }
   return NULL;
 }
 
 /*
- * Fill out[b][h][t][128] (row stride: head stride ld rows) with the rows of
- * positions t0 .. t0+n-1 for every (b, h), using nthreads threads.
- * tensor: 0 = Q (h is a query head), 1 = K, 2 = V.
+ * Fill out[b][h][t][128] (head stride ld rows) with the rows of positions
+ * t0 .. t0+n-1 of batch rows b0 .. b0+B-1 and heads h0 .. h0+H-1, using nthreads
+ * threads.  tensor: 0 = Q (heads are query heads), 1 = K, 2 = V.
  */
-int wl_fill(uint64_t seed, int tensor, int B, int H, int G, int64_t t0, int n, int64_t ld,
-            double theta, double key_scale, double query_scale, uint16_t* out, int nthreads) {
-  if (B <= 0 || H <= 0 || n <= 0 || ld < n || G <= 0 || !out) return 1;
+int wl_fill_block(uint64_t seed, int tensor, int b0, int B, int h0, int H, int G, int64_t t0, int n,
+                  int64_t ld, double theta, double key_scale, double query_scale, uint16_t* out,
+                  int nthreads) {
+  if (B <= 0 || H <= 0 || n <= 0 || ld < n || G <= 0 || !out || b0 < 0 || h0 < 0) return 1;
   if (nthreads < 1) nthreads = 1;
   if (nthreads > 256) nthreads = 256;
   int64_t rows = (int64_t)B * H * n;
@@ -212,6 +214,8 @@ int wl_fill(uint64_t seed, int tensor, int B, int H, int G, int64_t t0, int n, i
     J->P.theta = theta;
     J->P.key_scale = key_scale;
     J->P.query_scale = query_scale;
+    J->b0 = b0;
+    J->h0 = h0;
     J->B = B;
     J->H = H;
     J->n = n;
@@ -228,4 +232,11 @@ int wl_fill(uint64_t seed, int tensor, int B, int H, int G, int64_t t0, int n, i
   for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, wl_worker, &jobs[i]);
   for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
   return 0;
+}
+
+/* The whole batch from row 0 and head 0. */
+int wl_fill(uint64_t seed, int tensor, int B, int H, int G, int64_t t0, int n, int64_t ld,
+            double theta, double key_scale, double query_scale, uint16_t* out, int nthreads) {
+  return wl_fill_block(seed, tensor, 0, B, 0, H, G, t0, n, ld, theta, key_scale, query_scale, out,
+                       nthreads);
 }
