@@ -38,7 +38,7 @@ EXPORTED = [
     "pnmix_record_bytes", "pnmix_cache_bytes", "pnmix_cache_init", "pnmix_cache_reset",
     "pnmix_select_pairs", "pnmix_quantize_keys", "pnmix_quantize_values", "pnmix_append",
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
-    "pnmix_status_string", "pnmix_version",
+    "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
 ]
 
 
@@ -86,6 +86,7 @@ _SIGS = {
     "pnmix_read_error": (_i, [_KP, _i, ctypes.POINTER(ctypes.c_uint32)]),
     "pnmix_status_string": (ctypes.c_char_p, [_i]),
     "pnmix_version": (ctypes.c_char_p, []),
+    "pnmix_decode_attention_noalloc": (_i, [_CP, _vp, _KP, _i, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)

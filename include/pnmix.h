@@ -262,6 +262,24 @@ PNMIX_API pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uin
                                     const pnmix_cache* cache, int max_context, float* out,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * pnmix_decode_attention without a caller-provided workspace.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory (a plugin whose host runtime owns all device memory, or an interface
+ * with no slot for a workspace pointer).  Same arguments and result as
+ * pnmix_decode_attention minus the workspace: the split-K scratch comes from a
+ * 4 MiB array inside the library image, held on every device that loads the
+ * library until the process exits.  A call whose pnmix_workspace_bytes exceeds
+ * 4 MiB returns PNMIX_ERR_CAPACITY and enqueues nothing.  Every call on a device
+ * shares that array and clears the part it uses first (a memset on `stream`), so
+ * calls that overlap on the GPU race and must be serialised by the caller.  The
+ * first call on each device looks up the array's address with that device
+ * current; make it before any stream capture.  Allocates nothing.
+ */
+PNMIX_API pnmix_status pnmix_decode_attention_noalloc(const pnmix_config* cfg, const uint16_t* q,
+                                                      const pnmix_cache* cache, int max_context,
+                                                      float* out, void* stream);
+
 /* Synchronously read (and, if clear != 0, zero) the device error word.  Host pointer out. */
 PNMIX_API pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error);
 
