@@ -150,8 +150,7 @@ cudaError_t launch_quantize_values(const Geometry& g, const uint16_t* v, int L, 
 cudaError_t launch_append(const Geometry& g, const uint16_t* k_new, const uint16_t* v_new,
                           const pnmix_cache& c, cudaStream_t s);
 
-// Decode: split count for a batch / context bound, and the workspace it needs.
-int decode_splits(const Geometry& g, int max_context);
+// Decode: the workspace a batch / context bound needs, and the launch.
 size_t decode_workspace_bytes(const Geometry& g, int max_context);
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c,
                           int max_context, float* out, void* ws, cudaStream_t s);

@@ -1,10 +1,19 @@
-// decode_common.cuh -- split-K workspace and the fused combine of the decode kernels.
+// decode_common.cuh -- work partition, split-K workspace and fused combine of the decode
+// kernels.
 //
-// Every CTA of a (b, KV head) writes one partial (m, l, acc[128]) per query head of the
-// group; m is the running max in the log2 domain, l the sum of 2^(logit - m) and acc the
-// matching weighted sum of values.  The CTA that takes the last ticket of its unit merges
-// the S partials:  m* = max m_s,  out = sum_s acc_s 2^(m_s - m*) / sum_s l_s 2^(m_s - m*).
-// Nothing waits: the other CTAs simply exit after taking their ticket.
+// Work items.  Unit u = (b, h) owns len[b]/32 full-group items followed by one residual
+// item (the len[b] % 32 bf16 tokens, possibly none).  Items are numbered b-major, then h,
+// then item, T in total.  A grid of N CTAs splits [0, T) evenly: CTA i takes
+// [floor(i*T/N), floor((i+1)*T/N)).  Every CTA computes T from len[] itself, so the grid
+// is balanced for any mix of lengths without the host knowing them.
+//
+// Partials.  The piece of unit u that CTA i covers (a "segment") produces one partial
+// (m, l, acc[128]) per query head: m is the running max in the log2 domain, l the sum of
+// 2^(logit - m) and acc the matching weighted sum of values.  It goes to slot i + u; the
+// slots of u are contiguous and disjoint from other units'.  The CTA that takes the last
+// ticket of u (the partition tells how many segments u has) merges them:
+//     m* = max m_s,  out = sum_s acc_s 2^(m_s - m*) / sum_s l_s 2^(m_s - m*).
+// Nothing waits: the other CTAs take their ticket and move on.
 #pragma once
 
 #include "common.cuh"
@@ -12,61 +21,129 @@
 namespace pnmix {
 
 constexpr int kPartialStride = 2 + kHeadDim;   // m, l, acc[128]
+constexpr int kMaxDecodeCtas = 1024;           // grid cap of the decode kernels
 
 struct DecodeWs {
-  float* part;         // [units][S][G][kPartialStride]
+  float* part;         // [slots][G][kPartialStride]
   uint32_t* tickets;   // [units], zero between calls
+  int N;               // CTAs of the launch
 };
 
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-__host__ __device__ __forceinline__ size_t decode_partial_bytes(int units, int S, int G) {
-  return align256(sizeof(float) * static_cast<size_t>(units) * S * G * kPartialStride);
+__host__ __device__ __forceinline__ size_t decode_partial_bytes(int slots, int G) {
+  return align256(sizeof(float) * static_cast<size_t>(slots) * G * kPartialStride);
 }
 
-__device__ __forceinline__ void write_partial(const DecodeWs& ws, int unit, int split, int S, int G,
-                                              int hh, int c, float m, float l, float acc) {
-  float* p = ws.part + ((static_cast<size_t>(unit) * S + split) * G + hh) * kPartialStride;
-  if (c == 0) {
-    p[0] = m;
-    p[1] = l;
+// CTA that owns item x.
+__device__ __forceinline__ int cta_of(long long x, long long T, int N) {
+  return static_cast<int>(((x + 1) * N - 1) / T);
+}
+
+__device__ __forceinline__ long long total_items(const Geometry& g, const int32_t* len) {
+  long long T = 0;
+  for (int b = 0; b < g.B; ++b) T += static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+  return T;
+}
+
+struct Segment {
+  int b, h, unit;
+  int lo, hi;          // items [lo, hi) of the unit; item len/32 is the residual item
+  int ng, nr;          // full groups and residual tokens of the unit
+  int first, last;     // CTAs covering the unit
+};
+
+// Calls fn(seg) for every segment of this CTA, in item order.  All threads of the CTA
+// call it with the same arguments (the loop is uniform across the block).
+template <typename F>
+__device__ __forceinline__ void for_each_segment(const Geometry& g, const int32_t* len, int grid, F&& fn) {
+  const long long T = total_items(g, len);
+  // with more CTAs than items the surplus CTAs sit out, so every CTA of [0, N) owns >= 1 item
+  const int N = T < grid ? static_cast<int>(T) : grid;
+  const int i = blockIdx.x;
+  if (i >= N) return;
+  const long long a = T * i / N, e = T * (i + 1) / N;
+  long long cum = 0;   // first item of batch row b
+  int b = 0;
+  long long x = a;
+  while (x < e) {
+    long long per_b = static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+    while (b < g.B - 1 && cum + per_b <= x) {
+      cum += per_b;
+      ++b;
+      per_b = static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+    }
+    const int items = len[b] / kGroup + 1;
+    const int h = static_cast<int>((x - cum) / items);
+    const long long ustart = cum + static_cast<long long>(h) * items;
+    const long long uend = ustart + items;
+    Segment s;
+    s.b = b;
+    s.h = h;
+    s.unit = b * g.Hkv + h;
+    s.lo = static_cast<int>(x - ustart);
+    s.hi = static_cast<int>((uend < e ? uend : e) - ustart);
+    s.ng = len[b] / kGroup;
+    s.nr = len[b] % kGroup;
+    s.first = cta_of(ustart, T, N);
+    s.last = cta_of(uend - 1, T, N);
+    fn(s);
+    x = ustart + s.hi;
   }
-  p[2 + c] = acc;
 }
 
-// Called by every thread of a CTA after its partials are written.  out_unit points at
-// out[b][h*G][0] (G rows of 128 floats).
-__device__ __forceinline__ void combine_if_last(const DecodeWs& ws, int unit, int split, int S, int G,
+__device__ __forceinline__ float* partial_slot(const DecodeWs& ws, int unit, int G) {
+  return ws.part + static_cast<size_t>(blockIdx.x + unit) * G * kPartialStride;
+}
+
+// Called by every thread of the CTA after the segment's partials are in its slot.
+// out_unit points at out[b][h*G][0] (G rows of 128 floats).
+__device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G,
                                                 float* out_unit) {
   __shared__ int is_last;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(ws.tickets + unit, 1u) == static_cast<unsigned>(S - 1));
+  const unsigned nseg = static_cast<unsigned>(s.last - s.first + 1);
+  if (threadIdx.x == 0) is_last = (atomicAdd(ws.tickets + s.unit, 1u) == nseg - 1);
   __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const float* base = ws.part + static_cast<size_t>(unit) * S * G * kPartialStride;
-  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
-    const int hh = i / kHeadDim, c = i % kHeadDim;
-    float m = -INFINITY;
-    for (int s = 0; s < S; ++s) m = fmaxf(m, __ldcg(base + (static_cast<size_t>(s) * G + hh) * kPartialStride));
-    float den = 0.0f, num = 0.0f;
-    if (m != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float* p = base + (static_cast<size_t>(s) * G + hh) * kPartialStride;
-        float ms = __ldcg(p);
-        if (ms == -INFINITY) continue;
-        float f = exp2f(ms - m);
-        den = fmaf(__ldcg(p + 1), f, den);
-        num = fmaf(__ldcg(p + 2 + c), f, num);
+  if (is_last) {
+    __threadfence();
+    const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;
+    for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+      const int hh = i / kHeadDim, c = i % kHeadDim;
+      float m = -INFINITY;
+      for (unsigned k = 0; k < nseg; ++k)
+        m = fmaxf(m, __ldcg(base + (static_cast<size_t>(k) * G + hh) * kPartialStride));
+      float den = 0.0f, num = 0.0f;
+      if (m != -INFINITY) {
+        for (unsigned k = 0; k < nseg; ++k) {
+          const float* p = base + (static_cast<size_t>(k) * G + hh) * kPartialStride;
+          const float ms = __ldcg(p);
+          if (ms == -INFINITY) continue;
+          const float f = exp2f(ms - m);
+          den = fmaf(__ldcg(p + 1), f, den);
+          num = fmaf(__ldcg(p + 2 + c), f, num);
+        }
       }
+      out_unit[static_cast<size_t>(hh) * kHeadDim + c] = den > 0.0f ? num / den : 0.0f;
     }
-    out_unit[static_cast<size_t>(hh) * kHeadDim + c] = den > 0.0f ? num / den : 0.0f;
+    if (threadIdx.x == 0) ws.tickets[s.unit] = 0u;
   }
-  if (threadIdx.x == 0) ws.tickets[unit] = 0u;
+  __syncthreads();
 }
 
-cudaError_t launch_decode_simt(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int S,
+// Host side: CTAs a decode launch may use for this shape (the workspace is sized for it)
+// and the slots that gives.
+__host__ __forceinline__ int decode_max_ctas(const Geometry& g, int max_context) {
+  const long long units = static_cast<long long>(g.B) * g.Hkv;
+  const long long items = units * ((max_context > 0 ? max_context : 0) / kGroup + 1);
+  long long n = items < kMaxDecodeCtas ? items : kMaxDecodeCtas;
+  return static_cast<int>(n < 1 ? 1 : n);
+}
+
+cudaError_t launch_decode_simt(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                                float* out, DecodeWs ws, cudaStream_t s);
+cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
+                              float* out, DecodeWs ws, cudaStream_t s);
 
 }  // namespace pnmix

@@ -1,0 +1,671 @@
+// decode_mma.cu -- tensor-core decode attention over the packed cache.
+//
+// One CTA = one split of one (sequence, KV head) unit, 4 warps.  Every warp owns whole
+// 32-token group records (interleaved across the warps), stages them with cp.async
+// into its own 3-deep shared-memory ring, and keeps its own online softmax.  Per group:
+//
+//   logits  q . k^_t = sum_p q_p (s_p code_{p,t} + z_p)
+//          = [codes (32 tok x 128 pos)] x [q_p s_p]  +  [z broadcast] x [q]
+//   The codes become exact fp16 A fragments in registers (mask-and-OR into the mantissa
+//   of 1024.0, then one fp16 FMA removes the 1024 and the bit position).  The query is
+//   split into fp16 hi + lo halves held in interleaved B columns (head h -> columns 2h,
+//   2h+1) so the m16n8k16 product keeps ~22 bits; the per-group q_p s_p is formed with
+//   three fp16 FMAs per pair.  The zero-point term is one more MMA per slice with the z
+//   pairs broadcast over the rows.
+//   out     sum_t p_t v^_t = sum_t (p_t s_{t,j}) code_{t,c} + sum_t p_t z_{t,j}
+//          = [codes^T (channels x tokens)] x [p s]  +  [z rows] x [p]
+//   with p rounded to fp16 once (fp32 accumulation).
+//
+// The bit placement of the record (include/pnmix.h) is the fragment ownership of the
+// m16n8k16 tiles, so a lane's code words are exactly its A registers.  Splits merge
+// through decode_common.cuh (fused combine, no waiting).  The bf16 residual window is
+// attended by warp 0 of the last split with CUDA cores.
+#include "common.cuh"
+#include "decode_common.cuh"
+
+namespace pnmix {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));   // (a & b) | c
+  return d;
+}
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// (lo, hi) fp32 -> f16x2 with lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+// Codes as fp16 subnormals.  A code pair sitting at bit offset e of both 16-bit halves of
+// a word becomes an exact fp16x2 of (code * 2^(e-24)) with one AND: the exponent field
+// stays zero.  The tensor cores take subnormal fp16 operands exactly, so the bit offset
+// only scales the product, and the kernel removes that power of two afterwards.
+__device__ __forceinline__ uint32_t sub_pair(uint32_t w, uint32_t mask) { return w & mask; }
+
+// Bit offset of token row u (0..3) of a BITS-bit key slice in the A registers below.
+template <int BITS>
+__host__ __device__ constexpr int key_row_shift(int u) {
+  return BITS == 4 ? 4 * (u & 1) : (BITS == 2 ? 2 * u : u);
+}
+
+// A fragments (2 M-tiles x 4 registers) of one key slice from its code word(s).
+//   4-bit: words w0 (c = 0), w1 (c = 1); token rows u = 0,1 in bits 0-7, rows 2,3 in 8-15.
+//   2-bit: word w; c = 0 in bits 0-7, c = 1 in bits 8-15, row u at 2u.
+//   1-bit: word w holds two slices; the slice of parity o and half c sit at 4*(2o+c), row u at u.
+template <int BITS>
+__device__ __forceinline__ void key_slice_frags(uint32_t w0, uint32_t w1, int parity, uint32_t (&A)[2][4]) {
+  if constexpr (BITS == 4) {
+    const uint32_t s0 = w0 >> 8, s1 = w1 >> 8;
+    A[0][0] = sub_pair(w0, 0x000F000Fu); A[0][1] = sub_pair(w0, 0x00F000F0u);
+    A[1][0] = sub_pair(s0, 0x000F000Fu); A[1][1] = sub_pair(s0, 0x00F000F0u);
+    A[0][2] = sub_pair(w1, 0x000F000Fu); A[0][3] = sub_pair(w1, 0x00F000F0u);
+    A[1][2] = sub_pair(s1, 0x000F000Fu); A[1][3] = sub_pair(s1, 0x00F000F0u);
+  } else if constexpr (BITS == 2) {
+    const uint32_t s = w0 >> 8;
+    A[0][0] = sub_pair(w0, 0x00030003u); A[0][1] = sub_pair(w0, 0x000C000Cu);
+    A[1][0] = sub_pair(w0, 0x00300030u); A[1][1] = sub_pair(w0, 0x00C000C0u);
+    A[0][2] = sub_pair(s, 0x00030003u);  A[0][3] = sub_pair(s, 0x000C000Cu);
+    A[1][2] = sub_pair(s, 0x00300030u);  A[1][3] = sub_pair(s, 0x00C000C0u);
+  } else {
+    const uint32_t a = parity ? (w0 >> 8) : w0;     // half c = 0
+    const uint32_t b = parity ? (w0 >> 12) : (w0 >> 4);   // half c = 1
+    A[0][0] = sub_pair(a, 0x00010001u); A[0][1] = sub_pair(a, 0x00020002u);
+    A[1][0] = sub_pair(a, 0x00040004u); A[1][1] = sub_pair(a, 0x00080008u);
+    A[0][2] = sub_pair(b, 0x00010001u); A[0][3] = sub_pair(b, 0x00020002u);
+    A[1][2] = sub_pair(b, 0x00040004u); A[1][3] = sub_pair(b, 0x00080008u);
+  }
+}
+
+// ------------------------------------------------------------------ shared memory map
+
+struct SmemMap {
+  int qsets;     // [NT][4 sets][4 chunks][32 lanes][4 words]
+  int qnat;      // fp32 [kMaxG][128], natural channel order, log2-domain scale
+  int perm;      // 128 bytes
+  int resid;     // fp32 [kMaxG][kPartialStride]: partial of the residual item
+  int stages;    // [kWarps][kStages][R]
+  int part;      // fp32 [kWarps][kMaxG][kPartialStride], aliases the stages
+  int total;
+};
+
+__host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
+  SmemMap m;
+  m.qsets = 0;
+  m.qnat = NT * 4 * 4 * 32 * 16;
+  m.perm = m.qnat + kMaxG * kHeadDim * 4;
+  m.resid = m.perm + 128;
+  m.stages = m.resid + kMaxG * kPartialStride * 4;
+  int stage_bytes = kWarps * kStages * R;
+  int part_bytes = kWarps * kMaxG * kPartialStride * 4;
+  m.part = m.stages;
+  m.total = m.stages + (stage_bytes > part_bytes ? stage_bytes : part_bytes);
+  return m;
+}
+
+// ------------------------------------------------------------------ per-warp state
+
+template <int NT>
+struct WarpAcc {
+  float m[NT];          // running max (log2 domain) of head 4*nt + tq
+  float l[NT];          // this lane's partial sum of 2^(logit - m)
+  float pv[8][4];       // P.V accumulators: channels 16m + gq (+8), heads 2tq, 2tq+1
+  float bias[4];        // zero-point term: row gq = channel group, heads 2tq, 2tq+1
+};
+
+// One group record at `rec` (shared memory) folded into the warp's state.
+template <int BHI, int BLO, int NT, int NHS>
+__device__ __forceinline__ void process_group(const Geometry& g, const uint8_t* rec,
+                                              const uint32_t* qsets, WarpAcc<NT>& st) {
+  constexpr int WH = NHS * BHI / 2;   // key-code words per lane of the salient block
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int kc = g.kc_bytes;
+
+  // key scales / zeros of this lane: fp16x2 index sigma*2 + e, loaded per slice pair
+  const uint4* sp = reinterpret_cast<const uint4*>(rec + kc + tq * 64);
+  const uint4* zp = reinterpret_cast<const uint4*>(rec + kc + 256 + tq * 64);
+  uint4 s4 = make_uint4(0, 0, 0, 0), z4 = make_uint4(0, 0, 0, 0);
+  const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec);
+
+  // key-code products, kept apart per block because the two blocks' token-row bit
+  // offsets differ, and split by slice parity to halve the accumulation chains; the
+  // zero-point term separately (normal fp16 scale)
+  float acc_hi[NT][2][4], acc_lo[2][NT][2][4];
+  float dz[2][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc_hi[nt][0][i] = 0.f;
+      acc_hi[nt][1][i] = 0.f;
+#pragma unroll
+      for (int par = 0; par < 2; ++par) {
+        acc_lo[par][nt][0][i] = 0.f;
+        acc_lo[par][nt][1][i] = 0.f;
+        dz[par][nt][i] = 0.f;
+      }
+    }
+  }
+
+  uint4 qa4[NT], qb4[NT], qc4[NT], qz4[NT];
+#pragma unroll
+  for (int sigma = 0; sigma < 8; ++sigma) {
+    if ((sigma & 1) == 0) {
+      s4 = sp[sigma >> 1];
+      z4 = zp[sigma >> 1];
+      // q sets of this slice pair: one 16-byte load per set (entries 2*sigma .. 2*sigma+3)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4* qb = reinterpret_cast<const uint4*>(qsets) + ((nt * 4) * 4 + (sigma >> 1)) * 32 + lane;
+        qa4[nt] = qb[0];
+        qb4[nt] = qb[1 * 4 * 32];
+        qc4[nt] = qb[2 * 4 * 32];
+        qz4[nt] = qb[3 * 4 * 32];
+      }
+    }
+    // ---- A fragments of this slice (2 M-tiles x 4 registers)
+    uint32_t A[2][4];
+    const bool hi = sigma < NHS;
+    if (hi) {
+      if constexpr (BHI == 4)
+        key_slice_frags<4>(kw[(2 * sigma) * 32 + lane], kw[(2 * sigma + 1) * 32 + lane], 0, A);
+      else
+        key_slice_frags<BHI>(kw[sigma * 32 + lane], 0u, 0, A);
+    } else {
+      const int sl = sigma - NHS;   // slice inside the lo block
+      if constexpr (BLO == 2)
+        key_slice_frags<2>(kw[(WH + sl) * 32 + lane], 0u, 0, A);
+      else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
+        key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, sigma & 1, A);
+    }
+    // ---- B fragments: q'' = q * s (hi or lo half per column) and q (for z)
+    const int par = sigma & 1;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t qa0 = par ? qa4[nt].z : qa4[nt].x, qa1 = par ? qa4[nt].w : qa4[nt].y;
+      const uint32_t qb0 = par ? qb4[nt].z : qb4[nt].x, qb1 = par ? qb4[nt].w : qb4[nt].y;
+      const uint32_t qc0 = par ? qc4[nt].z : qc4[nt].x, qc1 = par ? qc4[nt].w : qc4[nt].y;
+      const uint32_t qz0 = par ? qz4[nt].z : qz4[nt].x, qz1 = par ? qz4[nt].w : qz4[nt].y;
+      const uint32_t s0 = par ? s4.z : s4.x, s1 = par ? s4.w : s4.y;
+      const uint32_t b0 = hfma2(qc0, s0, hfma2(qb0, s0, hmul2(qa0, s0)));
+      const uint32_t b1 = hfma2(qc1, s1, hfma2(qb1, s1, hmul2(qa1, s1)));
+      if (hi) {
+        mma16816(acc_hi[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+        mma16816(acc_hi[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+      } else {
+        mma16816(acc_lo[par][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+        mma16816(acc_lo[par][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+      }
+      const uint32_t z0 = par ? z4.z : z4.x, z1 = par ? z4.w : z4.y;
+      mma16816(dz[par][nt], z0, z0, z1, z1, qz0, qz1);
+    }
+  }
+
+  // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3;
+  // the product of a row-u token carries 2^(shift(u) - 24)
+  float lg[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float zb = (dz[0][nt][0] + dz[0][nt][1]) + (dz[1][nt][0] + dz[1][nt][1]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int mt = u >> 1, r = 2 * (u & 1);
+      const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23);
+      const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23);
+      const float vhi = acc_hi[nt][mt][r] + acc_hi[nt][mt][r + 1];
+      const float vlo = (acc_lo[0][nt][mt][r] + acc_lo[0][nt][mt][r + 1]) +
+                        (acc_lo[1][nt][mt][r] + acc_lo[1][nt][mt][r + 1]);
+      lg[nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
+    }
+  }
+
+  // ---- online softmax
+  float mnew[NT];
+  bool grow = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float mx = fmaxf(fmaxf(lg[nt][0], lg[nt][1]), fmaxf(lg[nt][2], lg[nt][3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    mnew[nt] = fmaxf(st.m[nt], mx);
+    grow |= mnew[nt] > st.m[nt];
+  }
+  if (__any_sync(0xffffffffu, grow)) {
+    float alpha[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      alpha[nt] = exp2f(st.m[nt] - mnew[nt]);
+      st.l[nt] *= alpha[nt];
+      st.m[nt] = mnew[nt];
+    }
+    // P.V columns of this lane are heads 2tq and 2tq+1
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+    float a0 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h0 & 3));
+    float a1 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h1 & 3));
+    if constexpr (NT == 2) {
+      const float b0 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h0 & 3));
+      const float b1 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h1 & 3));
+      if (h0 >= 4) a0 = b0;
+      if (h1 >= 4) a1 = b1;
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      st.pv[m][0] *= a0;
+      st.pv[m][1] *= a1;
+      st.pv[m][2] *= a0;
+      st.pv[m][3] *= a1;
+    }
+    st.bias[0] *= a0;
+    st.bias[1] *= a1;
+    st.bias[2] *= a0;
+    st.bias[3] *= a1;
+  }
+  float p[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      p[nt][i] = exp2f(lg[nt][i] - st.m[nt]);
+      st.l[nt] += p[nt][i];
+    }
+  }
+
+  // ---- P as B fragments: column gq = head gq, tokens 2tq + {0,1} (+8, +16, +24)
+  const int srcA = (2 * tq) * 4 + (gq & 3), srcB = (2 * tq + 1) * 4 + (gq & 3);
+  float pa[4], pb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pa[i] = __shfl_sync(0xffffffffu, p[0][i], srcA);
+    pb[i] = __shfl_sync(0xffffffffu, p[0][i], srcB);
+  }
+  if constexpr (NT == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float xa = __shfl_sync(0xffffffffu, p[1][i], srcA);
+      const float xb = __shfl_sync(0xffffffffu, p[1][i], srcB);
+      if (gq >= 4) {
+        pa[i] = xa;
+        pb[i] = xb;
+      }
+    }
+  }
+  uint32_t p16[4];
+  const bool col_ok = gq < g.G;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p16[i] = col_ok ? pack_f16x2(pa[i], pb[i]) : 0u;
+
+  // value scales: token pairs tp2 = tq + 4i, four channel groups each
+  const int vs_off = kc + 1536, vz_off = kc + 1792;
+  uint32_t vsr[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(rec + vs_off + (tq + 4 * i) * 16);
+    vsr[i][0] = v.x; vsr[i][1] = v.y; vsr[i][2] = v.z; vsr[i][3] = v.w;
+  }
+  // zero-point term: A rows = channel groups (rows 0..3), k = tokens
+  {
+    const int j = gq & 3;
+    uint32_t vz[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
+      vz[i] = gq < 4 ? v : 0u;
+    }
+    mma16816(st.bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
+    mma16816(st.bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
+  }
+  // value codes: words 0..7 of this lane (two 16-byte chunks).  Slot (r, p) of word m
+  // sits at bits 8r + 2p; taken from w >> (8r + 4*(p>>1)) at bit 2*(p&1), so odd token
+  // pairs carry an extra 2^2: the even-pair B columns are scaled by 4 to match.
+  const uint32_t four2 = 0x44004400u;   // fp16x2 (4, 4)
+  const uint32_t p16x4_0 = hmul2(p16[0], four2), p16x4_2 = hmul2(p16[2], four2);
+  const uint4 vw0 = *reinterpret_cast<const uint4*>(rec + kc + 512 + lane * 16);
+  const uint4 vw1 = *reinterpret_cast<const uint4*>(rec + kc + 512 + (32 + lane) * 16);
+  const uint32_t vw[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int j = m >> 1;
+    const uint32_t w = vw[m], w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
+    // (r, p) -> k-step p >> 1, register r + 2*(p & 1)
+    const uint32_t k0a0 = sub_pair(w, 0x00030003u), k0a2 = sub_pair(w, 0x000C000Cu);
+    const uint32_t k1a0 = sub_pair(w4, 0x00030003u), k1a2 = sub_pair(w4, 0x000C000Cu);
+    const uint32_t k0a1 = sub_pair(w8, 0x00030003u), k0a3 = sub_pair(w8, 0x000C000Cu);
+    const uint32_t k1a1 = sub_pair(w12, 0x00030003u), k1a3 = sub_pair(w12, 0x000C000Cu);
+    const uint32_t b00 = hmul2(p16x4_0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
+    const uint32_t b10 = hmul2(p16x4_2, vsr[2][j]), b11 = hmul2(p16[3], vsr[3][j]);
+    mma16816(st.pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
+    mma16816(st.pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
+  }
+}
+
+// The residual item: up to 31 bf16 tokens, with CUDA cores, heads h0, h0 + hstep, ...
+// one at a time (few registers).  Lane = token for the logit (its K row read with 16-byte loads, q in natural
+// channel order from shared memory), lane = channel for the values (rows read coalesced,
+// four tokens ahead).  Writes one partial per head into `slot`.
+__device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
+                                              int nr, const float* qnat, float* slot, int h0, int hstep) {
+  const int lane = threadIdx.x & 31;
+  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kHeadDim);
+#pragma unroll 1
+  for (int hh = h0; hh < g.G; hh += hstep) {
+    const float* qh = qnat + hh * kHeadDim;
+    float lg = 0.f;
+#pragma unroll
+    for (int c4 = 0; c4 < 16; c4 += 4) {
+      uint4 kv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kv[i] = __ldg(row + c4 + i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {kv[i].x, kv[i].y, kv[i].z, kv[i].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float k = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+          lg = fmaf(qh[(c4 + i) * 8 + e], k, lg);
+        }
+      }
+    }
+    if (lane >= nr) lg = -INFINITY;
+    float m = lg;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float pw = lane < nr ? exp2f(lg - m) : 0.f;
+    float l = pw;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int t0 = 0; t0 < nr; t0 += 4) {
+      float v[4][4];
+#pragma unroll
+      for (int dt = 0; dt < 4; ++dt) {
+        const int t = t0 + dt < nr ? t0 + dt : nr - 1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[dt][i] = bf16_bits_to_float(rv[t * kHeadDim + lane + 32 * i]);
+      }
+#pragma unroll
+      for (int dt = 0; dt < 4; ++dt) {
+        const float pt = __shfl_sync(0xffffffffu, pw, (t0 + dt) & 31);
+        if (t0 + dt < nr) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = fmaf(pt, v[dt][i], acc[i]);
+        }
+      }
+    }
+    float* s = slot + hh * kPartialStride;
+    if (lane == 0) {
+      s[0] = m;
+      s[1] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[2 + lane + 32 * i] = acc[i];
+  }
+}
+
+template <int BHI, int BLO, int NT, int NHS>
+__global__ void __launch_bounds__(kThreads, 3)
+decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
+                  DecodeWs ws) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int G = g.G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = g.record_bytes;
+  const SmemMap sm = smem_map(NT, R);
+  uint32_t* qsets = reinterpret_cast<uint32_t*>(smem + sm.qsets);
+  float* qnat = reinterpret_cast<float*>(smem + sm.qnat);
+  uint8_t* perm = smem + sm.perm;
+  float* rslot = reinterpret_cast<float*>(smem + sm.resid);
+  float* part = reinterpret_cast<float*>(smem + sm.part);
+  uint8_t* ring = smem + sm.stages + warp * kStages * R;
+  const int chunks = R >> 4;
+
+  for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
+    const int b = seg.b, h = seg.h, unit = seg.unit;
+    // ---- this warp's groups of the segment; stage the first ones right away
+    const int gend = seg.hi < seg.ng ? seg.hi : seg.ng;
+    const int my_first = seg.lo + warp;
+    const int my_count = my_first < gend ? (gend - my_first + kWarps - 1) / kWarps : 0;
+    const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
+    auto issue = [&](int i) {
+      if (i < my_count) {
+        const uint8_t* src = unit_rec + static_cast<size_t>(my_first + i * kWarps) * R;
+        uint8_t* dst = ring + (i % kStages) * R;
+        for (int k = lane; k < chunks; k += 32) cp_async16(dst + 16 * k, src + 16 * k);
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
+
+    // ---- query: log2-domain scale, natural order, then fp16 hi/lo column sets in
+    // position order
+    perm[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid];
+    const float qscale = g.scale * kLog2e;
+    for (int i = tid; i < kMaxG * kHeadDim; i += kThreads) {
+      const int hh = i / kHeadDim;
+      qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) * qscale
+                       : 0.f;
+    }
+    __syncthreads();
+    {
+      const int L = lane, chunk = warp;   // entries 4*chunk .. 4*chunk+3 (= sigma*2 + e)
+      const int tq = L & 3, gq = L >> 2;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int col = gq + 8 * nt, hh = col >> 1, hl = col & 1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int idx = chunk * 4 + i, sigma = idx >> 1, e = idx & 1;
+          const int p0 = 16 * sigma + 8 * e + 2 * tq;
+          uint32_t sets[4][2];
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const float x = hh < G ? qnat[hh * kHeadDim + perm[p0 + v]] : 0.f;
+            const __half hi = __float2half_rn(x);
+            const __half lo = __float2half_rn(x - __half2float(hi));
+            const uint32_t hib = __half_as_ushort(hi), lob = __half_as_ushort(lo);
+            sets[0][v] = hl ? (hib ^ 0x8000u) : hib;   // A: -hi on a lo column, hi otherwise
+            sets[1][v] = hl ? hib : 0u;                // B
+            sets[2][v] = hl ? lob : 0u;                // C
+            sets[3][v] = hl ? lob : hib;               // q half for the zero-point term
+          }
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            qsets[(((nt * 4 + s) * 4 + chunk) * 32 + L) * 4 + i] = sets[s][0] | (sets[s][1] << 16);
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- the residual item (CUDA cores): warp w takes heads w, w + 4
+    if (seg.hi > seg.ng && seg.nr > 0) {
+      const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
+      const uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
+      residual_partial(g, rk, rv, seg.nr, qnat, rslot, warp, kWarps);
+    } else if (warp == 0 && lane < G) {
+      rslot[lane * kPartialStride + 0] = -INFINITY;
+      rslot[lane * kPartialStride + 1] = 0.f;
+    }
+
+    // ---- the warp's groups
+    WarpAcc<NT> st;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      st.m[nt] = -INFINITY;
+      st.l[nt] = 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) st.pv[m][i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st.bias[i] = 0.f;
+
+    for (int i = 0; i < my_count; ++i) {
+      issue(i + kStages - 1);
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
+      process_group<BHI, BLO, NT, NHS>(g, ring + (i % kStages) * R, qsets, st);
+      __syncwarp();
+    }
+    cp_async_wait<0>();
+    __syncthreads();   // every ring is idle: the merge area may alias them
+
+    // ---- warp partials into shared memory
+    {
+      const int gq = lane >> 2, tq = lane & 3;
+      float lsum[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float v = st.l[nt];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        lsum[nt] = v;
+      }
+      float* wp = part + warp * kMaxG * kPartialStride;
+      if (gq == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hh = 4 * nt + tq;
+          if (hh < G) {
+            wp[hh * kPartialStride + 0] = my_count ? st.m[nt] : -INFINITY;
+            wp[hh * kPartialStride + 1] = my_count ? lsum[nt] : 0.f;
+          }
+        }
+      }
+      // zero-point term of channel group j for heads 2tq, 2tq+1 lives in lane (j, tq)
+      float bz[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bz[j][0] = __shfl_sync(0xffffffffu, st.bias[0], j * 4 + tq);
+        bz[j][1] = __shfl_sync(0xffffffffu, st.bias[1], j * 4 + tq);
+      }
+      const int h0 = 2 * tq, h1 = 2 * tq + 1;
+      const float pv_scale = 4194304.0f;   // 2^22: the codes' 2^-24 and the pairs' 2^2
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int j = m >> 1;
+        const int c0 = 16 * m + gq, c1 = c0 + 8;
+        if (h0 < G) {
+          wp[h0 * kPartialStride + 2 + c0] = fmaf(st.pv[m][0], pv_scale, bz[j][0]);
+          wp[h0 * kPartialStride + 2 + c1] = fmaf(st.pv[m][2], pv_scale, bz[j][0]);
+        }
+        if (h1 < G) {
+          wp[h1 * kPartialStride + 2 + c0] = fmaf(st.pv[m][1], pv_scale, bz[j][1]);
+          wp[h1 * kPartialStride + 2 + c1] = fmaf(st.pv[m][3], pv_scale, bz[j][1]);
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- CTA merge (thread = channel) into the segment's partial slot
+    float* slot = partial_slot(ws, unit, G);
+    for (int hh = 0; hh < G; ++hh) {
+      float m = rslot[hh * kPartialStride];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, part[(w * kMaxG + hh) * kPartialStride]);
+      float l = 0.f, a = 0.f;
+      if (m != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w <= kWarps; ++w) {
+          const float* p = w < kWarps ? part + (w * kMaxG + hh) * kPartialStride : rslot + hh * kPartialStride;
+          if (p[0] == -INFINITY) continue;
+          const float f = exp2f(p[0] - m);
+          l = fmaf(p[1], f, l);
+          a = fmaf(p[2 + tid], f, a);
+        }
+      }
+      float* o = slot + hh * kPartialStride;
+      if (tid == 0) {
+        o[0] = m;
+        o[1] = l;
+      }
+      o[2 + tid] = a;
+    }
+    combine_segment(ws, seg, G, out + (static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim);
+  });
+}
+
+template <int BHI, int BLO, int NT, int NHS>
+cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
+                         DecodeWs ws, cudaStream_t s) {
+  const SmemMap sm = smem_map(NT, g.record_bytes);
+  auto kern = decode_mma_kernel<BHI, BLO, NT, NHS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm.total);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, occ = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, sm.total);
+  if (e != cudaSuccess) return e;
+  const int n = sms * (occ > 0 ? occ : 1);
+  ws.N = n < nmax ? n : nmax;
+  kern<<<ws.N, kThreads, sm.total, s>>>(g, q, c, out, ws);
+  return cudaGetLastError();
+}
+
+template <int BHI, int BLO, int NT>
+cudaError_t launch_mma_nhs(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
+                           DecodeWs ws, cudaStream_t s) {
+  switch (g.nhs) {
+    case 0: return launch_mma_t<BHI, BLO, NT, 0>(g, q, c, nmax, out, ws, s);
+    case 2: return launch_mma_t<BHI, BLO, NT, 2>(g, q, c, nmax, out, ws, s);
+    case 4: return launch_mma_t<BHI, BLO, NT, 4>(g, q, c, nmax, out, ws, s);
+    case 8: return launch_mma_t<BHI, BLO, NT, 8>(g, q, c, nmax, out, ws, s);
+    default: break;
+  }
+  if constexpr (BLO == 2) {   // one salient slice (k = 8) only exists with 2-bit lo words
+    if (g.nhs == 1) return launch_mma_t<BHI, BLO, NT, 1>(g, q, c, nmax, out, ws, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
+                              float* out, DecodeWs ws, cudaStream_t s) {
+  const bool nt2 = g.G > 4;
+  if (g.bhi == 4 && g.blo == 2)
+    return nt2 ? launch_mma_nhs<4, 2, 2>(g, q, c, nmax, out, ws, s) : launch_mma_nhs<4, 2, 1>(g, q, c, nmax, out, ws, s);
+  if (g.bhi == 2 && g.blo == 1)
+    return nt2 ? launch_mma_nhs<2, 1, 2>(g, q, c, nmax, out, ws, s) : launch_mma_nhs<2, 1, 1>(g, q, c, nmax, out, ws, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pnmix

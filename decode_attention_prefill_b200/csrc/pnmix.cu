@@ -2,6 +2,7 @@
 // the launches.  No entry point allocates, frees or synchronises (except
 // pnmix_read_error, which is a synchronous read by definition).
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -90,30 +91,32 @@ static pnmix_status check_cache(const Geometry& g, const pnmix_cache* c) {
   return PNMIX_OK;
 }
 
-int decode_splits(const Geometry& g, int max_context) {
-  const int units = g.B * g.Hkv;
-  const int groups = max_context > 0 ? (max_context + kGroup - 1) / kGroup : 1;
-  int S = (4 * 148 + units - 1) / units;
-  if (S > groups) S = groups;
-  if (S > 256) S = 256;
-  if (S < 1) S = 1;
-  return S;
+// Which decode kernel runs: the tensor-core kernel (default) or, with the environment
+// variable PNMIX_DECODE_KERNEL=simt, the CUDA-core kernel (kept for A/B measurement).
+int decode_kernel_choice() {
+  static const int choice = [] {
+    const char* v = getenv("PNMIX_DECODE_KERNEL");
+    return (v && strcmp(v, "simt") == 0) ? 1 : 0;
+  }();
+  return choice;
 }
 
 size_t decode_workspace_bytes(const Geometry& g, int max_context) {
-  const int S = decode_splits(g, max_context);
+  const int nmax = decode_max_ctas(g, max_context);
   const int units = g.B * g.Hkv;
-  return decode_partial_bytes(units, S, g.G) + align256(sizeof(uint32_t) * units);
+  return decode_partial_bytes(nmax + units, g.G) + align256(sizeof(uint32_t) * units);
 }
 
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int max_context,
                           float* out, void* ws, cudaStream_t s) {
-  const int S = decode_splits(g, max_context);
+  const int nmax = decode_max_ctas(g, max_context);
   const int units = g.B * g.Hkv;
   DecodeWs w;
   w.part = static_cast<float*>(ws);
-  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(units, S, g.G));
-  return launch_decode_simt(g, q, c, S, out, w, s);
+  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(nmax + units, g.G));
+  w.N = nmax;
+  if (decode_kernel_choice() == 1) return launch_decode_simt(g, q, c, nmax, out, w, s);
+  return launch_decode_mma(g, q, c, nmax, out, w, s);
 }
 
 }  // namespace pnmix

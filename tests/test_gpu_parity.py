@@ -115,3 +115,16 @@ def test_sweep_128k_bit_points(k, bhi, blo):
     c.prefill()
     got, want = c.attend(c.query(131072))
     assert_close(got, want)
+
+
+def test_context_hint_smaller_than_the_cache_still_covers_every_token():
+    """The grid is sized from max_context; a smaller hint gives fewer CTAs, never fewer tokens."""
+    import decode_attention_prefill_b200 as pm
+    c = Case(4, 16, 4, 1000, seed=13)
+    c.prefill()
+    q = c.query(1000)
+    for mc in (0, 1, 64, 1000):
+        ws = torch.zeros(pm.workspace_bytes(c.cfg, 4, mc), dtype=torch.uint8, device="cuda")
+        out = torch.empty(4, 16, 128, dtype=torch.float32, device="cuda")
+        pm.pnmix_decode_attention(c.cfg, to_dev(q), c.cache, out, workspace=ws, max_context=mc)
+        assert_close(out.cpu().numpy(), c.ocache.attend(q))
