@@ -22,6 +22,7 @@ namespace pnmix {
 
 constexpr int kPartialStride = 2 + kHeadDim;   // m, l, acc[128]
 constexpr int kMaxDecodeCtas = 1024;           // grid cap of the decode kernels
+constexpr unsigned kMaxCombineSegs = 32;       // segments merged per pass of the combine
 
 struct DecodeWs {
   float* part;         // [slots][G][kPartialStride]
@@ -108,24 +109,41 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
   __syncthreads();
   if (is_last) {
     __threadfence();
+    // weights first (one thread per (head, segment)), then every thread sums its channels
+    // with independent loads
+    __shared__ float wsh[kMaxG][kMaxCombineSegs];
+    __shared__ float den_sh[kMaxG];
     const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;
-    for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
-      const int hh = i / kHeadDim, c = i % kHeadDim;
-      float m = -INFINITY;
-      for (unsigned k = 0; k < nseg; ++k)
-        m = fmaxf(m, __ldcg(base + (static_cast<size_t>(k) * G + hh) * kPartialStride));
-      float den = 0.0f, num = 0.0f;
-      if (m != -INFINITY) {
+    for (unsigned chunk = 0; chunk < nseg; chunk += kMaxCombineSegs) {
+      const unsigned n = nseg - chunk < kMaxCombineSegs ? nseg - chunk : kMaxCombineSegs;
+      if (threadIdx.x < G) {
+        const int hh = threadIdx.x;
+        float m = -INFINITY;
+        for (unsigned k = 0; k < nseg; ++k)
+          m = fmaxf(m, __ldcg(base + (static_cast<size_t>(k) * G + hh) * kPartialStride));
+        float den = 0.f;
         for (unsigned k = 0; k < nseg; ++k) {
           const float* p = base + (static_cast<size_t>(k) * G + hh) * kPartialStride;
           const float ms = __ldcg(p);
-          if (ms == -INFINITY) continue;
-          const float f = exp2f(ms - m);
+          const float f = (ms == -INFINITY || m == -INFINITY) ? 0.f : exp2f(ms - m);
           den = fmaf(__ldcg(p + 1), f, den);
-          num = fmaf(__ldcg(p + 2 + c), f, num);
+          if (k >= chunk && k < chunk + n) wsh[hh][k - chunk] = f;
         }
+        den_sh[hh] = den;
       }
-      out_unit[static_cast<size_t>(hh) * kHeadDim + c] = den > 0.0f ? num / den : 0.0f;
+      __syncthreads();
+      for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+        const int hh = i / kHeadDim, c = i % kHeadDim;
+        float num = chunk == 0 ? 0.f : out_unit[static_cast<size_t>(hh) * kHeadDim + c];
+#pragma unroll 4
+        for (unsigned k = 0; k < n; ++k)
+          num = fmaf(__ldcg(base + (static_cast<size_t>(chunk + k) * G + hh) * kPartialStride + 2 + c),
+                     wsh[hh][k], num);
+        const bool last_chunk = chunk + n == nseg;
+        out_unit[static_cast<size_t>(hh) * kHeadDim + c] =
+            last_chunk ? (den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f) : num;
+      }
+      __syncthreads();
     }
     if (threadIdx.x == 0) ws.tickets[s.unit] = 0u;
   }

@@ -28,16 +28,17 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 3;
+// Staging ring per warp: 6 slots when the warp consumes its groups in pairs (G <= 4),
+// 3 when it takes them one at a time (G <= 8).
+template <int NT>
+__host__ __device__ constexpr int stages_for() { return NT == 1 ? 6 : 3; }
+template <int NT>
+__host__ __device__ constexpr int groups_per_step() { return NT == 1 ? 2 : 1; }
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kResidKStride = kHeadDim + 8;   // bf16 per staged K row (+16 B: no bank conflicts)
 
 // ------------------------------------------------------------------ PTX helpers
 
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));   // (a & b) | c
-  return d;
-}
 __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -54,6 +55,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
+// 2^x with the hardware approximation (MUFU.EX2, ~2 ulp; inputs here are <= 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -62,13 +69,39 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem));
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// One bulk copy (TMA, no multicast) of `bytes` from global to this CTA's shared memory;
+// completion is signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(phase) : "memory");
+  return ok != 0;
+}
+// Orders this thread's earlier generic-proxy accesses of shared memory before later
+// async-proxy (TMA) writes to it.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// try_wait rounds before a staging wait gives up (each round may suspend the warp for a
+// while); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and the kernel stops consuming.
+constexpr uint32_t kWaitLimit = 1u << 22;
 
 // Codes as fp16 subnormals.  A code pair sitting at bit offset e of both 16-bit halves of
 // a word becomes an exact fp16x2 of (code * 2^(e-24)) with one AND: the exponent field
@@ -117,19 +150,24 @@ struct SmemMap {
   int qnat;      // fp32 [kMaxG][128], natural channel order, log2-domain scale
   int perm;      // 128 bytes
   int resid;     // fp32 [kMaxG][kPartialStride]: partial of the residual item
-  int stages;    // [kWarps][kStages][R]
+  int rrows;     // bf16 residual K rows [32][kResidKStride] then V rows [32][128]
+  int bars;      // uint64 [kWarps][stages] mbarriers
+  int stages;    // [kWarps][stages][R]
   int part;      // fp32 [kWarps][kMaxG][kPartialStride], aliases the stages
   int total;
 };
 
 __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
+  const int nst = NT == 1 ? stages_for<1>() : stages_for<2>();
   SmemMap m;
   m.qsets = 0;
   m.qnat = NT * 4 * 4 * 32 * 16;
   m.perm = m.qnat + kMaxG * kHeadDim * 4;
   m.resid = m.perm + 128;
-  m.stages = m.resid + kMaxG * kPartialStride * 4;
-  int stage_bytes = kWarps * kStages * R;
+  m.rrows = m.resid + kMaxG * kPartialStride * 4;
+  m.bars = m.rrows + kGroup * kResidKStride * 2 + kGroup * kHeadDim * 2;
+  m.stages = m.bars + ((kWarps * nst * 8 + 127) / 128) * 128;
+  int stage_bytes = kWarps * nst * R;
   int part_bytes = kWarps * kMaxG * kPartialStride * 4;
   m.part = m.stages;
   m.total = m.stages + (stage_bytes > part_bytes ? stage_bytes : part_bytes);
@@ -146,47 +184,43 @@ struct WarpAcc {
   float bias[4];        // zero-point term: row gq = channel group, heads 2tq, 2tq+1
 };
 
-// One group record at `rec` (shared memory) folded into the warp's state.
-template <int BHI, int BLO, int NT, int NHS>
-__device__ __forceinline__ void process_group(const Geometry& g, const uint8_t* rec,
-                                              const uint32_t* qsets, WarpAcc<NT>& st) {
+// NG group records at recs[0..NG) (shared memory, consecutive groups of this warp)
+// folded into the warp's state.  With NG = 2 the two groups' q.k^ chains interleave and
+// one online-softmax update covers both (64 tokens).
+template <int BHI, int BLO, int NT, int NHS, int NG>
+__device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
+                                               const uint32_t* qsets, WarpAcc<NT>& st) {
   constexpr int WH = NHS * BHI / 2;   // key-code words per lane of the salient block
+  constexpr int PAR = NG == 1 ? 2 : 1;   // accumulation chains per block (split by slice parity)
   const int lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int kc = g.kc_bytes;
 
-  // key scales / zeros of this lane: fp16x2 index sigma*2 + e, loaded per slice pair
-  const uint4* sp = reinterpret_cast<const uint4*>(rec + kc + tq * 64);
-  const uint4* zp = reinterpret_cast<const uint4*>(rec + kc + 256 + tq * 64);
-  uint4 s4 = make_uint4(0, 0, 0, 0), z4 = make_uint4(0, 0, 0, 0);
-  const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec);
-
   // key-code products, kept apart per block because the two blocks' token-row bit
-  // offsets differ, and split by slice parity to halve the accumulation chains; the
-  // zero-point term separately (normal fp16 scale)
-  float acc_hi[NT][2][4], acc_lo[2][NT][2][4];
-  float dz[2][NT][4];
+  // offsets differ; the zero-point term separately (normal fp16 scale)
+  float acc_hi[NG][NT][2][4], acc_lo[NG][PAR][NT][2][4], dz[NG][PAR][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc_hi[nt][0][i] = 0.f;
-      acc_hi[nt][1][i] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int par = 0; par < 2; ++par) {
-        acc_lo[par][nt][0][i] = 0.f;
-        acc_lo[par][nt][1][i] = 0.f;
-        dz[par][nt][i] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        acc_hi[gi][nt][0][i] = 0.f;
+        acc_hi[gi][nt][1][i] = 0.f;
+#pragma unroll
+        for (int pr = 0; pr < PAR; ++pr) {
+          acc_lo[gi][pr][nt][0][i] = 0.f;
+          acc_lo[gi][pr][nt][1][i] = 0.f;
+          dz[gi][pr][nt][i] = 0.f;
+        }
       }
-    }
-  }
 
   uint4 qa4[NT], qb4[NT], qc4[NT], qz4[NT];
+  uint4 s4[NG], z4[NG];
 #pragma unroll
   for (int sigma = 0; sigma < 8; ++sigma) {
-    if ((sigma & 1) == 0) {
-      s4 = sp[sigma >> 1];
-      z4 = zp[sigma >> 1];
+    const int par = sigma & 1, pr = PAR == 2 ? par : 0;
+    if (par == 0) {
       // q sets of this slice pair: one 16-byte load per set (entries 2*sigma .. 2*sigma+3)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -196,69 +230,96 @@ __device__ __forceinline__ void process_group(const Geometry& g, const uint8_t* 
         qc4[nt] = qb[2 * 4 * 32];
         qz4[nt] = qb[3 * 4 * 32];
       }
-    }
-    // ---- A fragments of this slice (2 M-tiles x 4 registers)
-    uint32_t A[2][4];
-    const bool hi = sigma < NHS;
-    if (hi) {
-      if constexpr (BHI == 4)
-        key_slice_frags<4>(kw[(2 * sigma) * 32 + lane], kw[(2 * sigma + 1) * 32 + lane], 0, A);
-      else
-        key_slice_frags<BHI>(kw[sigma * 32 + lane], 0u, 0, A);
-    } else {
-      const int sl = sigma - NHS;   // slice inside the lo block
-      if constexpr (BLO == 2)
-        key_slice_frags<2>(kw[(WH + sl) * 32 + lane], 0u, 0, A);
-      else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
-        key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, sigma & 1, A);
-    }
-    // ---- B fragments: q'' = q * s (hi or lo half per column) and q (for z)
-    const int par = sigma & 1;
+      // key scales / zeros of this lane: fp16x2 index sigma*2 + e
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t qa0 = par ? qa4[nt].z : qa4[nt].x, qa1 = par ? qa4[nt].w : qa4[nt].y;
-      const uint32_t qb0 = par ? qb4[nt].z : qb4[nt].x, qb1 = par ? qb4[nt].w : qb4[nt].y;
-      const uint32_t qc0 = par ? qc4[nt].z : qc4[nt].x, qc1 = par ? qc4[nt].w : qc4[nt].y;
-      const uint32_t qz0 = par ? qz4[nt].z : qz4[nt].x, qz1 = par ? qz4[nt].w : qz4[nt].y;
-      const uint32_t s0 = par ? s4.z : s4.x, s1 = par ? s4.w : s4.y;
-      const uint32_t b0 = hfma2(qc0, s0, hfma2(qb0, s0, hmul2(qa0, s0)));
-      const uint32_t b1 = hfma2(qc1, s1, hfma2(qb1, s1, hmul2(qa1, s1)));
-      if (hi) {
-        mma16816(acc_hi[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-        mma16816(acc_hi[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
-      } else {
-        mma16816(acc_lo[par][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-        mma16816(acc_lo[par][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+      for (int gi = 0; gi < NG; ++gi) {
+        s4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + tq * 64)[sigma >> 1];
+        z4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + 256 + tq * 64)[sigma >> 1];
       }
-      const uint32_t z0 = par ? z4.z : z4.x, z1 = par ? z4.w : z4.y;
-      mma16816(dz[par][nt], z0, z0, z1, z1, qz0, qz1);
+    }
+    const bool hi = sigma < NHS;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      // ---- A fragments of this slice (2 M-tiles x 4 registers)
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(recs[gi]);
+      uint32_t A[2][4];
+      if (hi) {
+        if constexpr (BHI == 4)
+          key_slice_frags<4>(kw[(2 * sigma) * 32 + lane], kw[(2 * sigma + 1) * 32 + lane], 0, A);
+        else
+          key_slice_frags<BHI>(kw[sigma * 32 + lane], 0u, 0, A);
+      } else {
+        const int sl = sigma - NHS;   // slice inside the lo block
+        if constexpr (BLO == 2)
+          key_slice_frags<2>(kw[(WH + sl) * 32 + lane], 0u, 0, A);
+        else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
+          key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, par, A);
+      }
+      // ---- B fragments: q'' = q * s (hi or lo half per column) and q (for z)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t qa0 = par ? qa4[nt].z : qa4[nt].x, qa1 = par ? qa4[nt].w : qa4[nt].y;
+        const uint32_t qb0 = par ? qb4[nt].z : qb4[nt].x, qb1 = par ? qb4[nt].w : qb4[nt].y;
+        const uint32_t qc0 = par ? qc4[nt].z : qc4[nt].x, qc1 = par ? qc4[nt].w : qc4[nt].y;
+        const uint32_t qz0 = par ? qz4[nt].z : qz4[nt].x, qz1 = par ? qz4[nt].w : qz4[nt].y;
+        const uint32_t s0 = par ? s4[gi].z : s4[gi].x, s1 = par ? s4[gi].w : s4[gi].y;
+        const uint32_t b0 = hfma2(qc0, s0, hfma2(qb0, s0, hmul2(qa0, s0)));
+        const uint32_t b1 = hfma2(qc1, s1, hfma2(qb1, s1, hmul2(qa1, s1)));
+        if (hi) {
+          mma16816(acc_hi[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+          mma16816(acc_hi[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+        } else {
+          mma16816(acc_lo[gi][pr][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+          mma16816(acc_lo[gi][pr][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+        }
+        if constexpr (NG == 1) {
+          const uint32_t z0 = par ? z4[0].z : z4[0].x, z1 = par ? z4[0].w : z4[0].y;
+          mma16816(dz[0][pr][nt], z0, z0, z1, z1, qz0, qz1);
+        } else if (gi == NG - 1) {
+          // both groups' zero points in one product: rows 0-7 group 0, rows 8-15 group 1
+          const uint32_t za0 = par ? z4[0].z : z4[0].x, za1 = par ? z4[0].w : z4[0].y;
+          const uint32_t zb0 = par ? z4[1].z : z4[1].x, zb1 = par ? z4[1].w : z4[1].y;
+          mma16816(dz[0][pr][nt], za0, zb0, za1, zb1, qz0, qz1);
+        }
+      }
     }
   }
 
   // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3;
   // the product of a row-u token carries 2^(shift(u) - 24)
-  float lg[NT][4];
+  float lg[NG][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const float zb = (dz[0][nt][0] + dz[0][nt][1]) + (dz[1][nt][0] + dz[1][nt][1]);
+  for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int mt = u >> 1, r = 2 * (u & 1);
-      const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23);
-      const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23);
-      const float vhi = acc_hi[nt][mt][r] + acc_hi[nt][mt][r + 1];
-      const float vlo = (acc_lo[0][nt][mt][r] + acc_lo[0][nt][mt][r + 1]) +
-                        (acc_lo[1][nt][mt][r] + acc_lo[1][nt][mt][r + 1]);
-      lg[nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
+    for (int nt = 0; nt < NT; ++nt) {
+      // zero-point term of this group: rows 0-7 (c0, c1) hold group 0, rows 8-15 (c2, c3)
+      // hold group 1 when two groups share the product
+      float zb = 0.f;
+#pragma unroll
+      for (int pr = 0; pr < PAR; ++pr)
+        zb += gi == 0 ? dz[0][pr][nt][0] + dz[0][pr][nt][1] : dz[0][pr][nt][2] + dz[0][pr][nt][3];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int mt = u >> 1, r = 2 * (u & 1);
+        const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23);
+        const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23);
+        const float vhi = acc_hi[gi][nt][mt][r] + acc_hi[gi][nt][mt][r + 1];
+        float vlo = 0.f;
+#pragma unroll
+        for (int pr = 0; pr < PAR; ++pr) vlo += acc_lo[gi][pr][nt][mt][r] + acc_lo[gi][pr][nt][mt][r + 1];
+        lg[gi][nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
+      }
     }
-  }
 
-  // ---- online softmax
+  // ---- online softmax over the NG groups
   float mnew[NT];
   bool grow = false;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    float mx = fmaxf(fmaxf(lg[nt][0], lg[nt][1]), fmaxf(lg[nt][2], lg[nt][3]));
+    float mx = -INFINITY;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi)
+      mx = fmaxf(mx, fmaxf(fmaxf(lg[gi][nt][0], lg[gi][nt][1]), fmaxf(lg[gi][nt][2], lg[gi][nt][3])));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -269,7 +330,7 @@ __device__ __forceinline__ void process_group(const Geometry& g, const uint8_t* 
     float alpha[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      alpha[nt] = exp2f(st.m[nt] - mnew[nt]);
+      alpha[nt] = ex2(st.m[nt] - mnew[nt]);
       st.l[nt] *= alpha[nt];
       st.m[nt] = mnew[nt];
     }
@@ -295,109 +356,108 @@ __device__ __forceinline__ void process_group(const Geometry& g, const uint8_t* 
     st.bias[2] *= a0;
     st.bias[3] *= a1;
   }
-  float p[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      p[nt][i] = exp2f(lg[nt][i] - st.m[nt]);
-      st.l[nt] += p[nt][i];
-    }
-  }
 
-  // ---- P as B fragments: column gq = head gq, tokens 2tq + {0,1} (+8, +16, +24)
   const int srcA = (2 * tq) * 4 + (gq & 3), srcB = (2 * tq + 1) * 4 + (gq & 3);
-  float pa[4], pb[4];
+  const bool col_ok = gq < g.G;
+  const uint32_t four2 = 0x44004400u;   // fp16x2 (4, 4)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    pa[i] = __shfl_sync(0xffffffffu, p[0][i], srcA);
-    pb[i] = __shfl_sync(0xffffffffu, p[0][i], srcB);
-  }
-  if constexpr (NT == 2) {
+  for (int gi = 0; gi < NG; ++gi) {
+    const uint8_t* rec = recs[gi];
+    float p[NT][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float xa = __shfl_sync(0xffffffffu, p[1][i], srcA);
-      const float xb = __shfl_sync(0xffffffffu, p[1][i], srcB);
-      if (gq >= 4) {
-        pa[i] = xa;
-        pb[i] = xb;
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        p[nt][i] = ex2(lg[gi][nt][i] - st.m[nt]);
+        st.l[nt] += p[nt][i];
       }
     }
-  }
-  uint32_t p16[4];
-  const bool col_ok = gq < g.G;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p16[i] = col_ok ? pack_f16x2(pa[i], pb[i]) : 0u;
-
-  // value scales: token pairs tp2 = tq + 4i, four channel groups each
-  const int vs_off = kc + 1536, vz_off = kc + 1792;
-  uint32_t vsr[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(rec + vs_off + (tq + 4 * i) * 16);
-    vsr[i][0] = v.x; vsr[i][1] = v.y; vsr[i][2] = v.z; vsr[i][3] = v.w;
-  }
-  // zero-point term: A rows = channel groups (rows 0..3), k = tokens
-  {
-    const int j = gq & 3;
-    uint32_t vz[4];
+    // ---- P as B fragments: column gq = head gq, tokens 2tq + {0,1} (+8, +16, +24)
+    float pa[4], pb[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
-      vz[i] = gq < 4 ? v : 0u;
+      pa[i] = __shfl_sync(0xffffffffu, p[0][i], srcA);
+      pb[i] = __shfl_sync(0xffffffffu, p[0][i], srcB);
     }
-    mma16816(st.bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
-    mma16816(st.bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
-  }
-  // value codes: words 0..7 of this lane (two 16-byte chunks).  Slot (r, p) of word m
-  // sits at bits 8r + 2p; taken from w >> (8r + 4*(p>>1)) at bit 2*(p&1), so odd token
-  // pairs carry an extra 2^2: the even-pair B columns are scaled by 4 to match.
-  const uint32_t four2 = 0x44004400u;   // fp16x2 (4, 4)
-  const uint32_t p16x4_0 = hmul2(p16[0], four2), p16x4_2 = hmul2(p16[2], four2);
-  const uint4 vw0 = *reinterpret_cast<const uint4*>(rec + kc + 512 + lane * 16);
-  const uint4 vw1 = *reinterpret_cast<const uint4*>(rec + kc + 512 + (32 + lane) * 16);
-  const uint32_t vw[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
+    if constexpr (NT == 2) {
 #pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int j = m >> 1;
-    const uint32_t w = vw[m], w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
-    // (r, p) -> k-step p >> 1, register r + 2*(p & 1)
-    const uint32_t k0a0 = sub_pair(w, 0x00030003u), k0a2 = sub_pair(w, 0x000C000Cu);
-    const uint32_t k1a0 = sub_pair(w4, 0x00030003u), k1a2 = sub_pair(w4, 0x000C000Cu);
-    const uint32_t k0a1 = sub_pair(w8, 0x00030003u), k0a3 = sub_pair(w8, 0x000C000Cu);
-    const uint32_t k1a1 = sub_pair(w12, 0x00030003u), k1a3 = sub_pair(w12, 0x000C000Cu);
-    const uint32_t b00 = hmul2(p16x4_0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
-    const uint32_t b10 = hmul2(p16x4_2, vsr[2][j]), b11 = hmul2(p16[3], vsr[3][j]);
-    mma16816(st.pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
-    mma16816(st.pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
+      for (int i = 0; i < 4; ++i) {
+        const float xa = __shfl_sync(0xffffffffu, p[1][i], srcA);
+        const float xb = __shfl_sync(0xffffffffu, p[1][i], srcB);
+        if (gq >= 4) {
+          pa[i] = xa;
+          pb[i] = xb;
+        }
+      }
+    }
+    uint32_t p16[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p16[i] = col_ok ? pack_f16x2(pa[i], pb[i]) : 0u;
+
+    // value scales: token pairs tp2 = tq + 4i, four channel groups each
+    const int vs_off = kc + 1536, vz_off = kc + 1792;
+    uint32_t vsr[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(rec + vs_off + (tq + 4 * i) * 16);
+      vsr[i][0] = v.x; vsr[i][1] = v.y; vsr[i][2] = v.z; vsr[i][3] = v.w;
+    }
+    // zero-point term: A rows = channel groups (rows 0..3), k = tokens
+    {
+      const int j = gq & 3;
+      uint32_t vz[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
+        vz[i] = gq < 4 ? v : 0u;
+      }
+      mma16816(st.bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
+      mma16816(st.bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
+    }
+    // value codes: words 0..7 of this lane (two 16-byte chunks).  Slot (r, p) of word m
+    // sits at bits 8r + 2p; taken from w >> (8r + 4*(p>>1)) at bit 2*(p&1), so odd token
+    // pairs carry an extra 2^2: the even-pair B columns are scaled by 4 to match.
+    const uint32_t p16x4_0 = hmul2(p16[0], four2), p16x4_2 = hmul2(p16[2], four2);
+    const uint4 vw0 = *reinterpret_cast<const uint4*>(rec + kc + 512 + lane * 16);
+    const uint4 vw1 = *reinterpret_cast<const uint4*>(rec + kc + 512 + (32 + lane) * 16);
+    const uint32_t vw[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int j = m >> 1;
+      const uint32_t w = vw[m], w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
+      // (r, p) -> k-step p >> 1, register r + 2*(p & 1)
+      const uint32_t k0a0 = sub_pair(w, 0x00030003u), k0a2 = sub_pair(w, 0x000C000Cu);
+      const uint32_t k1a0 = sub_pair(w4, 0x00030003u), k1a2 = sub_pair(w4, 0x000C000Cu);
+      const uint32_t k0a1 = sub_pair(w8, 0x00030003u), k0a3 = sub_pair(w8, 0x000C000Cu);
+      const uint32_t k1a1 = sub_pair(w12, 0x00030003u), k1a3 = sub_pair(w12, 0x000C000Cu);
+      const uint32_t b00 = hmul2(p16x4_0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
+      const uint32_t b10 = hmul2(p16x4_2, vsr[2][j]), b11 = hmul2(p16[3], vsr[3][j]);
+      mma16816(st.pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
+      mma16816(st.pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
+    }
   }
 }
 
-// The residual item: up to 31 bf16 tokens, with CUDA cores, heads h0, h0 + hstep, ...
-// one at a time (few registers).  Lane = token for the logit (its K row read with 16-byte loads, q in natural
-// channel order from shared memory), lane = channel for the values (rows read coalesced,
-// four tokens ahead).  Writes one partial per head into `slot`.
+// The residual item: up to 31 bf16 tokens staged in shared memory, with CUDA cores, heads
+// h0, h0 + hstep, ... one at a time (few registers).  Lane = token for the logit (its K
+// row, q in natural channel order), lane = channel for the values.  Writes one partial
+// per head into `slot`.
 __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
                                               int nr, const float* qnat, float* slot, int h0, int hstep) {
   const int lane = threadIdx.x & 31;
-  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kHeadDim);
+  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kResidKStride);
 #pragma unroll 1
   for (int hh = h0; hh < g.G; hh += hstep) {
     const float* qh = qnat + hh * kHeadDim;
     float lg = 0.f;
+#pragma unroll 4
+    for (int c8 = 0; c8 < 16; ++c8) {
+      const uint4 kv = row[c8];
+      const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-    for (int c4 = 0; c4 < 16; c4 += 4) {
-      uint4 kv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) kv[i] = __ldg(row + c4 + i);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t w[4] = {kv[i].x, kv[i].y, kv[i].z, kv[i].w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float k = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-          lg = fmaf(qh[(c4 + i) * 8 + e], k, lg);
-        }
+      for (int e = 0; e < 8; ++e) {
+        const float k = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        lg = fmaf(qh[c8 * 8 + e], k, lg);
       }
     }
     if (lane >= nr) lg = -INFINITY;
@@ -409,23 +469,11 @@ __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t*
 #pragma unroll
     for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int t0 = 0; t0 < nr; t0 += 4) {
-      float v[4][4];
+#pragma unroll 4
+    for (int t = 0; t < nr; ++t) {
+      const float pt = __shfl_sync(0xffffffffu, pw, t);
 #pragma unroll
-      for (int dt = 0; dt < 4; ++dt) {
-        const int t = t0 + dt < nr ? t0 + dt : nr - 1;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[dt][i] = bf16_bits_to_float(rv[t * kHeadDim + lane + 32 * i]);
-      }
-#pragma unroll
-      for (int dt = 0; dt < 4; ++dt) {
-        const float pt = __shfl_sync(0xffffffffu, pw, (t0 + dt) & 31);
-        if (t0 + dt < nr) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[i] = fmaf(pt, v[dt][i], acc[i]);
-        }
-      }
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(pt, bf16_bits_to_float(rv[t * kHeadDim + lane + 32 * i]), acc[i]);
     }
     float* s = slot + hh * kPartialStride;
     if (lane == 0) {
@@ -438,7 +486,7 @@ __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t*
 }
 
 template <int BHI, int BLO, int NT, int NHS>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 3)
 decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
                   DecodeWs ws) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -450,9 +498,21 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
   float* qnat = reinterpret_cast<float*>(smem + sm.qnat);
   uint8_t* perm = smem + sm.perm;
   float* rslot = reinterpret_cast<float*>(smem + sm.resid);
+  uint16_t* rrk = reinterpret_cast<uint16_t*>(smem + sm.rrows);
+  uint16_t* rrv = rrk + kGroup * kResidKStride;
   float* part = reinterpret_cast<float*>(smem + sm.part);
-  uint8_t* ring = smem + sm.stages + warp * kStages * R;
-  const int chunks = R >> 4;
+  constexpr int kS = stages_for<NT>();
+  uint8_t* ring = smem + sm.stages + warp * kS * R;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm.bars) + warp * kS;
+  if (lane == 0) {
+    for (int k = 0; k < kS; ++k) mbar_init(bars + k, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // A warp's staged groups are numbered in order across its segments: ordinal o lives in
+  // slot o % kS and completes phase (o / kS) & 1 of that slot's barrier.
+  uint32_t ord_base = 0;
+  bool failed = false;
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
@@ -461,16 +521,34 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     const int my_first = seg.lo + warp;
     const int my_count = my_first < gend ? (gend - my_first + kWarps - 1) / kWarps : 0;
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
-    auto issue = [&](int i) {
-      if (i < my_count) {
-        const uint8_t* src = unit_rec + static_cast<size_t>(my_first + i * kWarps) * R;
-        uint8_t* dst = ring + (i % kStages) * R;
-        for (int k = lane; k < chunks; k += 32) cp_async16(dst + 16 * k, src + 16 * k);
+    int issued = 0;   // groups of this segment handed to the copy engine
+    // Issue the warp's groups [issued, upto) of this segment.  Ordinal j may only be
+    // issued while j - (first unconsumed ordinal) < kS, which the callers keep.
+    auto issue_upto = [&](int upto) {
+      const int last = upto < my_count ? upto : my_count;
+      for (; issued < last; ++issued) {
+        if (lane == 0) {
+          const uint32_t o = ord_base + issued, slot = o % kS;
+          fence_proxy_async();
+          mbar_expect_tx(bars + slot, static_cast<uint32_t>(R));
+          bulk_g2s(ring + slot * R, unit_rec + static_cast<size_t>(my_first + issued * kWarps) * R,
+                   static_cast<uint32_t>(R), bars + slot);
+        }
       }
-      cp_async_commit();
     };
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) issue(i);
+    // wait until the group of ordinal ord_base + i has landed; returns its record
+    auto acquire = [&](int i) -> const uint8_t* {
+      const uint32_t o = ord_base + i, slot = o % kS, phase = (o / kS) & 1;
+      uint32_t spins = 0;
+      while (!failed && !mbar_try_wait(bars + slot, phase)) {
+        if (++spins >= kWaitLimit) {
+          failed = true;
+          if (lane == 0) atomicOr(c.error, PNMIX_DEVERR_TIMEOUT);
+        }
+      }
+      return ring + slot * R;
+    };
+    issue_upto(kS - groups_per_step<NT>());
 
     // ---- query: log2-domain scale, natural order, then fp16 hi/lo column sets in
     // position order
@@ -480,6 +558,16 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       const int hh = i / kHeadDim;
       qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) * qscale
                        : 0.f;
+    }
+    const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
+    if (seg_resid) {   // residual K and V rows into shared memory, 16-byte loads
+      const uint4* gk = reinterpret_cast<const uint4*>(c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim);
+      const uint4* gv = reinterpret_cast<const uint4*>(c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim);
+      for (int i = tid; i < seg.nr * 16; i += kThreads) {
+        const int r = i >> 4, cc = i & 15;
+        reinterpret_cast<uint4*>(rrk + r * kResidKStride)[cc] = __ldg(gk + i);
+        reinterpret_cast<uint4*>(rrv)[i] = __ldg(gv + i);
+      }
     }
     __syncthreads();
     {
@@ -513,10 +601,8 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     __syncthreads();
 
     // ---- the residual item (CUDA cores): warp w takes heads w, w + 4
-    if (seg.hi > seg.ng && seg.nr > 0) {
-      const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
-      const uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
-      residual_partial(g, rk, rv, seg.nr, qnat, rslot, warp, kWarps);
+    if (seg_resid) {
+      residual_partial(g, rrk, rrv, seg.nr, qnat, rslot, warp, kWarps);
     } else if (warp == 0 && lane < G) {
       rslot[lane * kPartialStride + 0] = -INFINITY;
       rslot[lane * kPartialStride + 1] = 0.f;
@@ -536,14 +622,31 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 #pragma unroll
     for (int i = 0; i < 4; ++i) st.bias[i] = 0.f;
 
-    for (int i = 0; i < my_count; ++i) {
-      issue(i + kStages - 1);
-      cp_async_wait<kStages - 1>();
+    int i = 0;
+    if constexpr (groups_per_step<NT>() == 2) {
+      for (; i + 1 < my_count; i += 2) {
+        issue_upto(i + kS);
+        const uint8_t* const recs[2] = {acquire(i), acquire(i + 1)};
+        __syncwarp();
+        if (!failed) process_groups<BHI, BLO, NT, NHS, 2>(g, recs, qsets, st);
+        __syncwarp();
+      }
+    }
+    for (; i < my_count; ++i) {
+      issue_upto(i + kS);
+      const uint8_t* const recs[1] = {acquire(i)};
       __syncwarp();
-      process_group<BHI, BLO, NT, NHS>(g, ring + (i % kStages) * R, qsets, st);
+      if (!failed) process_groups<BHI, BLO, NT, NHS, 1>(g, recs, qsets, st);
       __syncwarp();
     }
-    cp_async_wait<0>();
+    if (failed) {   // let copies still in flight land before the shared memory is reused
+      for (int k = 0; k < kS && k < my_count; ++k) {
+        const uint32_t o = ord_base + my_count - 1 - k;
+        for (uint32_t spins = 0; spins < kWaitLimit && !mbar_try_wait(bars + o % kS, (o / kS) & 1); ++spins) {
+        }
+      }
+    }
+    ord_base += my_count;
     __syncthreads();   // every ring is idle: the merge area may alias them
 
     // ---- warp partials into shared memory

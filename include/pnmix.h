@@ -133,6 +133,8 @@ typedef enum {
 
 /* Device error word bits (pnmix_read_error). */
 #define PNMIX_DEVERR_APPEND_FULL 0x1u  /* pnmix_append found len == capacity_tokens */
+#define PNMIX_DEVERR_TIMEOUT 0x2u      /* a bounded wait for staged cache data ran out in
+                                          pnmix_decode_attention (its output is then invalid) */
 
 /*
  * Method parameters.  Supported set:
