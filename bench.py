@@ -38,6 +38,15 @@ PREFILL, CONTEXT, WINDOW = 4096, 32768, 64
 K_SALIENT, BHI, BLO = 8, 4, 2
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM traffic of one decode launch from the committed ncu capture (profiles/
+# decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
+# of the decode sources it was taken on.  Reported only while the sources still match.
+DECODE_CAPTURE = {"sources_sha256_16": "9494d23a19085423", "traffic_bytes": 425101568,
+                  "algorithmic_bytes": 420855808}
+DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
+                  "decode_attention_prefill_b200/csrc/decode_common.cuh",
+                  "decode_attention_prefill_b200/csrc/common.cuh"]
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -62,6 +71,19 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def captured_traffic(alg_bytes_per_launch: float):
+    """Per-launch DRAM traffic scaled from the recorded capture, or None if the decode
+    sources changed since it was taken."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != DECODE_CAPTURE["sources_sha256_16"]:
+        return None
+    return DECODE_CAPTURE["traffic_bytes"] * alg_bytes_per_launch / DECODE_CAPTURE["algorithmic_bytes"]
 
 
 def decode_bytes(n_tokens: int, units: int, G: int, record_bytes: int) -> int:
@@ -380,7 +402,8 @@ def main():
                    "key_bits": [BHI, BLO], "value_bits": 2, "key_code_bits": 2.25,
                    "parallelism": f"dp{world}", "l2": "inputs larger than L2 (419 MB cache read per step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "pnmix decode attention",
+                     "frac": achieved / peak, "traffic": captured_traffic(sum(alg) / K),
+                     "algorithmic_bytes": sum(alg) / K, "kernel": "pnmix decode attention",
                      "peak_source": peak_kind, "frac_of_8tbs": achieved / 8000.0},
         "decode_kernel_us": 1e3 * sum(dec_ms) / K,
         "append_kernel_us": 1e3 * sum(app_ms) / K,

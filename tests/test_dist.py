@@ -1,0 +1,62 @@
+"""Multi-process host logic of the benchmark (gloo, world size 2, CPU).
+
+The decode path shards into independent (sequence, KV head) units, so ranks share no
+data; the only collectives are the barrier around the timed region and the max-over-ranks
+reduction of the measured time.  These tests run that logic on CPU ranks."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    w, r, local = bench.dist_setup(None)
+    assert (w, r, local) == (world, rank, rank)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # each rank: its own sequences (seed offset), its own measured time
+    seed = 0 + 7919 * rank
+    t = torch.tensor([10.0 + 5.0 * rank])
+    dist.barrier()
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    # whole-job value: all ranks' tokens over the slowest rank's time
+    value = world * bench.B * 4 / (float(t.item()) / 1e3)
+    q.put((rank, seed, float(t.item()), value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_shard_sequences_and_take_the_max_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    out = sorted(q.get(timeout=10) for _ in range(2))
+    assert out[0][1] != out[1][1]                 # distinct sequences per rank
+    assert out[0][2] == out[1][2] == 15.0         # the max over ranks
+    assert out[0][3] == out[1][3] == pytest.approx(2 * 16 * 4 / 0.015)
+
+
+def test_reference_arm_other_ranks_exit_quietly(capsys):
+    import bench
+
+    class A:
+        steps, warmup, seed = 1, 0, 0
+    assert bench.run_reference(A(), 2, 1) == 0
+    assert capsys.readouterr().out == ""
