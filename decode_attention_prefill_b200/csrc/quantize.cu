@@ -85,18 +85,37 @@ __device__ void quantize_key_group(const Geometry& g, GroupSmem& sm, uint8_t* re
 __device__ void quantize_value_group(const Geometry& g, GroupSmem& sm, uint8_t* rec) {
   {
     const int t = threadIdx.x >> 2, jg = threadIdx.x & 3;
-    float mn = bf16_bits_to_float(sm.tile[t][32 * jg]), mx = mn;
-#pragma unroll 8
+    // the thread's 32 channels with four 16-byte loads
+    float x[32];
+    const uint4* row = reinterpret_cast<const uint4*>(&sm.tile[t][32 * jg]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 v = row[k];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[8 * k + 2 * e] = __uint_as_float(w[e] << 16);
+        x[8 * k + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+    float mn = x[0], mx = x[0];
+#pragma unroll
     for (int i = 1; i < 32; ++i) {
-      float x = bf16_bits_to_float(sm.tile[t][32 * jg + i]);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+      mn = fminf(mn, x[i]);
+      mx = fmaxf(mx, x[i]);
     }
     QParams q = quant_params(mn, mx, g.bv);
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i)
-      sm.codes[t][32 * jg + i] =
-          static_cast<uint8_t>(quant_code(bf16_bits_to_float(sm.tile[t][32 * jg + i]), q, g.bv));
+    uint32_t packed[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t wv = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wv |= quant_code(x[4 * k + e], q, g.bv) << (8 * e);
+      packed[k] = wv;
+    }
+    uint4* crow = reinterpret_cast<uint4*>(&sm.codes[t][32 * jg]);
+    crow[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    crow[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     uint16_t* vs = reinterpret_cast<uint16_t*>(rec + rec_vscale(g));
     uint16_t* vz = reinterpret_cast<uint16_t*>(rec + rec_vzero(g));
     vs[vscale_index(t, jg)] = q.s16;

@@ -156,7 +156,8 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
   // scratch (max-norm accumulators and tickets) starts at zero for every call
   cudaError_t e = cudaMemsetAsync(c.scratch, 0, sizeof(uint32_t) * static_cast<size_t>(units) * 65, s);
   if (e != cudaSuccess) return e;
-  int want = (2 * 148 + units - 1) / units;
+  // about eight CTAs per SM so the max pass balances, with >= 128 tokens per CTA
+  int want = (8 * 148 + units - 1) / units;
   int max_split = (L + 127) / 128;
   int nsplit = want < max_split ? want : max_split;
   if (nsplit < 1) nsplit = 1;
