@@ -58,6 +58,15 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="stream_32k",
+                    choices=["stream_32k", "llama3_8b", "sweep_128k", "pipeline_32l"],
+                    help="stream_32k is the benchmark line; the others print per-workload "
+                         "measurements (decode GB/s and tokens/s; for the sweep the relative L2 "
+                         "error against unquantized bf16 attention; for the 32-layer pipeline the "
+                         "prefill latencies and the extrapolated end-to-end tokens/s)")
+    ap.add_argument("--pipeline-layers-generated", type=int, default=4,
+                    help="pipeline_32l: layers whose prefill inputs are generated (seed + layer); "
+                         "the others reuse them cyclically")
     ap.add_argument("--profile-decode", action="store_true",
                     help="build the 32K state, then run only --warmup + --steps decode launches "
                          "(small device footprint, for profiler captures); prints no bench line")
@@ -260,11 +269,206 @@ def run_reference(args, world, rank):
     return 0
 
 
+def exact_bf16_attention(q: np.ndarray, kin: np.ndarray, vin: np.ndarray) -> np.ndarray:
+    """softmax(q k^T / sqrt(128)) v over the unquantized bf16 rows, in fp64: the quality
+    yardstick of the bit sweep (q [G][128], kin / vin [n][128], all bf16 bits)."""
+    import workload
+    qf = workload.bf16_to_float(q).astype(np.float64)
+    kf = workload.bf16_to_float(kin).astype(np.float64)
+    vf = workload.bf16_to_float(vin).astype(np.float64)
+    logits = qf @ kf.T / np.sqrt(128.0)
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    return (p @ vf) / p.sum(axis=1, keepdims=True)
+
+
+def timed_launch(fn, flush, reps: int, warmup: int) -> float:
+    """Median device time (s) of fn() over reps launches, each after an L2 flush."""
+    import torch
+    times = []
+    for i in range(warmup + reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(times)
+
+
+def run_decode_workload(args):
+    """Decode-only measurements: llama3_8b (batch 8, 32/8 heads, one step at 8192) and
+    sweep_128k (batch 2, 28/4 heads, 131072 tokens, six bit points, each with the relative
+    L2 error against unquantized bf16 attention over every (sequence, KV head) unit).
+    These caches fit in L2, so every timed launch follows an L2 flush."""
+    import torch
+
+    import decode_attention_prefill_b200 as pm
+    import workload
+    wl = workload.WORKLOADS[args.workload]
+    Bw, Hq, Hkv, ctx = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.context
+    G = Hq // Hkv
+    points = wl.sweep if wl.sweep else (wl.bits,)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kin = workload.rows(args.seed, workload.K, Bw, Hkv, 0, ctx)
+    vin = workload.rows(args.seed, workload.V, Bw, Hkv, 0, ctx)
+    qwin = workload.rows(args.seed, workload.Q, Bw, Hq, ctx - WINDOW, WINDOW, group=G)
+    q = np.ascontiguousarray(workload.rows(args.seed, workload.Q, Bw, Hq, ctx, 1, group=G)[:, :, 0])
+    k_dev = torch.from_numpy(kin).view(torch.bfloat16).to(dev)
+    v_dev = torch.from_numpy(vin).view(torch.bfloat16).to(dev)
+    qwin_dev = torch.from_numpy(qwin).view(torch.bfloat16).to(dev)
+    q_dev = torch.from_numpy(q).view(torch.bfloat16).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # twice the 126 MB L2
+    peak, peak_kind = measured_peaks()
+    exact = None
+    if wl.sweep:
+        exact = {(b, h): exact_bf16_attention(q[b, h * G:(h + 1) * G], kin[b, h], vin[b, h])
+                 for b in range(Bw) for h in range(Hkv)}
+    results = []
+    with ClockSampler(0) as clocks:
+        for bp in points:
+            cfg = pm.Config.make(Hq, Hkv, bp.key_bits_hi, bp.key_bits_lo, bp.n_salient_pairs, WINDOW)
+            cache = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
+            cache.prefill(qwin_dev, k_dev, v_dev, ctx)
+            out = torch.empty(Bw, Hq, D, dtype=torch.float32, device=dev)
+            t = timed_launch(lambda: pm.pnmix_decode_attention(cfg, q_dev, cache, out), flush,
+                             args.steps, args.warmup)
+            assert cache.read_error() == 0
+            alg = decode_bytes(ctx, Bw * Hkv, G, cache.c.record_bytes)
+            r = {"key_bits": [bp.key_bits_hi, bp.key_bits_lo], "salient_pairs": bp.n_salient_pairs,
+                 "key_code_bits": bp.key_code_bits, "bytes_per_token_head": cache.c.record_bytes / 32,
+                 "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
+                 "frac_of_8tbs": alg / t / 8e12, "tokens_per_s": Bw / t}
+            if exact is not None:
+                got = out.cpu().numpy().astype(np.float64)
+                num = sum(float(np.sum((got[b, h * G:(h + 1) * G] - e) ** 2)) for (b, h), e in exact.items())
+                den = sum(float(np.sum(e ** 2)) for e in exact.values())
+                r["rel_l2_vs_bf16_attention"] = (num / den) ** 0.5
+            results.append(r)
+            del cache
+    line = {"workload": args.workload, "metric": "decode-attn GB/s (% of B200 HBM peak) + tokens/s",
+            "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "data": "synthetic", "dtype": "f32",
+            "config": {"batch": Bw, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": D,
+                       "context": ctx, "l2": "flushed (256 MB write) before every timed launch"},
+            "peak": peak, "peak_source": peak_kind, "points": results, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_pipeline(args):
+    """pipeline_32l: 32 layers, batch 32, 32/8 heads.  Per layer a 4096-token prefill
+    (saliency + quantize), then decode steps (append + attend in every layer) to 32768.
+    Prefill is timed on all 32 layers; the decode phase is timed at sampled contexts and
+    integrated over the 28672 steps (decode time is linear in the context), which the
+    output labels as extrapolated.  Layer l's inputs are those of seed + l for the
+    prefill; the decode-time caches past the prefill are filled by quantizing the
+    generated rows of layer 0 repeated along time (the decode cost does not depend on the
+    values), which keeps host generation to one layer."""
+    import torch
+
+    import decode_attention_prefill_b200 as pm
+    import workload
+    wl = workload.WORKLOADS["pipeline_32l"]
+    Bw, Hq, Hkv, L, C, NL = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.prefill, wl.context, wl.layers
+    G = Hq // Hkv
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n_gen = min(NL, max(1, args.pipeline_layers_generated))
+    cfg = pm.Config.make(Hq, Hkv, BHI, BLO, K_SALIENT, WINDOW)
+    caches = [pm.PNMixCache(cfg, Bw, C + 32, max_context=C) for _ in range(NL)]
+    inputs = []
+    for l in range(n_gen):
+        s = args.seed + l
+        inputs.append((torch.from_numpy(workload.rows(s, workload.Q, Bw, Hq, L - WINDOW, WINDOW, group=G))
+                       .view(torch.bfloat16).to(dev),
+                       torch.from_numpy(workload.rows(s, workload.K, Bw, Hkv, 0, L)).view(torch.bfloat16).to(dev),
+                       torch.from_numpy(workload.rows(s, workload.V, Bw, Hkv, 0, L)).view(torch.bfloat16).to(dev)))
+    # ---- prefill of all layers: saliency, then quantize, each layer in turn
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * NL)]
+    for rep in range(2):
+        for l in range(NL):
+            qw, kk, vv = inputs[l % n_gen]
+            caches[l].reset()
+            ev[3 * l].record()
+            pm.pnmix_select_pairs(cfg, qw, kk, L, caches[l])
+            ev[3 * l + 1].record()
+            pm.pnmix_quantize_keys(cfg, kk, L, caches[l])
+            pm.pnmix_quantize_values(cfg, vv, L, caches[l])
+            ev[3 * l + 2].record()
+        torch.cuda.synchronize()
+    sal_ms = sum(ev[3 * l].elapsed_time(ev[3 * l + 1]) for l in range(NL))
+    qnt_ms = sum(ev[3 * l + 1].elapsed_time(ev[3 * l + 2]) for l in range(NL))
+    prefill_ms = ev[0].elapsed_time(ev[3 * NL - 1])
+    # ---- decode phase at sampled contexts
+    reps = 8
+    k_rep = inputs[0][1].repeat(1, 1, C // L, 1)           # [B][Hkv][C][128]
+    v_rep = inputs[0][2].repeat(1, 1, C // L, 1)
+    steps_in = workload.rows(args.seed, workload.K, Bw, Hkv, L, reps)
+    kn = torch.from_numpy(np.ascontiguousarray(steps_in.transpose(2, 0, 1, 3))).view(torch.bfloat16).to(dev)
+    vn = torch.from_numpy(np.ascontiguousarray(
+        workload.rows(args.seed, workload.V, Bw, Hkv, L, reps).transpose(2, 0, 1, 3))).view(torch.bfloat16).to(dev)
+    qn = torch.from_numpy(np.ascontiguousarray(
+        workload.rows(args.seed, workload.Q, Bw, Hq, L, reps, group=G).transpose(2, 0, 1, 3))).view(torch.bfloat16).to(dev)
+    out = torch.empty(Bw, Hq, D, dtype=torch.float32, device=dev)
+    samples = []
+    contexts = [L + 1 + reps, 8192, 12288, 16384, 20480, 24576, 28672, C]
+    with ClockSampler(0) as clocks:
+        for ctx in contexts:
+            start = ctx - reps           # cache length before the first sampled step
+            for l in range(NL):
+                pm.pnmix_quantize_keys(cfg, k_rep, start, caches[l])
+                pm.pnmix_quantize_values(cfg, v_rep, start, caches[l])
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for i in range(reps):
+                if i == 2:
+                    e0.record()
+                for l in range(NL):
+                    pm.pnmix_append(cfg, kn[i], vn[i], caches[l])
+                    pm.pnmix_decode_attention(cfg, qn[i], caches[l], out)
+            e1.record()
+            torch.cuda.synchronize()
+            step_ms = e0.elapsed_time(e1) / (reps - 2)
+            samples.append({"context": start + 1 + (2 + reps - 1) / 2, "step_ms": step_ms})
+    assert all(c.read_error() == 0 for c in caches)
+    # integrate the step time over the decode steps (contexts L+1 .. C), trapezoid rule
+    xs = [s["context"] for s in samples]
+    ys = [s["step_ms"] for s in samples]
+    steps = C - L
+    grid = np.arange(L + 1, C + 1, dtype=np.float64)
+    total_ms = float(np.sum(np.interp(grid, xs, ys)))
+    line = {"workload": "pipeline_32l", "metric": "end-to-end attention-path tokens/s",
+            "unit": "tokens/s", "n_gpus": 1, "data": "synthetic", "dtype": "f32",
+            "config": {"layers": NL, "batch": Bw, "n_q_heads": Hq, "n_kv_heads": Hkv,
+                       "prefill": L, "context": C, "salient_pairs": K_SALIENT, "key_bits": [BHI, BLO],
+                       "prefill_inputs": f"seed + layer for {n_gen} generated layer(s), reused cyclically",
+                       "l2": "32 layers of cache between re-reads of a layer (>= 3 GB)"},
+            "prefill": {"saliency_ms_all_layers": sal_ms, "quantize_ms_all_layers": qnt_ms,
+                        "prefill_ms_all_layers": prefill_ms,
+                        "quantize_tokens_per_s": NL * Bw * L / (qnt_ms / 1e3)},
+            "decode_samples": samples,
+            "decode": {"steps": steps, "total_s_extrapolated": total_ms / 1e3,
+                       "tokens_per_s_extrapolated": Bw * steps / (total_ms / 1e3)},
+            "end_to_end": {"total_s_extrapolated": (total_ms + prefill_ms) / 1e3,
+                           "tokens_per_s_extrapolated": Bw * steps / ((total_ms + prefill_ms) / 1e3)},
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.workload == "pipeline_32l":
+        return run_pipeline(args)
+    if args.workload != "stream_32k":
+        return run_decode_workload(args)
 
     import torch
     if not torch.cuda.is_available():
