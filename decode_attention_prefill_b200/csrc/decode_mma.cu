@@ -6,12 +6,15 @@
 //
 //   logits  q . k^_t = sum_p q_p (s_p code_{p,t} + z_p)
 //          = [codes (32 tok x 128 pos)] x [q_p s_p]  +  [z broadcast] x [q]
-//   The codes become exact fp16 A fragments in registers (mask-and-OR into the mantissa
-//   of 1024.0, then one fp16 FMA removes the 1024 and the bit position).  The query is
-//   split into fp16 hi + lo halves held in interleaved B columns (head h -> columns 2h,
-//   2h+1) so the m16n8k16 product keeps ~22 bits; the per-group q_p s_p is formed with
-//   three fp16 FMAs per pair.  The zero-point term is one more MMA per slice with the z
-//   pairs broadcast over the rows.
+//   The codes become exact fp16 A fragments in registers: an AND leaves them as fp16
+//   subnormals code * 2^(offset-24), which the tensor cores multiply exactly.  The bf16
+//   query is exact in fp16; the product q_p s_p (19 significant bits) is carried exactly
+//   by two interleaved B columns (head h -> columns 2h, 2h+1): fp16(q s) and its rounding
+//   error fma(q, s, -fp16(q s)).  One lane-uniform sequence b = fma(X, s, fp16(Y s)) with
+//   per-lane constants (X, Y) = (0, q) on even columns and (q, -q) on odd ones gives both.
+//   The zero-point term is one more MMA per slice with the z pairs broadcast over the
+//   rows and X as B (the pair of columns then sums to q).  The softmax scale is applied
+//   to the fp32 logits.
 //   out     sum_t p_t v^_t = sum_t (p_t s_{t,j}) code_{t,c} + sum_t p_t z_{t,j}
 //          = [codes^T (channels x tokens)] x [p s]  +  [z rows] x [p]
 //   with p rounded to fp16 once (fp32 accumulation).
@@ -20,6 +23,8 @@
 // m16n8k16 tiles, so a lane's code words are exactly its A registers.  Splits merge
 // through decode_common.cuh (fused combine, no waiting).  The bf16 residual window is
 // attended by warp 0 of the last split with CUDA cores.
+#include <atomic>
+
 #include "common.cuh"
 #include "decode_common.cuh"
 
@@ -75,16 +80,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-// One bulk copy (TMA, no multicast) of `bytes` from global to this CTA's shared memory;
-// completion is signalled on `bar` as transaction bytes.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+// One staged group (a TMA bulk copy, no multicast): the issuing lane orders the warp's
+// earlier shared-memory reads of the slot before the copy's writes (fence.proxy.async),
+// arms the slot's barrier with the byte count and starts the copy.  Every lane executes
+// it; only `leader` acts (predicated, so the warp does not branch).
+__device__ __forceinline__ void stage_group(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                            bool leader) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " @p fence.proxy.async.shared::cta;\n"
+      " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %2;\n"
+      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "r"(static_cast<uint32_t>(leader))
+      : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   uint32_t ok;
@@ -94,9 +102,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(phase) : "memory");
   return ok != 0;
 }
-// Orders this thread's earlier generic-proxy accesses of shared memory before later
-// async-proxy (TMA) writes to it.
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
 // try_wait rounds before a staging wait gives up (each round may suspend the warp for a
@@ -146,8 +151,8 @@ __device__ __forceinline__ void key_slice_frags(uint32_t w0, uint32_t w1, int pa
 // ------------------------------------------------------------------ shared memory map
 
 struct SmemMap {
-  int qsets;     // [NT][4 sets][4 chunks][32 lanes][4 words]
-  int qnat;      // fp32 [kMaxG][128], natural channel order, log2-domain scale
+  int qsets;     // [NT][2 sets (X, Y)][4 slice pairs][32 lanes][4 words]
+  int qnat;      // fp32 [kMaxG][128], natural channel order, unscaled
   int perm;      // 128 bytes
   int resid;     // fp32 [kMaxG][kPartialStride]: partial of the residual item
   int rrows;     // bf16 residual K rows [32][kResidKStride] then V rows [32][128]
@@ -161,7 +166,7 @@ __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
   const int nst = NT == 1 ? stages_for<1>() : stages_for<2>();
   SmemMap m;
   m.qsets = 0;
-  m.qnat = NT * 4 * 4 * 32 * 16;
+  m.qnat = NT * 2 * 4 * 32 * 16;
   m.perm = m.qnat + kMaxG * kHeadDim * 4;
   m.resid = m.perm + 128;
   m.rrows = m.resid + kMaxG * kPartialStride * 4;
@@ -187,9 +192,16 @@ struct WarpAcc {
 // NG group records at recs[0..NG) (shared memory, consecutive groups of this warp)
 // folded into the warp's state.  With NG = 2 the two groups' q.k^ chains interleave and
 // one online-softmax update covers both (64 tokens).
+// The query constants of one lane, per slice pair c (entries 2*sigma + e of the pair):
+// X = (0 | q) and Y = (q | -q) on (even | odd) B columns, fp16x2.
+template <int NT>
+struct QFrags {
+  uint4 x[NT][4], y[NT][4];
+};
+
 template <int BHI, int BLO, int NT, int NHS, int NG>
 __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
-                                               const uint32_t* qsets, WarpAcc<NT>& st) {
+                                               const QFrags<NT>& qf, float qscale, WarpAcc<NT>& st) {
   constexpr int WH = NHS * BHI / 2;   // key-code words per lane of the salient block
   constexpr int PAR = NG == 1 ? 2 : 1;   // accumulation chains per block (split by slice parity)
   const int lane = threadIdx.x & 31;
@@ -215,21 +227,11 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
         }
       }
 
-  uint4 qa4[NT], qb4[NT], qc4[NT], qz4[NT];
   uint4 s4[NG], z4[NG];
 #pragma unroll
   for (int sigma = 0; sigma < 8; ++sigma) {
     const int par = sigma & 1, pr = PAR == 2 ? par : 0;
     if (par == 0) {
-      // q sets of this slice pair: one 16-byte load per set (entries 2*sigma .. 2*sigma+3)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint4* qb = reinterpret_cast<const uint4*>(qsets) + ((nt * 4) * 4 + (sigma >> 1)) * 32 + lane;
-        qa4[nt] = qb[0];
-        qb4[nt] = qb[1 * 4 * 32];
-        qc4[nt] = qb[2 * 4 * 32];
-        qz4[nt] = qb[3 * 4 * 32];
-      }
       // key scales / zeros of this lane: fp16x2 index sigma*2 + e
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
@@ -255,16 +257,17 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
         else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
           key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, par, A);
       }
-      // ---- B fragments: q'' = q * s (hi or lo half per column) and q (for z)
+      // ---- B fragments: fp16(q s) on even columns, its rounding error on odd ones;
+      // X alone (q on odd columns) for the zero-point term
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t qa0 = par ? qa4[nt].z : qa4[nt].x, qa1 = par ? qa4[nt].w : qa4[nt].y;
-        const uint32_t qb0 = par ? qb4[nt].z : qb4[nt].x, qb1 = par ? qb4[nt].w : qb4[nt].y;
-        const uint32_t qc0 = par ? qc4[nt].z : qc4[nt].x, qc1 = par ? qc4[nt].w : qc4[nt].y;
-        const uint32_t qz0 = par ? qz4[nt].z : qz4[nt].x, qz1 = par ? qz4[nt].w : qz4[nt].y;
+        const uint4& X = qf.x[nt][sigma >> 1];
+        const uint4& Y = qf.y[nt][sigma >> 1];
+        const uint32_t qx0 = par ? X.z : X.x, qx1 = par ? X.w : X.y;
+        const uint32_t qy0 = par ? Y.z : Y.x, qy1 = par ? Y.w : Y.y;
         const uint32_t s0 = par ? s4[gi].z : s4[gi].x, s1 = par ? s4[gi].w : s4[gi].y;
-        const uint32_t b0 = hfma2(qc0, s0, hfma2(qb0, s0, hmul2(qa0, s0)));
-        const uint32_t b1 = hfma2(qc1, s1, hfma2(qb1, s1, hmul2(qa1, s1)));
+        const uint32_t b0 = hfma2(qx0, s0, hmul2(qy0, s0));
+        const uint32_t b1 = hfma2(qx1, s1, hmul2(qy1, s1));
         if (hi) {
           mma16816(acc_hi[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
           mma16816(acc_hi[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
@@ -274,12 +277,12 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
         }
         if constexpr (NG == 1) {
           const uint32_t z0 = par ? z4[0].z : z4[0].x, z1 = par ? z4[0].w : z4[0].y;
-          mma16816(dz[0][pr][nt], z0, z0, z1, z1, qz0, qz1);
+          mma16816(dz[0][pr][nt], z0, z0, z1, z1, qx0, qx1);
         } else if (gi == NG - 1) {
           // both groups' zero points in one product: rows 0-7 group 0, rows 8-15 group 1
           const uint32_t za0 = par ? z4[0].z : z4[0].x, za1 = par ? z4[0].w : z4[0].y;
           const uint32_t zb0 = par ? z4[1].z : z4[1].x, zb1 = par ? z4[1].w : z4[1].y;
-          mma16816(dz[0][pr][nt], za0, zb0, za1, zb1, qz0, qz1);
+          mma16816(dz[0][pr][nt], za0, zb0, za1, zb1, qx0, qx1);
         }
       }
     }
@@ -298,11 +301,12 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
 #pragma unroll
       for (int pr = 0; pr < PAR; ++pr)
         zb += gi == 0 ? dz[0][pr][nt][0] + dz[0][pr][nt][1] : dz[0][pr][nt][2] + dz[0][pr][nt][3];
+      zb *= qscale;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int mt = u >> 1, r = 2 * (u & 1);
-        const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23);
-        const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23);
+        const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23) * qscale;
+        const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23) * qscale;
         const float vhi = acc_hi[gi][nt][mt][r] + acc_hi[gi][nt][mt][r + 1];
         float vlo = 0.f;
 #pragma unroll
@@ -415,23 +419,25 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
       mma16816(st.bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
     }
     // value codes: words 0..7 of this lane (two 16-byte chunks).  Slot (r, p) of word m
-    // sits at bits 8r + 2p; taken from w >> (8r + 4*(p>>1)) at bit 2*(p&1), so odd token
-    // pairs carry an extra 2^2: the even-pair B columns are scaled by 4 to match.
-    const uint32_t p16x4_0 = hmul2(p16[0], four2), p16x4_2 = hmul2(p16[2], four2);
+    // sits at bits 8r + 2p; it is taken in place from w >> 8r, so token block p carries
+    // 2^(2p).  The B rows of block p are scaled by 2^(2 - 2p) to leave a uniform 2^2.
+    const uint32_t bp0 = hmul2(p16[0], four2);                 // x 4
+    const uint32_t bp2 = hmul2(p16[2], 0x34003400u);           // x 1/4
+    const uint32_t bp3 = hmul2(p16[3], 0x2C002C00u);           // x 1/16
     const uint4 vw0 = *reinterpret_cast<const uint4*>(rec + kc + 512 + lane * 16);
     const uint4 vw1 = *reinterpret_cast<const uint4*>(rec + kc + 512 + (32 + lane) * 16);
     const uint32_t vw[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int j = m >> 1;
-      const uint32_t w = vw[m], w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
+      const uint32_t w = vw[m], w8 = w >> 8;
       // (r, p) -> k-step p >> 1, register r + 2*(p & 1)
       const uint32_t k0a0 = sub_pair(w, 0x00030003u), k0a2 = sub_pair(w, 0x000C000Cu);
-      const uint32_t k1a0 = sub_pair(w4, 0x00030003u), k1a2 = sub_pair(w4, 0x000C000Cu);
+      const uint32_t k1a0 = sub_pair(w, 0x00300030u), k1a2 = sub_pair(w, 0x00C000C0u);
       const uint32_t k0a1 = sub_pair(w8, 0x00030003u), k0a3 = sub_pair(w8, 0x000C000Cu);
-      const uint32_t k1a1 = sub_pair(w12, 0x00030003u), k1a3 = sub_pair(w12, 0x000C000Cu);
-      const uint32_t b00 = hmul2(p16x4_0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
-      const uint32_t b10 = hmul2(p16x4_2, vsr[2][j]), b11 = hmul2(p16[3], vsr[3][j]);
+      const uint32_t k1a1 = sub_pair(w8, 0x00300030u), k1a3 = sub_pair(w8, 0x00C000C0u);
+      const uint32_t b00 = hmul2(bp0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
+      const uint32_t b10 = hmul2(bp2, vsr[2][j]), b11 = hmul2(bp3, vsr[3][j]);
       mma16816(st.pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
       mma16816(st.pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
     }
@@ -443,7 +449,8 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
 // row, q in natural channel order), lane = channel for the values.  Writes one partial
 // per head into `slot`.
 __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
-                                              int nr, const float* qnat, float* slot, int h0, int hstep) {
+                                              int nr, const float* qnat, float qscale, float* slot, int h0,
+                                              int hstep) {
   const int lane = threadIdx.x & 31;
   const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kResidKStride);
 #pragma unroll 1
@@ -460,7 +467,7 @@ __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t*
         lg = fmaf(qh[c8 * 8 + e], k, lg);
       }
     }
-    if (lane >= nr) lg = -INFINITY;
+    lg = lane < nr ? lg * qscale : -INFINITY;
     float m = lg;
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -527,13 +534,9 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     auto issue_upto = [&](int upto) {
       const int last = upto < my_count ? upto : my_count;
       for (; issued < last; ++issued) {
-        if (lane == 0) {
-          const uint32_t o = ord_base + issued, slot = o % kS;
-          fence_proxy_async();
-          mbar_expect_tx(bars + slot, static_cast<uint32_t>(R));
-          bulk_g2s(ring + slot * R, unit_rec + static_cast<size_t>(my_first + issued * kWarps) * R,
-                   static_cast<uint32_t>(R), bars + slot);
-        }
+        const uint32_t o = ord_base + issued, slot = o % kS;
+        stage_group(ring + slot * R, unit_rec + static_cast<size_t>(my_first + issued * kWarps) * R,
+                    static_cast<uint32_t>(R), bars + slot, lane == 0);
       }
     };
     // wait until the group of ordinal ord_base + i has landed; returns its record
@@ -546,18 +549,18 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
           if (lane == 0) atomicOr(c.error, PNMIX_DEVERR_TIMEOUT);
         }
       }
+      failed = __any_sync(0xffffffffu, failed);   // keep the warp's control flow uniform
       return ring + slot * R;
     };
     issue_upto(kS - groups_per_step<NT>());
 
-    // ---- query: log2-domain scale, natural order, then fp16 hi/lo column sets in
-    // position order
+    // ---- query: unscaled fp32 in natural channel order, then the X / Y fp16 column sets
+    // in position order
     perm[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid];
     const float qscale = g.scale * kLog2e;
     for (int i = tid; i < kMaxG * kHeadDim; i += kThreads) {
       const int hh = i / kHeadDim;
-      qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) * qscale
-                       : 0.f;
+      qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) : 0.f;
     }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     if (seg_resid) {   // residual K and V rows into shared memory, 16-byte loads
@@ -580,21 +583,18 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
         for (int i = 0; i < 4; ++i) {
           const int idx = chunk * 4 + i, sigma = idx >> 1, e = idx & 1;
           const int p0 = 16 * sigma + 8 * e + 2 * tq;
-          uint32_t sets[4][2];
+          uint32_t sets[2][2];
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
+            // bf16 -> fp16 is exact in fp16's normal range (queries are assumed < 65504)
             const float x = hh < G ? qnat[hh * kHeadDim + perm[p0 + v]] : 0.f;
-            const __half hi = __float2half_rn(x);
-            const __half lo = __float2half_rn(x - __half2float(hi));
-            const uint32_t hib = __half_as_ushort(hi), lob = __half_as_ushort(lo);
-            sets[0][v] = hl ? (hib ^ 0x8000u) : hib;   // A: -hi on a lo column, hi otherwise
-            sets[1][v] = hl ? hib : 0u;                // B
-            sets[2][v] = hl ? lob : 0u;                // C
-            sets[3][v] = hl ? lob : hib;               // q half for the zero-point term
+            const uint32_t qb = __half_as_ushort(__float2half_rn(x));
+            sets[0][v] = hl ? qb : 0u;              // X
+            sets[1][v] = hl ? (qb ^ 0x8000u) : qb;  // Y
           }
 #pragma unroll
-          for (int s = 0; s < 4; ++s)
-            qsets[(((nt * 4 + s) * 4 + chunk) * 32 + L) * 4 + i] = sets[s][0] | (sets[s][1] << 16);
+          for (int s = 0; s < 2; ++s)
+            qsets[(((nt * 2 + s) * 4 + chunk) * 32 + L) * 4 + i] = sets[s][0] | (sets[s][1] << 16);
         }
       }
     }
@@ -602,13 +602,21 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 
     // ---- the residual item (CUDA cores): warp w takes heads w, w + 4
     if (seg_resid) {
-      residual_partial(g, rrk, rrv, seg.nr, qnat, rslot, warp, kWarps);
+      residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, warp, kWarps);
     } else if (warp == 0 && lane < G) {
       rslot[lane * kPartialStride + 0] = -INFINITY;
       rslot[lane * kPartialStride + 1] = 0.f;
     }
 
-    // ---- the warp's groups
+    // ---- the warp's groups; the query constants stay in registers for the segment
+    QFrags<NT> qf;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) {
+        qf.x[nt][cp] = reinterpret_cast<const uint4*>(qsets)[((nt * 2 + 0) * 4 + cp) * 32 + lane];
+        qf.y[nt][cp] = reinterpret_cast<const uint4*>(qsets)[((nt * 2 + 1) * 4 + cp) * 32 + lane];
+      }
     WarpAcc<NT> st;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -627,16 +635,14 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       for (; i + 1 < my_count; i += 2) {
         issue_upto(i + kS);
         const uint8_t* const recs[2] = {acquire(i), acquire(i + 1)};
-        __syncwarp();
-        if (!failed) process_groups<BHI, BLO, NT, NHS, 2>(g, recs, qsets, st);
+        if (!failed) process_groups<BHI, BLO, NT, NHS, 2>(g, recs, qf, qscale, st);
         __syncwarp();
       }
     }
     for (; i < my_count; ++i) {
       issue_upto(i + kS);
       const uint8_t* const recs[1] = {acquire(i)};
-      __syncwarp();
-      if (!failed) process_groups<BHI, BLO, NT, NHS, 1>(g, recs, qsets, st);
+      if (!failed) process_groups<BHI, BLO, NT, NHS, 1>(g, recs, qf, qscale, st);
       __syncwarp();
     }
     if (failed) {   // let copies still in flight land before the shared memory is reused
@@ -725,20 +731,35 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
   });
 }
 
+// Resident CTAs of one full wave of a kernel instance, per device: the shared-memory
+// attribute and the occupancy query run once per (instance, device), not on every decode
+// step (they cost more host time than a small launch's kernel).  The record size is fixed
+// by the instance's bit widths, so the shared-memory footprint is too.
+constexpr int kMaxDevices = 64;
+
 template <int BHI, int BLO, int NT, int NHS>
 cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                          DecodeWs ws, cudaStream_t s) {
+  static std::atomic<int> wave_cache[kMaxDevices];   // 0 until known
   const SmemMap sm = smem_map(NT, g.record_bytes);
   auto kern = decode_mma_kernel<BHI, BLO, NT, NHS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm.total);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, occ = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, sm.total);
-  if (e != cudaSuccess) return e;
-  const int n = sms * (occ > 0 ? occ : 1);
-  ws.N = n < nmax ? n : nmax;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  int wave = cacheable ? wave_cache[dev].load(std::memory_order_relaxed) : 0;
+  if (wave == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm.total);
+    if (e != cudaSuccess) return e;
+    int sms = 148, occ = 1;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, sm.total);
+    if (e != cudaSuccess) return e;
+    wave = sms * (occ > 0 ? occ : 1);
+    if (cacheable) wave_cache[dev].store(wave, std::memory_order_relaxed);
+  }
+  ws.N = wave < nmax ? wave : nmax;
   kern<<<ws.N, kThreads, sm.total, s>>>(g, q, c, out, ws);
   return cudaGetLastError();
 }
