@@ -103,14 +103,29 @@ __device__ __forceinline__ QParams quant_params(float mn, float mx, int bits) {
   return q;
 }
 
-// code = clamp(rint(fl(fl(x - z) / s)), 0, 2^b - 1); 0 when s == 0.
-__device__ __forceinline__ uint32_t quant_code(float x, const QParams& q, int bits) {
-  if (q.s == 0.0f) return 0u;
-  float d = __fsub_rn(x, q.z);
-  float r = rintf(__fdiv_rn(d, q.s));
-  float levels = static_cast<float>((1 << bits) - 1);
-  r = fminf(fmaxf(r, 0.0f), levels);
-  return static_cast<uint32_t>(r);
+// The code of the reference definition, code = clamp(rint(fl(fl(x - z) / s)), 0, 2^b - 1)
+// (0 when s == 0, handled by the callers), with one multiply by the correctly rounded
+// reciprocal inv = rcp_rn(s) in place of the division.  t = fl(d * inv) differs from d / s by at most |d / s| * 2^-23
+// (two roundings of 2^-24).  Only quotients below 16 decide a code (beyond, the clamp
+// does), and there t and the rounded quotient fl(d / s) differ by less than 2^-18, so rint
+// gives the same integer for both unless t lies within that distance of a half-integer.
+// Elements with |t - rint(t)| >= 0.5 - 2^-17 take the exact division instead.  rint is
+// formed by adding and removing 1.5 * 2^23 (round-to-nearest-even in the add), whose low
+// bits are then the integer.  Needs s > 0.
+__device__ __forceinline__ uint32_t quant_code_rcp(float x, float z, float s, float inv, int levels) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  const float d = __fsub_rn(x, z);
+  const float t = __fmul_rn(d, inv);
+  const float y = __fadd_rn(t, kMagic);
+  const float r = __fsub_rn(y, kMagic);
+  int code;
+  if (fabsf(__fsub_rn(t, r)) < 0.5f - 0x1p-17f) {
+    code = __float_as_int(y) - 0x4B400000;
+  } else {
+    const float e = fminf(fmaxf(rintf(__fdiv_rn(d, s)), -1.0f), static_cast<float>(levels + 1));
+    code = static_cast<int>(e);
+  }
+  return static_cast<uint32_t>(min(max(code, 0), levels));
 }
 
 // Squared pair norm fl(fl(a*a) + fl(b*b)).

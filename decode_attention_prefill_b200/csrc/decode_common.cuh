@@ -163,5 +163,7 @@ cudaError_t launch_decode_simt(const Geometry& g, const uint16_t* q, const pnmix
                                float* out, DecodeWs ws, cudaStream_t s);
 cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                               float* out, DecodeWs ws, cudaStream_t s);
+cudaError_t launch_decode_ws(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
+                             float* out, DecodeWs ws, cudaStream_t s);
 
 }  // namespace pnmix

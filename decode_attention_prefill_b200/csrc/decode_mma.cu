@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "decode_common.cuh"
+#include "decode_frag.cuh"
 
 namespace pnmix {
 namespace {
@@ -39,115 +40,6 @@ template <int NT>
 __host__ __device__ constexpr int stages_for() { return NT == 1 ? 6 : 3; }
 template <int NT>
 __host__ __device__ constexpr int groups_per_step() { return NT == 1 ? 2 : 1; }
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kResidKStride = kHeadDim + 8;   // bf16 per staged K row (+16 B: no bank conflicts)
-
-// ------------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-// (lo, hi) fp32 -> f16x2 with lo in the low half.
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-// 2^x with the hardware approximation (MUFU.EX2, ~2 ulp; inputs here are <= 0).
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-// One staged group (a TMA bulk copy, no multicast): the issuing lane orders the warp's
-// earlier shared-memory reads of the slot before the copy's writes (fence.proxy.async),
-// arms the slot's barrier with the byte count and starts the copy.  Every lane executes
-// it; only `leader` acts (predicated, so the warp does not branch).
-__device__ __forceinline__ void stage_group(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                                            bool leader) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
-      " @p fence.proxy.async.shared::cta;\n"
-      " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %2;\n"
-      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "r"(static_cast<uint32_t>(leader))
-      : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(phase) : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-
-// try_wait rounds before a staging wait gives up (each round may suspend the warp for a
-// while); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and the kernel stops consuming.
-constexpr uint32_t kWaitLimit = 1u << 22;
-
-// Codes as fp16 subnormals.  A code pair sitting at bit offset e of both 16-bit halves of
-// a word becomes an exact fp16x2 of (code * 2^(e-24)) with one AND: the exponent field
-// stays zero.  The tensor cores take subnormal fp16 operands exactly, so the bit offset
-// only scales the product, and the kernel removes that power of two afterwards.
-__device__ __forceinline__ uint32_t sub_pair(uint32_t w, uint32_t mask) { return w & mask; }
-
-// Bit offset of token row u (0..3) of a BITS-bit key slice in the A registers below.
-template <int BITS>
-__host__ __device__ constexpr int key_row_shift(int u) {
-  return BITS == 4 ? 4 * (u & 1) : (BITS == 2 ? 2 * u : u);
-}
-
-// A fragments (2 M-tiles x 4 registers) of one key slice from its code word(s).
-//   4-bit: words w0 (c = 0), w1 (c = 1); token rows u = 0,1 in bits 0-7, rows 2,3 in 8-15.
-//   2-bit: word w; c = 0 in bits 0-7, c = 1 in bits 8-15, row u at 2u.
-//   1-bit: word w holds two slices; the slice of parity o and half c sit at 4*(2o+c), row u at u.
-template <int BITS>
-__device__ __forceinline__ void key_slice_frags(uint32_t w0, uint32_t w1, int parity, uint32_t (&A)[2][4]) {
-  if constexpr (BITS == 4) {
-    const uint32_t s0 = w0 >> 8, s1 = w1 >> 8;
-    A[0][0] = sub_pair(w0, 0x000F000Fu); A[0][1] = sub_pair(w0, 0x00F000F0u);
-    A[1][0] = sub_pair(s0, 0x000F000Fu); A[1][1] = sub_pair(s0, 0x00F000F0u);
-    A[0][2] = sub_pair(w1, 0x000F000Fu); A[0][3] = sub_pair(w1, 0x00F000F0u);
-    A[1][2] = sub_pair(s1, 0x000F000Fu); A[1][3] = sub_pair(s1, 0x00F000F0u);
-  } else if constexpr (BITS == 2) {
-    const uint32_t s = w0 >> 8;
-    A[0][0] = sub_pair(w0, 0x00030003u); A[0][1] = sub_pair(w0, 0x000C000Cu);
-    A[1][0] = sub_pair(w0, 0x00300030u); A[1][1] = sub_pair(w0, 0x00C000C0u);
-    A[0][2] = sub_pair(s, 0x00030003u);  A[0][3] = sub_pair(s, 0x000C000Cu);
-    A[1][2] = sub_pair(s, 0x00300030u);  A[1][3] = sub_pair(s, 0x00C000C0u);
-  } else {
-    const uint32_t a = parity ? (w0 >> 8) : w0;     // half c = 0
-    const uint32_t b = parity ? (w0 >> 12) : (w0 >> 4);   // half c = 1
-    A[0][0] = sub_pair(a, 0x00010001u); A[0][1] = sub_pair(a, 0x00020002u);
-    A[1][0] = sub_pair(a, 0x00040004u); A[1][1] = sub_pair(a, 0x00080008u);
-    A[0][2] = sub_pair(b, 0x00010001u); A[0][3] = sub_pair(b, 0x00020002u);
-    A[1][2] = sub_pair(b, 0x00040004u); A[1][3] = sub_pair(b, 0x00080008u);
-  }
-}
-
 // ------------------------------------------------------------------ shared memory map
 
 struct SmemMap {
@@ -192,12 +84,6 @@ struct WarpAcc {
 // NG group records at recs[0..NG) (shared memory, consecutive groups of this warp)
 // folded into the warp's state.  With NG = 2 the two groups' q.k^ chains interleave and
 // one online-softmax update covers both (64 tokens).
-// The query constants of one lane, per slice pair c (entries 2*sigma + e of the pair):
-// X = (0 | q) and Y = (q | -q) on (even | odd) B columns, fp16x2.
-template <int NT>
-struct QFrags {
-  uint4 x[NT][4], y[NT][4];
-};
 
 template <int BHI, int BLO, int NT, int NHS, int NG>
 __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
@@ -441,54 +327,6 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
       mma16816(st.pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
       mma16816(st.pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
     }
-  }
-}
-
-// The residual item: up to 31 bf16 tokens staged in shared memory, with CUDA cores, heads
-// h0, h0 + hstep, ... one at a time (few registers).  Lane = token for the logit (its K
-// row, q in natural channel order), lane = channel for the values.  Writes one partial
-// per head into `slot`.
-__device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
-                                              int nr, const float* qnat, float qscale, float* slot, int h0,
-                                              int hstep) {
-  const int lane = threadIdx.x & 31;
-  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kResidKStride);
-#pragma unroll 1
-  for (int hh = h0; hh < g.G; hh += hstep) {
-    const float* qh = qnat + hh * kHeadDim;
-    float lg = 0.f;
-#pragma unroll 4
-    for (int c8 = 0; c8 < 16; ++c8) {
-      const uint4 kv = row[c8];
-      const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float k = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-        lg = fmaf(qh[c8 * 8 + e], k, lg);
-      }
-    }
-    lg = lane < nr ? lg * qscale : -INFINITY;
-    float m = lg;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float pw = lane < nr ? exp2f(lg - m) : 0.f;
-    float l = pw;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int t = 0; t < nr; ++t) {
-      const float pt = __shfl_sync(0xffffffffu, pw, t);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(pt, bf16_bits_to_float(rv[t * kHeadDim + lane + 32 * i]), acc[i]);
-    }
-    float* s = slot + hh * kPartialStride;
-    if (lane == 0) {
-      s[0] = m;
-      s[1] = l;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s[2 + lane + 32 * i] = acc[i];
   }
 }
 
@@ -741,6 +579,7 @@ template <int BHI, int BLO, int NT, int NHS>
 cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                          DecodeWs ws, cudaStream_t s) {
   static std::atomic<int> wave_cache[kMaxDevices];   // 0 until known
+  if (g.record_bytes != record_bytes_of<BHI, BLO, NHS>()) return cudaErrorInvalidValue;
   const SmemMap sm = smem_map(NT, g.record_bytes);
   auto kern = decode_mma_kernel<BHI, BLO, NT, NHS>;
   int dev = 0;

@@ -91,14 +91,18 @@ static pnmix_status check_cache(const Geometry& g, const pnmix_cache* c) {
   return PNMIX_OK;
 }
 
-// Which decode kernel runs: the tensor-core kernel (default) or, with the environment
-// variable PNMIX_DECODE_KERNEL=simt, the CUDA-core kernel (kept for A/B measurement).
+// Which decode kernel runs.  By default the single-role tensor-core kernel
+// (decode_mma.cu) for up to 4 query heads per KV head and the warp-specialized one
+// (decode_ws.cu) above, the faster of the two on the measured workloads.  The environment
+// variable PNMIX_DECODE_KERNEL = mma | ws | simt forces one (read at every call, so tests
+// can run each kernel on every shape; simt is the CUDA-core baseline).
 int decode_kernel_choice() {
-  static const int choice = [] {
-    const char* v = getenv("PNMIX_DECODE_KERNEL");
-    return (v && strcmp(v, "simt") == 0) ? 1 : 0;
-  }();
-  return choice;
+  const char* v = getenv("PNMIX_DECODE_KERNEL");
+  if (!v) return 0;
+  if (strcmp(v, "simt") == 0) return 1;
+  if (strcmp(v, "mma") == 0) return 2;
+  if (strcmp(v, "ws") == 0) return 3;
+  return 0;
 }
 
 size_t decode_workspace_bytes(const Geometry& g, int max_context) {
@@ -115,8 +119,13 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   w.part = static_cast<float*>(ws);
   w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(nmax + units, g.G));
   w.N = nmax;
-  if (decode_kernel_choice() == 1) return launch_decode_simt(g, q, c, nmax, out, w, s);
-  return launch_decode_mma(g, q, c, nmax, out, w, s);
+  switch (decode_kernel_choice()) {
+    case 1: return launch_decode_simt(g, q, c, nmax, out, w, s);
+    case 2: return launch_decode_mma(g, q, c, nmax, out, w, s);
+    case 3: return launch_decode_ws(g, q, c, nmax, out, w, s);
+    default:   // measured: single-role kernel for up to 4 heads per KV head, pairs above
+      return g.G <= 4 ? launch_decode_mma(g, q, c, nmax, out, w, s) : launch_decode_ws(g, q, c, nmax, out, w, s);
+  }
 }
 
 }  // namespace pnmix

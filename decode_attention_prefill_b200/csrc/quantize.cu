@@ -21,7 +21,7 @@ constexpr int kTileStride = kHeadDim + 8;   // bf16 elements per shared row (+16
 
 struct GroupSmem {
   uint16_t tile[kGroup][kTileStride];
-  uint8_t codes[kGroup][kHeadDim];
+  uint32_t vcodes[kGroup][8];   // value codes of token t, channels 16i .. 16i+15 in word i
   uint8_t perm[kHeadDim];
 };
 
@@ -34,58 +34,89 @@ __device__ __forceinline__ void load_tile(GroupSmem& sm, const uint16_t* src, si
   }
 }
 
-// Keys of the staged group -> key part of `rec`.
+// Keys of the staged group -> key part of `rec`.  Thread j owns position j (channel
+// perm[j]) and its 32 tokens.  Its codes go to the words of the 8 lanes gq (tokens
+// gq + 8u, u = 0..3, in consecutive slots of one word); the positions sharing a word
+// (the two halves, and the two 8-position blocks c of a slice at 2 bits, or also the two
+// slices at 1 bit) are 1, 8 and 16 threads apart, so the words are completed with warp
+// shuffles and every word is stored once, by one of the threads that hold it.
 __device__ void quantize_key_group(const Geometry& g, GroupSmem& sm, uint8_t* rec) {
-  const int j = threadIdx.x;   // position
-  {
-    const int ch = sm.perm[j];
-    const int bits = j < g.nhi ? g.bhi : g.blo;
-    float mn = bf16_bits_to_float(sm.tile[0][ch]), mx = mn;
-#pragma unroll 8
-    for (int t = 1; t < kGroup; ++t) {
-      float x = bf16_bits_to_float(sm.tile[t][ch]);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
-    }
-    QParams q = quant_params(mn, mx, bits);
-#pragma unroll 8
-    for (int t = 0; t < kGroup; ++t)
-      sm.codes[t][j] = static_cast<uint8_t>(quant_code(bf16_bits_to_float(sm.tile[t][ch]), q, bits));
-    uint16_t* ks = reinterpret_cast<uint16_t*>(rec + rec_kscale(g));
-    uint16_t* kz = reinterpret_cast<uint16_t*>(rec + rec_kzero(g));
-    ks[kscale_index(j)] = q.s16;
-    kz[kscale_index(j)] = q.z16;
+  const int j = threadIdx.x;
+  const int ch = sm.perm[j];
+  const bool hi = j < g.nhi;
+  const int bits = hi ? g.bhi : g.blo;
+  const int levels = (1 << bits) - 1;
+  float x[kGroup];
+#pragma unroll
+  for (int t = 0; t < kGroup; ++t) x[t] = bf16_bits_to_float(sm.tile[t][ch]);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int t = 1; t < kGroup; ++t) {
+    mn = fminf(mn, x[t]);
+    mx = fmaxf(mx, x[t]);
   }
-  __syncthreads();
-  // pack: word (w, L) for every lane L and lane-local word w
-  const int words = (g.wh + g.wl) * 32;
+  const QParams q = quant_params(mn, mx, bits);
+  uint16_t* ks = reinterpret_cast<uint16_t*>(rec + rec_kscale(g));
+  uint16_t* kz = reinterpret_cast<uint16_t*>(rec + rec_kzero(g));
+  ks[kscale_index(j)] = q.s16;
+  kz[kscale_index(j)] = q.z16;
+
+  // slot of (token gq + 8u) in this position's word: n = 8 * slice + 4 * c + u
+  const int sigma = j >> 4, rem = j & 15, cc = rem >> 3, tq = (rem & 7) >> 1, half = rem & 1;
+  const int sl = hi ? sigma : sigma - g.nhs;
+  const int m = 16 / bits;
+  const int n0 = sl * 8 + cc * 4;
+  const int w = (hi ? 0 : g.wh) + n0 / m;
+  const int shift0 = 16 * half + bits * (n0 % m);
+  uint32_t pw[8];
+  if (q.s == 0.0f) {
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) pw[gq] = 0u;
+  } else {
+    const float inv = __frcp_rn(q.s);
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        word |= quant_code_rcp(x[gq + 8 * u], q.z, q.s, inv, levels) << (shift0 + bits * u);
+      pw[gq] = word;
+    }
+  }
+  const bool join8 = bits <= 2, join16 = bits == 1;
+  const bool any8 = __any_sync(0xffffffffu, join8), any16 = __any_sync(0xffffffffu, join16);
+#pragma unroll
+  for (int gq = 0; gq < 8; ++gq) pw[gq] |= __shfl_xor_sync(0xffffffffu, pw[gq], 1);
+  if (any8) {
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, pw[gq], 8);
+      if (join8) pw[gq] |= o;
+    }
+  }
+  if (any16) {
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, pw[gq], 16);
+      if (join16) pw[gq] |= o;
+    }
+  }
+  // holders of a word: 2 (4-bit), 4 (2-bit) or 8 (1-bit) threads; holder `rank` stores
+  // the words of the lanes gq = rank (mod holders)
+  const int holders = bits == 4 ? 2 : (bits == 2 ? 4 : 8);
+  const int rank = half + (bits <= 2 ? 2 * cc : 0) + (bits == 1 ? 4 * (sl & 1) : 0);
   uint32_t* kw = reinterpret_cast<uint32_t*>(rec);
-  for (int i = threadIdx.x; i < words; i += kThreads) {
-    const int w = i >> 5, L = i & 31;
-    const int gq = L >> 2, tq = L & 3;
-    const bool hi = w < g.wh;
-    const int bits = hi ? g.bhi : g.blo;
-    const int m = 16 / bits;
-    const int wl = hi ? w : w - g.wh;
-    const int sigma0 = hi ? 0 : g.nhs;
-    uint32_t word = 0;
-    for (int r = 0; r < m; ++r) {
-      const int n = wl * m + r;
-      const int sigma = sigma0 + (n >> 3), cc = (n >> 2) & 1, u = n & 3;
-      const int p0 = 16 * sigma + 2 * tq + 8 * cc;
-      const int tau = gq + 8 * u;
-      word |= static_cast<uint32_t>(sm.codes[tau][p0]) << (bits * r);
-      word |= static_cast<uint32_t>(sm.codes[tau][p0 + 1]) << (16 + bits * r);
-    }
-    kw[i] = word;
-  }
+#pragma unroll
+  for (int gq = 0; gq < 8; ++gq)
+    if ((gq & (holders - 1)) == rank) kw[w * 32 + gq * 4 + tq] = pw[gq];
 }
 
-// Values of the staged group -> value part of `rec`.
+// Values of the staged group -> value part of `rec`.  Thread (t, jg) quantizes token t
+// over channels 32 jg .. 32 jg + 31 and keeps the 2-bit codes as two 16-channel words;
+// then every thread assembles two record words from those.
 __device__ void quantize_value_group(const Geometry& g, GroupSmem& sm, uint8_t* rec) {
   {
     const int t = threadIdx.x >> 2, jg = threadIdx.x & 3;
-    // the thread's 32 channels with four 16-byte loads
     float x[32];
     const uint4* row = reinterpret_cast<const uint4*>(&sm.tile[t][32 * jg]);
 #pragma unroll
@@ -104,37 +135,36 @@ __device__ void quantize_value_group(const Geometry& g, GroupSmem& sm, uint8_t* 
       mn = fminf(mn, x[i]);
       mx = fmaxf(mx, x[i]);
     }
-    QParams q = quant_params(mn, mx, g.bv);
-    uint32_t packed[8];
+    const QParams q = quant_params(mn, mx, g.bv);
+    const int levels = (1 << g.bv) - 1;
+    uint32_t cw[2] = {0u, 0u};
+    if (q.s != 0.0f) {
+      const float inv = __frcp_rn(q.s);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t wv = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) wv |= quant_code(x[4 * k + e], q, g.bv) << (8 * e);
-      packed[k] = wv;
+      for (int i = 0; i < 32; ++i) cw[i >> 4] |= quant_code_rcp(x[i], q.z, q.s, inv, levels) << (2 * (i & 15));
     }
-    uint4* crow = reinterpret_cast<uint4*>(&sm.codes[t][32 * jg]);
-    crow[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    crow[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    sm.vcodes[t][2 * jg] = cw[0];
+    sm.vcodes[t][2 * jg + 1] = cw[1];
     uint16_t* vs = reinterpret_cast<uint16_t*>(rec + rec_vscale(g));
     uint16_t* vz = reinterpret_cast<uint16_t*>(rec + rec_vzero(g));
     vs[vscale_index(t, jg)] = q.s16;
     vz[vscale_index(t, jg)] = q.z16;
   }
   __syncthreads();
+  // word (m, L): slot q = 4r + p holds channel 16m + gq + 8r of tokens 2tq + 8p (+1)
   uint8_t* vc = rec + rec_vcode(g);
   for (int i = threadIdx.x; i < 8 * 32; i += kThreads) {
     const int m = i >> 5, L = i & 31;
     const int gq = L >> 2, tq = L & 3;
     uint32_t word = 0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int r = q >> 2, p = q & 3;
-      const int ch = 16 * m + gq + 8 * r;
-      const int t0 = 2 * tq + 8 * p;
-      word |= static_cast<uint32_t>(sm.codes[t0][ch]) << (2 * q);
-      word |= static_cast<uint32_t>(sm.codes[t0 + 1][ch]) << (16 + 2 * q);
-    }
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t v = sm.vcodes[2 * tq + 8 * p + hf][m] >> (2 * gq);
+        word |= (v & 3u) << (2 * p + 16 * hf);
+        word |= ((v >> 16) & 3u) << (2 * (4 + p) + 16 * hf);
+      }
     *reinterpret_cast<uint32_t*>(vc + vword_offset(m, L)) = word;
   }
 }

@@ -18,7 +18,7 @@ def test_tiny_workload_end_to_end():
     assert_close(got, want)
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", [
+SHAPES = [
     (1, 1, 1, 1, 8, 4, 2),
     (1, 4, 1, 31, 8, 4, 2),
     (2, 8, 2, 32, 8, 4, 2),
@@ -30,12 +30,39 @@ def test_tiny_workload_end_to_end():
     (2, 4, 4, 300, 32, 4, 2),
     (1, 8, 1, 64, 0, 2, 1),
     (4, 32, 8, 1000, 8, 4, 2),
-])
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", SHAPES)
 def test_prefill_and_decode_shapes(B, Hq, Hkv, L, k, bhi, blo):
     c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + k)
     c.prefill()
     got, want = c.attend(c.query(L))
     assert_close(got, want)
+
+
+# The library routes decode to one of two tensor-core kernels by the number of query heads
+# per KV head; each one is forced here on every shape (the variable is read per call).
+@pytest.mark.parametrize("kernel", ["mma", "ws"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", SHAPES)
+def test_each_decode_kernel_on_every_shape(kernel, B, Hq, Hkv, L, k, bhi, blo, monkeypatch):
+    monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + k + 1)
+    c.prefill()
+    got, want = c.attend(c.query(L))
+    assert_close(got, want)
+
+
+@pytest.mark.parametrize("kernel", ["mma", "ws"])
+def test_each_decode_kernel_over_a_long_append_stream(kernel, monkeypatch):
+    monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+    c = Case(2, 14, 2, 3000, extra_tokens=70, seed=11)
+    c.prefill()
+    for t in range(3000, 3070):
+        c.append(t)
+        if t in (3007, 3039, 3069):
+            got, want = c.attend(c.query(t))
+            assert_close(got, want)
 
 
 def test_append_stream_crosses_flush_boundaries():
@@ -128,3 +155,40 @@ def test_context_hint_smaller_than_the_cache_still_covers_every_token():
         out = torch.empty(4, 16, 128, dtype=torch.float32, device="cuda")
         pm.pnmix_decode_attention(c.cfg, to_dev(q), c.cache, out, workspace=ws, max_context=mc)
         assert_close(out.cpu().numpy(), c.ocache.attend(q))
+
+
+def _bf16(a):
+    u = np.asarray(a, dtype=np.float32).view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0)
+    return (u >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("bhi,blo,k", [(4, 2, 8), (2, 1, 16)])
+def test_quantizer_ties_are_bit_exact(bhi, blo, k):
+    """Every key channel and value group spans [0, 2^b - 1] with scale 1 and zero 0, and the
+    other entries sit on half-integers: each of those quotients is an exact tie, which the
+    GPU must round half-to-even like the oracle (the kernels divide by a reciprocal and fall
+    back to the IEEE quotient near ties)."""
+    rng = np.random.default_rng(7 + k)
+    L = 96
+    c = Case(1, 4, 1, L, k, bhi, blo, seed=5)
+    kf = rng.integers(0, 2 * 15 + 1, (L, 128)).astype(np.float32) / 2       # 0, 0.5, ..., 15
+    vf = rng.integers(0, 2 * 3 + 1, (L, 128)).astype(np.float32) / 2        # 0, 0.5, ..., 3
+    for g in range(L // 32):
+        kf[32 * g] = 0.0
+        vf[32 * g: 32 * g + 32, ::32] = 0.0
+        vf[32 * g: 32 * g + 32, 1::32] = 3.0
+    # key channels of lo precision (2 or 1 bits) get the range [0, 2^b_lo - 1]; the
+    # saliency pass decides which channels are hi, so use a range every channel shares:
+    # scale (max - min) / (2^b - 1) is a power of two for both widths when max = 2^b - 1
+    lo_levels = (1 << blo) - 1
+    kf = np.minimum(kf, lo_levels)
+    for g in range(L // 32):
+        kf[32 * g + 1] = lo_levels
+    c.kin = _bf16(kf)[None, None].copy()
+    c.vin = _bf16(vf)[None, None].copy()
+    c.k_dev = to_dev(c.kin)
+    c.v_dev = to_dev(c.vin)
+    c.prefill()          # checks records, scales, zeros and residual bit-exactly
+    got, want = c.attend(c.query(L))
+    assert_close(got, want)
