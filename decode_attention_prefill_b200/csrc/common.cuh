@@ -27,6 +27,7 @@ struct Geometry {
   int capacity;   // tokens per sequence
   int gcap;       // records per (b, h) = capacity / 32
   float scale;    // softmax scale
+  int score;      // saliency statistic, PNMIX_SCORE_*
 };
 
 // Record part offsets.
@@ -150,8 +151,13 @@ __host__ __device__ __forceinline__ size_t scratch_select_ticket_offset(int B, i
 __host__ __device__ __forceinline__ size_t scratch_append_ticket_offset(int B, int Hkv) {
   return static_cast<size_t>(B) * Hkv * 65;
 }
-__host__ __device__ __forceinline__ size_t scratch_words(int B, int Hkv) {
+// per unit, ordered-key images of the channel minima [128] then maxima [128] (the
+// range statistic of pnmix_select_pairs)
+__host__ __device__ __forceinline__ size_t scratch_range_offset(int B, int Hkv) {
   return static_cast<size_t>(B) * Hkv * 65 + B;
+}
+__host__ __device__ __forceinline__ size_t scratch_words(int B, int Hkv) {
+  return static_cast<size_t>(B) * Hkv * (65 + 256) + B;
 }
 
 // Launchers (one translation unit each).

@@ -28,6 +28,8 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   const int nhs = 2 * k / 16;
   if ((nhs * cfg->key_bits_hi) % 2 || ((8 - nhs) * cfg->key_bits_lo) % 2) return PNMIX_ERR_UNSUPPORTED;
   if (cfg->saliency_window < 1 || cfg->saliency_window > 1024) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->saliency_score < PNMIX_SCORE_PNMIX || cfg->saliency_score > PNMIX_SCORE_RANGE_QUERY)
+    return PNMIX_ERR_UNSUPPORTED;
   g->B = batch;
   g->Hq = cfg->n_q_heads;
   g->Hkv = cfg->n_kv_heads;
@@ -45,6 +47,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->capacity = capacity;
   g->gcap = capacity / kGroup;
   g->scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale : 1.0f / sqrtf(128.0f);
+  g->score = cfg->saliency_score;
   return PNMIX_OK;
 }
 

@@ -6,10 +6,12 @@
 //   every CTA reduces max_t (k_{t,p}^2 + k_{t,p+64}^2) over its token slice with 16-byte
 //   loads and merges it into a per-unit scratch array with atomicMax on the float bits
 //   (non-negative floats order like their bit patterns, and max is order-free, so the
-//   split is exact);
+//   split is exact); for the range statistic it also reduces every channel's min and max
+//   (atomicMin / atomicMax on an order-preserving integer image of the float);
 //   the last CTA of a unit (atomic ticket, no waiting) forms the query pair norms of the
 //   G x W window, sums them sequentially in the reference order (heads outer, tokens
-//   inner), builds the scores and selects the top k with warp shuffles.
+//   inner), builds the scores of the configured statistic and selects the top k with
+//   warp shuffles.
 #include "common.cuh"
 
 namespace pnmix {
@@ -19,19 +21,42 @@ constexpr int kThreads = 256;
 constexpr int kRowsPerIter = kThreads / 8;   // 8 threads per 128-channel row
 
 // Pair norms of 8 consecutive pairs p = 8*c .. 8*c+7 of one row, from the two 16-byte
-// chunks (channels 8c..8c+7 and 64+8c..64+8c+7).
-__device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float out[8]) {
+// chunks (channels 8c..8c+7 and 64+8c..64+8c+7); with RANGE also the 16 channel values.
+template <bool RANGE = false>
+__device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float out[8],
+                                               float* mn = nullptr, float* mx = nullptr) {
   uint4 lo = __ldg(reinterpret_cast<const uint4*>(row) + c);
   uint4 hi = __ldg(reinterpret_cast<const uint4*>(row) + 8 + c);
   const uint16_t* a = reinterpret_cast<const uint16_t*>(&lo);
   const uint16_t* b = reinterpret_cast<const uint16_t*>(&hi);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = pair_norm2(bf16_bits_to_float(a[i]), bf16_bits_to_float(b[i]));
+  for (int i = 0; i < 8; ++i) {
+    const float x = bf16_bits_to_float(a[i]), y = bf16_bits_to_float(b[i]);
+    out[i] = pair_norm2(x, y);
+    if constexpr (RANGE) {
+      mn[i] = fminf(mn[i], x);
+      mx[i] = fmaxf(mx[i], x);
+      mn[8 + i] = fminf(mn[8 + i], y);
+      mx[8 + i] = fmaxf(mx[8 + i], y);
+    }
+  }
 }
 
+// Order-preserving map of non-NaN floats to unsigned integers (and back), so that
+// integer atomics compute float min / max.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ordered_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+template <int SCORE>
 __global__ void __launch_bounds__(kThreads)
 select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_window,
                     const uint16_t* __restrict__ k, int L, int ld, pnmix_cache c) {
+  constexpr bool RANGE = SCORE == PNMIX_SCORE_RANGE_QUERY;
   const int unit = blockIdx.y;
   const int b = unit / g.Hkv, h = unit % g.Hkv;
   const int nsplit = gridDim.x, split = blockIdx.x;
@@ -42,21 +67,32 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
   __shared__ float red[kThreads / 32][64];
   __shared__ float qn[kRowsPerIter][64];
   __shared__ float score_s[64];
+  __shared__ float rmin[RANGE ? kThreads / 32 : 1][128], rmax[RANGE ? kThreads / 32 : 1][128];
   __shared__ int is_last;
 
   uint32_t* kmax = c.scratch + scratch_kmax_offset() + static_cast<size_t>(unit) * 64;
   uint32_t* ticket = c.scratch + scratch_select_ticket_offset(g.B, g.Hkv) + unit;
+  uint32_t* cmin = c.scratch + scratch_range_offset(g.B, g.Hkv) + static_cast<size_t>(unit) * 256;
+  uint32_t* cmax = cmin + 128;
 
-  // ---- key pair-norm max over this split's tokens
+  // ---- key pair-norm max (and channel min / max) over this split's tokens
   const int t0 = static_cast<int>(static_cast<long long>(L) * split / nsplit);
   const int t1 = static_cast<int>(static_cast<long long>(L) * (split + 1) / nsplit);
   const uint16_t* kbase = k + unit_index(g, b, h) * static_cast<size_t>(ld) * kHeadDim;
   float m8[8];
+  float mn16[RANGE ? 16 : 1], mx16[RANGE ? 16 : 1];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m8[i] = 0.0f;
+  if constexpr (RANGE) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      mn16[i] = INFINITY;
+      mx16[i] = -INFINITY;
+    }
+  }
   for (int t = t0 + rsub; t < t1; t += kRowsPerIter) {
     float n2[8];
-    row_pair_norm2(kbase + static_cast<size_t>(t) * kHeadDim, cidx, n2);
+    row_pair_norm2<RANGE>(kbase + static_cast<size_t>(t) * kHeadDim, cidx, n2, mn16, mx16);
 #pragma unroll
     for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], n2[i]);
   }
@@ -65,6 +101,24 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
   for (int i = 0; i < 8; ++i) {
     m8[i] = fmaxf(m8[i], __shfl_xor_sync(0xffffffffu, m8[i], 8));
     m8[i] = fmaxf(m8[i], __shfl_xor_sync(0xffffffffu, m8[i], 16));
+  }
+  if constexpr (RANGE) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      mn16[i] = fminf(mn16[i], __shfl_xor_sync(0xffffffffu, mn16[i], 8));
+      mn16[i] = fminf(mn16[i], __shfl_xor_sync(0xffffffffu, mn16[i], 16));
+      mx16[i] = fmaxf(mx16[i], __shfl_xor_sync(0xffffffffu, mx16[i], 8));
+      mx16[i] = fmaxf(mx16[i], __shfl_xor_sync(0xffffffffu, mx16[i], 16));
+    }
+    if (lane < 8) {   // channels 8*lane + i and 64 + 8*lane + i
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        rmin[warp][8 * lane + i] = mn16[i];
+        rmax[warp][8 * lane + i] = mx16[i];
+        rmin[warp][64 + 8 * lane + i] = mn16[8 + i];
+        rmax[warp][64 + 8 * lane + i] = mx16[8 + i];
+      }
+    }
   }
   if (lane < 8) {
 #pragma unroll
@@ -75,6 +129,17 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
     float v = 0.0f;
     for (int w = 0; w < kThreads / 32; ++w) v = fmaxf(v, red[w][tid]);
     atomicMax(kmax + tid, __float_as_uint(v));
+  }
+  if constexpr (RANGE) {
+    if (tid < 128 && t1 > t0) {
+      float lo = INFINITY, hi = -INFINITY;
+      for (int w = 0; w < kThreads / 32; ++w) {
+        lo = fminf(lo, rmin[w][tid]);
+        hi = fmaxf(hi, rmax[w][tid]);
+      }
+      atomicMin(cmin + tid, ordered_key(lo));
+      atomicMax(cmax + tid, ordered_key(hi));
+    }
   }
   __threadfence();
   __syncthreads();
@@ -107,7 +172,16 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
   if (tid < 64) {
     float kp = __fsqrt_rn(__uint_as_float(__ldcg(kmax + tid)));
     float qp = __fdiv_rn(qsum, static_cast<float>(rows));
-    float s = __fmul_rn(qp, kp);
+    float s;
+    if constexpr (SCORE == PNMIX_SCORE_KEY_ONLY) {
+      s = kp;
+    } else if constexpr (RANGE) {
+      const float r0 = __fsub_rn(ordered_value(__ldcg(cmax + tid)), ordered_value(__ldcg(cmin + tid)));
+      const float r1 = __fsub_rn(ordered_value(__ldcg(cmax + 64 + tid)), ordered_value(__ldcg(cmin + 64 + tid)));
+      s = __fmul_rn(qp, __fsqrt_rn(__fadd_rn(__fmul_rn(r0, r0), __fmul_rn(r1, r1))));
+    } else {
+      s = __fmul_rn(qp, kp);
+    }
     score_s[tid] = s;
     c.pair_scores[static_cast<size_t>(unit) * 64 + tid] = s;
   }
@@ -153,9 +227,17 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
                                 const uint16_t* k, int L, int ld, const pnmix_cache& c,
                                 cudaStream_t s) {
   const int units = g.B * g.Hkv;
-  // scratch (max-norm accumulators and tickets) starts at zero for every call
+  // scratch (max-norm accumulators and tickets) starts at zero for every call; the range
+  // statistic's channel minima start at the largest key, maxima at the smallest
   cudaError_t e = cudaMemsetAsync(c.scratch, 0, sizeof(uint32_t) * static_cast<size_t>(units) * 65, s);
   if (e != cudaSuccess) return e;
+  if (g.score == PNMIX_SCORE_RANGE_QUERY) {
+    uint32_t* cm = c.scratch + scratch_range_offset(g.B, g.Hkv);
+    e = cudaMemset2DAsync(cm, 1024, 0xFF, 512, units, s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset2DAsync(cm + 128, 1024, 0x00, 512, units, s);
+    if (e != cudaSuccess) return e;
+  }
   // about eight CTAs per SM so the max pass balances, with >= 128 tokens per CTA
   int want = (8 * 148 + units - 1) / units;
   int max_split = (L + 127) / 128;
@@ -163,7 +245,16 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
   if (nsplit < 1) nsplit = 1;
   if (nsplit > 512) nsplit = 512;
   dim3 grid(nsplit, units);
-  select_pairs_kernel<<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
+  switch (g.score) {
+    case PNMIX_SCORE_KEY_ONLY:
+      select_pairs_kernel<PNMIX_SCORE_KEY_ONLY><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
+      break;
+    case PNMIX_SCORE_RANGE_QUERY:
+      select_pairs_kernel<PNMIX_SCORE_RANGE_QUERY><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
+      break;
+    default:
+      select_pairs_kernel<PNMIX_SCORE_PNMIX><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
+  }
   return cudaGetLastError();
 }
 

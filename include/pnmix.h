@@ -143,7 +143,8 @@ typedef enum {
  *   n_salient_pairs k in {0, 8, 16, 32, 64} with WH and WL (see the layout) whole
  *     numbers, i.e. every k for (4,2) and k in {0, 16, 32, 64} for (2,1);
  *   G = n_q_heads / n_kv_heads in [1, 8];
- *   saliency_window W in [1, 1024].
+ *   saliency_window W in [1, 1024];
+ *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*).
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
  */
 typedef struct {
@@ -159,7 +160,25 @@ typedef struct {
   int32_t value_group;
   int32_t saliency_window;
   float softmax_scale;
+  int32_t saliency_score;   /* statistic that ranks the pairs, PNMIX_SCORE_* (0 = PN-Mix) */
 } pnmix_config;
+
+/*
+ * Pair statistics pnmix_select_pairs can rank by (all per (b, kv head), fp32, one
+ * rounding per operation; K_p and Q_p as defined at pnmix_select_pairs):
+ *   PNMIX_SCORE_PNMIX        s_p = Q_p * K_p, the PN-Mix pair-norm product (default).
+ *   PNMIX_SCORE_KEY_ONLY     s_p = K_p: key statistics alone, the channel-saliency
+ *                            estimate of the earlier mixed-precision methods that the
+ *                            PN-Mix abstract compares against.
+ *   PNMIX_SCORE_RANGE_QUERY  s_p = Q_p * sqrt(r_p^2 + r_{p+64}^2), r_c = max_t k - min_t k
+ *                            of channel c over the L rows: quantization difficulty (the
+ *                            range the min-max code must span) times query relevance, the
+ *                            two factors named by the MixKVQ abstract.  The page gives no
+ *                            formula; this is its plainest pair-level reading.
+ */
+#define PNMIX_SCORE_PNMIX 0
+#define PNMIX_SCORE_KEY_ONLY 1
+#define PNMIX_SCORE_RANGE_QUERY 2
 
 /* Device pointers into one caller-owned buffer; filled by pnmix_cache_init. */
 typedef struct {
@@ -175,7 +194,7 @@ typedef struct {
   uint64_t* pair_mask;       /* [B][Hkv] */
   uint8_t* perm;             /* [B][Hkv][128] */
   float* pair_scores;        /* [B][Hkv][64] */
-  uint32_t* scratch;         /* library-internal counters; zero between calls */
+  uint32_t* scratch;         /* library-internal counters and reduction space */
   uint32_t* error;           /* device error word */
   void* base;
   size_t total_bytes;
@@ -206,9 +225,11 @@ PNMIX_API pnmix_status pnmix_cache_reset(const pnmix_cache* cache, void* stream)
 /*
  * Prefill step 1 (PN-Mix abstract: salient pairs are picked once at prefill from
  * the query-key pair-norm product).  For every (b, kv head h):
- *   K_p from the first L rows of k, Q_p from the n_window rows of q_window of the
- *   G query heads h*G .. h*G+G-1, s_p = Q_p * K_p; the k = n_salient_pairs pairs
- *   with the largest s_p (ties to the lower p) become salient.
+ *   K_p = sqrt(max over the first L rows of k of k_p^2 + k_{p+64}^2), Q_p = the mean
+ *   over the n_window rows of q_window of the G query heads h*G .. h*G+G-1 of
+ *   sqrt(q_p^2 + q_{p+64}^2) (heads outer, rows inner), s_p = Q_p * K_p (or the
+ *   statistic cfg->saliency_score names); the k = n_salient_pairs pairs with the
+ *   largest s_p (ties to the lower p) become salient.
  * q_window: bf16 [B][Hq][n_window][128] -- the LAST n_window prefill queries, after RoPE.
  * k:        bf16 [B][Hkv][ld_tokens][128], rows [0, L) used, after RoPE.
  * n_window must equal min(L, saliency_window); 1 <= L <= ld_tokens.

@@ -57,6 +57,7 @@ def lib():
                 "orc_f32_from_f16": (f, [ctypes.c_uint16]),
                 "orc_f16_from_f32": (ctypes.c_uint16, [f]),
                 "orc_pair_scores": (None, [i, i, i, vp, vp, vp, vp, vp]),
+                "orc_pair_scores_mode": (None, [i, i, i, i, vp, vp, vp]),
                 "orc_topk": (None, [vp, i, vp, vp]),
                 "orc_position_order": (i, [ctypes.c_uint64, vp]),
                 "orc_minmax_quant": (None, [vp, i, i, vp, vp, vp]),
@@ -114,6 +115,19 @@ def pair_scores(qwin: np.ndarray, k: np.ndarray):
     return s, kn, qn
 
 
+SCORE_PNMIX, SCORE_KEY_ONLY, SCORE_RANGE_QUERY = 0, 1, 2
+
+
+def pair_scores_mode(mode: int, qwin: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """Scores fp32 [64] under statistic `mode` (SCORE_*), see orc_pair_scores_mode."""
+    qwin = np.ascontiguousarray(qwin, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    G, W, _ = qwin.shape
+    s = np.zeros(64, np.float32)
+    lib().orc_pair_scores_mode(mode, G, W, k.shape[0], _p(qwin), _p(k), _p(s))
+    return s
+
+
 def topk(scores: np.ndarray, k: int):
     """-> (idx uint8 [k] ascending, mask int)."""
     scores = np.ascontiguousarray(scores, dtype=np.float32)
@@ -129,9 +143,9 @@ def position_order(mask: int):
     return perm, nhi
 
 
-def select_unit(qwin: np.ndarray, k: np.ndarray, n_salient: int):
+def select_unit(qwin: np.ndarray, k: np.ndarray, n_salient: int, mode: int = SCORE_PNMIX):
     """Full step 1 of one (b, KV head): scores, idx, mask, perm."""
-    s, _, _ = pair_scores(qwin, k)
+    s = pair_scores(qwin, k)[0] if mode == SCORE_PNMIX else pair_scores_mode(mode, qwin, k)
     idx, mask = topk(s, n_salient)
     perm, _ = position_order(mask)
     return s, idx, mask, perm
@@ -210,9 +224,10 @@ def unpack_record(k, bhi, blo, rec):
 class Cache:
     """Host image of the cache regions the tests compare with the device."""
 
-    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2):
+    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2, score=SCORE_PNMIX):
         self.batch, self.n_kv, self.capacity = batch, n_kv, capacity
         self.k, self.bhi, self.blo, self.bv = k, bhi, blo, bv
+        self.score = score
         self.R = record_bytes(k, bhi, blo)
         if not self.R:
             raise ValueError("unsupported bit point")
@@ -229,7 +244,7 @@ class Cache:
         """qwin bf16 [B][Hq][W][128]; kin bf16 [B][Hkv][>=L][128]."""
         G = qwin.shape[1] // self.n_kv
         for b, h in units or [(b, h) for b in range(self.batch) for h in range(self.n_kv)]:
-            s, idx, mask, perm = select_unit(qwin[b, h * G:(h + 1) * G], kin[b, h, :L], self.k)
+            s, idx, mask, perm = select_unit(qwin[b, h * G:(h + 1) * G], kin[b, h, :L], self.k, self.score)
             self.scores[b, h] = s
             self.idx[b, h, :self.k] = idx
             self.mask[b, h] = mask

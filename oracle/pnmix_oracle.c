@@ -144,6 +144,46 @@ void orc_pair_scores(int G, int W, int L, const uint16_t* qwin, const uint16_t* 
 }
 
 /*
+ * Saliency scores under the three statistics the path supports (mode):
+ *   0  PN-Mix: s_p = Q_p * K_p as in orc_pair_scores (query pair norm times key pair
+ *      norm; PN-Mix abstract).
+ *   1  key statistics only: s_p = K_p (the channel-saliency estimate of the earlier
+ *      mixed-precision methods that the PN-Mix abstract contrasts with).
+ *   2  quantization difficulty times query relevance (the MixKVQ abstract's two factors):
+ *      D_p = sqrt(r_p*r_p + r_{p+64}*r_{p+64}) with r_c = max_t k[t][c] - min_t k[t][c],
+ *      the pair norm of the two channels' ranges; s_p = Q_p * D_p.
+ * Every operation is one fp32 rounding, in the order written.
+ */
+void orc_pair_scores_mode(int mode, int G, int W, int L, const uint16_t* qwin, const uint16_t* k,
+                          float* scores) {
+  float s0[64], kn[64], qn[64];
+  orc_pair_scores(G, W, L, qwin, k, s0, kn, qn);
+  for (int p = 0; p < 64; ++p) {
+    if (mode == 0) {
+      scores[p] = s0[p];
+    } else if (mode == 1) {
+      scores[p] = kn[p];
+    } else {
+      float r[2];
+      for (int e = 0; e < 2; ++e) {
+        const int c = p + 64 * e;
+        float mn = orc_f32_from_bf16(k[c]), mx = mn;
+        for (int t = 1; t < L; ++t) {
+          const float x = orc_f32_from_bf16(k[(size_t)t * 128 + c]);
+          if (x < mn) mn = x;
+          if (x > mx) mx = x;
+        }
+        r[e] = mx - mn;
+      }
+      const float r0 = r[0] * r[0];
+      const float r1 = r[1] * r[1];
+      const float d = sqrtf(r0 + r1);
+      scores[p] = qn[p] * d;
+    }
+  }
+}
+
+/*
  * The k pairs with the largest score; among equal scores the lower pair index
  * wins.  idx receives them in ascending pair order, mask has bit p set for
  * every chosen p.

@@ -49,6 +49,8 @@ def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
     (dict(n_q_heads=30, n_kv_heads=4), pm.ERR_INVALID_ARG),   # not a multiple
     (dict(value_bits=4), pm.ERR_UNSUPPORTED),
     (dict(saliency_window=0), pm.ERR_UNSUPPORTED),
+    (dict(saliency_score=3), pm.ERR_UNSUPPORTED),
+    (dict(saliency_score=-1), pm.ERR_UNSUPPORTED),
 ])
 def test_config_validation(change, status):
     cfg = pm.Config.make(32, 8)

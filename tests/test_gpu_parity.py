@@ -192,3 +192,19 @@ def test_quantizer_ties_are_bit_exact(bhi, blo, k):
     c.prefill()          # checks records, scales, zeros and residual bit-exactly
     got, want = c.attend(c.query(L))
     assert_close(got, want)
+
+
+@pytest.mark.parametrize("score", [1, 2])
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", [
+    (1, 4, 1, 1, 8, 4, 2),
+    (2, 8, 2, 517, 16, 4, 2),
+    (3, 28, 4, 2049, 32, 2, 1),
+    (2, 32, 8, 4000, 8, 4, 2),
+])
+def test_saliency_statistics_select_like_the_oracle(score, B, Hq, Hkv, L, k, bhi, blo):
+    """Key-only (1) and key-range x query (2) statistics: scores bit-exact (so the same
+    pairs, permutation and records) and the decode over the resulting cache."""
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + score, score=score)
+    c.prefill()
+    got, want = c.attend(c.query(L))
+    assert_close(got, want)

@@ -139,6 +139,97 @@ def test_topk_matches_exact_brute_force_with_ties(seed):
         assert mask == sum(1 << p for p in want)
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_key_only_score_is_the_exact_key_pair_norm_and_ignores_queries(seed):
+    """Key-only statistic on Pythagorean integer keys: K_p is an exact integer (the
+    largest hypotenuse over the tokens); two unrelated query windows give the same scores."""
+    rng = np.random.default_rng(40 + seed)
+    G, W, L = 2, 3, 5
+    kint = np.zeros((L, 128), np.int64)
+    for p in range(64):
+        for t in range(L):
+            a, b = PYTH[rng.integers(0, len(PYTH))]
+            kint[t, p], kint[t, p + 64] = a * rng.choice([-1, 1]), b * rng.choice([-1, 1])
+    want = [max(math.isqrt(int(a) ** 2 + int(b) ** 2) for a, b in zip(kint[:, p], kint[:, p + 64]))
+            for p in range(64)]
+    kb = bf16_bits(kint.astype(np.float32))
+    q1 = bf16_bits(rng.integers(-8, 9, (G, W, 128)).astype(np.float32))
+    q2 = bf16_bits(rng.integers(-8, 9, (G, W, 128)).astype(np.float32))
+    s1 = oracle.pair_scores_mode(oracle.SCORE_KEY_ONLY, q1, kb)
+    s2 = oracle.pair_scores_mode(oracle.SCORE_KEY_ONLY, q2, kb)
+    np.testing.assert_array_equal(s1, np.array(want, np.float32))
+    np.testing.assert_array_equal(s1, s2)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_range_score_on_pythagorean_ranges(seed):
+    """Range statistic: channel ranges (max - min over tokens) form Pythagorean pairs per
+    RoPE pair and the query pair norms are exact, so s_p = Q_p * hypot(r_p, r_{p+64}) is
+    an exact small rational; the key pair norms play no part."""
+    rng = np.random.default_rng(60 + seed)
+    G, W, L = 2, 2, 6    # G*W = 4: the query mean is exact in binary32
+    kint = np.zeros((L, 128), np.int64)
+    qint = np.zeros((G, W, 128), np.int64)
+    want = []
+    for p in range(64):
+        ra, rb = PYTH[rng.integers(0, len(PYTH))]
+        for c, r in ((p, ra), (p + 64, rb)):
+            lo = int(rng.integers(-20, 20))
+            col = lo + rng.integers(0, r + 1, L)
+            i_lo, i_hi = rng.choice(L, 2, replace=False)
+            col[i_lo], col[i_hi] = lo, lo + r
+            if r == 0:
+                col[:] = lo
+            kint[:, c] = col
+        qs = 0
+        for h in range(G):
+            for t in range(W):
+                a, b = PYTH[rng.integers(0, len(PYTH))]
+                qint[h, t, p], qint[h, t, p + 64] = a, -b
+                qs += math.isqrt(a * a + b * b)
+        want.append(Fraction(qs, G * W) * math.isqrt(ra * ra + rb * rb))
+    got = oracle.pair_scores_mode(oracle.SCORE_RANGE_QUERY, bf16_bits(qint.astype(np.float32)),
+                                  bf16_bits(kint.astype(np.float32)))
+    np.testing.assert_array_equal(got.astype(np.float64), [float(w) for w in want])
+
+
+def test_range_score_ignores_a_channel_shift_that_moves_the_pnmix_score():
+    """Adding a constant to a key channel leaves its range, hence the range statistic,
+    unchanged, while the pair-norm product (which sees the magnitude) changes."""
+    rng = np.random.default_rng(3)
+    kf = rng.integers(-4, 5, (40, 128)).astype(np.float32)
+    qb = bf16_bits(rng.integers(-4, 5, (3, 8, 128)).astype(np.float32))
+    shifted = kf.copy()
+    shifted[:, 5] += 16.0
+    shifted[:, 64 + 9] -= 32.0
+    a = oracle.pair_scores_mode(oracle.SCORE_RANGE_QUERY, qb, bf16_bits(kf))
+    b = oracle.pair_scores_mode(oracle.SCORE_RANGE_QUERY, qb, bf16_bits(shifted))
+    np.testing.assert_array_equal(a, b)
+    p0 = oracle.pair_scores_mode(oracle.SCORE_PNMIX, qb, bf16_bits(kf))
+    p1 = oracle.pair_scores_mode(oracle.SCORE_PNMIX, qb, bf16_bits(shifted))
+    assert p1[5] > p0[5] and p1[9] > p0[9]
+    np.testing.assert_array_equal(p0, oracle.pair_scores(qb, bf16_bits(kf))[0])
+
+
+def test_key_only_selection_misses_the_query_outlier_pairs():
+    """On the tiny workload the planted x4 query pairs rank only by the query factor, so
+    the key-only statistic leaves them out of its top 8 while the pair-norm product keeps
+    them (the difference the PN-Mix abstract draws between the two estimates)."""
+    L, W = 512, 64
+    k = workload.rows(0, workload.K, 1, 1, 0, L)[0, 0]
+    qwin = workload.rows(0, workload.Q, 1, 1, L - W, W)[0]
+    qpairs = set(workload.outlier_pairs(0, True, 0, 0))
+    kpairs = set(workload.outlier_pairs(0, False, 0, 0))
+    sel = {}
+    for mode in (oracle.SCORE_PNMIX, oracle.SCORE_KEY_ONLY):
+        s = oracle.pair_scores_mode(mode, qwin, k)
+        idx, _ = oracle.topk(s, 8)
+        sel[mode] = set(int(i) for i in idx)
+    assert kpairs <= sel[oracle.SCORE_PNMIX] and (qpairs - kpairs) <= sel[oracle.SCORE_PNMIX]
+    assert kpairs <= sel[oracle.SCORE_KEY_ONLY]
+    assert not (qpairs - kpairs) <= sel[oracle.SCORE_KEY_ONLY]
+
+
 def test_topk_all_equal_scores_take_lowest_pairs():
     idx, mask = oracle.topk(np.full(64, 3.0, np.float32), 8)
     assert list(idx) == list(range(8)) and mask == 0xFF
