@@ -59,11 +59,12 @@ def parse():
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="stream_32k",
-                    choices=["stream_32k", "llama3_8b", "sweep_128k", "pipeline_32l"],
+                    choices=["stream_32k", "llama3_8b", "sweep_128k", "pipeline_32l", "verify_32k"],
                     help="stream_32k is the benchmark line; the others print per-workload "
                          "measurements (decode GB/s and tokens/s; for the sweep the relative L2 "
                          "error against unquantized bf16 attention; for the 32-layer pipeline the "
-                         "prefill latencies and the extrapolated end-to-end tokens/s)")
+                         "prefill latencies and the extrapolated end-to-end tokens/s; verify_32k: "
+                         "two new tokens per sequence attended at once at 32K)")
     ap.add_argument("--pipeline-layers-generated", type=int, default=4,
                     help="pipeline_32l: layers whose prefill inputs are generated (seed + layer); "
                          "the others reuse them cyclically")
@@ -191,7 +192,7 @@ def gen_inputs(seed: int, T_total: int, q_positions: list[int]):
     vin = workload.rows(seed, workload.V, B, HKV, 0, T_total)
     qwin = workload.rows(seed, workload.Q, B, HQ, PREFILL - WINDOW, WINDOW, group=HQ // HKV)
     qs = np.stack([workload.rows(seed, workload.Q, B, HQ, p, 1, group=HQ // HKV)[:, :, 0]
-                   for p in q_positions])
+                   for p in q_positions]) if q_positions else None
     return kin, vin, qwin, qs
 
 
@@ -376,6 +377,65 @@ def run_decode_workload(args):
     return 0
 
 
+def run_verify(args):
+    """verify_32k: the stream_32k shape (16 x 32/8 heads, 32768 tokens) with T = 2 new
+    tokens per sequence attended at once (pnmix_decode_attention_multi after two appends),
+    against one single-query decode of the same cache.  The 419 MB cache exceeds L2."""
+    import torch
+
+    import decode_attention_prefill_b200 as pm
+    T = 2
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n0 = CONTEXT - T
+    kin, vin, qwin, _ = gen_inputs(args.seed, CONTEXT, [])
+    qm = workload_rows_q(args.seed, CONTEXT - T, T)                      # [B][T][Hq][128]
+    cfg = pm.Config.make(HQ, HKV, BHI, BLO, K_SALIENT, WINDOW)
+    cache = pm.PNMixCache(cfg, B, CONTEXT + 32, max_context=CONTEXT, max_queries=T)
+    k_dev = torch.from_numpy(kin).view(torch.bfloat16).to(dev)
+    v_dev = torch.from_numpy(vin).view(torch.bfloat16).to(dev)
+    pm.pnmix_select_pairs(cfg, torch.from_numpy(qwin).view(torch.bfloat16).to(dev), k_dev, PREFILL, cache)
+    pm.pnmix_quantize_keys(cfg, k_dev, n0, cache)
+    pm.pnmix_quantize_values(cfg, v_dev, n0, cache)
+    for t in range(n0, CONTEXT):
+        pm.pnmix_append(cfg, k_dev[:, :, t].contiguous(), v_dev[:, :, t].contiguous(), cache)
+    del k_dev, v_dev
+    q_dev = torch.from_numpy(qm).view(torch.bfloat16).to(dev)
+    out_m = torch.empty(B, T, HQ, D, dtype=torch.float32, device=dev)
+    out_1 = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
+    q1 = q_dev[:, T - 1].contiguous()
+    with ClockSampler(0) as clocks:
+        t_multi = timed_rotation([lambda: pm.pnmix_decode_attention_multi(cfg, q_dev, cache, out_m)],
+                                 args.steps, args.warmup)
+        t_single = timed_rotation([lambda: pm.pnmix_decode_attention(cfg, q1, cache, out_1)],
+                                  args.steps, args.warmup)
+    assert cache.read_error() == 0
+    G = HQ // HKV
+    rec = cache.c.record_bytes
+    alg_m = decode_bytes(CONTEXT, B * HKV, G * T, rec)
+    alg_1 = decode_bytes(CONTEXT, B * HKV, G, rec)
+    peak, peak_kind = measured_peaks()
+    line = {"workload": "verify_32k", "metric": "multi-token decode attention at 32K", "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic", "dtype": "f32",
+            "config": {"batch": B, "n_q_heads": HQ, "n_kv_heads": HKV, "context": CONTEXT,
+                       "queries_per_sequence": T, "key_code_bits": 2.25,
+                       "l2": "inputs larger than L2 (419 MB cache per launch)"},
+            "multi": {"decode_us": t_multi * 1e6, "tokens_per_s": B * T / t_multi,
+                      "decode_gbs": alg_m / t_multi / 1e9, "frac": alg_m / t_multi / 1e9 / peak},
+            "single": {"decode_us": t_single * 1e6, "tokens_per_s": B / t_single,
+                       "decode_gbs": alg_1 / t_single / 1e9, "frac": alg_1 / t_single / 1e9 / peak},
+            "peak": peak, "peak_source": peak_kind, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_rows_q(seed: int, pos0: int, n: int) -> np.ndarray:
+    """Queries of positions pos0 .. pos0+n-1 of the bench workload: bf16 [B][n][Hq][128]."""
+    import workload
+    q = workload.rows(seed, workload.Q, B, HQ, pos0, n, group=HQ // HKV)
+    return np.ascontiguousarray(q.transpose(0, 2, 1, 3))
+
+
 def run_pipeline(args):
     """pipeline_32l: 32 layers, batch 32, 32/8 heads.  Per layer a 4096-token prefill
     (saliency + quantize), then decode steps (append + attend in every layer) to 32768.
@@ -484,6 +544,8 @@ def main():
         return run_reference(args, world, rank)
     if args.workload == "pipeline_32l":
         return run_pipeline(args)
+    if args.workload == "verify_32k":
+        return run_verify(args)
     if args.workload != "stream_32k":
         return run_decode_workload(args)
 

@@ -39,6 +39,7 @@ EXPORTED = [
     "pnmix_select_pairs", "pnmix_quantize_keys", "pnmix_quantize_values", "pnmix_append",
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
+    "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi",
 ]
 
 
@@ -88,6 +89,8 @@ _SIGS = {
     "pnmix_status_string": (ctypes.c_char_p, [_i]),
     "pnmix_version": (ctypes.c_char_p, []),
     "pnmix_decode_attention_noalloc": (_i, [_CP, _vp, _KP, _i, _vp, _vp]),
+    "pnmix_workspace_bytes_multi": (_sz, [_CP, _i, _i, _i]),
+    "pnmix_decode_attention_multi": (_i, [_CP, _vp, _i, _KP, _i, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -180,13 +183,29 @@ def pnmix_decode_attention(cfg: Config, q: torch.Tensor, cache: "PNMixCache", ou
                                        _stream(stream)), "pnmix_decode_attention")
 
 
+def workspace_bytes_multi(cfg: Config, batch: int, max_context: int, n_queries: int) -> int:
+    return int(_lib.pnmix_workspace_bytes_multi(ctypes.byref(cfg), batch, max_context, n_queries))
+
+
+def pnmix_decode_attention_multi(cfg: Config, q: torch.Tensor, cache: "PNMixCache", out: torch.Tensor,
+                                 workspace: torch.Tensor | None = None, max_context: int | None = None,
+                                 stream=None):
+    """q bf16 [B][T][Hq][128] -> out fp32 [B][T][Hq][128]; query j over the first len - T + 1 + j tokens."""
+    ws = cache.workspace if workspace is None else workspace
+    mc = cache.max_context if max_context is None else max_context
+    _check(_lib.pnmix_decode_attention_multi(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q"), q.shape[1],
+                                             ctypes.byref(cache.c), mc, _dev(out, torch.float32, "out"),
+                                             _dev(ws, torch.uint8, "workspace"), ws.numel(),
+                                             _stream(stream)), "pnmix_decode_attention_multi")
+
+
 # ---------------------------------------------------------------- owner of device buffers
 
 class PNMixCache:
     """Cache + decode workspace of one layer, allocated with torch on `device`."""
 
     def __init__(self, cfg: Config, batch: int, capacity_tokens: int, device="cuda",
-                 max_context: int | None = None, stream=None):
+                 max_context: int | None = None, stream=None, max_queries: int = 1):
         self.cfg = cfg
         self.batch = batch
         self.capacity = capacity_tokens
@@ -198,7 +217,8 @@ class PNMixCache:
         _check(_lib.pnmix_cache_init(ctypes.byref(cfg), batch, capacity_tokens, ctypes.c_void_p(base),
                                      nbytes, ctypes.byref(self.c)), "pnmix_cache_init")
         self._base_off = base - self.buffer.data_ptr()
-        ws = workspace_bytes(cfg, batch, self.max_context)
+        ws = max(workspace_bytes(cfg, batch, self.max_context),
+                 workspace_bytes_multi(cfg, batch, self.max_context, max_queries) if max_queries > 1 else 0)
         self.workspace = torch.zeros(ws + 256, dtype=torch.uint8, device=device)
         # 256-byte aligned view
         off = (-self.workspace.data_ptr()) % 256
@@ -257,6 +277,13 @@ class PNMixCache:
 
     def append(self, k_new, v_new, stream=None):
         pnmix_append(self.cfg, k_new, v_new, self, stream)
+
+    def attend_multi(self, q, out=None, stream=None) -> torch.Tensor:
+        """q bf16 [B][T][Hq][128] of T tokens already appended -> fp32 [B][T][Hq][128]."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        pnmix_decode_attention_multi(self.cfg, q, self, out, stream=stream)
+        return out
 
     def attend(self, q, out=None, stream=None) -> torch.Tensor:
         if out is None:

@@ -28,6 +28,8 @@ struct Geometry {
   int gcap;       // records per (b, h) = capacity / 32
   float scale;    // softmax scale
   int score;      // saliency statistic, PNMIX_SCORE_*
+  int tq;         // decode queries per sequence (1, or T of a multi-query step)
+  int rows;       // query rows per (b, KV head) in decode: G * tq (row v = query v / G, head v % G)
 };
 
 // Record part offsets.

@@ -97,10 +97,23 @@ __device__ __forceinline__ float* partial_slot(const DecodeWs& ws, int unit, int
   return ws.part + static_cast<size_t>(blockIdx.x + unit) * G * kPartialStride;
 }
 
-// Called by every thread of the CTA after the segment's partials are in its slot.
-// out_unit points at out[b][h*G][0] (G rows of 128 floats).
+// Query row v of unit (b, h) is query v / G of sequence b, head h*G + v % G; q and out
+// are [B][tq][Hq][128] (tq = 1: [B][Hq][128]).
+__device__ __forceinline__ size_t row_offset(const Geometry& g, int b, int h, int v) {
+  const int j = v / g.G, hg = v - j * g.G;
+  return ((static_cast<size_t>(b) * g.tq + j) * g.Hq + h * g.G + hg) * kHeadDim;
+}
+
+// Tokens visible to query row v: a multi-query step appended its tq tokens before
+// attending, and query j sees the cache up to its own token (len - tq + 1 + j).
+__device__ __forceinline__ int visible_tokens(const Geometry& g, int len, int v) {
+  return len - g.tq + 1 + v / g.G;
+}
+
+// Called by every thread of the CTA after the segment's partials are in its slot: the
+// CTA that takes the unit's last ticket writes the unit's G = g.rows output rows.
 __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G,
-                                                float* out_unit) {
+                                                float* out, const Geometry& geo) {
   __shared__ int is_last;
   __threadfence();
   __syncthreads();
@@ -134,14 +147,14 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
       __syncthreads();
       for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
         const int hh = i / kHeadDim, c = i % kHeadDim;
-        float num = chunk == 0 ? 0.f : out_unit[static_cast<size_t>(hh) * kHeadDim + c];
+        float* out_row = out + row_offset(geo, s.b, s.h, hh);
+        float num = chunk == 0 ? 0.f : out_row[c];
 #pragma unroll 4
         for (unsigned k = 0; k < n; ++k)
           num = fmaf(__ldcg(base + (static_cast<size_t>(chunk + k) * G + hh) * kPartialStride + 2 + c),
                      wsh[hh][k], num);
         const bool last_chunk = chunk + n == nseg;
-        out_unit[static_cast<size_t>(hh) * kHeadDim + c] =
-            last_chunk ? (den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f) : num;
+        out_row[c] = last_chunk ? (den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f) : num;
       }
       __syncthreads();
     }

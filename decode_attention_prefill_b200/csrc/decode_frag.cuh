@@ -144,11 +144,13 @@ struct QFrags {
 // per head into `slot`.
 __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
                                               int nr, const float* qnat, float qscale, float* slot, int h0,
-                                              int hstep) {
+                                              int hstep, int tok0, int vis_base) {
   const int lane = threadIdx.x & 31;
   const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kResidKStride);
 #pragma unroll 1
-  for (int hh = h0; hh < g.G; hh += hstep) {
+  for (int hh = h0; hh < g.rows; hh += hstep) {
+    // residual row `lane` is token tok0 + lane; row hh sees tokens below vis_base + hh / G
+    const bool vis = lane < nr && tok0 + lane < vis_base + hh / g.G;
     const float* qh = qnat + hh * kHeadDim;
     float lg = 0.f;
 #pragma unroll 4
@@ -161,11 +163,11 @@ __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t*
         lg = fmaf(qh[c8 * 8 + e], k, lg);
       }
     }
-    lg = lane < nr ? lg * qscale : -INFINITY;
+    lg = vis ? lg * qscale : -INFINITY;
     float m = lg;
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float pw = lane < nr ? exp2f(lg - m) : 0.f;
+    const float pw = vis ? exp2f(lg - m) : 0.f;   // (m = -inf only when no token is visible)
     float l = pw;
 #pragma unroll
     for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);

@@ -85,13 +85,16 @@ struct WarpAcc {
 // folded into the warp's state.  With NG = 2 the two groups' q.k^ chains interleave and
 // one online-softmax update covers both (64 tokens).
 
-template <int BHI, int BLO, int NT, int NHS, int NG>
-__device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
-                                               const QFrags<NT>& qf, float qscale, WarpAcc<NT>& st) {
+// Key side of NG group records: the log2-domain logits lg[gi][nt][u] of head 4*nt + tq at
+// tokens gq + 8u of group gi.
+template <int BHI, int BLO, int NT, int NHS, int NG, bool MQ>
+__device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* const (&recs)[NG],
+                                             const QFrags<NT>& qf, float qscale, const int (&tok0)[NG],
+                                             int vis_base, float (&lg)[NG][NT][4]) {
   constexpr int WH = NHS * BHI / 2;   // key-code words per lane of the salient block
   constexpr int PAR = NG == 1 ? 2 : 1;   // accumulation chains per block (split by slice parity)
   const int lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq = lane & 3;
+  const int tq = lane & 3;
   const int kc = g.kc_bytes;
 
   // key-code products, kept apart per block because the two blocks' token-row bit
@@ -176,7 +179,6 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
 
   // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3;
   // the product of a row-u token carries 2^(shift(u) - 24)
-  float lg[NG][NT][4];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
@@ -200,6 +202,34 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
         lg[gi][nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
       }
     }
+
+  // ---- multi-query steps: row v sees tokens below vis_base + v / G (only the newest
+  // tokens of a unit can be hidden, so only a group reaching them takes this branch)
+  if constexpr (MQ) {
+    const int gq = lane >> 2;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      if (tok0[gi] + kGroup > vis_base) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int lim = vis_base + (4 * nt + tq) / g.G;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (tok0[gi] + gq + 8 * u >= lim) lg[gi][nt][u] = -INFINITY;
+        }
+      }
+    }
+  }
+}
+
+// Value side of NG group records with their logits: online softmax update, P as B
+// fragments, P x V into the warp's accumulators.
+template <int NT, int NG>
+__device__ __forceinline__ void group_softmax_values(const Geometry& g, const uint8_t* const (&recs)[NG],
+                                                     const float (&lg)[NG][NT][4], WarpAcc<NT>& st) {
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int kc = g.kc_bytes;
 
   // ---- online softmax over the NG groups
   float mnew[NT];
@@ -248,7 +278,7 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
   }
 
   const int srcA = (2 * tq) * 4 + (gq & 3), srcB = (2 * tq + 1) * 4 + (gq & 3);
-  const bool col_ok = gq < g.G;
+  const bool col_ok = gq < g.rows;
   const uint32_t four2 = 0x44004400u;   // fp16x2 (4, 4)
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
@@ -330,12 +360,23 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
   }
 }
 
-template <int BHI, int BLO, int NT, int NHS>
+template <int BHI, int BLO, int NT, int NHS, int NG, bool MQ>
+__device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
+                                               const QFrags<NT>& qf, float qscale, const int (&tok0)[NG],
+                                               int vis_base, WarpAcc<NT>& st) {
+  float lg[NG][NT][4];
+  group_logits<BHI, BLO, NT, NHS, NG, MQ>(g, recs, qf, qscale, tok0, vis_base, lg);
+  group_softmax_values<NT, NG>(g, recs, lg, st);
+}
+
+// MQ: several queries per sequence (rows = G * tq), with the causal mask on the newest
+// tokens; a separate instance so the one-query kernel carries none of it.
+template <int BHI, int BLO, int NT, int NHS, bool MQ>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 3)
 decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
                   DecodeWs ws) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int G = g.G;
+  const int G = g.rows;   // query rows per unit
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = g.record_bytes;
   const SmemMap sm = smem_map(NT, R);
@@ -361,6 +402,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
+    const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
     // ---- this warp's groups of the segment; stage the first ones right away
     const int gend = seg.hi < seg.ng ? seg.hi : seg.ng;
     const int my_first = seg.lo + warp;
@@ -398,7 +440,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     const float qscale = g.scale * kLog2e;
     for (int i = tid; i < kMaxG * kHeadDim; i += kThreads) {
       const int hh = i / kHeadDim;
-      qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) : 0.f;
+      qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
     }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     if (seg_resid) {   // residual K and V rows into shared memory, 16-byte loads
@@ -440,7 +482,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 
     // ---- the residual item (CUDA cores): warp w takes heads w, w + 4
     if (seg_resid) {
-      residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, warp, kWarps);
+      residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, warp, kWarps, seg.ng * kGroup, vis_base);
     } else if (warp == 0 && lane < G) {
       rslot[lane * kPartialStride + 0] = -INFINITY;
       rslot[lane * kPartialStride + 1] = 0.f;
@@ -473,14 +515,16 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       for (; i + 1 < my_count; i += 2) {
         issue_upto(i + kS);
         const uint8_t* const recs[2] = {acquire(i), acquire(i + 1)};
-        if (!failed) process_groups<BHI, BLO, NT, NHS, 2>(g, recs, qf, qscale, st);
+        const int tok[2] = {(my_first + i * kWarps) * kGroup, (my_first + (i + 1) * kWarps) * kGroup};
+        if (!failed) process_groups<BHI, BLO, NT, NHS, 2, MQ>(g, recs, qf, qscale, tok, vis_base, st);
         __syncwarp();
       }
     }
     for (; i < my_count; ++i) {
       issue_upto(i + kS);
       const uint8_t* const recs[1] = {acquire(i)};
-      if (!failed) process_groups<BHI, BLO, NT, NHS, 1>(g, recs, qf, qscale, st);
+      const int tok[1] = {(my_first + i * kWarps) * kGroup};
+      if (!failed) process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, recs, qf, qscale, tok, vis_base, st);
       __syncwarp();
     }
     if (failed) {   // let copies still in flight land before the shared memory is reused
@@ -565,7 +609,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       }
       o[2 + tid] = a;
     }
-    combine_segment(ws, seg, G, out + (static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim);
+    combine_segment(ws, seg, G, out, g);
   });
 }
 
@@ -575,13 +619,13 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 // by the instance's bit widths, so the shared-memory footprint is too.
 constexpr int kMaxDevices = 64;
 
-template <int BHI, int BLO, int NT, int NHS>
+template <int BHI, int BLO, int NT, int NHS, bool MQ>
 cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                          DecodeWs ws, cudaStream_t s) {
   static std::atomic<int> wave_cache[kMaxDevices];   // 0 until known
   if (g.record_bytes != record_bytes_of<BHI, BLO, NHS>()) return cudaErrorInvalidValue;
   const SmemMap sm = smem_map(NT, g.record_bytes);
-  auto kern = decode_mma_kernel<BHI, BLO, NT, NHS>;
+  auto kern = decode_mma_kernel<BHI, BLO, NT, NHS, MQ>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -603,31 +647,38 @@ cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache
   return cudaGetLastError();
 }
 
-template <int BHI, int BLO, int NT>
+template <int BHI, int BLO, int NT, bool MQ>
 cudaError_t launch_mma_nhs(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                            DecodeWs ws, cudaStream_t s) {
   switch (g.nhs) {
-    case 0: return launch_mma_t<BHI, BLO, NT, 0>(g, q, c, nmax, out, ws, s);
-    case 2: return launch_mma_t<BHI, BLO, NT, 2>(g, q, c, nmax, out, ws, s);
-    case 4: return launch_mma_t<BHI, BLO, NT, 4>(g, q, c, nmax, out, ws, s);
-    case 8: return launch_mma_t<BHI, BLO, NT, 8>(g, q, c, nmax, out, ws, s);
+    case 0: return launch_mma_t<BHI, BLO, NT, 0, MQ>(g, q, c, nmax, out, ws, s);
+    case 2: return launch_mma_t<BHI, BLO, NT, 2, MQ>(g, q, c, nmax, out, ws, s);
+    case 4: return launch_mma_t<BHI, BLO, NT, 4, MQ>(g, q, c, nmax, out, ws, s);
+    case 8: return launch_mma_t<BHI, BLO, NT, 8, MQ>(g, q, c, nmax, out, ws, s);
     default: break;
   }
   if constexpr (BLO == 2) {   // one salient slice (k = 8) only exists with 2-bit lo words
-    if (g.nhs == 1) return launch_mma_t<BHI, BLO, NT, 1>(g, q, c, nmax, out, ws, s);
+    if (g.nhs == 1) return launch_mma_t<BHI, BLO, NT, 1, MQ>(g, q, c, nmax, out, ws, s);
   }
   return cudaErrorInvalidValue;
+}
+
+template <int BHI, int BLO, int NT>
+cudaError_t launch_mma_mq(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
+                          DecodeWs ws, cudaStream_t s) {
+  return g.tq > 1 ? launch_mma_nhs<BHI, BLO, NT, true>(g, q, c, nmax, out, ws, s)
+                  : launch_mma_nhs<BHI, BLO, NT, false>(g, q, c, nmax, out, ws, s);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                               float* out, DecodeWs ws, cudaStream_t s) {
-  const bool nt2 = g.G > 4;
+  const bool nt2 = g.rows > 4;
   if (g.bhi == 4 && g.blo == 2)
-    return nt2 ? launch_mma_nhs<4, 2, 2>(g, q, c, nmax, out, ws, s) : launch_mma_nhs<4, 2, 1>(g, q, c, nmax, out, ws, s);
+    return nt2 ? launch_mma_mq<4, 2, 2>(g, q, c, nmax, out, ws, s) : launch_mma_mq<4, 2, 1>(g, q, c, nmax, out, ws, s);
   if (g.bhi == 2 && g.blo == 1)
-    return nt2 ? launch_mma_nhs<2, 1, 2>(g, q, c, nmax, out, ws, s) : launch_mma_nhs<2, 1, 1>(g, q, c, nmax, out, ws, s);
+    return nt2 ? launch_mma_mq<2, 1, 2>(g, q, c, nmax, out, ws, s) : launch_mma_mq<2, 1, 1>(g, q, c, nmax, out, ws, s);
   return cudaErrorInvalidValue;
 }
 

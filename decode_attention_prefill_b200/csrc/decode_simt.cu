@@ -175,7 +175,7 @@ decode_simt_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, fl
       }
       p[2 + tid] = a;
     }
-    combine_segment(ws, s, G, out + (static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim);
+    combine_segment(ws, s, G, out, g);   // one query per sequence here (g.tq == 1)
   });
 }
 

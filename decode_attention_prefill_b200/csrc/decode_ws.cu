@@ -97,9 +97,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 // Logits of one group for the heads of this lane (log2 domain): lane (gq, tq) gets head
 // 4*nt + tq at tokens gq + 8u, u = 0..3.
-template <int BHI, int BLO, int NT, int NHS, bool QREG>
+template <int BHI, int BLO, int NT, int NHS, bool QREG, bool MQ>
 __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* rec, const QFrags<NT>& qf,
-                                             const uint4* qsets, float qscale, float (&lg)[NT][4]) {
+                                             const uint4* qsets, float qscale, int tok0, int vis_base,
+                                             float (&lg)[NT][4]) {
   constexpr int WH = NHS * BHI / 2;
   constexpr int kc = key_code_bytes<BHI, BLO, NHS>();
   const int lane = threadIdx.x & 31;
@@ -175,6 +176,18 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* r
       lg[nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
     }
   }
+  // multi-query steps: row v sees tokens below vis_base + v / G (only a group that
+  // reaches the newest tokens of its unit takes this branch)
+  if (MQ && tok0 + kGroup > vis_base) {
+    const int gq = lane >> 2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int lim = vis_base + (4 * nt + tq) / g.G;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (tok0 + gq + 8 * u >= lim) lg[nt][u] = -INFINITY;
+    }
+  }
 }
 
 // Value side of one group: acc (channels 16m + gq (+8), heads 2tq, 2tq+1) and the zero-point
@@ -226,7 +239,9 @@ __device__ __forceinline__ void group_values(const uint8_t* rec, const uint4& p4
   }
 }
 
-template <int BHI, int BLO, int NT, int NHS>
+// MQ: several queries per sequence (rows = G * tq) with the causal mask on the newest
+// tokens; a separate instance so the one-query kernel carries none of it.
+template <int BHI, int BLO, int NT, int NHS, bool MQ>
 __global__ void __launch_bounds__(kWsThreads, 2)
 decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
                  DecodeWs ws) {
@@ -235,7 +250,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   constexpr bool QREG = NT == 1;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int stop_flag;
-  const int G = g.G;
+  const int G = g.rows;   // query rows per unit
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool is_qk = warp < kPairs;
   const int pair = is_qk ? warp : warp - kPairs;
@@ -273,6 +288,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
+    const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
     const int gend = seg.hi < seg.ng ? seg.hi : seg.ng;
     const int my_first = seg.lo + pair;
     const int my_count = my_first < gend ? (gend - my_first + kPairs - 1) / kPairs : 0;
@@ -293,7 +309,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     const float qscale = g.scale * kLog2e;
     for (int i = tid; i < kMaxG * kHeadDim; i += kWsThreads) {
       const int hh = i / kHeadDim;
-      qnat[i] = hh < G ? bf16_bits_to_float(q[(static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim + i]) : 0.f;
+      qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
     }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     if (seg_resid) {
@@ -362,8 +378,8 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         const uint32_t o = ord_base + i;
         if (!__all_sync(0xffffffffu, ws_wait(full + o % S, (o / S) & 1, stop, c.error))) break;
         float lg[NT][4];
-        group_logits<BHI, BLO, NT, NHS, QREG>(g, ring + (o % S) * R, qf,
-                                             reinterpret_cast<const uint4*>(qsets), qscale, lg);
+        group_logits<BHI, BLO, NT, NHS, QREG, MQ>(g, ring + (o % S) * R, qf, reinterpret_cast<const uint4*>(qsets),
+                                             qscale, (my_first + i * kPairs) * kGroup, vis_base, lg);
         // lazy running max per head (4*nt + tq), over the group's 32 tokens
         bool raise = false;
         float mx[NT];
@@ -411,7 +427,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     } else {
       // ================================================================ PV warp
       if (seg_resid) {
-        residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, pair, kPairs);
+        residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, pair, kPairs, seg.ng * kGroup, vis_base);
       } else if (pair == 0 && lane < G) {
         rslot[lane * kPartialStride + 0] = -INFINITY;
         rslot[lane * kPartialStride + 1] = 0.f;
@@ -529,13 +545,13 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       }
       o[2 + ch] = a;
     }
-    combine_segment(ws, seg, G, out + (static_cast<size_t>(b) * g.Hq + h * G) * kHeadDim);
+    combine_segment(ws, seg, G, out, g);
   });
 }
 
 constexpr int kMaxDevices = 64;
 
-template <int BHI, int BLO, int NT, int NHS>
+template <int BHI, int BLO, int NT, int NHS, bool MQ>
 cudaError_t launch_ws_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                         DecodeWs ws, cudaStream_t s) {
   constexpr int R = record_bytes_of<BHI, BLO, NHS>();
@@ -544,7 +560,7 @@ cudaError_t launch_ws_t(const Geometry& g, const uint16_t* q, const pnmix_cache&
   static std::atomic<int> wave_cache[kMaxDevices];   // resident CTAs of a full wave, 0 until known
   if (g.record_bytes != R) return cudaErrorInvalidValue;
   const WsSmem sm = ws_smem(NT, R, S);
-  auto kern = decode_ws_kernel<BHI, BLO, NT, NHS>;
+  auto kern = decode_ws_kernel<BHI, BLO, NT, NHS, MQ>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -566,31 +582,38 @@ cudaError_t launch_ws_t(const Geometry& g, const uint16_t* q, const pnmix_cache&
   return cudaGetLastError();
 }
 
-template <int BHI, int BLO, int NT>
+template <int BHI, int BLO, int NT, bool MQ>
 cudaError_t launch_ws_nhs(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
                           DecodeWs ws, cudaStream_t s) {
   switch (g.nhs) {
-    case 0: return launch_ws_t<BHI, BLO, NT, 0>(g, q, c, nmax, out, ws, s);
-    case 2: return launch_ws_t<BHI, BLO, NT, 2>(g, q, c, nmax, out, ws, s);
-    case 4: return launch_ws_t<BHI, BLO, NT, 4>(g, q, c, nmax, out, ws, s);
-    case 8: return launch_ws_t<BHI, BLO, NT, 8>(g, q, c, nmax, out, ws, s);
+    case 0: return launch_ws_t<BHI, BLO, NT, 0, MQ>(g, q, c, nmax, out, ws, s);
+    case 2: return launch_ws_t<BHI, BLO, NT, 2, MQ>(g, q, c, nmax, out, ws, s);
+    case 4: return launch_ws_t<BHI, BLO, NT, 4, MQ>(g, q, c, nmax, out, ws, s);
+    case 8: return launch_ws_t<BHI, BLO, NT, 8, MQ>(g, q, c, nmax, out, ws, s);
     default: break;
   }
   if constexpr (BLO == 2) {   // one salient slice (k = 8) only exists with 2-bit lo words
-    if (g.nhs == 1) return launch_ws_t<BHI, BLO, NT, 1>(g, q, c, nmax, out, ws, s);
+    if (g.nhs == 1) return launch_ws_t<BHI, BLO, NT, 1, MQ>(g, q, c, nmax, out, ws, s);
   }
   return cudaErrorInvalidValue;
+}
+
+template <int BHI, int BLO, int NT>
+cudaError_t launch_ws_mq(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out,
+                         DecodeWs ws, cudaStream_t s) {
+  return g.tq > 1 ? launch_ws_nhs<BHI, BLO, NT, true>(g, q, c, nmax, out, ws, s)
+                  : launch_ws_nhs<BHI, BLO, NT, false>(g, q, c, nmax, out, ws, s);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_ws(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                              float* out, DecodeWs ws, cudaStream_t s) {
-  const bool nt2 = g.G > 4;
+  const bool nt2 = g.rows > 4;
   if (g.bhi == 4 && g.blo == 2)
-    return nt2 ? launch_ws_nhs<4, 2, 2>(g, q, c, nmax, out, ws, s) : launch_ws_nhs<4, 2, 1>(g, q, c, nmax, out, ws, s);
+    return nt2 ? launch_ws_mq<4, 2, 2>(g, q, c, nmax, out, ws, s) : launch_ws_mq<4, 2, 1>(g, q, c, nmax, out, ws, s);
   if (g.bhi == 2 && g.blo == 1)
-    return nt2 ? launch_ws_nhs<2, 1, 2>(g, q, c, nmax, out, ws, s) : launch_ws_nhs<2, 1, 1>(g, q, c, nmax, out, ws, s);
+    return nt2 ? launch_ws_mq<2, 1, 2>(g, q, c, nmax, out, ws, s) : launch_ws_mq<2, 1, 1>(g, q, c, nmax, out, ws, s);
   return cudaErrorInvalidValue;
 }
 

@@ -48,6 +48,8 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->gcap = capacity / kGroup;
   g->scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale : 1.0f / sqrtf(128.0f);
   g->score = cfg->saliency_score;
+  g->tq = 1;
+  g->rows = G;
   return PNMIX_OK;
 }
 
@@ -111,7 +113,7 @@ int decode_kernel_choice() {
 size_t decode_workspace_bytes(const Geometry& g, int max_context) {
   const int nmax = decode_max_ctas(g, max_context);
   const int units = g.B * g.Hkv;
-  return decode_partial_bytes(nmax + units, g.G) + align256(sizeof(uint32_t) * units);
+  return decode_partial_bytes(nmax + units, g.rows) + align256(sizeof(uint32_t) * units);
 }
 
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int max_context,
@@ -120,14 +122,14 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   const int units = g.B * g.Hkv;
   DecodeWs w;
   w.part = static_cast<float*>(ws);
-  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(nmax + units, g.G));
+  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(nmax + units, g.rows));
   w.N = nmax;
-  switch (decode_kernel_choice()) {
+  switch (g.tq > 1 && decode_kernel_choice() == 1 ? 0 : decode_kernel_choice()) {   // simt: one query
     case 1: return launch_decode_simt(g, q, c, nmax, out, w, s);
     case 2: return launch_decode_mma(g, q, c, nmax, out, w, s);
     case 3: return launch_decode_ws(g, q, c, nmax, out, w, s);
     default:   // measured: single-role kernel for up to 4 heads per KV head, pairs above
-      return g.G <= 4 ? launch_decode_mma(g, q, c, nmax, out, w, s) : launch_decode_ws(g, q, c, nmax, out, w, s);
+      return g.rows <= 4 ? launch_decode_mma(g, q, c, nmax, out, w, s) : launch_decode_ws(g, q, c, nmax, out, w, s);
   }
 }
 
@@ -263,6 +265,33 @@ pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
   if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
   if (!q || !out || !workspace || max_context < 0) return PNMIX_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
+  return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch, int max_context, int n_queries) {
+  Geometry g;
+  if (batch <= 0 || n_queries < 1 || make_geometry(cfg, batch, 32, &g) != PNMIX_OK) return 0;
+  if (g.G * n_queries > kMaxG) return 0;
+  g.tq = n_queries;
+  g.rows = g.G * n_queries;
+  return decode_workspace_bytes(g, max_context);
+}
+
+pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_t* q, int n_queries,
+                                          const pnmix_cache* cache, int max_context, float* out,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, &g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
+  if (!q || !out || !workspace || max_context < 0 || n_queries < 1) return PNMIX_ERR_INVALID_ARG;
+  if (g.G * n_queries > kMaxG) return PNMIX_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  g.tq = n_queries;
+  g.rows = g.G * n_queries;
   if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
   return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
                                    static_cast<cudaStream_t>(stream)));

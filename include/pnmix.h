@@ -20,6 +20,7 @@
  *   pnmix_quantize_values -- prefill: per-token 32-channel groups at b_v bits
  *   pnmix_append          -- decode: write one new K/V row, quantize every full 32-token group
  *   pnmix_decode_attention-- decode: split-K attention over the packed cache + bf16 residual
+ *   (pnmix_decode_attention_multi: the same for several new tokens per sequence, causal)
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -133,8 +134,8 @@ typedef enum {
 
 /* Device error word bits (pnmix_read_error). */
 #define PNMIX_DEVERR_APPEND_FULL 0x1u  /* pnmix_append found len == capacity_tokens */
-#define PNMIX_DEVERR_TIMEOUT 0x2u      /* a bounded wait for staged cache data ran out in
-                                          pnmix_decode_attention (its output is then invalid) */
+#define PNMIX_DEVERR_TIMEOUT 0x2u      /* a bounded wait for staged cache data ran out in a
+                                          decode call (its output is then invalid) */
 
 /*
  * Method parameters.  Supported set:
@@ -284,6 +285,29 @@ PNMIX_API size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int m
 PNMIX_API pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
                                     const pnmix_cache* cache, int max_context, float* out,
                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes pnmix_decode_attention_multi needs for n_queries queries per
+ * sequence (n_queries = 1 gives pnmix_workspace_bytes); 0 if unsupported.
+ */
+PNMIX_API size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch, int max_context,
+                                             int n_queries);
+
+/*
+ * Decode attention of T = n_queries new tokens per sequence at once (a speculative
+ * verify or chunked decode step), after all T of their K/V rows were appended with
+ * pnmix_append.  q: bf16 [B][T][Hq][128] (after RoPE); out: fp32 [B][T][Hq][128].
+ * Query j (0-based) of sequence b attends causally over the first len[b] - T + 1 + j
+ * cached tokens: the cache before the step plus the new tokens up to its own.  The
+ * pages have no such call; it is the multi-token neighbour of pnmix_decode_attention
+ * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 8 (PNMIX_ERR_UNSUPPORTED
+ * otherwise).  A query that sees no token gets zeros.  Workspace from
+ * pnmix_workspace_bytes_multi with the same T.
+ */
+PNMIX_API pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_t* q,
+                                                    int n_queries, const pnmix_cache* cache,
+                                                    int max_context, float* out, void* workspace,
+                                                    size_t workspace_bytes, void* stream);
 
 /*
  * pnmix_decode_attention without a caller-provided workspace.  The pages have no

@@ -58,6 +58,7 @@ def lib():
                 "orc_f16_from_f32": (ctypes.c_uint16, [f]),
                 "orc_pair_scores": (None, [i, i, i, vp, vp, vp, vp, vp]),
                 "orc_pair_scores_mode": (None, [i, i, i, i, vp, vp, vp]),
+                "orc_attend_unit_rows": (i, [i, vp, d, i, i, i, vp, vp, i, vp, vp, i, vp, vp]),
                 "orc_topk": (None, [vp, i, vp, vp]),
                 "orc_position_order": (i, [ctypes.c_uint64, vp]),
                 "orc_minmax_quant": (None, [vp, i, i, vp, vp, vp]),
@@ -288,6 +289,33 @@ class Cache:
                                    _p(self.records[b, h]), n // 32, _p(self.resid_k[b, h]),
                                    _p(self.resid_v[b, h]), n % 32, None, None, _p(out))
         assert rc == 0
+        return out
+
+    def attend_rows(self, q: np.ndarray, n_visible, b: int, h: int, scale: float | None = None) -> np.ndarray:
+        """q bf16 [rows][128] of KV head h of sequence b, row r over the first n_visible[r]
+        cached tokens -> fp64 [rows][128]."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        nv = np.ascontiguousarray(n_visible, dtype=np.int32)
+        n = int(self.len[b])
+        out = np.zeros((q.shape[0], 128), np.float64)
+        rc = lib().orc_attend_unit_rows(q.shape[0], _p(q), scale if scale else 1.0 / np.sqrt(128.0),
+                                        self.k, self.bhi, self.blo, _p(self.perm[b, h]),
+                                        _p(self.records[b, h]), n // 32, _p(self.resid_k[b, h]),
+                                        _p(self.resid_v[b, h]), n % 32, _p(nv), _p(out))
+        assert rc == 0
+        return out
+
+    def attend_multi(self, q: np.ndarray, heads=None) -> np.ndarray:
+        """T new queries per sequence after their T tokens were appended: q bf16
+        [B][T][Hq][128] -> fp64 [B][T][Hq][128], query j over the first len - T + 1 + j
+        tokens (only the listed (b, kv head) units)."""
+        B, T, Hq, _ = q.shape
+        G = Hq // self.n_kv
+        out = np.full((B, T, Hq, 128), np.nan)
+        for b, h in heads or [(b, h) for b in range(B) for h in range(self.n_kv)]:
+            rows = np.ascontiguousarray(q[b, :, h * G:(h + 1) * G].reshape(T * G, 128))
+            nv = [int(self.len[b]) - T + 1 + j for j in range(T) for _ in range(G)]
+            out[b, :, h * G:(h + 1) * G] = self.attend_rows(rows, nv, b, h).reshape(T, G, 128)
         return out
 
     def attend(self, q: np.ndarray, heads=None) -> np.ndarray:

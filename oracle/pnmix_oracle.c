@@ -608,6 +608,52 @@ int orc_attend_unit(int G, const uint16_t* q, double scale, int k, int bhi, int 
   return 0;
 }
 
+/*
+ * Several query rows per (b, KV head), each over its own prefix of the cache: row r
+ * (bf16 q[r][128]) attends over the first n_visible[r] of the n_groups*32 + n_resid
+ * tokens (the cache dequantized as in orc_attend_unit).  A verify or chunked decode step
+ * appends T new tokens first; its query j then sees len - T + 1 + j tokens (causal among
+ * the new ones).  A row that sees no token gets zeros.
+ */
+int orc_attend_unit_rows(int rows, const uint16_t* q, double scale, int k, int bhi, int blo,
+                         const uint8_t* perm, const uint8_t* records, int n_groups,
+                         const uint16_t* resid_k, const uint16_t* resid_v, int n_resid,
+                         const int* n_visible, double* out) {
+  long R = orc_record_bytes(k, bhi, blo);
+  if (!R) return 1;
+  long n = (long)n_groups * 32 + n_resid;
+  double* khat = (double*)malloc(sizeof(double) * 128 * (size_t)(n > 0 ? n : 1));
+  double* vhat = (double*)malloc(sizeof(double) * 128 * (size_t)(n > 0 ? n : 1));
+  if (!khat || !vhat) {
+    free(khat);
+    free(vhat);
+    return 2;
+  }
+  for (int g = 0; g < n_groups; ++g)
+    orc_dequant_record(k, bhi, blo, perm, records + (size_t)g * R, khat + (size_t)g * 4096,
+                       vhat + (size_t)g * 4096);
+  for (int r = 0; r < n_resid; ++r) {
+    long t = (long)n_groups * 32 + r;
+    for (int c = 0; c < 128; ++c) {
+      khat[t * 128 + c] = (double)orc_f32_from_bf16(resid_k[r * 128 + c]);
+      vhat[t * 128 + c] = (double)orc_f32_from_bf16(resid_v[r * 128 + c]);
+    }
+  }
+  for (int r = 0; r < rows; ++r) {
+    double qd[128];
+    for (int c = 0; c < 128; ++c) qd[c] = (double)orc_f32_from_bf16(q[r * 128 + c]);
+    long nv = n_visible[r] < 0 ? 0 : (n_visible[r] > n ? n : n_visible[r]);
+    if (nv == 0) {
+      for (int c = 0; c < 128; ++c) out[r * 128 + c] = 0.0;
+      continue;
+    }
+    orc_attention_core(1, qd, khat, vhat, nv, scale, out + (size_t)r * 128);
+  }
+  free(khat);
+  free(vhat);
+  return 0;
+}
+
 /* Plain softmax attention over unquantized bf16 K and V ([n][128]). */
 void orc_exact_attention(int G, const uint16_t* q, const uint16_t* kin, const uint16_t* vin,
                          long n, double scale, double* out) {

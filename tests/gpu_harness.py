@@ -34,7 +34,8 @@ class Case:
         self.vin = workload.rows(seed, workload.V, B, Hkv, 0, max(total, 1))
         self.qwin = workload.rows(seed, workload.Q, B, Hq, L - self.W, max(self.W, 1), group=self.G) \
             if L > 0 else None
-        self.cache = pm.PNMixCache(self.cfg, B, self.capacity, max_context=max_context)
+        self.cache = pm.PNMixCache(self.cfg, B, self.capacity, max_context=max_context,
+                                   max_queries=max(1, 8 // self.G))
         self.ocache = oracle.Cache(B, Hkv, self.capacity, k, bhi, blo, score=score)
         self.k_dev = to_dev(self.kin)
         self.v_dev = to_dev(self.vin)
@@ -58,6 +59,17 @@ class Case:
 
     def query(self, pos: int) -> np.ndarray:
         return workload.rows(self.seed, workload.Q, self.B, self.Hq, pos, 1, group=self.G)[:, :, 0]
+
+    def query_multi(self, pos0: int, T: int) -> np.ndarray:
+        """Queries of positions pos0 .. pos0+T-1: bf16 [B][T][Hq][128]."""
+        q = workload.rows(self.seed, workload.Q, self.B, self.Hq, pos0, T, group=self.G)
+        return np.ascontiguousarray(q.transpose(0, 2, 1, 3))
+
+    def attend_multi(self, q: np.ndarray):
+        """GPU multi-query decode vs the oracle's causal rows: fp32 and fp64 [B][T][Hq][128]."""
+        out = self.cache.attend_multi(to_dev(q)).cpu().numpy()
+        want = self.ocache.attend_multi(q)
+        return out, want
 
     def check_state(self, units=None):
         c, o = self.cache, self.ocache

@@ -208,3 +208,26 @@ def test_saliency_statistics_select_like_the_oracle(score, B, Hq, Hkv, L, k, bhi
     c.prefill()
     got, want = c.attend(c.query(L))
     assert_close(got, want)
+
+
+@pytest.mark.parametrize("kernel", [None, "mma", "ws"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,T", [
+    (1, 1, 1, 40, 3),      # all new tokens in the residual
+    (2, 2, 1, 30, 4),      # the step crosses a flush: hidden tokens in the last record too
+    (2, 8, 2, 95, 2),      # 8 rows per unit
+    (3, 4, 4, 61, 8),      # 8 queries of one head
+    (1, 28, 4, 1000, 1),   # one query equals the single-query call
+    (2, 32, 8, 2047, 2),   # the step fills a group exactly
+])
+def test_multi_query_decode_is_causal_like_the_oracle(kernel, B, Hq, Hkv, L, T, monkeypatch):
+    if kernel:
+        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + T)
+    c.prefill()
+    for t in range(L, L + T):
+        c.append(t)
+    got, want = c.attend_multi(c.query_multi(L, T))
+    assert_close(got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128))
+    if T == 1:   # the multi-query call with one query is the single-query call
+        single, _ = c.attend(c.query(L))
+        np.testing.assert_allclose(got[:, 0], single, rtol=0, atol=1e-6)

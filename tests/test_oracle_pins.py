@@ -617,3 +617,41 @@ def test_lossless_cache_reproduces_exact_attention(k, bhi, blo):
     got = c.attend_unit(q, 0, 0)
     want = oracle.exact_attention(q, kb, vb)
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_multi_query_rows_with_one_query_equal_the_single_query_oracle():
+    rng_seed, L = 4, 77
+    k = workload.rows(rng_seed, workload.K, 2, 2, 0, L)
+    v = workload.rows(rng_seed, workload.V, 2, 2, 0, L)
+    qwin = workload.rows(rng_seed, workload.Q, 2, 8, L - 64, 64, group=4)
+    c = oracle.Cache(2, 2, 128, 8, 4, 2)
+    c.select(qwin, k, L)
+    c.prefill(k, v, L)
+    q = workload.rows(rng_seed, workload.Q, 2, 8, L, 1, group=4)[:, :, 0]
+    np.testing.assert_array_equal(c.attend_multi(q[:, None]), c.attend(q)[:, None])
+
+
+@pytest.mark.parametrize("L,T", [(40, 3), (70, 8), (5, 2)])
+def test_multi_query_rows_are_causal(L, T):
+    """After T appends (none completing a group, so every new token stays in the bf16
+    residual), query j of the step equals a single query over a cache that holds only the
+    first L + j + 1 tokens: an independent construction of the causal mask."""
+    assert (L % 32) + T <= 32
+    G, Hkv = 2, 1
+    k = workload.rows(9, workload.K, 1, Hkv, 0, L + T)
+    v = workload.rows(9, workload.V, 1, Hkv, 0, L + T)
+    qwin = workload.rows(9, workload.Q, 1, G, max(L - 64, 0), min(L, 64), group=G)
+    q = workload.rows(9, workload.Q, 1, G, L, T, group=G).transpose(0, 2, 1, 3).copy()
+    full = oracle.Cache(1, Hkv, 128, 8, 4, 2)
+    full.select(qwin, k, L)
+    full.prefill(k, v, L)
+    for t in range(L, L + T):
+        full.append(np.ascontiguousarray(k[:, :, t]), np.ascontiguousarray(v[:, :, t]))
+    got = full.attend_multi(q)
+    for j in range(T):
+        part = oracle.Cache(1, Hkv, 128, 8, 4, 2)
+        part.select(qwin, k, L)
+        part.prefill(k, v, L)
+        for t in range(L, L + j + 1):
+            part.append(np.ascontiguousarray(k[:, :, t]), np.ascontiguousarray(v[:, :, t]))
+        np.testing.assert_allclose(got[:, j], part.attend(np.ascontiguousarray(q[:, j])), rtol=0, atol=1e-12)
