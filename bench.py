@@ -41,11 +41,12 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one decode launch from the committed ncu capture (profiles/
 # decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
 # of the decode sources it was taken on.  Reported only while the sources still match.
-DECODE_CAPTURE = {"sources_sha256_16": "9494d23a19085423", "traffic_bytes": 425101568,
+DECODE_CAPTURE = {"sources_sha256_16": "7568204654d154d6", "traffic_bytes": 425442304,
                   "algorithmic_bytes": 420855808}
 DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
                   "decode_attention_prefill_b200/csrc/decode_common.cuh",
-                  "decode_attention_prefill_b200/csrc/common.cuh"]
+                  "decode_attention_prefill_b200/csrc/common.cuh",
+                  "decode_attention_prefill_b200/csrc/decode_frag.cuh"]
 
 
 def parse():
@@ -194,6 +195,43 @@ def gen_inputs(seed: int, T_total: int, q_positions: list[int]):
     qs = np.stack([workload.rows(seed, workload.Q, B, HQ, p, 1, group=HQ // HKV)[:, :, 0]
                    for p in q_positions]) if q_positions else None
     return kin, vin, qwin, qs
+
+
+def _oracle_unit_seconds(args):
+    """Worker of the all-cores CPU baseline: build one (sequence, KV head) unit in the
+    oracle at n_tokens context and time its decode attention (seconds)."""
+    seed, b, h, n_tokens = args
+    import oracle
+    import workload
+    G = HQ // HKV
+    kin = workload.unit_rows(seed, workload.K, b, h, 1, 0, n_tokens, threads=1)[None]
+    vin = workload.unit_rows(seed, workload.V, b, h, 1, 0, n_tokens, threads=1)[None]
+    qwin = workload.unit_rows(seed, workload.Q, b, h * G, G, PREFILL - WINDOW, WINDOW, group=G, threads=1)
+    q = workload.unit_rows(seed, workload.Q, b, h * G, G, n_tokens, 1, group=G, threads=1)[:, 0]
+    oc = oracle.Cache(1, 1, (n_tokens + 32) // 32 * 32, K_SALIENT, BHI, BLO)
+    oc.select(qwin[None], kin, PREFILL)
+    oc.prefill(kin, vin, n_tokens)
+    t0 = time.perf_counter()
+    oc.attend_unit(np.ascontiguousarray(q), 0, 0)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_all_cores(seed: int, n_tokens: int):
+    """The same oracle unit decode spread over every host core (one process per core,
+    started with spawn), on min(128, 2 x cores) units; the step time is the wall time of
+    the attention calls scaled to 128 units."""
+    import concurrent.futures
+    import multiprocessing
+    cores = os.cpu_count() or 1
+    units = [(seed, b, h, n_tokens) for b in range(B) for h in range(HKV)][:min(B * HKV, 2 * cores)]
+    with concurrent.futures.ProcessPoolExecutor(max_workers=cores,
+                                                mp_context=multiprocessing.get_context("spawn")) as ex:
+        secs = list(ex.map(_oracle_unit_seconds, units))
+    # the attention calls of `cores` workers overlap: per-unit cost / cores
+    step_s = (sum(secs) / len(secs)) * (B * HKV) / min(cores, len(units))
+    return {"value": B / step_s, "unit": "tokens/s", "cores": min(cores, len(units)), "kind": "oracle",
+            "sample": f"oracle decode attention of {len(units)} (sequence, KV head) units at {n_tokens} "
+                      f"tokens on {min(cores, len(units))} processes, scaled to a full {B}-sequence step"}
 
 
 def cpu_baseline(seed: int, budget_s: float, n_tokens: int):
@@ -700,6 +738,10 @@ def main():
     }
     if rank == 0 and not args.no_cpu_baseline:
         out_line["cpu_baseline"] = cpu_baseline(args.seed, args.cpu_seconds, CONTEXT)
+        try:
+            out_line["cpu_baseline"]["all_cores"] = cpu_baseline_all_cores(args.seed, CONTEXT)
+        except Exception as e:   # the host may forbid process pools; the one-core figure stands
+            out_line["cpu_baseline"]["all_cores"] = {"unavailable": str(e)[:200]}
     if pg:
         pg.barrier()
         pg.destroy_process_group()
