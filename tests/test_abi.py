@@ -112,3 +112,28 @@ def test_entry_points_reject_bad_arguments_before_launching():
     assert L.pnmix_decode_attention(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, odd, ws, None) == pm.ERR_ALIGNMENT
     other = pm.Config.make(8, 2, n_salient_pairs=16)   # record size differs from the cache's
     assert L.pnmix_decode_attention(ctypes.byref(other), P, ctypes.byref(c), 256, P, P, ws, None) == pm.ERR_INVALID_ARG
+
+
+def test_multi_query_workspace_follows_the_rows():
+    cfg = pm.Config.make(8, 2)                      # G = 4
+    one = pm.workspace_bytes(cfg, 2, 256)
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 1) == one
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 2) > one
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 3) == 0   # 12 rows per KV head: unsupported
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 0) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_multi_query_entry_rejects_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2)
+    c = _fake_cache(cfg)
+    P = ctypes.c_void_p(1 << 41)
+    L = pm._lib
+    ws = pm.workspace_bytes_multi(cfg, 2, 256, 2)
+    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 3, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_UNSUPPORTED
+    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 0, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_INVALID_ARG
+    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 2, ctypes.byref(c), 256, P, P, ws - 1,
+                                          None) == pm.ERR_CAPACITY
