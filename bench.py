@@ -652,19 +652,57 @@ def main():
     rec_bytes = cache.c.record_bytes
 
     # ---- end-to-end through host buffers (pinned), e2e steps T0 .. T0+n_e2e-1
+    # Double-buffered: step i+1's inputs go host -> device on a copy stream while step i
+    # appends and attends; step i's output goes device -> host on a third stream.
     q_host = torch.from_numpy(qs).view(torch.bfloat16).pin_memory()
     kn_host = kn_dev[:n_e2e].cpu().pin_memory()
     vn_host = vn_dev[:n_e2e].cpu().pin_memory()
-    out_host = torch.empty(B, HQ, D, dtype=torch.float32).pin_memory()
-    staging = {}
+    out_host = [torch.empty(B, HQ, D, dtype=torch.float32).pin_memory() for _ in range(2)]
+    comp_s = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = [{"q": torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev),
+             "k": torch.empty(B, HKV, D, dtype=torch.bfloat16, device=dev),
+             "v": torch.empty(B, HKV, D, dtype=torch.bfloat16, device=dev),
+             "out": torch.empty(B, HQ, D, dtype=torch.float32, device=dev)} for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of a buffer landed
+    ev_used = [torch.cuda.Event() for _ in range(2)]    # append + decode done with a buffer
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # its output copied to the host
+    used = [False, False]
+
+    def stage(i):
+        j = i % 2
+        if used[j]:
+            h2d_s.wait_event(ev_used[j])
+        with torch.cuda.stream(h2d_s):
+            bufs[j]["q"].copy_(q_host[i], non_blocking=True)
+            bufs[j]["k"].copy_(kn_host[i], non_blocking=True)
+            bufs[j]["v"].copy_(vn_host[i], non_blocking=True)
+            ev_in[j].record(h2d_s)
+
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(n_e2e):
+        j = i % 2
         if i == W:
             if pg:
                 pg.barrier()
             torch.cuda.synchronize()
             e0.record()
-        pm.decode_step_host(cache, q_host[i], kn_host[i], vn_host[i], out_host, staging)
+        if i == 0 or i == W:
+            stage(i)
+        if i + 1 < n_e2e and i + 1 != W:
+            stage(i + 1)
+        comp_s.wait_event(ev_in[j])
+        if used[j]:
+            comp_s.wait_event(ev_out[j])     # the previous output of this buffer has left
+        pm.pnmix_append(cfg, bufs[j]["k"], bufs[j]["v"], cache)
+        pm.pnmix_decode_attention(cfg, bufs[j]["q"], cache, bufs[j]["out"])
+        ev_used[j].record(comp_s)
+        d2h_s.wait_event(ev_used[j])
+        with torch.cuda.stream(d2h_s):
+            out_host[j].copy_(bufs[j]["out"], non_blocking=True)
+            ev_out[j].record(d2h_s)
+        used[j] = True
+    comp_s.wait_stream(d2h_s)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -732,7 +770,8 @@ def main():
                     "quantize_tokens_per_s": B * PREFILL / (quant_ms / 1e3)},
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(q_host[0].numel() * 2 + kn_host[0].numel() * 2 * 2),
-                "d2h_bytes_per_step": int(out_host.numel() * 4)},
+                "d2h_bytes_per_step": int(out_host[0].numel() * 4),
+                "overlap": "inputs of step i+1 and the output of step i-1 copy during step i"},
         "gpu_launches": 2 * K,
         "clocks": clocks.summary(),
     }
