@@ -1,8 +1,9 @@
-// decode_mma.cu -- tensor-core decode attention over the packed cache.
+// decode_mma.cu -- tensor-core decode attention over the packed cache, one role per warp.
 //
-// One CTA = one split of one (sequence, KV head) unit, 4 warps.  Every warp owns whole
-// 32-token group records (interleaved across the warps), stages them with cp.async
-// into its own 3-deep shared-memory ring, and keeps its own online softmax.  Per group:
+// One CTA = one slice of the work partition (decode_common.cuh), 4 warps.  Every warp
+// owns whole 32-token group records (interleaved across the warps), stages them with TMA
+// bulk copies into its own shared-memory ring (6 slots when it takes its groups in pairs),
+// and keeps its own online softmax.  Per group:
 //
 //   logits  q . k^_t = sum_p q_p (s_p code_{p,t} + z_p)
 //          = [codes (32 tok x 128 pos)] x [q_p s_p]  +  [z broadcast] x [q]
@@ -22,7 +23,7 @@
 // The bit placement of the record (include/pnmix.h) is the fragment ownership of the
 // m16n8k16 tiles, so a lane's code words are exactly its A registers.  Splits merge
 // through decode_common.cuh (fused combine, no waiting).  The bf16 residual window is
-// attended by warp 0 of the last split with CUDA cores.
+// attended with CUDA cores by the CTA whose slice holds it (one query row per warp).
 #include <atomic>
 
 #include "common.cuh"
