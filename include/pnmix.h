@@ -46,13 +46,15 @@
  *   key norm     K_p = sqrt(max_t (k_{t,p}^2 + k_{t,p+64}^2)) over all L prefill tokens;
  *   query norm   Q_p = (sum over heads h of the group, then tokens of the window,
  *                       of sqrt(q_{h,t,p}^2 + q_{h,t,p+64}^2)) / (G * W');
- *   score        s_p = Q_p * K_p, top k by (s desc, p asc);
+ *   score        s_p = Q_p * K_p (or the statistic cfg->saliency_score names, see
+ *                PNMIX_SCORE_*), top k by (s desc, p asc);
  *   quantizer    mn, mx over the group; s16 = fp16(fl(mx - mn) / (2^b - 1));
  *                z16 = fp16(mn); code = clamp(rint((x - z) / s), 0, 2^b - 1)
  *                with s, z the fp32 values of s16, z16; all codes 0 when s16 == 0.
  * Attention is  out_h = sum_t softmax_t(q_h . k^_t * scale) v^_t  over every
- * cached token, with k^ = code*s + z for packed tokens and the bf16 value for
- * residual tokens; it is accumulated in fp32 and returned in fp32.
+ * cached token (over a causal prefix in pnmix_decode_attention_multi), with
+ * k^ = code*s + z for packed tokens and the bf16 value for residual tokens; it is
+ * accumulated in fp32 and returned in fp32.
  *
  * Packed cache layout (the contract the oracle and the kernels share)
  * ------------------------------------------------------------------
