@@ -353,10 +353,14 @@ def run_decode_workload(args):
     G = Hq // Hkv
     # (bit point, saliency statistic): the sweep adds the key-only (1) and key-range x
     # query (2) statistics at two bit points for comparison with the pair-norm product (0)
-    points = [(bp, 0) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
+    # (bit point, saliency statistic, pruned query pairs): the sweep adds the key-only (1)
+    # and key-range x query (2) statistics at two bit points, and 40 % dynamic query-channel
+    # pruning (26 of 64 pairs) at 2.25 bits
+    points = [(bp, 0, 0) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
     if wl.sweep:
-        points += [(workload.BitPoint(4, 2, 8), 1), (workload.BitPoint(4, 2, 8), 2),
-                   (workload.BitPoint(2, 1, 16), 1), (workload.BitPoint(2, 1, 16), 2)]
+        points += [(workload.BitPoint(4, 2, 8), 1, 0), (workload.BitPoint(4, 2, 8), 2, 0),
+                   (workload.BitPoint(2, 1, 16), 1, 0), (workload.BitPoint(2, 1, 16), 2, 0),
+                   (workload.BitPoint(4, 2, 8), 0, 26)]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     kin = workload.rows(args.seed, workload.K, Bw, Hkv, 0, ctx)
@@ -375,9 +379,9 @@ def run_decode_workload(args):
                  for b in range(Bw) for h in range(Hkv)}
     results = []
     with ClockSampler(0) as clocks:
-        for bp, score in points:
+        for bp, score, prune in points:
             cfg = pm.Config.make(Hq, Hkv, bp.key_bits_hi, bp.key_bits_lo, bp.n_salient_pairs, WINDOW,
-                                 saliency_score=score)
+                                 saliency_score=score, n_pruned_pairs=prune)
             cache = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
             cache.prefill(qwin_dev, k_dev, v_dev, ctx)
             n_rep = max(3, -(-3 * l2_bytes // pm.cache_bytes(cfg, Bw, ctx + 32)))
@@ -394,6 +398,7 @@ def run_decode_workload(args):
             alg = decode_bytes(ctx, Bw * Hkv, G, cache.c.record_bytes)
             r = {"key_bits": [bp.key_bits_hi, bp.key_bits_lo], "salient_pairs": bp.n_salient_pairs,
                  "saliency_score": ["pair-norm product", "key only", "key range x query"][score],
+                 "pruned_query_pairs": prune,
                  "key_code_bits": bp.key_code_bits, "bytes_per_token_head": cache.c.record_bytes / 32,
                  "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
                  "frac_of_8tbs": alg / t / 8e12, "tokens_per_s": Bw / t, "replicas": n_rep}

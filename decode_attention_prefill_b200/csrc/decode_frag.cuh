@@ -138,6 +138,46 @@ struct QFrags {
   uint4 x[NT][4], y[NT][4];
 };
 
+// Dynamic query-channel pruning of the unit's query rows in shared memory (qnat, fp32
+// [kMaxG][128], natural channel order): row v drops the g.n_prune pairs of smallest
+// squared pair norm fl(fl(a*a) + fl(b*b)), never pair 0, the higher pair index first among
+// equal norms, by zeroing both channels.  Warp w handles rows w, w + nwarps, ...; lane l
+// ranks pairs l and l + 32 against all 63 candidates with shuffles.
+__device__ __forceinline__ void prune_query_rows(const Geometry& g, float* qnat, int warp, int nwarps) {
+  const int lane = threadIdx.x & 31;
+  for (int v = warp; v < g.rows; v += nwarps) {
+    float* row = qnat + v * kHeadDim;
+    float n2[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) n2[e] = pair_norm2(row[lane + 32 * e], row[lane + 32 * e + 64]);
+    // pair p is pruned when fewer than n_prune candidates (pairs 1..63) precede it in the
+    // order (norm ascending, index descending)
+    int before[2] = {0, 0};
+#pragma unroll 4
+    for (int src = 0; src < 32; ++src) {
+#pragma unroll
+      for (int e2 = 0; e2 < 2; ++e2) {
+        const float o = __shfl_sync(0xffffffffu, n2[e2], src);
+        const int po = src + 32 * e2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int p = lane + 32 * e;
+          before[e] += (po >= 1 && po != p && (o < n2[e] || (o == n2[e] && po > p))) ? 1 : 0;
+        }
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int p = lane + 32 * e;
+      if (p >= 1 && before[e] < g.n_prune) {
+        row[p] = 0.f;
+        row[p + 64] = 0.f;
+      }
+    }
+  }
+}
+
 // The residual item: up to 31 bf16 tokens staged in shared memory, with CUDA cores, heads
 // h0, h0 + hstep, ... one at a time (few registers).  Lane = token for the logit (its K
 // row, q in natural channel order), lane = channel for the values.  Writes one partial

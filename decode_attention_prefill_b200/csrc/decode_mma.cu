@@ -453,6 +453,10 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
         reinterpret_cast<uint4*>(rrv)[i] = __ldg(gv + i);
       }
     }
+    if (g.n_prune > 0) {   // dynamic query-channel pruning of the staged query rows
+      __syncthreads();
+      prune_query_rows(g, qnat, warp, kWarps);
+    }
     __syncthreads();
     {
       const int L = lane, chunk = warp;   // entries 4*chunk .. 4*chunk+3 (= sigma*2 + e)

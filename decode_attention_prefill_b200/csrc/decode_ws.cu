@@ -321,6 +321,10 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         reinterpret_cast<uint4*>(rrv)[i] = __ldg(gv + i);
       }
     }
+    if (g.n_prune > 0) {   // dynamic query-channel pruning of the staged query rows
+      __syncthreads();
+      prune_query_rows(g, qnat, warp, kWsWarps);
+    }
     __syncthreads();
     if (is_qk) {   // QK warp w builds slice pair w of the sets
       const int tq = lane & 3, gq = lane >> 2, chunk = warp;

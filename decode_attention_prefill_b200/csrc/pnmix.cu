@@ -30,6 +30,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   if (cfg->saliency_window < 1 || cfg->saliency_window > 1024) return PNMIX_ERR_UNSUPPORTED;
   if (cfg->saliency_score < PNMIX_SCORE_PNMIX || cfg->saliency_score > PNMIX_SCORE_RANGE_QUERY)
     return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->n_pruned_pairs < 0 || cfg->n_pruned_pairs > 63) return PNMIX_ERR_UNSUPPORTED;
   g->B = batch;
   g->Hq = cfg->n_q_heads;
   g->Hkv = cfg->n_kv_heads;
@@ -48,6 +49,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->gcap = capacity / kGroup;
   g->scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale : 1.0f / sqrtf(128.0f);
   g->score = cfg->saliency_score;
+  g->n_prune = cfg->n_pruned_pairs;
   g->tq = 1;
   g->rows = G;
   return PNMIX_OK;

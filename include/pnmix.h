@@ -147,8 +147,17 @@ typedef enum {
  *     numbers, i.e. every k for (4,2) and k in {0, 16, 32, 64} for (2,1);
  *   G = n_q_heads / n_kv_heads in [1, 8];
  *   saliency_window W in [1, 1024];
- *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*).
+ *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*);
+ *   n_pruned_pairs in [0, 63].
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ *
+ * Dynamic query-channel pruning (n_pruned_pairs > 0; the query-channel pruning of the
+ * "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches" abstract, applied
+ * to RoPE pairs): in every decode call each query row drops the n_pruned_pairs pairs with
+ * the smallest squared pair norm fl(fl(q_p^2) + fl(q_{p+64}^2)), never pair 0 (the
+ * abstract's channel-0 protection), the higher pair index first among equal norms.  A
+ * dropped pair contributes nothing to that row's logits (its query channels count as
+ * zero).  The packed records are still read whole; what changes is the arithmetic.
  */
 typedef struct {
   int32_t head_dim;
@@ -164,6 +173,7 @@ typedef struct {
   int32_t saliency_window;
   float softmax_scale;
   int32_t saliency_score;   /* statistic that ranks the pairs, PNMIX_SCORE_* (0 = PN-Mix) */
+  int32_t n_pruned_pairs;   /* decode: query pairs each query row drops, 0..63 (0 = none) */
 } pnmix_config;
 
 /*

@@ -59,6 +59,8 @@ def lib():
                 "orc_pair_scores": (None, [i, i, i, vp, vp, vp, vp, vp]),
                 "orc_pair_scores_mode": (None, [i, i, i, i, vp, vp, vp]),
                 "orc_attend_unit_rows": (i, [i, vp, d, i, i, i, vp, vp, i, vp, vp, i, vp, vp]),
+                "orc_pruned_pairs": (ctypes.c_uint64, [vp, i]),
+                "orc_prune_queries": (None, [i, vp, i, vp]),
                 "orc_topk": (None, [vp, i, vp, vp]),
                 "orc_position_order": (i, [ctypes.c_uint64, vp]),
                 "orc_minmax_quant": (None, [vp, i, i, vp, vp, vp]),
@@ -117,6 +119,23 @@ def pair_scores(qwin: np.ndarray, k: np.ndarray):
 
 
 SCORE_PNMIX, SCORE_KEY_ONLY, SCORE_RANGE_QUERY = 0, 1, 2
+
+
+def pruned_pairs(q_row: np.ndarray, n_prune: int) -> int:
+    """Mask of the pairs one query row (bf16 [128]) prunes, see orc_pruned_pairs."""
+    q_row = np.ascontiguousarray(q_row, dtype=np.uint16)
+    return int(lib().orc_pruned_pairs(_p(q_row), n_prune))
+
+
+def prune_queries(q: np.ndarray, n_prune: int) -> np.ndarray:
+    """bf16 [..., 128] query rows with each row's pruned pairs zeroed."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    out = np.empty_like(q)
+    if n_prune <= 0:
+        out[...] = q
+        return out
+    lib().orc_prune_queries(q.size // 128, _p(q), n_prune, _p(out))
+    return out
 
 
 def pair_scores_mode(mode: int, qwin: np.ndarray, k: np.ndarray) -> np.ndarray:
@@ -225,10 +244,11 @@ def unpack_record(k, bhi, blo, rec):
 class Cache:
     """Host image of the cache regions the tests compare with the device."""
 
-    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2, score=SCORE_PNMIX):
+    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2, score=SCORE_PNMIX, n_prune=0):
         self.batch, self.n_kv, self.capacity = batch, n_kv, capacity
         self.k, self.bhi, self.blo, self.bv = k, bhi, blo, bv
         self.score = score
+        self.n_prune = n_prune   # query pairs each decode row drops (0: none)
         self.R = record_bytes(k, bhi, blo)
         if not self.R:
             raise ValueError("unsupported bit point")
@@ -280,7 +300,7 @@ class Cache:
 
     def attend_unit(self, q: np.ndarray, b: int, h: int, scale: float | None = None) -> np.ndarray:
         """q bf16 [G][128] of KV head h of sequence b -> fp64 [G][128]."""
-        q = np.ascontiguousarray(q, dtype=np.uint16)
+        q = prune_queries(q, self.n_prune)
         G = q.shape[0]
         n = int(self.len[b])
         out = np.zeros((G, 128), np.float64)
@@ -294,7 +314,7 @@ class Cache:
     def attend_rows(self, q: np.ndarray, n_visible, b: int, h: int, scale: float | None = None) -> np.ndarray:
         """q bf16 [rows][128] of KV head h of sequence b, row r over the first n_visible[r]
         cached tokens -> fp64 [rows][128]."""
-        q = np.ascontiguousarray(q, dtype=np.uint16)
+        q = prune_queries(q, self.n_prune)
         nv = np.ascontiguousarray(n_visible, dtype=np.int32)
         n = int(self.len[b])
         out = np.zeros((q.shape[0], 128), np.float64)

@@ -654,6 +654,45 @@ int orc_attend_unit_rows(int rows, const uint16_t* q, double scale, int k, int b
   return 0;
 }
 
+/*
+ * Dynamic query-channel pruning (the Dual-QK abstract's query-channel pruning, at the
+ * RoPE-pair level of PN-Mix): for one query row q (bf16 [128]) the n_prune pairs with
+ * the smallest squared pair norm n2_p = fl(fl(a*a) + fl(b*b)), (a, b) = (q[p], q[p+64]),
+ * are pruned, pair 0 never (the abstract's channel-0 protection); among equal norms the
+ * higher pair index is pruned first.  Returns the mask of pruned pairs.
+ */
+uint64_t orc_pruned_pairs(const uint16_t* q, int n_prune) {
+  float n2[64];
+  for (int p = 0; p < 64; ++p) {
+    const float a = orc_f32_from_bf16(q[p]);
+    const float b = orc_f32_from_bf16(q[p + 64]);
+    const float aa = a * a;
+    const float bb = b * b;
+    n2[p] = aa + bb;
+  }
+  uint64_t mask = 0;
+  for (int i = 0; i < n_prune && i < 63; ++i) {
+    int best = -1;
+    for (int p = 63; p >= 1; --p) {   /* scan high to low: ties keep the higher p */
+      if ((mask >> p) & 1ull) continue;
+      if (best < 0 || n2[p] < n2[best]) best = p;
+    }
+    mask |= 1ull << best;
+  }
+  return mask;
+}
+
+/* Copy of the query rows q (bf16 [rows][128]) with the channels of the pairs each row
+ * prunes (orc_pruned_pairs) set to zero: attention with that copy drops exactly their
+ * contributions, q_c * k_c = 0 for every token. */
+void orc_prune_queries(int rows, const uint16_t* q, int n_prune, uint16_t* out) {
+  for (int r = 0; r < rows; ++r) {
+    const uint64_t mask = orc_pruned_pairs(q + (size_t)r * 128, n_prune);
+    for (int c = 0; c < 128; ++c)
+      out[(size_t)r * 128 + c] = ((mask >> (c & 63)) & 1ull) ? 0 : q[(size_t)r * 128 + c];
+  }
+}
+
 /* Plain softmax attention over unquantized bf16 K and V ([n][128]). */
 void orc_exact_attention(int G, const uint16_t* q, const uint16_t* kin, const uint16_t* vin,
                          long n, double scale, double* out) {

@@ -51,6 +51,8 @@ def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
     (dict(saliency_window=0), pm.ERR_UNSUPPORTED),
     (dict(saliency_score=3), pm.ERR_UNSUPPORTED),
     (dict(saliency_score=-1), pm.ERR_UNSUPPORTED),
+    (dict(n_pruned_pairs=64), pm.ERR_UNSUPPORTED),
+    (dict(n_pruned_pairs=-1), pm.ERR_UNSUPPORTED),
 ])
 def test_config_validation(change, status):
     cfg = pm.Config.make(32, 8)

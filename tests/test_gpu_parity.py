@@ -231,3 +231,27 @@ def test_multi_query_decode_is_causal_like_the_oracle(kernel, B, Hq, Hkv, L, T, 
     if T == 1:   # the multi-query call with one query is the single-query call
         single, _ = c.attend(c.query(L))
         np.testing.assert_allclose(got[:, 0], single, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("kernel", [None, "mma", "ws"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,n_prune,T", [
+    (1, 1, 1, 77, 26, 1),
+    (2, 8, 2, 1000, 26, 1),
+    (2, 28, 4, 517, 40, 1),
+    (2, 32, 8, 2100, 10, 1),
+    (2, 8, 2, 300, 26, 2),     # with two queries per sequence
+    (1, 4, 1, 64, 63, 1),      # only pair 0 left
+])
+def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T, monkeypatch):
+    if kernel:
+        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + n_prune, n_prune=n_prune)
+    c.prefill()
+    if T == 1:
+        got, want = c.attend(c.query(L))
+    else:
+        for t in range(L, L + T):
+            c.append(t)
+        got, want = c.attend_multi(c.query_multi(L, T))
+        got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
+    assert_close(got, want)

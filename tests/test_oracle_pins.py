@@ -655,3 +655,51 @@ def test_multi_query_rows_are_causal(L, T):
         for t in range(L, L + j + 1):
             part.append(np.ascontiguousarray(k[:, :, t]), np.ascontiguousarray(v[:, :, t]))
         np.testing.assert_allclose(got[:, j], part.attend(np.ascontiguousarray(q[:, j])), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_pruned_pairs_match_a_sort_of_exact_integer_norms(seed):
+    """Query-channel pruning on integer queries (exact squared pair norms, many ties): the
+    pruned set is the first n of pairs 1..63 sorted by (norm, higher index first)."""
+    rng = np.random.default_rng(80 + seed)
+    q = rng.integers(-3, 4, 128).astype(np.float32)
+    n2 = [int(q[p]) ** 2 + int(q[p + 64]) ** 2 for p in range(64)]
+    qb = bf16_bits(q)
+    for n in (0, 1, 10, 26, 40, 63):
+        order = sorted(range(1, 64), key=lambda p: (n2[p], -p))
+        want = sum(1 << p for p in order[:n])
+        assert oracle.pruned_pairs(qb, n) == want
+
+
+def test_pair_zero_is_never_pruned():
+    q = np.full(128, 2.0, np.float32)
+    q[0] = q[64] = 0.0                       # pair 0 has the smallest norm
+    mask = oracle.pruned_pairs(bf16_bits(q), 63)
+    assert mask == (1 << 64) - 2
+
+
+def test_pruned_key_channels_do_not_change_the_pruned_attention():
+    """The pruned pairs' key channels can hold anything: with pruning the output is the
+    same to the last bit, without pruning it changes (so the pruning is what hides them)."""
+    rng = np.random.default_rng(5)
+    n = 3 * 32 + 7
+    kf = rng.integers(-6, 7, (n, 128)).astype(np.float32) / 2
+    vf = _grid_rows(rng, n)
+    qf = rng.integers(-4, 5, (1, 128)).astype(np.float32)
+    qb = bf16_bits(qf)
+    mask = oracle.pruned_pairs(qb[0], 26)
+    kf2 = kf.copy()
+    for p in range(64):
+        if (mask >> p) & 1:   # token-dependent changes (a constant would cancel in softmax)
+            kf2[:, p] += rng.integers(-4, 5, n) * 1.5
+            kf2[:, p + 64] -= rng.integers(-4, 5, n) * 2.0
+    outs = {}
+    for name, kk in (("orig", kf), ("changed", kf2)):
+        for prune in (0, 26):
+            c = oracle.Cache(1, 1, 128, 8, 4, 2, n_prune=prune)
+            c.perm[0, 0] = np.arange(128)
+            c.mask[0, 0] = 0xFF
+            c.prefill(bf16_bits(kk)[None, None], bf16_bits(vf)[None, None], n)
+            outs[name, prune] = c.attend_unit(qb, 0, 0)
+    np.testing.assert_array_equal(outs["orig", 26], outs["changed", 26])
+    assert np.abs(outs["orig", 0] - outs["changed", 0]).max() > 1e-3
