@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one decode launch from the committed ncu capture (profiles/
 # decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
 # of the decode sources it was taken on.  Reported only while the sources still match.
-DECODE_CAPTURE = {"sources_sha256_16": "670a2a5cb0582fdb", "traffic_bytes": 425442304,
+DECODE_CAPTURE = {"sources_sha256_16": "9a9c8d0b626a1eb8", "traffic_bytes": 424529664,
                   "algorithmic_bytes": 420855808}
 DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
                   "decode_attention_prefill_b200/csrc/decode_common.cuh",
@@ -60,12 +60,14 @@ def parse():
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="stream_32k",
-                    choices=["stream_32k", "llama3_8b", "sweep_128k", "pipeline_32l", "verify_32k"],
+                    choices=["stream_32k", "llama3_8b", "sweep_128k", "pipeline_32l", "verify_32k",
+                             "stream_full"],
                     help="stream_32k is the benchmark line; the others print per-workload "
                          "measurements (decode GB/s and tokens/s; for the sweep the relative L2 "
                          "error against unquantized bf16 attention; for the 32-layer pipeline the "
                          "prefill latencies and the extrapolated end-to-end tokens/s; verify_32k: "
-                         "two new tokens per sequence attended at once at 32K)")
+                         "two new tokens per sequence attended at once at 32K; stream_full: the "
+                         "whole 4096 -> 32768 stream, measured)")
     ap.add_argument("--pipeline-layers-generated", type=int, default=4,
                     help="pipeline_32l: layers whose prefill inputs are generated (seed + layer); "
                          "the others reuse them cyclically")
@@ -472,6 +474,57 @@ def run_verify(args):
     return 0
 
 
+def run_stream_full(args):
+    """stream_full: the whole stream_32k stream, measured rather than sampled: a 4096-token
+    prefill (saliency + quantize), then all 28672 append + decode steps to 32768 tokens,
+    one token per sequence per step.  K/V rows are the generator's at their true
+    positions; the queries of 1024 consecutive positions are reused cyclically (the decode
+    cost does not depend on the query values).  Reports the whole-stream time and the
+    average decode tokens/s."""
+    import torch
+
+    import decode_attention_prefill_b200 as pm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kin, vin, qwin, _ = gen_inputs(args.seed, CONTEXT, [])
+    n_q = 1024
+    q_dev = torch.from_numpy(workload_rows_q(args.seed, PREFILL, n_q)).view(torch.bfloat16).to(dev) \
+        .permute(1, 0, 2, 3).contiguous()           # [n_q][B][Hq][128]
+    cfg = pm.Config.make(HQ, HKV, BHI, BLO, K_SALIENT, WINDOW)
+    cache = pm.PNMixCache(cfg, B, CONTEXT + 32, max_context=CONTEXT)
+    k_dev = torch.from_numpy(kin).view(torch.bfloat16).to(dev)
+    v_dev = torch.from_numpy(vin).view(torch.bfloat16).to(dev)
+    kn = k_dev.permute(2, 0, 1, 3).contiguous()     # [T][B][Hkv][128]
+    vn = v_dev.permute(2, 0, 1, 3).contiguous()
+    qwin_dev = torch.from_numpy(qwin).view(torch.bfloat16).to(dev)
+    out = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        e[0].record()
+        cache.prefill(qwin_dev, k_dev, v_dev, PREFILL)
+        e[1].record()
+        for t in range(PREFILL, CONTEXT):
+            pm.pnmix_append(cfg, kn[t], vn[t], cache)
+            pm.pnmix_decode_attention(cfg, q_dev[(t - PREFILL) % n_q], cache, out)
+        e[2].record()
+        torch.cuda.synchronize()
+    assert cache.read_error() == 0 and int(cache.lengths().min().item()) == CONTEXT
+    prefill_s = e[0].elapsed_time(e[1]) / 1e3
+    stream_s = e[1].elapsed_time(e[2]) / 1e3
+    steps = CONTEXT - PREFILL
+    line = {"workload": "stream_full", "metric": "whole-stream time, 4096 -> 32768 tokens",
+            "unit": "s", "n_gpus": 1, "data": "synthetic", "dtype": "f32",
+            "config": {"batch": B, "n_q_heads": HQ, "n_kv_heads": HKV, "prefill": PREFILL,
+                       "context": CONTEXT, "key_code_bits": 2.25,
+                       "queries": f"{n_q} consecutive positions reused cyclically"},
+            "prefill_s": prefill_s, "stream_s": stream_s, "steps": steps,
+            "decode_tokens_per_s": B * steps / stream_s, "mean_step_us": stream_s / steps * 1e6,
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_rows_q(seed: int, pos0: int, n: int) -> np.ndarray:
     """Queries of positions pos0 .. pos0+n-1 of the bench workload: bf16 [B][n][Hq][128]."""
     import workload
@@ -589,6 +642,8 @@ def main():
         return run_pipeline(args)
     if args.workload == "verify_32k":
         return run_verify(args)
+    if args.workload == "stream_full":
+        return run_stream_full(args)
     if args.workload != "stream_32k":
         return run_decode_workload(args)
 
