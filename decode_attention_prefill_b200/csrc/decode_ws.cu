@@ -154,13 +154,13 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* r
       const uint32_t b0 = hfma2(qx0, s0, hmul2(qy0, s0));
       const uint32_t b1 = hfma2(qx1, s1, hmul2(qy1, s1));
       if (hi) {
-        mma16816(acc_hi[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-        mma16816(acc_hi[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+        mma16816_free(acc_hi[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+        mma16816_free(acc_hi[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
       } else {
-        mma16816(acc_lo[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-        mma16816(acc_lo[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+        mma16816_free(acc_lo[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+        mma16816_free(acc_lo[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
       }
-      mma16816(dz[nt], z0, z0, z1, z1, qx0, qx1);
+      mma16816_free(dz[nt], z0, z0, z1, z1, qx0, qx1);
     }
   }
 #pragma unroll
@@ -213,8 +213,8 @@ __device__ __forceinline__ void group_values(const uint8_t* rec, const uint4& p4
       const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
       vz[i] = gq < 4 ? v : 0u;
     }
-    mma16816(bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
-    mma16816(bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
+    mma16816_free(bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
+    mma16816_free(bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
   }
   // slot (r, p) of value word m sits at bits 8r + 2p and is taken in place from w >> 8r,
   // so token block p carries 2^(2p); its B rows are scaled by 2^(2 - 2p)
@@ -234,8 +234,8 @@ __device__ __forceinline__ void group_values(const uint8_t* rec, const uint4& p4
     const uint32_t k1a1 = sub_pair(w8, 0x00300030u), k1a3 = sub_pair(w8, 0x00C000C0u);
     const uint32_t b00 = hmul2(bp0, vsr[0][j]), b01 = hmul2(p16[1], vsr[1][j]);
     const uint32_t b10 = hmul2(bp2, vsr[2][j]), b11 = hmul2(bp3, vsr[3][j]);
-    mma16816(pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
-    mma16816(pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
+    mma16816_free(pv[m], k0a0, k0a1, k0a2, k0a3, b00, b01);
+    mma16816_free(pv[m], k1a0, k1a1, k1a2, k1a3, b10, b11);
   }
 }
 
