@@ -139,6 +139,7 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* r
     }
     const uint32_t s0 = par ? s4.z : s4.x, s1 = par ? s4.w : s4.y;
     const uint32_t z0 = par ? z4.z : z4.x, z1 = par ? z4.w : z4.y;
+    uint32_t qxs[NT][2];   // this slice's X registers of each tile (for the zero-point term)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       uint4 X, Y;
@@ -160,12 +161,33 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* r
         mma16816_free(acc_lo[nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
         mma16816_free(acc_lo[nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
       }
-      mma16816_free(dz[nt], z0, z0, z1, z1, qx0, qx1);
+      qxs[nt][0] = qx0;
+      qxs[nt][1] = qx1;
     }
+    if constexpr (NT == 1) {
+      mma16816_free(dz[0], z0, z0, z1, z1, qxs[0][0], qxs[0][1]);
+    } else {
+      // zero-point term of both tiles in one product: A = X transposed (row = query column:
+      // rows gq and gq + 8 are column gq of tile 0 and tile 1, exactly this lane's X
+      // registers), B = z (the same in every column).  Row c of the result is
+      // sum_p X[p][c] z_p.
+      mma16816_free(dz[0], qxs[0][0], qxs[1][0], qxs[0][1], qxs[1][1], z0, z1);
+    }
+  }
+  // zero-point sums per head: columns 2tq and 2tq+1 of each tile
+  float zsum[NT];
+  if constexpr (NT == 1) {
+    zsum[0] = dz[0][0] + dz[0][1];
+  } else {
+    // row c of the transposed product sits in lanes 4c .. 4c+3 (c < 8: element 0, tile 0;
+    // element 2: tile 1)
+    const int src0 = (2 * tq) * 4, src1 = (2 * tq + 1) * 4;
+    zsum[0] = __shfl_sync(0xffffffffu, dz[0][0], src0) + __shfl_sync(0xffffffffu, dz[0][0], src1);
+    zsum[1] = __shfl_sync(0xffffffffu, dz[0][2], src0) + __shfl_sync(0xffffffffu, dz[0][2], src1);
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float zb = (dz[nt][0] + dz[nt][1]) * qscale;
+    const float zb = zsum[nt] * qscale;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int mt = u >> 1, r = 2 * (u & 1);
