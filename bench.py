@@ -182,6 +182,22 @@ class ClockSampler:
                 "reasons": sorted(active), "samples": len(self.samples), "source": "nvml"}
 
 
+def max_over_ranks(ms: float, pg, dev) -> float:
+    """The slowest rank's time (every rank takes part; pg is torch.distributed or None)."""
+    if not pg:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, steps: int, ms: float) -> float:
+    """Tokens of all ranks (B sequences each, one token per sequence per step) over the
+    slowest rank's time."""
+    return world * B * steps / (ms / 1e3)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -765,12 +781,8 @@ def main():
     comp_s.wait_stream(d2h_s)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * B * K / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+    e2e_value = whole_job_tokens_per_s(world, K, e2e_ms)
 
     # ---- device-resident steps, two passes of W + K steps each.  Pass 1 (the bench value):
     # K whole steps between two events.  Pass 2 (the kernel roofline): the next steps with
@@ -807,10 +819,7 @@ def main():
     torch.cuda.synchronize()
     dec_ms = [ev[1][i].elapsed_time(ev[2][i]) for i in range(K)]
     app_ms = [ev[0][i].elapsed_time(ev[1][i]) for i in range(K)]
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, pg, dev)
     err = cache.read_error()
     lens = cache.lengths().cpu().numpy()
     assert err == 0 and int(lens.min()) == CONTEXT, (err, lens)
@@ -821,7 +830,7 @@ def main():
     avg_dec_s = sum(dec_ms) / K / 1e3
     achieved = sum(alg) / K / avg_dec_s / 1e9
     peak, peak_kind = measured_peaks()
-    value = world * B * K / (total_ms / 1e3)
+    value = whole_job_tokens_per_s(world, K, total_ms)
     out_line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",

@@ -25,14 +25,13 @@ def _rank_main(rank, world, port, q):
     w, r, local = bench.dist_setup(None)
     assert (w, r, local) == (world, rank, rank)
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    # each rank: its own sequences (seed offset), its own measured time
+    # each rank: its own sequences (seed offset), its own measured time; the bench's own
+    # helpers reduce it to the slowest rank's and form the whole-job value
     seed = 0 + 7919 * rank
-    t = torch.tensor([10.0 + 5.0 * rank])
     dist.barrier()
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    # whole-job value: all ranks' tokens over the slowest rank's time
-    value = world * bench.B * 4 / (float(t.item()) / 1e3)
-    q.put((rank, seed, float(t.item()), value))
+    ms = bench.max_over_ranks(10.0 + 5.0 * rank, dist, torch.device("cpu"))
+    value = bench.whole_job_tokens_per_s(world, 4, ms)
+    q.put((rank, seed, ms, value))
     dist.barrier()
     dist.destroy_process_group()
 
