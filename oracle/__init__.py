@@ -60,6 +60,8 @@ def lib():
                 "orc_pair_scores_mode": (None, [i, i, i, i, vp, vp, vp]),
                 "orc_attend_unit_rows": (i, [i, vp, d, i, i, i, vp, vp, i, vp, vp, i, vp, vp]),
                 "orc_pruned_pairs": (ctypes.c_uint64, [vp, i]),
+                "orc_ers": (ctypes.c_uint32, [ctypes.c_uint32, i]),
+                "orc_shrink_record": (i, [i, i, i, vp, vp]),
                 "orc_prune_queries": (None, [i, vp, i, vp]),
                 "orc_topk": (None, [vp, i, vp, vp]),
                 "orc_position_order": (i, [ctypes.c_uint64, vp]),
@@ -146,6 +148,11 @@ def pair_scores_mode(mode: int, qwin: np.ndarray, k: np.ndarray) -> np.ndarray:
     s = np.zeros(64, np.float32)
     lib().orc_pair_scores_mode(mode, G, W, k.shape[0], _p(qwin), _p(k), _p(s))
     return s
+
+
+def ers(x: int, b: int) -> int:
+    """Equivalent right shift of a 2b-bit code to b bits, see orc_ers."""
+    return int(lib().orc_ers(x, b))
 
 
 def topk(scores: np.ndarray, k: int):
@@ -309,6 +316,24 @@ class Cache:
                                    _p(self.records[b, h]), n // 32, _p(self.resid_k[b, h]),
                                    _p(self.resid_v[b, h]), n % 32, None, None, _p(out))
         assert rc == 0
+        return out
+
+    def shrunk(self) -> "Cache":
+        """The cache with its salient key positions shrunk from b_hi to b_lo = b_hi / 2 bits
+        (orc_shrink_record on every full group): a k = 0 cache in the same position order."""
+        out = Cache(self.batch, self.n_kv, self.capacity, 0, self.bhi, self.blo, self.bv,
+                    self.score, self.n_prune)
+        out.perm[:] = self.perm
+        out.scores[:] = self.scores
+        out.len[:] = self.len
+        out.resid_k[:] = self.resid_k
+        out.resid_v[:] = self.resid_v
+        for b in range(self.batch):
+            for h in range(self.n_kv):
+                for g in range(int(self.len[b]) // 32):
+                    rc = lib().orc_shrink_record(self.k, self.bhi, self.blo, _p(self.records[b, h, g]),
+                                                 _p(out.records[b, h, g]))
+                    assert rc == 0
         return out
 
     def attend_rows(self, q: np.ndarray, n_visible, b: int, h: int, scale: float | None = None) -> np.ndarray:

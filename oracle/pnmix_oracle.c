@@ -454,6 +454,39 @@ int orc_unpack_record(int k, int bhi, int blo, const uint8_t* rec, uint8_t* kcod
   return 0;
 }
 
+/*
+ * Equivalent right shift (PM-KVQ review page, the bit-width shrinking step of its
+ * progressive quantization): a 2b-bit code X becomes the b-bit code
+ *   X_b = ((2^(2b) - 2^b + 1) * (X + 2^(b-1))) >> 3b,
+ * the integer form of round(X / (2^b + 1)), with the scale multiplied by 2^b + 1 and the
+ * zero point kept.
+ */
+uint32_t orc_ers(uint32_t x, int b) {
+  const uint32_t mul = (1u << (2 * b)) - (1u << b) + 1u;
+  return (mul * (x + (1u << (b - 1)))) >> (3 * b);
+}
+
+/*
+ * Shrink one record of the (bhi, blo, k) layout to the (bhi, blo, 0) layout (every
+ * position at blo = bhi / 2 bits, same position order): the codes of the salient
+ * positions [0, 2k) go through orc_ers with b = blo and their scale becomes
+ * fp16(fl(s * (2^blo + 1))); every other byte is carried over.
+ */
+int orc_shrink_record(int k, int bhi, int blo, const uint8_t* src, uint8_t* dst) {
+  if (bhi != 2 * blo) return 1;
+  uint8_t kcodes[32 * 128], vcodes[32 * 128];
+  uint16_t ks[128], kz[128], vs[32 * 4], vz[32 * 4];
+  if (orc_unpack_record(k, bhi, blo, src, kcodes, ks, kz, vcodes, vs, vz)) return 1;
+  const int nhi = 2 * k;
+  const float mul = (float)((1 << blo) + 1);
+  for (int j = 0; j < nhi; ++j) {
+    for (int t = 0; t < 32; ++t) kcodes[t * 128 + j] = (uint8_t)orc_ers(kcodes[t * 128 + j], blo);
+    const float s = orc_f32_from_f16(ks[j]) * mul;
+    ks[j] = orc_f16_from_f32(s);
+  }
+  return orc_pack_record(0, bhi, blo, kcodes, ks, kz, vcodes, vs, vz, dst);
+}
+
 /* Quantize 32 K rows and 32 V rows (bf16 [32][128] each) into one record. */
 int orc_make_record(int k, int bhi, int blo, int bv, const uint8_t* perm, const uint16_t* krows,
                     const uint16_t* vrows, uint8_t* rec) {

@@ -703,3 +703,57 @@ def test_pruned_key_channels_do_not_change_the_pruned_attention():
             outs[name, prune] = c.attend_unit(qb, 0, 0)
     np.testing.assert_array_equal(outs["orig", 26], outs["changed", 26])
     assert np.abs(outs["orig", 0] - outs["changed", 0]).max() > 1e-3
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8])
+def test_equivalent_right_shift_is_round_of_the_division_exhaustively(b):
+    """The shift formula equals round(X / (2^b + 1)) for every 2b-bit X (no value sits
+    exactly between two integers, since 2^b + 1 is odd)."""
+    d = (1 << b) + 1
+    for x in range(1 << (2 * b)):
+        want = int(Fraction(x, d) + Fraction(1, 2))
+        assert oracle.ers(x, b) == want, (x, b)
+
+
+@pytest.mark.parametrize("bhi,blo,k", [(4, 2, 8), (4, 2, 32), (2, 1, 16)])
+def test_shrinking_codes_on_the_coarse_grid_changes_nothing(bhi, blo, k):
+    """Salient key channels whose codes are multiples of 2^blo + 1 (and power-of-two scales)
+    sit on the coarse grid too: after the shift the dequantized keys, hence the attention,
+    are exactly the same; the other channels' codes are carried over unchanged."""
+    rng = np.random.default_rng(30 + k + bhi)
+    G, ng, nr = 2, 3, 5
+    n = ng * 32 + nr
+    mask = 0
+    for p in rng.choice(64, k, replace=False):
+        mask |= 1 << int(p)
+    perm, nhi = oracle.position_order(mask)
+    d = (1 << blo) + 1
+    kf = np.zeros((n, 128), np.float32)
+    for g in range(ng + 1):
+        for j in range(128):
+            hi = j < nhi
+            bits = bhi if hi else blo
+            levels = (1 << bits) - 1
+            z = float(rng.integers(-16, 16)) / 8
+            s = float(2.0 ** rng.integers(-2, 2))
+            if hi:
+                c = rng.integers(0, levels // d + 1, 32) * d      # 0, d, 2d, ... up to levels
+            else:
+                c = rng.integers(0, levels + 1, 32)
+            c[0], c[1] = 0, levels
+            rows = slice(32 * g, min(32 * g + 32, n))
+            kf[rows, perm[j]] = (z + c * s)[: rows.stop - rows.start]
+    vf = _grid_rows(rng, n)
+    c = oracle.Cache(1, 1, 256, k, bhi, blo)
+    c.mask[0, 0], c.perm[0, 0] = mask, perm
+    c.prefill(bf16_bits(kf)[None, None], bf16_bits(vf)[None, None], n)
+    small = c.shrunk()
+    assert small.R == oracle.record_bytes(0, bhi, blo) < c.R
+    q = bf16_bits_round(rng.standard_normal((G, 128)))
+    np.testing.assert_array_equal(small.attend_unit(q, 0, 0), c.attend_unit(q, 0, 0))
+    # codes of the non-salient positions are the same before and after
+    for g in range(ng):
+        a = oracle.unpack_record(k, bhi, blo, c.records[0, 0, g])[0]
+        b2 = oracle.unpack_record(0, bhi, blo, small.records[0, 0, g])[0]
+        np.testing.assert_array_equal(a[:, nhi:], b2[:, nhi:])
+        np.testing.assert_array_equal(b2[:, :nhi], a[:, :nhi] // d)
