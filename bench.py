@@ -358,8 +358,9 @@ def timed_rotation(fns, reps: int, warmup: int) -> float:
 
 def run_decode_workload(args):
     """Decode-only measurements: llama3_8b (batch 8, 32/8 heads, one step at 8192) and
-    sweep_128k (batch 2, 28/4 heads, 131072 tokens, six bit points, each with the relative
-    L2 error against unquantized bf16 attention over every (sequence, KV head) unit).
+    sweep_128k (batch 2, 28/4 heads, 131072 tokens, six bit points and the statistic,
+    pruning and shrinking variants, each with the relative L2 error against unquantized
+    bf16 attention over every (sequence, KV head) unit).
     These caches fit in L2, so the timed launches rotate over enough identical cache
     replicas to exceed it three times over."""
     import torch
@@ -369,16 +370,16 @@ def run_decode_workload(args):
     wl = workload.WORKLOADS[args.workload]
     Bw, Hq, Hkv, ctx = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.context
     G = Hq // Hkv
-    # (bit point, saliency statistic): the sweep adds the key-only (1) and key-range x
-    # query (2) statistics at two bit points for comparison with the pair-norm product (0)
-    # (bit point, saliency statistic, pruned query pairs): the sweep adds the key-only (1)
-    # and key-range x query (2) statistics at two bit points, and 40 % dynamic query-channel
-    # pruning (26 of 64 pairs) at 2.25 bits
-    points = [(bp, 0, 0) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
+    # (bit point, saliency statistic, pruned query pairs, shrunk): the sweep adds the
+    # key-only (1) and key-range x query (2) statistics at two bit points, 40 % dynamic
+    # query-channel pruning (26 of 64 pairs) at 2.25 bits, and two caches whose salient
+    # keys were shrunk to the low bit width after quantization (pnmix_shrink_keys)
+    points = [(bp, 0, 0, False) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
     if wl.sweep:
-        points += [(workload.BitPoint(4, 2, 8), 1, 0), (workload.BitPoint(4, 2, 8), 2, 0),
-                   (workload.BitPoint(2, 1, 16), 1, 0), (workload.BitPoint(2, 1, 16), 2, 0),
-                   (workload.BitPoint(4, 2, 8), 0, 26)]
+        points += [(workload.BitPoint(4, 2, 8), 1, 0, False), (workload.BitPoint(4, 2, 8), 2, 0, False),
+                   (workload.BitPoint(2, 1, 16), 1, 0, False), (workload.BitPoint(2, 1, 16), 2, 0, False),
+                   (workload.BitPoint(4, 2, 8), 0, 26, False),
+                   (workload.BitPoint(4, 2, 8), 0, 0, True), (workload.BitPoint(2, 1, 16), 0, 0, True)]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     kin = workload.rows(args.seed, workload.K, Bw, Hkv, 0, ctx)
@@ -397,17 +398,27 @@ def run_decode_workload(args):
                  for b in range(Bw) for h in range(Hkv)}
     results = []
     with ClockSampler(0) as clocks:
-        for bp, score, prune in points:
-            cfg = pm.Config.make(Hq, Hkv, bp.key_bits_hi, bp.key_bits_lo, bp.n_salient_pairs, WINDOW,
-                                 saliency_score=score, n_pruned_pairs=prune)
-            cache = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
-            cache.prefill(qwin_dev, k_dev, v_dev, ctx)
+        for bp, score, prune, shrink in points:
+            qcfg = pm.Config.make(Hq, Hkv, bp.key_bits_hi, bp.key_bits_lo, bp.n_salient_pairs, WINDOW,
+                                  saliency_score=score, n_pruned_pairs=prune)
+            cfg = qcfg.without_salient() if shrink else qcfg
+            src = pm.PNMixCache(qcfg, Bw, ctx + 32, max_context=ctx)
+            src.prefill(qwin_dev, k_dev, v_dev, ctx)
             n_rep = max(3, -(-3 * l2_bytes // pm.cache_bytes(cfg, Bw, ctx + 32)))
-            replicas = [cache]
-            for _ in range(n_rep - 1):
-                r = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
-                r.prefill(qwin_dev, k_dev, v_dev, ctx)
-                replicas.append(r)
+            shrink_us = None
+            if shrink:
+                replicas = [src.shrunk() for _ in range(n_rep)]
+                shrink_us = timed_rotation([lambda: pm.pnmix_shrink_keys(qcfg, src, replicas[0])],
+                                           max(args.steps, 5), args.warmup) * 1e6
+                pm.pnmix_shrink_keys(qcfg, src, replicas[0])
+                del src
+            else:
+                replicas = [src]
+                for _ in range(n_rep - 1):
+                    r = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
+                    r.prefill(qwin_dev, k_dev, v_dev, ctx)
+                    replicas.append(r)
+            cache = replicas[0]
             out = torch.empty(Bw, Hq, D, dtype=torch.float32, device=dev)
             fns = [(lambda c_=c_: pm.pnmix_decode_attention(cfg, q_dev, c_, out)) for c_ in replicas]
             t = timed_rotation(fns, max(args.steps, 3 * n_rep), args.warmup)
@@ -416,8 +427,9 @@ def run_decode_workload(args):
             alg = decode_bytes(ctx, Bw * Hkv, G, cache.c.record_bytes)
             r = {"key_bits": [bp.key_bits_hi, bp.key_bits_lo], "salient_pairs": bp.n_salient_pairs,
                  "saliency_score": ["pair-norm product", "key only", "key range x query"][score],
-                 "pruned_query_pairs": prune,
-                 "key_code_bits": bp.key_code_bits, "bytes_per_token_head": cache.c.record_bytes / 32,
+                 "pruned_query_pairs": prune, "shrunk_to_low_bits": shrink, "shrink_us": shrink_us,
+                 "key_code_bits": bp.key_bits_lo if shrink else bp.key_code_bits,
+                 "bytes_per_token_head": cache.c.record_bytes / 32,
                  "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
                  "frac_of_8tbs": alg / t / 8e12, "tokens_per_s": Bw / t, "replicas": n_rep}
             if exact is not None:

@@ -39,7 +39,7 @@ EXPORTED = [
     "pnmix_select_pairs", "pnmix_quantize_keys", "pnmix_quantize_values", "pnmix_append",
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
-    "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi",
+    "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi", "pnmix_shrink_keys",
 ]
 
 
@@ -60,6 +60,12 @@ class Config(ctypes.Structure):
     @property
     def group(self) -> int:
         return self.n_q_heads // self.n_kv_heads
+
+    def without_salient(self) -> "Config":
+        """The same config with no salient pair (the layout pnmix_shrink_keys writes)."""
+        c = Config.from_buffer_copy(self)
+        c.n_salient_pairs = 0
+        return c
 
 
 class Cache(ctypes.Structure):
@@ -92,6 +98,7 @@ _SIGS = {
     "pnmix_decode_attention_noalloc": (_i, [_CP, _vp, _KP, _i, _vp, _vp]),
     "pnmix_workspace_bytes_multi": (_sz, [_CP, _i, _i, _i]),
     "pnmix_decode_attention_multi": (_i, [_CP, _vp, _i, _KP, _i, _vp, _vp, _sz, _vp]),
+    "pnmix_shrink_keys": (_i, [_CP, _KP, _KP, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -200,6 +207,12 @@ def pnmix_decode_attention_multi(cfg: Config, q: torch.Tensor, cache: "PNMixCach
                                              _stream(stream)), "pnmix_decode_attention_multi")
 
 
+def pnmix_shrink_keys(cfg: Config, src: "PNMixCache", dst: "PNMixCache", stream=None):
+    """src: a cache of cfg (b_hi = 2 b_lo, k > 0); dst: a cache of cfg with n_salient_pairs = 0."""
+    _check(_lib.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src.c), ctypes.byref(dst.c), _stream(stream)),
+           "pnmix_shrink_keys")
+
+
 # ---------------------------------------------------------------- owner of device buffers
 
 class PNMixCache:
@@ -278,6 +291,13 @@ class PNMixCache:
 
     def append(self, k_new, v_new, stream=None):
         pnmix_append(self.cfg, k_new, v_new, self, stream)
+
+    def shrunk(self, stream=None, max_queries: int = 1) -> "PNMixCache":
+        """A new cache holding this one with its salient keys shrunk to key_bits_lo bits."""
+        dst = PNMixCache(self.cfg.without_salient(), self.batch, self.capacity, device=self.buffer.device,
+                         max_context=self.max_context, stream=stream, max_queries=max_queries)
+        pnmix_shrink_keys(self.cfg, self, dst, stream)
+        return dst
 
     def attend_multi(self, q, out=None, stream=None) -> torch.Tensor:
         """q bf16 [B][T][Hq][128] of T tokens already appended -> fp32 [B][T][Hq][128]."""

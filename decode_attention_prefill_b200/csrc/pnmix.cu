@@ -299,6 +299,23 @@ pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_
                                    static_cast<cudaStream_t>(stream)));
 }
 
+pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_cache* src, pnmix_cache* dst,
+                               void* stream) {
+  if (!cfg || !src || !dst) return PNMIX_ERR_INVALID_ARG;
+  Geometry gs, gd;
+  pnmix_status st = make_geometry(cfg, src->batch, src->capacity_tokens, &gs);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(gs, src)) != PNMIX_OK) return st;
+  if (gs.bhi != 2 * gs.blo || gs.k == 0) return PNMIX_ERR_UNSUPPORTED;
+  pnmix_config small = *cfg;
+  small.n_salient_pairs = 0;
+  if ((st = make_geometry(&small, src->batch, src->capacity_tokens, &gd)) != PNMIX_OK) return st;
+  if (dst->batch != src->batch || dst->capacity_tokens != src->capacity_tokens) return PNMIX_ERR_INVALID_ARG;
+  if ((st = check_cache(gd, dst)) != PNMIX_OK) return st;
+  if (dst->base == src->base) return PNMIX_ERR_INVALID_ARG;
+  return cuda_status(launch_shrink(gs, gd, *src, *dst, static_cast<cudaStream_t>(stream)));
+}
+
 pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error) {
   if (!cache || !cache->error || !host_error) return PNMIX_ERR_INVALID_ARG;
   cudaError_t e = cudaMemcpy(host_error, cache->error, sizeof(uint32_t), cudaMemcpyDeviceToHost);

@@ -139,3 +139,32 @@ def test_multi_query_entry_rejects_bad_arguments_before_launching():
                                           None) == pm.ERR_INVALID_ARG
     assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 2, ctypes.byref(c), 256, P, P, ws - 1,
                                           None) == pm.ERR_CAPACITY
+
+
+def _fake_cache_at(cfg, base, B=2, cap=256):
+    c = pm.Cache()
+    nbytes = pm.cache_bytes(cfg, B, cap)
+    assert pm._lib.pnmix_cache_init(ctypes.byref(cfg), B, cap, ctypes.c_void_p(base), nbytes,
+                                    ctypes.byref(c)) == pm.OK
+    return c
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_shrink_entry_rejects_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2, key_bits_hi=4, key_bits_lo=2, n_salient_pairs=8)
+    small = cfg.without_salient()
+    assert small.n_salient_pairs == 0 and cfg.n_salient_pairs == 8
+    src = _fake_cache_at(cfg, 1 << 40)
+    dst = _fake_cache_at(small, 1 << 42)
+    L = pm._lib
+    # the destination must have the no-salient layout, its own memory, the same shape
+    assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(src), None) == pm.ERR_INVALID_ARG
+    same = _fake_cache_at(small, 1 << 40)
+    assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(same), None) == pm.ERR_INVALID_ARG
+    wide = _fake_cache_at(small, 1 << 42, cap=512)
+    assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(wide), None) == pm.ERR_INVALID_ARG
+    assert L.pnmix_shrink_keys(ctypes.byref(cfg), None, ctypes.byref(dst), None) == pm.ERR_INVALID_ARG
+    # there must be salient pairs to shrink (both supported bit pairs have b_hi = 2 b_lo)
+    s0 = _fake_cache_at(small, 1 << 40)
+    assert L.pnmix_shrink_keys(ctypes.byref(small), ctypes.byref(s0), ctypes.byref(dst), None) == pm.ERR_UNSUPPORTED

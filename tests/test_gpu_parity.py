@@ -255,3 +255,47 @@ def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T
         got, want = c.attend_multi(c.query_multi(L, T))
         got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
     assert_close(got, want)
+
+
+# Bit-width shrinking of the salient keys (the PM-KVQ review page's equivalent right shift):
+# the shrunk GPU cache is byte-identical to the oracle's, decodes like it, and keeps taking
+# appends in the no-salient layout.
+@pytest.mark.parametrize("kernel", [None, "mma", "ws"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", [
+    (2, 8, 2, 300, 8, 4, 2),
+    (1, 28, 4, 517, 32, 4, 2),
+    (2, 16, 2, 200, 16, 2, 1),
+    (1, 8, 1, 64, 64, 4, 2),
+    (1, 4, 1, 20, 8, 4, 2),     # no full group yet: only the residual window carries over
+])
+def test_shrunk_cache_matches_the_oracle_and_decodes_like_it(kernel, B, Hq, Hkv, L, k, bhi, blo,
+                                                              monkeypatch):
+    if kernel:
+        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+    extra = 40
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + 3 * k, extra_tokens=extra)
+    c.prefill()
+    small = c.cache.shrunk()
+    want = c.ocache.shrunk()
+    torch.cuda.synchronize()
+    assert small.c.record_bytes < c.cache.c.record_bytes
+    ng = L // 32
+    np.testing.assert_array_equal(small.records().cpu().numpy()[:, :, :ng], want.records[:, :, :ng])
+    np.testing.assert_array_equal(small.lengths().cpu().numpy(), want.len)
+    np.testing.assert_array_equal(small.perm().cpu().numpy(), want.perm)
+    np.testing.assert_array_equal(small.pair_scores().cpu().numpy().view(np.uint32), want.scores.view(np.uint32))
+    assert not small.pair_mask().cpu().numpy().any()
+    r = L % 32
+    np.testing.assert_array_equal(small.resid("k").cpu().numpy().view(np.uint16)[:, :, :r], want.resid_k[:, :, :r])
+    q = c.query(L)
+    assert_close(small.attend(to_dev(q)).cpu().numpy(), want.attend(q))
+    for t in range(L, L + extra):
+        kn = np.ascontiguousarray(c.kin[:, :, t])
+        vn = np.ascontiguousarray(c.vin[:, :, t])
+        small.append(to_dev(kn), to_dev(vn))
+        want.append(kn, vn)
+    torch.cuda.synchronize()
+    ng = (L + extra) // 32
+    np.testing.assert_array_equal(small.records().cpu().numpy()[:, :, :ng], want.records[:, :, :ng])
+    q = c.query(L + extra)
+    assert_close(small.attend(to_dev(q)).cpu().numpy(), want.attend(q))
