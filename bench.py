@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--pipeline-layers-generated", type=int, default=4,
                     help="pipeline_32l: layers whose prefill inputs are generated (seed + layer); "
                          "the others reuse them cyclically")
+    ap.add_argument("--shrunk-only", action="store_true",
+                    help="sweep_128k: run only the points whose cache was shrunk (pnmix_shrink_keys)")
     ap.add_argument("--profile-decode", action="store_true",
                     help="build the 32K state, then run only --warmup + --steps decode launches "
                          "(small device footprint, for profiler captures); prints no bench line")
@@ -380,6 +382,8 @@ def run_decode_workload(args):
                    (workload.BitPoint(2, 1, 16), 1, 0, False), (workload.BitPoint(2, 1, 16), 2, 0, False),
                    (workload.BitPoint(4, 2, 8), 0, 26, False),
                    (workload.BitPoint(4, 2, 8), 0, 0, True), (workload.BitPoint(2, 1, 16), 0, 0, True)]
+        if args.shrunk_only:
+            points = [p_ for p_ in points if p_[3]]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     kin = workload.rows(args.seed, workload.K, Bw, Hkv, 0, ctx)
@@ -405,11 +409,23 @@ def run_decode_workload(args):
             src = pm.PNMixCache(qcfg, Bw, ctx + 32, max_context=ctx)
             src.prefill(qwin_dev, k_dev, v_dev, ctx)
             n_rep = max(3, -(-3 * l2_bytes // pm.cache_bytes(cfg, Bw, ctx + 32)))
-            shrink_us = None
+            shrink_us = shrink_gbs = None
             if shrink:
                 replicas = [src.shrunk() for _ in range(n_rep)]
-                shrink_us = timed_rotation([lambda: pm.pnmix_shrink_keys(qcfg, src, replicas[0])],
-                                           max(args.steps, 5), args.warmup) * 1e6
+                # one shrink reads every source record and writes every destination record,
+                # and copies both residual windows
+                ng = ctx // 32
+                shrink_bytes = Bw * Hkv * (ng * (src.c.record_bytes + replicas[0].c.record_bytes)
+                                           + 2 * 2 * 32 * D * 2)
+                # two sources alternate and the destinations rotate, so each launch finds
+                # neither its source nor its destination in L2
+                src2 = pm.PNMixCache(qcfg, Bw, ctx + 32, max_context=ctx)
+                src2.prefill(qwin_dev, k_dev, v_dev, ctx)
+                sfns = [(lambda s_=(src, src2)[i % 2], d_=r_: pm.pnmix_shrink_keys(qcfg, s_, d_))
+                        for i, r_ in enumerate(replicas + replicas[:1] if n_rep % 2 else replicas)]
+                t_s = timed_rotation(sfns, max(args.steps, 2 * len(sfns)), args.warmup)
+                del src2
+                shrink_us, shrink_gbs = t_s * 1e6, shrink_bytes / t_s / 1e9
                 pm.pnmix_shrink_keys(qcfg, src, replicas[0])
                 del src
             else:
@@ -428,6 +444,7 @@ def run_decode_workload(args):
             r = {"key_bits": [bp.key_bits_hi, bp.key_bits_lo], "salient_pairs": bp.n_salient_pairs,
                  "saliency_score": ["pair-norm product", "key only", "key range x query"][score],
                  "pruned_query_pairs": prune, "shrunk_to_low_bits": shrink, "shrink_us": shrink_us,
+                 "shrink_gbs": shrink_gbs,
                  "key_code_bits": bp.key_bits_lo if shrink else bp.key_code_bits,
                  "bytes_per_token_head": cache.c.record_bytes / 32,
                  "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,

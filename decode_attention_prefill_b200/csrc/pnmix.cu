@@ -312,7 +312,8 @@ pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_cache* src, 
   if ((st = make_geometry(&small, src->batch, src->capacity_tokens, &gd)) != PNMIX_OK) return st;
   if (dst->batch != src->batch || dst->capacity_tokens != src->capacity_tokens) return PNMIX_ERR_INVALID_ARG;
   if ((st = check_cache(gd, dst)) != PNMIX_OK) return st;
-  if (dst->base == src->base) return PNMIX_ERR_INVALID_ARG;
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src->base), d0 = reinterpret_cast<uintptr_t>(dst->base);
+  if (s0 < d0 + dst->total_bytes && d0 < s0 + src->total_bytes) return PNMIX_ERR_INVALID_ARG;   // overlap
   return cuda_status(launch_shrink(gs, gd, *src, *dst, static_cast<cudaStream_t>(stream)));
 }
 

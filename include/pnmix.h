@@ -323,16 +323,22 @@ PNMIX_API pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, con
 
 /*
  * Shrink the salient key positions of a cache from b_hi to b_lo = b_hi / 2 bits (the
- * equivalent right shift of the PM-KVQ review page: the bit-width shrinking step of its
- * progressive quantization).  src holds a cache of cfg (key_bits_hi = 2 * key_bits_lo,
- * n_salient_pairs > 0); dst must be a distinct cache of the same batch and capacity laid
- * out for cfg with n_salient_pairs = 0.  Every full group record of src is written to dst
- * with all positions at b_lo bits in the SAME position order: for positions [0, 2k) the
- * code X becomes ((2^(2b) - 2^b + 1) * (X + 2^(b-1))) >> 3b with b = b_lo (which is
- * round(X / (2^b + 1))) and the scale fp16(fl(s * (2^b + 1))); zero points, the other
- * positions, the value part, the residual window, len, perm and pair_scores are copied,
- * pair_idx and pair_mask cleared.  Decode dst with the n_salient_pairs = 0 config (its
- * records are record_bytes(cfg) - 128 * WH_hi + 128 * WH_lo bytes).
+ * equivalent right shift of the PM-KVQ review page, "key_machinery": the bit-width
+ * shrinking step of its progressive quantization).
+ *   cfg  the configuration src was built with (key_bits_hi = 2 * key_bits_lo, which holds
+ *        for both supported pairs, and n_salient_pairs > 0).
+ *   src  a cache of cfg; read only.
+ *   dst  a cache of the same batch and capacity laid out for cfg with n_salient_pairs = 0
+ *        (pnmix_cache_init with that config), in memory that does not overlap src's.
+ * Every full group record of src is written to dst with all positions at b_lo bits in the
+ * SAME position order: for positions [0, 2k) the code X becomes
+ * ((2^(2b) - 2^b + 1) * (X + 2^(b-1))) >> 3b with b = b_lo, which is round(X / (2^b + 1)),
+ * and the scale becomes fp16(fl(s * (2^b + 1))); zero points, the other positions, the value
+ * part, the residual window, len, perm and pair_scores are copied, and pair_idx and
+ * pair_mask cleared.  Decode dst with the n_salient_pairs = 0 config.  One launch on
+ * `stream`, asynchronous.  Errors: INVALID_ARG for null pointers, a dst of another shape
+ * or layout, or overlapping caches; UNSUPPORTED for k = 0 or a configuration outside the
+ * supported set; CUDA for a launch failure.
  */
 PNMIX_API pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_cache* src, pnmix_cache* dst,
                                          void* stream);

@@ -162,6 +162,8 @@ def test_shrink_entry_rejects_bad_arguments_before_launching():
     assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(src), None) == pm.ERR_INVALID_ARG
     same = _fake_cache_at(small, 1 << 40)
     assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(same), None) == pm.ERR_INVALID_ARG
+    tail = _fake_cache_at(small, (1 << 40) + pm.cache_bytes(cfg, 2, 256) - 256)   # overlaps src's end
+    assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(tail), None) == pm.ERR_INVALID_ARG
     wide = _fake_cache_at(small, 1 << 42, cap=512)
     assert L.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(wide), None) == pm.ERR_INVALID_ARG
     assert L.pnmix_shrink_keys(ctypes.byref(cfg), None, ctypes.byref(dst), None) == pm.ERR_INVALID_ARG
