@@ -173,8 +173,6 @@ cudaError_t launch_quantize_values(const Geometry& g, const uint16_t* v, int L, 
                                    const pnmix_cache& c, cudaStream_t s);
 cudaError_t launch_append(const Geometry& g, const uint16_t* k_new, const uint16_t* v_new,
                           const pnmix_cache& c, cudaStream_t s);
-cudaError_t launch_shrink(const Geometry& gs, const Geometry& gd, const pnmix_cache& src,
-                          const pnmix_cache& dst, cudaStream_t s);
 
 // Decode: the workspace a batch / context bound needs, and the launch.
 size_t decode_workspace_bytes(const Geometry& g, int max_context);

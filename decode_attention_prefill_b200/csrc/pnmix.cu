@@ -135,6 +135,10 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   }
 }
 
+// csrc/shrink.cu: salient keys from b_hi to b_lo bits, src geometry gs -> dst geometry gd.
+cudaError_t launch_shrink(const Geometry& gs, const Geometry& gd, const pnmix_cache& src,
+                          const pnmix_cache& dst, cudaStream_t s);
+
 }  // namespace pnmix
 
 using namespace pnmix;
