@@ -144,6 +144,28 @@ def test_sweep_128k_bit_points(k, bhi, blo):
     assert_close(got, want)
 
 
+@pytest.mark.slow
+def test_stream_32k_full_size_every_append_through_the_abi():
+    """Batch 16, 32/8 heads: prefill 4096, then 28672 single-token appends through the C ABI
+    up to 32768 tokens.  Appending folds each full residual window with the salient set
+    fixed at prefill, so the oracle's state is its bulk quantization of the 32768 tokens
+    under that set: every record, residual row and length equal it byte for byte, and the
+    decode step at 32768 (the launch the streaming benchmark times) matches on every head."""
+    T0, T = 4096, 32768
+    c = Case(16, 32, 8, T0, seed=0, extra_tokens=T - T0)
+    c.prefill(check=False)
+    kt = c.k_dev.permute(2, 0, 1, 3).contiguous()     # [token][B][Hkv][128]
+    vt = c.v_dev.permute(2, 0, 1, 3).contiguous()
+    for t in range(T0, T):
+        c.cache.append(kt[t], vt[t])
+    del kt, vt
+    c.ocache.prefill(c.kin, c.vin, T)
+    c.check_state()
+    assert c.cache.read_error() == 0
+    got, want = c.attend(c.query(T))
+    assert_close(got, want)
+
+
 def test_context_hint_smaller_than_the_cache_still_covers_every_token():
     """The grid is sized from max_context; a smaller hint gives fewer CTAs, never fewer tokens."""
     import decode_attention_prefill_b200 as pm
