@@ -71,7 +71,7 @@ decode_simt_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, fl
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& s) {
     const int b = s.b, h = s.h, unit = s.unit;
-    perm_s[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid];
+    perm_s[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid] & (kHeadDim - 1);
     __syncthreads();
     const float qscale = g.scale * 1.4426950408889634f;   // logits in the log2 domain
     for (int i = tid; i < G * kHeadDim; i += kThreads) {

@@ -193,7 +193,7 @@ quantize_prefill_kernel(Geometry g, const uint16_t* __restrict__ x, int L, int l
     copy_tail(src, ng * kGroup, L, resid);
     return;
   }
-  if (kKeys) sm.perm[threadIdx.x] = c.perm[unit_index(g, b, h) * kHeadDim + threadIdx.x];
+  if (kKeys) sm.perm[threadIdx.x] = c.perm[unit_index(g, b, h) * kHeadDim + threadIdx.x] & (kHeadDim - 1);
   load_tile(sm, src + static_cast<size_t>(grp) * kGroup * kHeadDim, kHeadDim);
   __syncthreads();
   uint8_t* rec = record_ptr(g, c.records, b, h, grp);
@@ -213,7 +213,7 @@ append_kernel(Geometry g, const uint16_t* __restrict__ k_new, const uint16_t* __
   __shared__ GroupSmem sm;
   const int h = blockIdx.x, b = blockIdx.y;
   const int n = c.len[b];
-  if (n >= g.capacity) {
+  if (n < 0 || n >= g.capacity) {
     if (h == 0 && threadIdx.x == 0) atomicOr(c.error, PNMIX_DEVERR_APPEND_FULL);
     return;
   }
@@ -231,7 +231,7 @@ append_kernel(Geometry g, const uint16_t* __restrict__ k_new, const uint16_t* __
   if (slot == kGroup - 1) {
     __syncthreads();
     uint8_t* rec = record_ptr(g, c.records, b, h, n / kGroup);
-    sm.perm[threadIdx.x] = c.perm[u * kHeadDim + threadIdx.x];
+    sm.perm[threadIdx.x] = c.perm[u * kHeadDim + threadIdx.x] & (kHeadDim - 1);
     for (int i = threadIdx.x; i < kGroup * 16; i += kThreads) {
       int r = i >> 4, cc = i & 15;
       *reinterpret_cast<uint4*>(&sm.tile[r][cc * 8]) = reinterpret_cast<const uint4*>(rk + r * kHeadDim)[cc];

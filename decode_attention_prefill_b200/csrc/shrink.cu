@@ -92,7 +92,8 @@ shrink_kernel(Geometry gs, Geometry gd, pnmix_cache src, pnmix_cache dst) {
     if (threadIdx.x == 0) dst.pair_mask[u] = 0;
     if (threadIdx.x == 0 && h == 0) dst.len[b] = src.len[b];
   }
-  if (grp >= src.len[b] / kGroup) return;
+  const int n = src.len[b];
+  if (grp >= (n < 0 ? 0 : (n > gs.capacity ? gs.capacity : n)) / kGroup) return;
   const uint32_t* ws = reinterpret_cast<const uint32_t*>(record_ptr(gs, src.records, b, h, grp));
   uint32_t* wd = reinterpret_cast<uint32_t*>(record_ptr(gd, dst.records, b, h, grp));
   // ---- key words: the salient block shrinks, the low block moves down unchanged.  All

@@ -35,6 +35,12 @@
  *  - Conditions only the device can see (a full cache on append, a bounded wait
  *    that ran out) set bits in the cache's device error word; read it with
  *    pnmix_read_error.  No kernel traps or asserts.
+ *  - A cache's device state (lengths, permutation, records) is valid only once
+ *    pnmix_cache_reset has run on it, and is kept valid by these calls alone: the
+ *    caller orders every call after the work it depends on (the zero fill and reset
+ *    of the cache memory included) when it uses more than one stream.  The decode
+ *    kernels take the lengths as they find them; append and shrink clamp them to
+ *    [0, capacity], and the quantizers mask permutation entries to a channel index.
  *  - head_dim is 128; rows of K, V and Q are 128 contiguous bf16 values.
  *
  * Numerical contract
