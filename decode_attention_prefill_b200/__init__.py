@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_PKG, "libpnmix.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m decode_attention_prefill_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python decode_attention_prefill_b200/build.py` "
         "(there is no fallback implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)
