@@ -78,6 +78,10 @@ def lib():
                 "orc_attend_unit": (i, [i, vp, d, i, i, i, vp, vp, i, vp, vp, i, vp, vp, vp]),
                 "orc_exact_attention": (None, [i, vp, vp, vp, ctypes.c_long, d, vp]),
                 "orc_key_code_bits": (d, [i, i, i]),
+                "orc_mean_query": (None, [i, i, vp, vp]),
+                "orc_group_scores": (None, [vp, i, vp, vp]),
+                "orc_route_groups": (None, [i, vp, i, vp]),
+                "orc_attend_two": (i, [i, vp, d, i, i, i, vp, vp, i, i, vp, vp, i, vp, vp, i, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -370,6 +374,104 @@ class Cache:
         out = np.full((B, Hq, 128), np.nan)
         for b, h in heads or [(b, h) for b in range(B) for h in range(self.n_kv)]:
             out[b, h * G:(h + 1) * G] = self.attend_unit(q[b, h * G:(h + 1) * G], b, h)
+        return out
+
+
+# ---------------------------------------------------------------- two-precision mixing
+# SemKV abstract (token-level mixing of two adjacent precisions by a model-internal
+# rank), with 32-token groups as the unit and two salient-pair counts as the precisions.
+
+def mean_query(qwin_unit: np.ndarray) -> np.ndarray:
+    """qwin_unit bf16 [G][W][128] -> fp32 [128] (orc_mean_query)."""
+    q = np.ascontiguousarray(qwin_unit, dtype=np.uint16)
+    out = np.zeros(128, np.float32)
+    lib().orc_mean_query(q.shape[0], q.shape[1], _p(q), _p(out))
+    return out
+
+
+def group_scores(qbar: np.ndarray, k_unit: np.ndarray, L: int) -> np.ndarray:
+    """Largest mean-query logit of each full 32-token group of k_unit (bf16 [>=L][128])."""
+    kk = np.ascontiguousarray(k_unit[:L], dtype=np.uint16)
+    qb = np.ascontiguousarray(qbar, dtype=np.float32)
+    out = np.zeros(max(L // 32, 1), np.float32)
+    lib().orc_group_scores(_p(qb), L, _p(kk), _p(out))
+    return out[:L // 32]
+
+
+def route_groups(scores: np.ndarray, n_hi: int) -> np.ndarray:
+    """uint8 [ng]: 1 for the n_hi best-ranked groups (ties: lower index first)."""
+    sc = np.ascontiguousarray(scores, dtype=np.float32)
+    out = np.zeros(max(len(sc), 1), np.uint8)
+    lib().orc_route_groups(len(sc), _p(sc), n_hi, _p(out))
+    return out[:len(sc)]
+
+
+def hi_groups(ng: int, percent: int) -> int:
+    """Groups of a unit at the high precision: floor(ng * percent / 100)."""
+    return ng * percent // 100
+
+
+class TwoPrecision:
+    """Host image of a two-precision cache: per (sequence, KV head) the full groups of the
+    prefill are ranked by group_scores of the saliency window's mean query; the best
+    hi_groups(ng, percent) of them are quantized with k_hi salient pairs into `hi`, the
+    others with k_lo into `lo`, each part in ascending group order.  The residual tail
+    and every appended token go to `lo`.  Both parts take their salient pairs from the
+    same prefill statistic (top k_hi and top k_lo of one score vector)."""
+
+    def __init__(self, batch, n_kv, capacity, k_hi, k_lo, bhi, blo, percent, score=SCORE_PNMIX):
+        if not 0 <= percent <= 100:
+            raise ValueError("percent outside [0, 100]")
+        self.batch, self.n_kv, self.percent = batch, n_kv, percent
+        self.hi = Cache(batch, n_kv, capacity, k_hi, bhi, blo, score=score)
+        self.lo = Cache(batch, n_kv, capacity, k_lo, bhi, blo, score=score)
+        self.route = np.zeros((batch, n_kv, capacity // 32), np.uint8)
+
+    def prefill(self, qwin: np.ndarray, kin: np.ndarray, vin: np.ndarray, L: int):
+        """qwin bf16 [B][Hq][W][128] (the saliency window); kin, vin bf16 [B][Hkv][>=L][128]."""
+        self.hi.select(qwin, kin, L)
+        self.lo.select(qwin, kin, L)
+        G = qwin.shape[1] // self.n_kv
+        ng = L // 32
+        n_hi = hi_groups(ng, self.percent)
+        for b in range(self.batch):
+            for h in range(self.n_kv):
+                qbar = mean_query(qwin[b, h * G:(h + 1) * G])
+                route = route_groups(group_scores(qbar, kin[b, h], L), n_hi)
+                self.route[b, h, :ng] = route
+                for part, take in ((self.hi, 1), (self.lo, 0)):
+                    rows = [np.arange(32 * g, 32 * g + 32) for g in range(ng) if route[g] == take]
+                    if take == 0:
+                        rows.append(np.arange(32 * ng, L))
+                    idx = np.concatenate(rows) if rows else np.zeros(0, np.int64)
+                    kk = np.ascontiguousarray(kin[b, h, idx], dtype=np.uint16)
+                    vv = np.ascontiguousarray(vin[b, h, idx], dtype=np.uint16)
+                    rc = lib().orc_prefill_unit(part.k, part.bhi, part.blo, part.bv, _p(part.perm[b, h]),
+                                                len(idx), _p(kk), _p(vv), _p(part.records[b, h]),
+                                                _p(part.resid_k[b, h]), _p(part.resid_v[b, h]))
+                    assert rc == 0
+            self.hi.len[b] = 32 * n_hi
+            self.lo.len[b] = L - 32 * n_hi
+
+    def append(self, knew: np.ndarray, vnew: np.ndarray):
+        self.lo.append(knew, vnew)
+
+    def attend(self, q: np.ndarray, heads=None) -> np.ndarray:
+        """q bf16 [B][Hq][128] -> fp64 [B][Hq][128]: softmax over both parts' tokens."""
+        B, Hq, _ = q.shape
+        G = Hq // self.n_kv
+        hi, lo = self.hi, self.lo
+        out = np.full((B, Hq, 128), np.nan)
+        for b, h in heads or [(b, h) for b in range(B) for h in range(self.n_kv)]:
+            qq = np.ascontiguousarray(q[b, h * G:(h + 1) * G], dtype=np.uint16)
+            o = np.zeros((G, 128), np.float64)
+            n_lo = int(lo.len[b])
+            rc = lib().orc_attend_two(G, _p(qq), 1.0 / np.sqrt(128.0), hi.bhi, hi.blo,
+                                      hi.k, _p(hi.perm[b, h]), _p(hi.records[b, h]), int(hi.len[b]) // 32,
+                                      lo.k, _p(lo.perm[b, h]), _p(lo.records[b, h]), n_lo // 32,
+                                      _p(lo.resid_k[b, h]), _p(lo.resid_v[b, h]), n_lo % 32, _p(o))
+            assert rc == 0
+            out[b, h * G:(h + 1) * G] = o
         return out
 
 

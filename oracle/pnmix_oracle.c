@@ -35,7 +35,10 @@
  * inputs with ties, outlier-union selection on the tiny workload, grid-exact
  * round trips, the s/2 round-trip bound, half-even ties, code-bit accounting,
  * fp16 rounding against numpy, layout bijection, append == bulk prefill, and
- * the 16-bit pass-through reducing to plain softmax attention.
+ * the 16-bit pass-through reducing to plain softmax attention; for the two-
+ * precision mixing: exact means of identical rows, exact integer group scores,
+ * the route against a stable sort, and the union of two equal-precision parts
+ * against one cache.
  */
 #include <math.h>
 #include <stdint.h>
@@ -747,4 +750,106 @@ double orc_key_code_bits(int k, int bhi, int blo) {
   long R = orc_record_bytes(k, bhi, blo);
   if (!R) return 0.0;
   return (double)(R - 2048) * 8.0 / (32.0 * 128.0);
+}
+
+/* ------------------------------------------------------------------ */
+/* Token-level two-precision mixing (SemKV).                           */
+/* ------------------------------------------------------------------ */
+/*
+ * "SemKV: Semantic Mixed-Precision KV Cache Quantization Guided by the Quality Cliff for
+ * Long-Context LLM Inference", abstract: every token is kept, tokens are ranked by a
+ * model-internal score, and two adjacent precisions are assigned by rank.  In this path
+ * the unit of assignment is a 32-token group (its tokens share the per-channel key
+ * statistics), the two precisions are two salient-pair counts k_hi > k_lo of the same bit
+ * pair, and the score of a group is the largest logit that the mean query of the saliency
+ * window gives one of its tokens.
+ */
+
+/*
+ * Mean query of one KV head's saliency window: qbar[c] = (sum_h sum_t q[h][t][c]) / (G*W),
+ * heads outer, tokens inner, one fp32 rounding per operation.  qwin: bf16 [G][W][128].
+ */
+void orc_mean_query(int G, int W, const uint16_t* qwin, float* qbar) {
+  for (int c = 0; c < 128; ++c) {
+    float s = 0.0f;
+    for (int h = 0; h < G; ++h)
+      for (int t = 0; t < W; ++t) s = s + orc_f32_from_bf16(qwin[((size_t)h * W + t) * 128 + c]);
+    qbar[c] = s / (float)(G * W);
+  }
+}
+
+/*
+ * Group scores of the L / 32 full groups of k (bf16 [L][128]):
+ *   l_t = sum_c qbar[c] * k[t][c], channels 0..127 in order, one fp32 rounding per
+ *         product and per sum;
+ *   score[g] = max over t in [32g, 32g + 32) of l_t.
+ */
+void orc_group_scores(const float* qbar, int L, const uint16_t* k, float* score) {
+  for (int g = 0; g < L / 32; ++g) {
+    float best = -INFINITY;
+    for (int t = 32 * g; t < 32 * g + 32; ++t) {
+      float acc = 0.0f;
+      for (int c = 0; c < 128; ++c) {
+        float p = qbar[c] * orc_f32_from_bf16(k[(size_t)t * 128 + c]);
+        acc = acc + p;
+      }
+      if (acc > best) best = acc;
+    }
+    score[g] = best;
+  }
+}
+
+/*
+ * Route of ng groups: group g ranks r_g = #{g' : score[g'] > score[g], or equal with
+ * g' < g}; it takes the high precision (route[g] = 1) when r_g < n_hi, else 0.
+ */
+void orc_route_groups(int ng, const float* score, int n_hi, uint8_t* route) {
+  for (int g = 0; g < ng; ++g) {
+    int r = 0;
+    for (int o = 0; o < ng; ++o)
+      if (score[o] > score[g] || (score[o] == score[g] && o < g)) ++r;
+    route[g] = (uint8_t)(r < n_hi);
+  }
+}
+
+/*
+ * Decode attention of one (b, KV head) over a two-precision cache: the G query rows q
+ * (bf16 [G][128]) attend over the union of the n_hi records of the high-precision part
+ * (k_hi salient pairs, permutation perm_hi), the n_lo records of the low-precision part
+ * (k_lo, perm_lo) and the n_resid bf16 residual rows: plain softmax attention over all
+ * of these tokens (its value does not depend on their order).
+ */
+int orc_attend_two(int G, const uint16_t* q, double scale, int bhi, int blo, int k_hi,
+                   const uint8_t* perm_hi, const uint8_t* rec_hi, int n_hi, int k_lo,
+                   const uint8_t* perm_lo, const uint8_t* rec_lo, int n_lo,
+                   const uint16_t* resid_k, const uint16_t* resid_v, int n_resid, double* out) {
+  long Rh = orc_record_bytes(k_hi, bhi, blo), Rl = orc_record_bytes(k_lo, bhi, blo);
+  if (!Rh || !Rl || G > 8) return 1;
+  long n = (long)(n_hi + n_lo) * 32 + n_resid;
+  double* khat = (double*)malloc(sizeof(double) * 128 * (size_t)(n > 0 ? n : 1));
+  double* vhat = (double*)malloc(sizeof(double) * 128 * (size_t)(n > 0 ? n : 1));
+  double qd[8 * 128];
+  if (!khat || !vhat) {
+    free(khat);
+    free(vhat);
+    return 2;
+  }
+  for (int i = 0; i < G * 128; ++i) qd[i] = (double)orc_f32_from_bf16(q[i]);
+  for (int g = 0; g < n_hi; ++g)
+    orc_dequant_record(k_hi, bhi, blo, perm_hi, rec_hi + (size_t)g * Rh, khat + (size_t)g * 4096,
+                       vhat + (size_t)g * 4096);
+  for (int g = 0; g < n_lo; ++g)
+    orc_dequant_record(k_lo, bhi, blo, perm_lo, rec_lo + (size_t)g * Rl,
+                       khat + (size_t)(n_hi + g) * 4096, vhat + (size_t)(n_hi + g) * 4096);
+  for (int r = 0; r < n_resid; ++r) {
+    long t = (long)(n_hi + n_lo) * 32 + r;
+    for (int c = 0; c < 128; ++c) {
+      khat[t * 128 + c] = (double)orc_f32_from_bf16(resid_k[r * 128 + c]);
+      vhat[t * 128 + c] = (double)orc_f32_from_bf16(resid_v[r * 128 + c]);
+    }
+  }
+  orc_attention_core(G, qd, khat, vhat, n, scale, out);
+  free(khat);
+  free(vhat);
+  return 0;
 }

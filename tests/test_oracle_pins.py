@@ -757,3 +757,118 @@ def test_shrinking_codes_on_the_coarse_grid_changes_nothing(bhi, blo, k):
         b2 = oracle.unpack_record(0, bhi, blo, small.records[0, 0, g])[0]
         np.testing.assert_array_equal(a[:, nhi:], b2[:, nhi:])
         np.testing.assert_array_equal(b2[:, :nhi], a[:, :nhi] // d)
+
+
+# ------------------------------------------------------------------ two-precision mixing
+
+@pytest.mark.parametrize("G,W", [(4, 64), (7, 64), (1, 3)])
+def test_mean_query_of_identical_rows_is_that_row(G, W):
+    """G*W copies of one bf16 row: each partial sum n*x needs at most 8 + 10 significant
+    bits, so every fp32 sum is exact and the mean is the row itself."""
+    rng = np.random.default_rng(G * W)
+    row = bf16_bits(np.round(rng.standard_normal(128) * 64) / 64)
+    qwin = np.broadcast_to(row, (G, W, 128))
+    qbar = oracle.mean_query(qwin)
+    np.testing.assert_array_equal(qbar, oracle.bf16_to_f32(row))
+
+
+def test_group_scores_are_the_exact_integer_maxima_on_small_integers():
+    """Integer queries and keys small enough that every product and partial sum is an
+    exact fp32 integer: the scores equal the maxima of exact integer dot products."""
+    rng = np.random.default_rng(5)
+    L = 32 * 5 + 7                                    # five full groups and a ragged tail
+    qrow = rng.integers(-8, 9, 128)
+    qwin = np.broadcast_to(bf16_bits(qrow.astype(np.float32)), (2, 4, 128))
+    k = rng.integers(-16, 17, (L, 128))
+    scores = oracle.group_scores(oracle.mean_query(qwin), bf16_bits(k.astype(np.float32)), L)
+    logits = k.astype(np.int64) @ qrow.astype(np.int64)
+    want = logits[:32 * 5].reshape(5, 32).max(axis=1)
+    assert scores.shape == (5,)
+    np.testing.assert_array_equal(scores, want.astype(np.float32))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_route_takes_the_first_n_of_a_stable_descending_sort(seed):
+    rng = np.random.default_rng(seed)
+    ng = 40
+    scores = rng.integers(-5, 6, ng).astype(np.float32)   # many ties
+    for n_hi in (0, 1, 13, 39, 40):
+        route = oracle.route_groups(scores, n_hi)
+        order = np.argsort(-scores, kind="stable")       # equal scores keep index order
+        want = np.zeros(ng, np.uint8)
+        want[order[:n_hi]] = 1
+        np.testing.assert_array_equal(route, want)
+
+
+def _two_precision_case(seed, L, k_hi, k_lo, percent, B=2, Hq=8, Hkv=2):
+    G = Hq // Hkv
+    kin = workload.rows(seed, workload.K, B, Hkv, 0, L)
+    vin = workload.rows(seed, workload.V, B, Hkv, 0, L)
+    qwin = workload.rows(seed, workload.Q, B, Hq, L - min(L, 64), min(L, 64), group=G)
+    q = workload.rows(seed, workload.Q, B, Hq, L, 1, group=G)[:, :, 0]
+    cap = (L + 31) // 32 * 32 + 32
+    two = oracle.TwoPrecision(B, Hkv, cap, k_hi, k_lo, 4, 2, percent)
+    two.prefill(qwin, kin, vin, L)
+    return two, kin, vin, qwin, q, cap
+
+
+@pytest.mark.parametrize("L,percent", [(300, 50), (517, 25), (64, 100), (100, 0)])
+def test_two_precision_with_equal_precisions_is_the_single_cache_attention(L, percent):
+    """With k_hi == k_lo both parts hold the same records a single cache holds, only
+    reordered; softmax attention does not depend on the order, so the union equals the
+    single cache's attention (up to binary64 summation order)."""
+    two, kin, vin, qwin, q, cap = _two_precision_case(L + percent, L, 8, 8, percent)
+    one = oracle.Cache(2, 2, cap, 8, 4, 2)
+    one.select(qwin, kin, L)
+    one.prefill(kin, vin, L)
+    np.testing.assert_allclose(two.attend(q), one.attend(q), rtol=0, atol=1e-12)
+    ng = L // 32
+    assert int(two.route[0, 0, :ng].sum()) == ng * percent // 100
+    assert two.hi.len[0] + two.lo.len[0] == L
+
+
+def test_two_precision_parts_hold_each_group_at_its_own_precision():
+    """Record i of the high part is the i-th routed group quantized with k_hi salient pairs,
+    record j of the low part the j-th other group with k_lo, and the low part's residual
+    holds the ragged tail; the routed groups are the best-scored ones."""
+    L = 32 * 9 + 5
+    two, kin, vin, qwin, q, cap = _two_precision_case(3, L, 16, 8, 40)
+    ng = L // 32
+    for b in range(2):
+        for h in range(2):
+            route = two.route[b, h, :ng]
+            hi_g = [g for g in range(ng) if route[g]]
+            lo_g = [g for g in range(ng) if not route[g]]
+            assert len(hi_g) == ng * 40 // 100
+            qbar = oracle.mean_query(qwin[b, h * 4:(h + 1) * 4])
+            sc = oracle.group_scores(qbar, kin[b, h], L)
+            assert min(sc[hi_g]) >= max(sc[lo_g])
+            for part, groups in ((two.hi, hi_g), (two.lo, lo_g)):
+                for i, g in enumerate(groups):
+                    rec = np.zeros(part.R, np.uint8)
+                    rc = oracle.lib().orc_make_record(
+                        part.k, 4, 2, 2, oracle._p(part.perm[b, h]),
+                        oracle._p(np.ascontiguousarray(kin[b, h, 32 * g:32 * g + 32])),
+                        oracle._p(np.ascontiguousarray(vin[b, h, 32 * g:32 * g + 32])), oracle._p(rec))
+                    assert rc == 0
+                    np.testing.assert_array_equal(part.records[b, h, i], rec)
+            np.testing.assert_array_equal(two.lo.resid_k[b, h, :L % 32], kin[b, h, 32 * ng:L])
+    assert two.hi.perm[0, 0].tolist() != two.lo.perm[0, 0].tolist()   # 16 vs 8 salient pairs
+
+
+def test_two_precision_mix_lies_between_its_precisions_on_the_tiny_workload():
+    """Relative L2 error against exact attention: the mixed cache is no worse than the
+    low precision alone and no better than the high precision alone, on the tiny
+    single-head workload and its neighbours (the data follow the workload recipe)."""
+    for seed in range(3):
+        L = 512
+        two, kin, vin, qwin, q, cap = _two_precision_case(seed, L, 32, 0, 50, B=1, Hq=1, Hkv=1)
+        exact = oracle.exact_attention(q[0], kin[0, 0], vin[0, 0])
+        errs = {}
+        for name, k in (("hi", 32), ("lo", 0)):
+            c = oracle.Cache(1, 1, cap, k, 4, 2)
+            c.select(qwin, kin, L)
+            c.prefill(kin, vin, L)
+            errs[name] = np.linalg.norm(c.attend(q)[0] - exact) / np.linalg.norm(exact)
+        mix = np.linalg.norm(two.attend(q)[0] - exact) / np.linalg.norm(exact)
+        assert errs["hi"] <= mix <= errs["lo"], (seed, errs, mix)
