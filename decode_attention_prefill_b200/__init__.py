@@ -40,6 +40,7 @@ EXPORTED = [
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
     "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi", "pnmix_shrink_keys",
+    "pnmix_split_groups",
 ]
 
 
@@ -99,6 +100,8 @@ _SIGS = {
     "pnmix_workspace_bytes_multi": (_sz, [_CP, _i, _i, _i]),
     "pnmix_decode_attention_multi": (_i, [_CP, _vp, _i, _KP, _i, _vp, _vp, _sz, _vp]),
     "pnmix_shrink_keys": (_i, [_CP, _KP, _KP, _vp]),
+    "pnmix_split_groups": (_i, [_CP, _i, _vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -211,6 +214,40 @@ def pnmix_shrink_keys(cfg: Config, src: "PNMixCache", dst: "PNMixCache", stream=
     """src: a cache of cfg (b_hi = 2 b_lo, k > 0); dst: a cache of cfg with n_salient_pairs = 0."""
     _check(_lib.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src.c), ctypes.byref(dst.c), _stream(stream)),
            "pnmix_shrink_keys")
+
+
+def split_sizes(L: int, hi_percent: int) -> tuple[int, int]:
+    """(L_hi, L_lo): tokens of the high and low parts of a two-precision prefill."""
+    n_hi = (L // 32) * hi_percent // 100
+    return 32 * n_hi, L - 32 * n_hi
+
+
+def pnmix_split_groups(cfg: Config, q_window: torch.Tensor, k: torch.Tensor, v: torch.Tensor, L: int,
+                       hi_percent: int, stream=None) -> dict:
+    """Rank the 32-token groups of a prefill and split K / V into a high and a low part.
+    q_window bf16 [B][Hq][W'][128]; k, v bf16 [B][Hkv][ld][128].  Returns the device tensors
+    scores fp32 / route uint8 / dest int32 [B][Hkv][L/32] and k_hi, v_hi [B][Hkv][L_hi][128],
+    k_lo, v_lo [B][Hkv][L_lo][128]."""
+    B, Hkv = k.shape[0], k.shape[1]
+    ng = L // 32
+    L_hi, L_lo = split_sizes(L, hi_percent)
+    dev = k.device
+    r = {"scores": torch.empty(B, Hkv, ng, dtype=torch.float32, device=dev),
+         "route": torch.empty(B, Hkv, ng, dtype=torch.uint8, device=dev),
+         "dest": torch.empty(B, Hkv, ng, dtype=torch.int32, device=dev),
+         "k_hi": torch.empty(B, Hkv, L_hi, 128, dtype=torch.bfloat16, device=dev),
+         "v_hi": torch.empty(B, Hkv, L_hi, 128, dtype=torch.bfloat16, device=dev),
+         "k_lo": torch.empty(B, Hkv, L_lo, 128, dtype=torch.bfloat16, device=dev),
+         "v_lo": torch.empty(B, Hkv, L_lo, 128, dtype=torch.bfloat16, device=dev)}
+
+    def ptr(t):
+        return t.data_ptr() if t.numel() else None
+    _check(_lib.pnmix_split_groups(ctypes.byref(cfg), B, _dev(q_window, torch.bfloat16, "q_window"),
+                                   q_window.shape[2], _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
+                                   L, k.shape[2], hi_percent, ptr(r["scores"]), ptr(r["route"]), ptr(r["dest"]),
+                                   ptr(r["k_hi"]), ptr(r["v_hi"]), ptr(r["k_lo"]), ptr(r["v_lo"]),
+                                   _stream(stream)), "pnmix_split_groups")
+    return r
 
 
 # ---------------------------------------------------------------- owner of device buffers

@@ -135,6 +135,12 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   }
 }
 
+// csrc/mix.cu: group scores, route and the split of K / V rows into two parts.
+cudaError_t launch_split_groups(const Geometry& g, const uint16_t* q_window, int nw, const uint16_t* k,
+                                const uint16_t* v, int L, int ld, int n_hi, float* scores, uint8_t* route,
+                                int32_t* dest, uint16_t* k_hi, uint16_t* v_hi, uint16_t* k_lo, uint16_t* v_lo,
+                                cudaStream_t s);
+
 // csrc/shrink.cu: salient keys from b_hi to b_lo bits, src geometry gs -> dst geometry gd.
 cudaError_t launch_shrink(const Geometry& gs, const Geometry& gd, const pnmix_cache& src,
                           const pnmix_cache& dst, cudaStream_t s);
@@ -319,6 +325,32 @@ pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_cache* src, 
   const uintptr_t s0 = reinterpret_cast<uintptr_t>(src->base), d0 = reinterpret_cast<uintptr_t>(dst->base);
   if (s0 < d0 + dst->total_bytes && d0 < s0 + src->total_bytes) return PNMIX_ERR_INVALID_ARG;   // overlap
   return cuda_status(launch_shrink(gs, gd, *src, *dst, static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_split_groups(const pnmix_config* cfg, int batch, const uint16_t* q_window, int n_window,
+                                const uint16_t* k, const uint16_t* v, int L, int ld_tokens, int hi_percent,
+                                float* scores, uint8_t* route, int32_t* dest, uint16_t* k_hi, uint16_t* v_hi,
+                                uint16_t* k_lo, uint16_t* v_lo, void* stream) {
+  if (!cfg || batch < 0 || L < 1 || ld_tokens < L) return PNMIX_ERR_INVALID_ARG;
+  Geometry g;
+  const pnmix_status st = make_geometry(cfg, batch, (L + kGroup - 1) / kGroup * kGroup, &g);
+  if (st != PNMIX_OK) return st;
+  if (!q_window || !k || !v) return PNMIX_ERR_INVALID_ARG;
+  if (hi_percent < 0 || hi_percent > 100) return PNMIX_ERR_INVALID_ARG;
+  const int want_w = L < cfg->saliency_window ? L : cfg->saliency_window;
+  if (n_window != want_w) return PNMIX_ERR_INVALID_ARG;
+  const int ng = L / kGroup;
+  const int n_hi = static_cast<int>(static_cast<long long>(ng) * hi_percent / 100);
+  const int L_hi = kGroup * n_hi, L_lo = L - L_hi;
+  if (ng > 0 && (!scores || !route || !dest)) return PNMIX_ERR_INVALID_ARG;
+  if (L_hi > 0 && (!k_hi || !v_hi)) return PNMIX_ERR_INVALID_ARG;
+  if (L_lo > 0 && (!k_lo || !v_lo)) return PNMIX_ERR_INVALID_ARG;
+  for (const void* p : {static_cast<const void*>(q_window), static_cast<const void*>(k),
+                        static_cast<const void*>(v), static_cast<const void*>(k_hi), static_cast<const void*>(v_hi),
+                        static_cast<const void*>(k_lo), static_cast<const void*>(v_lo)})
+    if (p && !aligned(p, 16)) return PNMIX_ERR_ALIGNMENT;
+  return cuda_status(launch_split_groups(g, q_window, n_window, k, v, L, ld_tokens, n_hi, scores, route, dest,
+                                         k_hi, v_hi, k_lo, v_lo, static_cast<cudaStream_t>(stream)));
 }
 
 pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error) {

@@ -350,6 +350,42 @@ PNMIX_API pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_ca
                                          void* stream);
 
 /*
+ * Token-level two-precision mixing, prefill side ("SemKV: Semantic Mixed-Precision KV
+ * Cache Quantization Guided by the Quality Cliff for Long-Context LLM Inference",
+ * abstract: tokens ranked by a model-internal score take one of two adjacent precisions).
+ * The unit of assignment is a 32-token group.  Per (sequence b, KV head h), with
+ * ng = L / 32 full groups and n_hi = floor(ng * hi_percent / 100):
+ *   qbar[c]  = (sum over the G heads of h and the window tokens of q_window[c]) / (G * W'),
+ *              heads outer, tokens inner, fp32;
+ *   score[g] = max over the tokens t of group g of sum_c qbar[c] * k[t][c] (channels in
+ *              order; every product and sum one fp32 rounding; first maximum kept);
+ *   route[g] = 1 for the n_hi best-ranked groups (score descending, ties: lower g), else 0;
+ *   dest[g]  = the number of groups before g with the same route.
+ * Group g's 32 K and V rows are copied to rows [32 dest[g], 32 dest[g] + 32) of the high
+ * part (route 1) or the low part (route 0); the L mod 32 tail rows end the low part.
+ *   cfg, batch    the configuration and batch of the caches the parts will fill (only its
+ *                 head counts and saliency_window are read here).
+ *   q_window      bf16 [batch][Hq][n_window][128], n_window = min(L, saliency_window), as
+ *                 for pnmix_select_pairs.
+ *   k, v          bf16 [batch][Hkv][ld_tokens][128], tokens [0, L) read.
+ *   hi_percent    0..100.
+ *   scores        fp32 [batch][Hkv][ng], route uint8 [batch][Hkv][ng], dest int32
+ *                 [batch][Hkv][ng]: written (may be NULL when ng = 0).
+ *   k_hi, v_hi    bf16 [batch][Hkv][L_hi][128], L_hi = 32 n_hi (NULL allowed if L_hi = 0).
+ *   k_lo, v_lo    bf16 [batch][Hkv][L_lo][128], L_lo = L - L_hi (NULL allowed if L_lo = 0).
+ * A mixed cache is then two caches: pnmix_select_pairs of each on the full k (its own
+ * n_salient_pairs), and pnmix_quantize_keys / _values of each part with L_hi / L_lo.
+ * Two launches on `stream`; the ranking costs ng^2 comparisons per (b, h).  Errors:
+ * INVALID_ARG (null pointers, L < 1, ld_tokens < L, n_window, hi_percent outside 0..100),
+ * UNSUPPORTED (head counts), ALIGNMENT (bf16 pointers not 16-byte aligned), CUDA.
+ */
+PNMIX_API pnmix_status pnmix_split_groups(const pnmix_config* cfg, int batch, const uint16_t* q_window,
+                                          int n_window, const uint16_t* k, const uint16_t* v, int L,
+                                          int ld_tokens, int hi_percent, float* scores, uint8_t* route,
+                                          int32_t* dest, uint16_t* k_hi, uint16_t* v_hi, uint16_t* k_lo,
+                                          uint16_t* v_lo, void* stream);
+
+/*
  * pnmix_decode_attention without a caller-provided workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory (a plugin whose host runtime owns all device memory, or an interface

@@ -321,3 +321,60 @@ def test_shrunk_cache_matches_the_oracle_and_decodes_like_it(kernel, B, Hq, Hkv,
     np.testing.assert_array_equal(small.records().cpu().numpy()[:, :, :ng], want.records[:, :, :ng])
     q = c.query(L + extra)
     assert_close(small.attend(to_dev(q)).cpu().numpy(), want.attend(q))
+
+
+# Two-precision mixing, prefill side (the SemKV abstract's ranked two-precision
+# assignment): group scores and route bit-exact, and the two parts quantized into two
+# caches byte-equal to the oracle's.
+@pytest.mark.parametrize("B,Hq,Hkv,L,k_hi,k_lo,percent", [
+    (2, 8, 2, 300, 16, 8, 50),
+    (1, 28, 4, 517, 32, 8, 25),
+    (2, 8, 2, 64, 16, 8, 100),
+    (1, 4, 1, 100, 16, 8, 0),
+    (2, 32, 8, 1000, 16, 0, 40),
+])
+def test_split_groups_and_two_precision_caches_match_the_oracle(B, Hq, Hkv, L, k_hi, k_lo, percent):
+    import decode_attention_prefill_b200 as pm
+    import oracle
+    import workload
+    G = Hq // Hkv
+    W = min(L, 64)
+    kin = workload.rows(L, workload.K, B, Hkv, 0, L)
+    vin = workload.rows(L, workload.V, B, Hkv, 0, L)
+    qwin = workload.rows(L, workload.Q, B, Hq, L - W, W, group=G)
+    cap = (L + 31) // 32 * 32 + 32
+    want = oracle.TwoPrecision(B, Hkv, cap, k_hi, k_lo, 4, 2, percent)
+    want.prefill(qwin, kin, vin, L)
+
+    q_dev, k_dev, v_dev = to_dev(qwin), to_dev(kin), to_dev(vin)
+    cfg_hi = pm.Config.make(Hq, Hkv, 4, 2, k_hi, 64)
+    cfg_lo = pm.Config.make(Hq, Hkv, 4, 2, k_lo, 64)
+    parts = pm.pnmix_split_groups(cfg_hi, q_dev, k_dev, v_dev, L, percent)
+    torch.cuda.synchronize()
+    ng = L // 32
+    np.testing.assert_array_equal(parts["route"].cpu().numpy(), want.route[:, :, :ng])
+    route = want.route[:, :, :ng].astype(np.int64)
+    same_before = np.where(route == 1, np.cumsum(route, axis=2) - 1, np.cumsum(1 - route, axis=2) - 1)
+    np.testing.assert_array_equal(parts["dest"].cpu().numpy(), same_before)
+    for b in range(B):
+        for h in range(Hkv):
+            qbar = oracle.mean_query(qwin[b, h * G:(h + 1) * G])
+            np.testing.assert_array_equal(parts["scores"][b, h].cpu().numpy(), oracle.group_scores(qbar, kin[b, h], L))
+
+    L_hi, L_lo = pm.split_sizes(L, percent)
+    for cfg, part, k_part, v_part, Lp in ((cfg_hi, want.hi, parts["k_hi"], parts["v_hi"], L_hi),
+                                         (cfg_lo, want.lo, parts["k_lo"], parts["v_lo"], L_lo)):
+        cache = pm.PNMixCache(cfg, B, cap)
+        pm.pnmix_select_pairs(cfg, q_dev, k_dev, L, cache)
+        if Lp > 0:
+            pm.pnmix_quantize_keys(cfg, k_part, Lp, cache)
+            pm.pnmix_quantize_values(cfg, v_part, Lp, cache)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(cache.lengths().cpu().numpy(), part.len)
+        np.testing.assert_array_equal(cache.perm().cpu().numpy(), part.perm)
+        n = int(part.len[0])
+        np.testing.assert_array_equal(cache.records().cpu().numpy()[:, :, :n // 32], part.records[:, :, :n // 32])
+        if n % 32:
+            np.testing.assert_array_equal(cache.resid("k").cpu().numpy().view(np.uint16)[:, :, :n % 32],
+                                          part.resid_k[:, :, :n % 32])
+        assert cache.read_error() == 0
