@@ -170,3 +170,28 @@ def test_shrink_entry_rejects_bad_arguments_before_launching():
     # there must be salient pairs to shrink (both supported bit pairs have b_hi = 2 b_lo)
     s0 = _fake_cache_at(small, 1 << 40)
     assert L.pnmix_shrink_keys(ctypes.byref(small), ctypes.byref(s0), ctypes.byref(dst), None) == pm.ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_split_groups_rejects_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2)
+    P = ctypes.c_void_p(1 << 41)
+    odd = ctypes.c_void_p((1 << 41) + 2)
+    L = pm._lib
+    def call(q=P, nw=64, k=P, v=P, n=300, ld=300, pct=50, sc=P, rt=P, ds=P, kh=P, vh=P, kl=P, vl=P, cf=cfg):
+        return L.pnmix_split_groups(ctypes.byref(cf), 2, q, nw, k, v, n, ld, pct, sc, rt, ds, kh, vh, kl, vl, None)
+    assert call(nw=63) == pm.ERR_INVALID_ARG                  # window must be min(L, W)
+    assert call(ld=299) == pm.ERR_INVALID_ARG
+    assert call(pct=101) == pm.ERR_INVALID_ARG
+    assert call(pct=-1) == pm.ERR_INVALID_ARG
+    assert call(n=0, nw=0) == pm.ERR_INVALID_ARG
+    assert call(sc=None) == pm.ERR_INVALID_ARG                # 9 full groups need the outputs
+    assert call(kh=None) == pm.ERR_INVALID_ARG                # 4 groups go to the high part
+    assert call(pct=0, kh=None, vh=None, n=20, nw=20, ld=20, sc=None, rt=None, ds=None, kl=odd) == pm.ERR_ALIGNMENT
+    assert call(v=odd) == pm.ERR_ALIGNMENT
+    bad = pm.Config.make(8, 3)                                # 8 query heads over 3 KV heads
+    assert call(cf=bad) == pm.ERR_INVALID_ARG
+    assert pm.split_sizes(300, 50) == (128, 172)
+    assert pm.split_sizes(64, 100) == (64, 0)
+    assert pm.split_sizes(20, 100) == (0, 20)
