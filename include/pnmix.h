@@ -376,8 +376,9 @@ PNMIX_API pnmix_status pnmix_shrink_keys(const pnmix_config* cfg, const pnmix_ca
  * A mixed cache is then two caches: pnmix_select_pairs of each on the full k (its own
  * n_salient_pairs), and pnmix_quantize_keys / _values of each part with L_hi / L_lo.
  * Two launches on `stream`; the ranking costs ng^2 comparisons per (b, h).  Errors:
- * INVALID_ARG (null pointers, L < 1, ld_tokens < L, n_window, hi_percent outside 0..100),
- * UNSUPPORTED (head counts), ALIGNMENT (bf16 pointers not 16-byte aligned), CUDA.
+ * INVALID_ARG (null pointers, L < 1, ld_tokens < L, n_window, hi_percent outside 0..100,
+ * query heads not a multiple of KV heads), UNSUPPORTED (a configuration outside the
+ * supported set), ALIGNMENT (bf16 pointers not 16-byte aligned), CUDA.
  */
 PNMIX_API pnmix_status pnmix_split_groups(const pnmix_config* cfg, int batch, const uint16_t* q_window,
                                           int n_window, const uint16_t* k, const uint16_t* v, int L,
