@@ -59,3 +59,25 @@ def test_reference_arm_other_ranks_exit_quietly(capsys):
         steps, warmup, seed = 1, 0, 0
     assert bench.run_reference(A(), 2, 1) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    """Rank 0 of the reference arm times the oracle and prints one JSON line with the
+    contract's keys, its own cpu_baseline and an e2e block that moves no bytes."""
+    import json
+
+    import bench
+
+    class A:
+        steps, warmup, seed = 1, 0, 0
+    assert bench.run_reference(A(), 1, 0) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "stream_32k"
