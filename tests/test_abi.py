@@ -195,3 +195,16 @@ def test_split_groups_rejects_bad_arguments_before_launching():
     assert pm.split_sizes(300, 50) == (128, 172)
     assert pm.split_sizes(64, 100) == (64, 0)
     assert pm.split_sizes(20, 100) == (0, 20)
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])
+def test_header_is_plain_c_and_cxx(lang, std, tmp_path):
+    """include/pnmix.h parses on its own as C99 and as C++ (no torch or CUDA types)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", std, "-x", lang, HEADER],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
