@@ -33,6 +33,10 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_ALIGNMENT, ERR_DEVICE = range(7)
 DEVERR_APPEND_FULL = 0x1
+DEVERR_TIMEOUT = 0x2
+# decode kernels (Config.decode_kernel)
+DECODE_AUTO, DECODE_SIMT, DECODE_MMA, DECODE_PAIRS = range(4)
+DECODE_KERNELS = {"auto": DECODE_AUTO, "simt": DECODE_SIMT, "mma": DECODE_MMA, "ws": DECODE_PAIRS}
 
 EXPORTED = [
     "pnmix_record_bytes", "pnmix_cache_bytes", "pnmix_cache_init", "pnmix_cache_reset",
@@ -40,7 +44,7 @@ EXPORTED = [
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
     "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi", "pnmix_shrink_keys",
-    "pnmix_split_groups",
+    "pnmix_split_groups", "pnmix_debug_decode_stall",
 ]
 
 
@@ -49,14 +53,14 @@ class Config(ctypes.Structure):
         "head_dim", "n_q_heads", "n_kv_heads", "group_tokens", "residual_tokens", "key_bits_hi",
         "key_bits_lo", "n_salient_pairs", "value_bits", "value_group", "saliency_window")] + [
         ("softmax_scale", ctypes.c_float), ("saliency_score", ctypes.c_int32),
-        ("n_pruned_pairs", ctypes.c_int32)]
+        ("n_pruned_pairs", ctypes.c_int32), ("decode_kernel", ctypes.c_int32)]
 
     @classmethod
     def make(cls, n_q_heads: int, n_kv_heads: int, key_bits_hi: int = 4, key_bits_lo: int = 2,
              n_salient_pairs: int = 8, saliency_window: int = 64, softmax_scale: float = 0.0,
-             saliency_score: int = 0, n_pruned_pairs: int = 0):
+             saliency_score: int = 0, n_pruned_pairs: int = 0, decode_kernel: int = 0):
         return cls(128, n_q_heads, n_kv_heads, 32, 32, key_bits_hi, key_bits_lo, n_salient_pairs,
-                   2, 32, saliency_window, softmax_scale, saliency_score, n_pruned_pairs)
+                   2, 32, saliency_window, softmax_scale, saliency_score, n_pruned_pairs, decode_kernel)
 
     @property
     def group(self) -> int:
@@ -102,6 +106,7 @@ _SIGS = {
     "pnmix_shrink_keys": (_i, [_CP, _KP, _KP, _vp]),
     "pnmix_split_groups": (_i, [_CP, _i, _vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp]),
+    "pnmix_debug_decode_stall": (_i, [_CP, _vp, _KP, _i, _vp, _vp, _sz, _i, ctypes.c_uint32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)

@@ -31,7 +31,15 @@ struct Geometry {
   int n_prune;    // decode: query pairs each query row drops (0: none)
   int tq;         // decode queries per sequence (1, or T of a multi-query step)
   int rows;       // query rows per (b, KV head) in decode: G * tq (row v = query v / G, head v % G)
+  int kernel;     // decode kernel, PNMIX_DECODE_*
+  uint32_t wait_limit;   // decode: try_wait rounds before a staging wait gives up
+  int skip_unit;         // decode test hook: the unit whose records are never staged (-1: none)
 };
+
+// try_wait rounds before a decode staging wait gives up (each round may suspend the warp
+// for a while); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and the kernel stops
+// consuming.
+constexpr uint32_t kDecodeWaitLimit = 1u << 22;
 
 // Record part offsets.
 __host__ __device__ __forceinline__ int rec_kscale(const Geometry& g) { return g.kc_bytes; }
@@ -174,8 +182,13 @@ cudaError_t launch_quantize_values(const Geometry& g, const uint16_t* v, int L, 
 cudaError_t launch_append(const Geometry& g, const uint16_t* k_new, const uint16_t* v_new,
                           const pnmix_cache& c, cudaStream_t s);
 
-// Decode: the workspace a batch / context bound needs, and the launch.
+// Decode: host-side validation of a decode call's arguments (everything but the
+// workspace), the workspace a batch / context bound needs, the byte offset of its ticket
+// words (the only part that must be zero before a launch), and the launch.
+pnmix_status check_decode_args(const pnmix_config* cfg, const uint16_t* q, const pnmix_cache* cache,
+                               int max_context, const float* out, Geometry* g);
 size_t decode_workspace_bytes(const Geometry& g, int max_context);
+size_t decode_ticket_offset(const Geometry& g, int max_context);
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c,
                           int max_context, float* out, void* ws, cudaStream_t s);
 

@@ -2,7 +2,8 @@
 // kernels.
 //
 // Work items.  Unit u = (b, h) owns len[b]/32 full-group items followed by one residual
-// item (the len[b] % 32 bf16 tokens, possibly none).  Items are numbered b-major, then h,
+// item (the len[b] % 32 bf16 tokens, possibly none); len[b] is taken clamped to
+// [0, capacity].  Items are numbered b-major, then h,
 // then item, T in total.  A grid of N CTAs splits [0, T) evenly: CTA i takes
 // [floor(i*T/N), floor((i+1)*T/N)).  Every CTA computes T from len[] itself, so the grid
 // is balanced for any mix of lengths without the host knowing them.
@@ -41,9 +42,16 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int N) {
   return static_cast<int>(((x + 1) * N - 1) / T);
 }
 
+// Length of sequence b as the partition uses it: len[b] clamped to [0, capacity], so a
+// length array holding anything else (stale memory, a caller's ordering mistake) cannot
+// send a record read outside the cache.
+__device__ __forceinline__ int seq_len(const Geometry& g, const int32_t* len, int b) {
+  return min(max(len[b], 0), g.capacity);
+}
+
 __device__ __forceinline__ long long total_items(const Geometry& g, const int32_t* len) {
   long long T = 0;
-  for (int b = 0; b < g.B; ++b) T += static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+  for (int b = 0; b < g.B; ++b) T += static_cast<long long>(g.Hkv) * (seq_len(g, len, b) / kGroup + 1);
   return T;
 }
 
@@ -68,13 +76,15 @@ __device__ __forceinline__ void for_each_segment(const Geometry& g, const int32_
   int b = 0;
   long long x = a;
   while (x < e) {
-    long long per_b = static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+    int lb = seq_len(g, len, b);
+    long long per_b = static_cast<long long>(g.Hkv) * (lb / kGroup + 1);
     while (b < g.B - 1 && cum + per_b <= x) {
       cum += per_b;
       ++b;
-      per_b = static_cast<long long>(g.Hkv) * (len[b] / kGroup + 1);
+      lb = seq_len(g, len, b);
+      per_b = static_cast<long long>(g.Hkv) * (lb / kGroup + 1);
     }
-    const int items = len[b] / kGroup + 1;
+    const int items = lb / kGroup + 1;
     const int h = static_cast<int>((x - cum) / items);
     const long long ustart = cum + static_cast<long long>(h) * items;
     const long long uend = ustart + items;
@@ -84,8 +94,8 @@ __device__ __forceinline__ void for_each_segment(const Geometry& g, const int32_
     s.unit = b * g.Hkv + h;
     s.lo = static_cast<int>(x - ustart);
     s.hi = static_cast<int>((uend < e ? uend : e) - ustart);
-    s.ng = len[b] / kGroup;
-    s.nr = len[b] % kGroup;
+    s.ng = lb / kGroup;
+    s.nr = lb % kGroup;
     s.first = cta_of(ustart, T, N);
     s.last = cta_of(uend - 1, T, N);
     fn(s);

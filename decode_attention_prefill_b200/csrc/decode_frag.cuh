@@ -98,9 +98,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
 }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
-// try_wait rounds before a staging wait gives up (each round may suspend the warp for a
-// while); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and the kernel stops consuming.
-constexpr uint32_t kWaitLimit = 1u << 22;
 
 // Codes as fp16 subnormals.  A code pair sitting at bit offset e of both 16-bit halves of
 // a word becomes an exact fp16x2 of (code * 2^(e-24)) with one AND: the exponent field

@@ -399,7 +399,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
   // A warp's staged groups are numbered in order across its segments: ordinal o lives in
   // slot o % kS and completes phase (o / kS) & 1 of that slot's barrier.
   uint32_t ord_base = 0;
-  bool failed = false;
+  bool failed = false;   // a staging wait ran out: stage and consume nothing more
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
@@ -409,11 +409,14 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     const int my_first = seg.lo + warp;
     const int my_count = my_first < gend ? (gend - my_first + kWarps - 1) / kWarps : 0;
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
-    int issued = 0;   // groups of this segment handed to the copy engine
+    int issued = 0;     // groups of this segment handed to the copy engine
+    int consumed = 0;   // groups of this segment whose copies have landed and been taken
+    const bool stage = unit != g.skip_unit;   // false only under the timeout test hook
     // Issue the warp's groups [issued, upto) of this segment.  Ordinal j may only be
     // issued while j - (first unconsumed ordinal) < kS, which the callers keep.
     auto issue_upto = [&](int upto) {
       const int last = upto < my_count ? upto : my_count;
+      if (failed || !stage) return;
       for (; issued < last; ++issued) {
         const uint32_t o = ord_base + issued, slot = o % kS;
         stage_group(ring + slot * R, unit_rec + static_cast<size_t>(my_first + issued * kWarps) * R,
@@ -425,12 +428,13 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       const uint32_t o = ord_base + i, slot = o % kS, phase = (o / kS) & 1;
       uint32_t spins = 0;
       while (!failed && !mbar_try_wait(bars + slot, phase)) {
-        if (++spins >= kWaitLimit) {
+        if (++spins >= g.wait_limit) {
           failed = true;
           if (lane == 0) atomicOr(c.error, PNMIX_DEVERR_TIMEOUT);
         }
       }
       failed = __any_sync(0xffffffffu, failed);   // keep the warp's control flow uniform
+      if (!failed) consumed = i + 1;
       return ring + slot * R;
     };
     issue_upto(kS - groups_per_step<NT>());
@@ -532,10 +536,10 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       if (!failed) process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, recs, qf, qscale, tok, vis_base, st);
       __syncwarp();
     }
-    if (failed) {   // let copies still in flight land before the shared memory is reused
-      for (int k = 0; k < kS && k < my_count; ++k) {
-        const uint32_t o = ord_base + my_count - 1 - k;
-        for (uint32_t spins = 0; spins < kWaitLimit && !mbar_try_wait(bars + o % kS, (o / kS) & 1); ++spins) {
+    if (failed) {   // let the copies issued and not yet taken land before the shared memory is reused
+      for (int k = consumed; k < issued; ++k) {
+        const uint32_t o = ord_base + k;
+        for (uint32_t spins = 0; spins < g.wait_limit && !mbar_try_wait(bars + o % kS, (o / kS) & 1); ++spins) {
         }
       }
     }

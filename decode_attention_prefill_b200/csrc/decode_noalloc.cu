@@ -13,45 +13,36 @@
 //    (pnmix_workspace_bytes for the same config, batch and max_context) is larger
 //    is rejected with PNMIX_ERR_CAPACITY before anything is enqueued;
 //  - every device that loads the library keeps those 4 MiB until the process exits;
-//  - all calls on a device share the one array and it keeps what the last call left,
-//    so each call first clears the part it uses (cudaMemsetAsync on `stream`);
-//    calls whose work overlaps on the GPU (other streams, other threads) race on
-//    the array and must be serialised by the caller;
-//  - the first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress) with that device current; make that first call before
-//    any stream capture.
+//  - all calls on a device share the one array and it keeps what the last call left.
+//    Only the split-K ticket words must start at zero (every partial slot is written
+//    before it is read in the same launch), so each call clears just those words
+//    (cudaMemsetAsync on `stream`) before its launch; calls whose work overlaps on the
+//    GPU (other streams, other threads) race on the array and must be serialised by
+//    the caller;
+//  - the array's device address is looked up (cudaGetSymbolAddress) on every call,
+//    with the caller's current device, so it stays right after a device reset or a new
+//    primary context.  The first call on a device also loads the library's device code
+//    there; make that first call before any stream capture.  `stream` must belong to
+//    the current device.
 // Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
-#include <mutex>
-
 #include "common.cuh"
+#include "decode_common.cuh"
 
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
-constexpr int kMaxDevices = 64;
 
 // The scratch.  In host code this name is only a stand-in for the device
 // variable; its device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices];
-
 pnmix_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PNMIX_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) return PNMIX_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) return PNMIX_ERR_CUDA;
+  *out = p;
   return PNMIX_OK;
 }
-
-bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
 
@@ -60,22 +51,19 @@ extern "C" PNMIX_API pnmix_status pnmix_decode_attention_noalloc(const pnmix_con
                                                                  const pnmix_cache* cache,
                                                                  int max_context, float* out,
                                                                  void* stream) {
-  // Everything pnmix_decode_attention would reject is rejected here first, so a
-  // failing call enqueues nothing (not even the clearing memset).
-  if (!cfg || !cache || !cache->base || !cache->records || !q || !out || max_context < 0)
-    return PNMIX_ERR_INVALID_ARG;
-  const size_t rb = pnmix_record_bytes(cfg);
-  if (rb == 0) return PNMIX_ERR_UNSUPPORTED;
-  if (cache->n_kv_heads != cfg->n_kv_heads || static_cast<size_t>(cache->record_bytes) != rb)
-    return PNMIX_ERR_INVALID_ARG;
-  if (!is_aligned(q, 16) || !is_aligned(out, 16)) return PNMIX_ERR_ALIGNMENT;
-  const size_t need = pnmix_workspace_bytes(cfg, cache->batch, max_context);
-  if (need == 0) return PNMIX_ERR_INVALID_ARG;
+  // The same validation as pnmix_decode_attention, all before anything is enqueued: a
+  // rejected call leaves the shared array alone.
+  pnmix::Geometry g;
+  pnmix_status st = pnmix::check_decode_args(cfg, q, cache, max_context, out, &g);
+  if (st != PNMIX_OK) return st;
+  const size_t need = pnmix::decode_workspace_bytes(g, max_context);
   if (need > kNoAllocScratchBytes) return PNMIX_ERR_CAPACITY;
   void* ws = nullptr;
-  pnmix_status st = scratch_address(&ws);
-  if (st != PNMIX_OK) return st;
-  if (cudaMemsetAsync(ws, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if ((st = scratch_address(&ws)) != PNMIX_OK) return st;
+  const size_t tickets = pnmix::decode_ticket_offset(g, max_context);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(static_cast<char*>(ws) + tickets, 0, need - tickets, s) != cudaSuccess)
     return PNMIX_ERR_CUDA;
-  return pnmix_decode_attention(cfg, q, cache, max_context, out, ws, need, stream);
+  return pnmix::launch_decode(g, q, *cache, max_context, out, ws, s) == cudaSuccess ? PNMIX_OK
+                                                                                      : PNMIX_ERR_CUDA;
 }

@@ -19,7 +19,7 @@
 // 2^kLazyMax), so the value accumulators are rescaled a few times per segment instead of
 // at every increase.
 //
-// Every wait is bounded (kWaitLimit); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and a
+// Every wait is bounded (Geometry::wait_limit rounds); a wait that runs out sets PNMIX_DEVERR_TIMEOUT and a
 // shared flag that makes every warp of the CTA stop consuming.
 #include <atomic>
 
@@ -78,11 +78,12 @@ __host__ __device__ __forceinline__ WsSmem ws_smem(int NT, int R, int S) {
 
 // Bounded wait on phase `parity` of `bar`.  Returns false (and raises the CTA's stop flag
 // and the cache error word) when the wait runs out or another warp already stopped.
-__device__ __forceinline__ bool ws_wait(uint64_t* bar, uint32_t parity, volatile int* stop, uint32_t* err) {
+__device__ __forceinline__ bool ws_wait(uint64_t* bar, uint32_t parity, volatile int* stop, uint32_t* err,
+                                       uint32_t limit) {
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*stop) return false;
-    if (++spins >= kWaitLimit) {
+    if (++spins >= limit) {
       *stop = 1;
       if ((threadIdx.x & 31) == 0) atomicOr(err, PNMIX_DEVERR_TIMEOUT);
       return false;
@@ -317,12 +318,15 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
     auto rec_src = [&](int i) { return unit_rec + static_cast<size_t>(my_first + i * kPairs) * R; };
 
-    // the PV warp owns the pair's ring: stage the first groups right away
-    if (!is_qk) {
+    // the PV warp owns the pair's ring: stage the first groups right away (nothing once a
+    // wait of this CTA has run out, or for the unit the timeout test hook leaves unstaged)
+    const bool stage = unit != g.skip_unit;
+    int issued = 0;
+    if (!is_qk && stage && !*stop) {
       const int n0 = my_count < S ? my_count : S;
-      for (int i = 0; i < n0; ++i) {
-        const uint32_t o = ord_base + i;
-        stage_group(ring + (o % S) * R, rec_src(i), static_cast<uint32_t>(R), full + o % S, lane == 0);
+      for (; issued < n0; ++issued) {
+        const uint32_t o = ord_base + issued;
+        stage_group(ring + (o % S) * R, rec_src(issued), static_cast<uint32_t>(R), full + o % S, lane == 0);
       }
     }
 
@@ -402,7 +406,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       }
       for (int i = 0; i < my_count; ++i) {
         const uint32_t o = ord_base + i;
-        if (!__all_sync(0xffffffffu, ws_wait(full + o % S, (o / S) & 1, stop, c.error))) break;
+        if (!__all_sync(0xffffffffu, ws_wait(full + o % S, (o / S) & 1, stop, c.error, g.wait_limit))) break;
         float lg[NT][4];
         group_logits<BHI, BLO, NT, NHS, QREG, MQ>(g, ring + (o % S) * R, qf, reinterpret_cast<const uint4*>(qsets),
                                              qscale, (my_first + i * kPairs) * kGroup, vis_base, lg);
@@ -422,7 +426,7 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         const uint32_t pb = o & 1;
         uint8_t* P = pbuf + pb * kPBufBytes;
         // the P buffer's previous use (ordinal o - 2) must have been read by the PV warp
-        if (o >= 2 && !__all_sync(0xffffffffu, ws_wait(pempty + pb, ((o >> 1) + 1) & 1, stop, c.error))) break;
+        if (o >= 2 && !__all_sync(0xffffffffu, ws_wait(pempty + pb, ((o >> 1) + 1) & 1, stop, c.error, g.wait_limit))) break;
         if (any_raise) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
@@ -463,8 +467,8 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         const uint32_t o = ord_base + i;
         const uint32_t pb = o & 1;
         const uint8_t* P = pbuf + pb * kPBufBytes;
-        if (!__all_sync(0xffffffffu, ws_wait(pfull + pb, (o >> 1) & 1, stop, c.error))) break;
-        if (!__all_sync(0xffffffffu, ws_wait(full + o % S, (o / S) & 1, stop, c.error))) break;
+        if (!__all_sync(0xffffffffu, ws_wait(pfull + pb, (o >> 1) & 1, stop, c.error, g.wait_limit))) break;
+        if (!__all_sync(0xffffffffu, ws_wait(full + o % S, (o / S) & 1, stop, c.error, g.wait_limit))) break;
         const uint4 p4 = reinterpret_cast<const uint4*>(P)[lane];
         const int rescale = *reinterpret_cast<const volatile int*>(P + 512);
         float a0 = 1.f, a1 = 1.f;
@@ -490,17 +494,18 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         group_values<key_code_bytes<BHI, BLO, NHS>()>(ring + (o % S) * R, p4, pv, bias);
         consumed = i + 1;
         __syncwarp();
-        if (i + S < my_count) {
-          const uint32_t on = o + S;
-          stage_group(ring + (on % S) * R, rec_src(i + S), static_cast<uint32_t>(R), full + on % S, lane == 0);
+        if (issued < my_count && stage && !*stop) {
+          const uint32_t on = ord_base + issued;
+          stage_group(ring + (on % S) * R, rec_src(issued), static_cast<uint32_t>(R), full + on % S, lane == 0);
+          ++issued;
         }
       }
       if (consumed < my_count) {
-        // stopped early: let the copies still in flight land before the shared memory is reused
-        const int issued = my_count < consumed + S ? my_count : consumed + S;
+        // stopped early: let the copies issued and not yet taken land before the shared
+        // memory is reused
         for (int k = consumed; k < issued; ++k) {
           const uint32_t o = ord_base + k;
-          for (uint32_t spins = 0; spins < kWaitLimit && !mbar_try_wait(full + o % S, (o / S) & 1); ++spins) {
+          for (uint32_t spins = 0; spins < g.wait_limit && !mbar_try_wait(full + o % S, (o / S) & 1); ++spins) {
           }
         }
       }

@@ -2,7 +2,6 @@
 // the launches.  No entry point allocates, frees or synchronises (except
 // pnmix_read_error, which is a synchronous read by definition).
 #include <math.h>
-#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -31,6 +30,9 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   if (cfg->saliency_score < PNMIX_SCORE_PNMIX || cfg->saliency_score > PNMIX_SCORE_RANGE_QUERY)
     return PNMIX_ERR_UNSUPPORTED;
   if (cfg->n_pruned_pairs < 0 || cfg->n_pruned_pairs > 63) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->decode_kernel < PNMIX_DECODE_AUTO || cfg->decode_kernel > PNMIX_DECODE_PAIRS)
+    return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->decode_kernel == PNMIX_DECODE_SIMT && cfg->n_pruned_pairs > 0) return PNMIX_ERR_UNSUPPORTED;
   g->B = batch;
   g->Hq = cfg->n_q_heads;
   g->Hkv = cfg->n_kv_heads;
@@ -52,6 +54,9 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->n_prune = cfg->n_pruned_pairs;
   g->tq = 1;
   g->rows = G;
+  g->kernel = cfg->decode_kernel;
+  g->wait_limit = kDecodeWaitLimit;
+  g->skip_unit = -1;
   return PNMIX_OK;
 }
 
@@ -98,39 +103,38 @@ static pnmix_status check_cache(const Geometry& g, const pnmix_cache* c) {
   return PNMIX_OK;
 }
 
-// Which decode kernel runs.  By default the single-role tensor-core kernel
-// (decode_mma.cu) for up to 4 query heads per KV head and the warp-specialized one
-// (decode_ws.cu) above, the faster of the two on the measured workloads.  The environment
-// variable PNMIX_DECODE_KERNEL = mma | ws | simt forces one (read at every call, so tests
-// can run each kernel on every shape; simt is the CUDA-core baseline).
-int decode_kernel_choice() {
-  const char* v = getenv("PNMIX_DECODE_KERNEL");
-  if (!v) return 0;
-  if (strcmp(v, "simt") == 0) return 1;
-  if (strcmp(v, "mma") == 0) return 2;
-  if (strcmp(v, "ws") == 0) return 3;
-  return 0;
+size_t decode_ticket_offset(const Geometry& g, int max_context) {
+  const int nmax = decode_max_ctas(g, max_context);
+  return decode_partial_bytes(nmax + g.B * g.Hkv, g.rows);
 }
 
 size_t decode_workspace_bytes(const Geometry& g, int max_context) {
-  const int nmax = decode_max_ctas(g, max_context);
-  const int units = g.B * g.Hkv;
-  return decode_partial_bytes(nmax + units, g.rows) + align256(sizeof(uint32_t) * units);
+  return decode_ticket_offset(g, max_context) + align256(sizeof(uint32_t) * g.B * g.Hkv);
+}
+
+pnmix_status check_decode_args(const pnmix_config* cfg, const uint16_t* q, const pnmix_cache* cache,
+                               int max_context, const float* out, Geometry* g) {
+  if (!cache) return PNMIX_ERR_INVALID_ARG;
+  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, g);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_cache(*g, cache)) != PNMIX_OK) return st;
+  if (!q || !out || max_context < 0) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return PNMIX_ERR_ALIGNMENT;
+  return PNMIX_OK;
 }
 
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int max_context,
                           float* out, void* ws, cudaStream_t s) {
   const int nmax = decode_max_ctas(g, max_context);
-  const int units = g.B * g.Hkv;
   DecodeWs w;
   w.part = static_cast<float*>(ws);
-  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_partial_bytes(nmax + units, g.rows));
+  w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_ticket_offset(g, max_context));
   w.N = nmax;
-  switch (g.tq > 1 && decode_kernel_choice() == 1 ? 0 : decode_kernel_choice()) {   // simt: one query
-    case 1: return launch_decode_simt(g, q, c, nmax, out, w, s);
-    case 2: return launch_decode_mma(g, q, c, nmax, out, w, s);
-    case 3: return launch_decode_ws(g, q, c, nmax, out, w, s);
-    default:   // measured: single-role kernel for up to 4 heads per KV head, pairs above
+  switch (g.kernel) {
+    case PNMIX_DECODE_SIMT: return launch_decode_simt(g, q, c, nmax, out, w, s);
+    case PNMIX_DECODE_MMA: return launch_decode_mma(g, q, c, nmax, out, w, s);
+    case PNMIX_DECODE_PAIRS: return launch_decode_ws(g, q, c, nmax, out, w, s);
+    default:   // measured: single-role kernel for up to 4 rows per KV head, pairs above
       return g.rows <= 4 ? launch_decode_mma(g, q, c, nmax, out, w, s) : launch_decode_ws(g, q, c, nmax, out, w, s);
   }
 }
@@ -270,16 +274,29 @@ size_t pnmix_workspace_bytes(const pnmix_config* cfg, int batch, int max_context
 pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
                                     const pnmix_cache* cache, int max_context, float* out,
                                     void* workspace, size_t workspace_bytes, void* stream) {
-  if (!cache) return PNMIX_ERR_INVALID_ARG;
   Geometry g;
-  pnmix_status st = make_geometry(cfg, cache->batch, cache->capacity_tokens, &g);
+  pnmix_status st = check_decode_args(cfg, q, cache, max_context, out, &g);
   if (st != PNMIX_OK) return st;
-  if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
-  if (!q || !out || !workspace || max_context < 0) return PNMIX_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  if (!workspace) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
   if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
   return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_debug_decode_stall(const pnmix_config* cfg, const uint16_t* q, const pnmix_cache* cache,
+                                      int max_context, float* out, void* workspace, size_t workspace_bytes,
+                                      int skip_unit, uint32_t wait_rounds, void* stream) {
+  Geometry g;
+  pnmix_status st = check_decode_args(cfg, q, cache, max_context, out, &g);
+  if (st != PNMIX_OK) return st;
+  if (!workspace || skip_unit < 0 || skip_unit >= g.B * g.Hkv || wait_rounds < 1) return PNMIX_ERR_INVALID_ARG;
+  if (g.kernel == PNMIX_DECODE_SIMT) return PNMIX_ERR_UNSUPPORTED;
+  if (!aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
+  g.skip_unit = skip_unit;
+  g.wait_limit = wait_rounds;
+  return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch, int max_context, int n_queries) {
@@ -301,6 +318,7 @@ pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_
   if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
   if (!q || !out || !workspace || max_context < 0 || n_queries < 1) return PNMIX_ERR_INVALID_ARG;
   if (g.G * n_queries > kMaxG) return PNMIX_ERR_UNSUPPORTED;
+  if (g.kernel == PNMIX_DECODE_SIMT && n_queries > 1) return PNMIX_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
   g.tq = n_queries;
   g.rows = g.G * n_queries;

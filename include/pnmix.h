@@ -143,7 +143,8 @@ typedef enum {
 /* Device error word bits (pnmix_read_error). */
 #define PNMIX_DEVERR_APPEND_FULL 0x1u  /* pnmix_append found len == capacity_tokens */
 #define PNMIX_DEVERR_TIMEOUT 0x2u      /* a bounded wait for staged cache data ran out in a
-                                          decode call (its output is then invalid) */
+                                          decode call (its output is then invalid); see
+                                          pnmix_debug_decode_stall */
 
 /*
  * Method parameters.  Supported set:
@@ -154,7 +155,8 @@ typedef enum {
  *   G = n_q_heads / n_kv_heads in [1, 8];
  *   saliency_window W in [1, 1024];
  *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*);
- *   n_pruned_pairs in [0, 63].
+ *   n_pruned_pairs in [0, 63];
+ *   decode_kernel in {0, 1, 2, 3} (PNMIX_DECODE_*).
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
  *
  * Dynamic query-channel pruning (n_pruned_pairs > 0; the query-channel pruning of the
@@ -180,7 +182,24 @@ typedef struct {
   float softmax_scale;
   int32_t saliency_score;   /* statistic that ranks the pairs, PNMIX_SCORE_* (0 = PN-Mix) */
   int32_t n_pruned_pairs;   /* decode: query pairs each query row drops, 0..63 (0 = none) */
+  int32_t decode_kernel;    /* decode: which kernel runs, PNMIX_DECODE_* (0 = automatic) */
 } pnmix_config;
+
+/*
+ * Decode kernels (cfg->decode_kernel).  All give the result of the numerical contract
+ * above; they differ in speed.  The choice is part of the configuration, so it costs no
+ * host work per call.
+ *   PNMIX_DECODE_AUTO   the faster tensor-core kernel for the shape (one role per warp for
+ *                       up to 4 query rows per KV head, warp pairs above).
+ *   PNMIX_DECODE_SIMT   CUDA cores only (a baseline): one query per sequence and no query
+ *                       pruning (PNMIX_ERR_UNSUPPORTED otherwise).
+ *   PNMIX_DECODE_MMA    tensor cores, every warp scores and accumulates its own groups.
+ *   PNMIX_DECODE_PAIRS  tensor cores, a key-side and a value-side warp per group stream.
+ */
+#define PNMIX_DECODE_AUTO 0
+#define PNMIX_DECODE_SIMT 1
+#define PNMIX_DECODE_MMA 2
+#define PNMIX_DECODE_PAIRS 3
 
 /*
  * Pair statistics pnmix_select_pairs can rank by (all per (b, kv head), fp32, one
@@ -390,19 +409,37 @@ PNMIX_API pnmix_status pnmix_split_groups(const pnmix_config* cfg, int batch, co
  * pnmix_decode_attention without a caller-provided workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory (a plugin whose host runtime owns all device memory, or an interface
- * with no slot for a workspace pointer).  Same arguments and result as
+ * with no slot for a workspace pointer).  Same arguments, validation and result as
  * pnmix_decode_attention minus the workspace: the split-K scratch comes from a
  * 4 MiB array inside the library image, held on every device that loads the
  * library until the process exits.  A call whose pnmix_workspace_bytes exceeds
- * 4 MiB returns PNMIX_ERR_CAPACITY and enqueues nothing.  Every call on a device
- * shares that array and clears the part it uses first (a memset on `stream`), so
- * calls that overlap on the GPU race and must be serialised by the caller.  The
- * first call on each device looks up the array's address with that device
- * current; make it before any stream capture.  Allocates nothing.
+ * 4 MiB returns PNMIX_ERR_CAPACITY, and every rejected call enqueues nothing.
+ * Every call on a device shares that array and first clears the words of it that
+ * must start at zero (a memset on `stream`), so calls that overlap on the GPU race
+ * and must be serialised by the caller.  The array's address is looked up on every
+ * call for the current device, which `stream` must belong to; the first call on a
+ * device also loads the library's device code there, so make it before any stream
+ * capture.  Allocates nothing.
  */
 PNMIX_API pnmix_status pnmix_decode_attention_noalloc(const pnmix_config* cfg, const uint16_t* q,
                                                       const pnmix_cache* cache, int max_context,
                                                       float* out, void* stream);
+
+/*
+ * Test hook of the bounded staging wait; the pages have no counterpart.  Runs
+ * pnmix_decode_attention (same arguments and validation) with two changes: the
+ * packed records of unit skip_unit (= b * n_kv_heads + h, in [0, batch * n_kv_heads))
+ * are never staged, and every staging wait gives up after wait_rounds (>= 1) rounds of
+ * mbarrier try_wait.  The waits for that unit's records therefore run out: the kernel
+ * sets PNMIX_DEVERR_TIMEOUT in the cache's error word, lets every copy it issued land,
+ * and returns.  The output of the call is then invalid; the cache, the workspace and
+ * the CUDA context stay usable.  Needs a tensor-core decode kernel (PNMIX_ERR_UNSUPPORTED
+ * with PNMIX_DECODE_SIMT, which stages nothing).
+ */
+PNMIX_API pnmix_status pnmix_debug_decode_stall(const pnmix_config* cfg, const uint16_t* q,
+                                                const pnmix_cache* cache, int max_context, float* out,
+                                                void* workspace, size_t workspace_bytes, int skip_unit,
+                                                uint32_t wait_rounds, void* stream);
 
 /* Synchronously read (and, if clear != 0, zero) the device error word.  Host pointer out. */
 PNMIX_API pnmix_status pnmix_read_error(const pnmix_cache* cache, int clear, uint32_t* host_error);

@@ -21,7 +21,7 @@ class Case:
     """One workload instance: inputs on host and device, a GPU cache and an oracle cache."""
 
     def __init__(self, B, Hq, Hkv, L, k=8, bhi=4, blo=2, capacity=None, seed=0, W=64,
-                 max_context=None, extra_tokens=0, score=0, n_prune=0):
+                 max_context=None, extra_tokens=0, score=0, n_prune=0, kernel=None):
         import decode_attention_prefill_b200 as pm
         self.pm = pm
         self.B, self.Hq, self.Hkv, self.G, self.L = B, Hq, Hkv, Hq // Hkv, L
@@ -29,7 +29,8 @@ class Case:
         self.W = min(L, W)
         total = L + extra_tokens
         self.capacity = capacity or ((total + 31) // 32 * 32 + 32)
-        self.cfg = pm.Config.make(Hq, Hkv, bhi, blo, k, W, saliency_score=score, n_pruned_pairs=n_prune)
+        self.cfg = pm.Config.make(Hq, Hkv, bhi, blo, k, W, saliency_score=score, n_pruned_pairs=n_prune,
+                                  decode_kernel=pm.DECODE_KERNELS[kernel or "auto"])
         self.kin = workload.rows(seed, workload.K, B, Hkv, 0, max(total, 1))
         self.vin = workload.rows(seed, workload.V, B, Hkv, 0, max(total, 1))
         self.qwin = workload.rows(seed, workload.Q, B, Hq, L - self.W, max(self.W, 1), group=self.G) \

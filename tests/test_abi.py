@@ -53,6 +53,9 @@ def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
     (dict(saliency_score=-1), pm.ERR_UNSUPPORTED),
     (dict(n_pruned_pairs=64), pm.ERR_UNSUPPORTED),
     (dict(n_pruned_pairs=-1), pm.ERR_UNSUPPORTED),
+    (dict(decode_kernel=4), pm.ERR_UNSUPPORTED),
+    (dict(decode_kernel=-1), pm.ERR_UNSUPPORTED),
+    (dict(decode_kernel=pm.DECODE_SIMT, n_pruned_pairs=5), pm.ERR_UNSUPPORTED),   # simt has no pruning
 ])
 def test_config_validation(change, status):
     cfg = pm.Config.make(32, 8)
@@ -208,3 +211,78 @@ def test_header_is_plain_c_and_cxx(lang, std, tmp_path):
     r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", std, "-x", lang, HEADER],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of pnmix_config and pnmix_cache have the header's size and field
+    offsets (a C program built against include/pnmix.h prints them)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "pnmix.h"', 'int main(void) {']
+    for cname, cls in (("pnmix_config", pm.Config), ("pnmix_cache", pm.Cache)):
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    r = subprocess.run([cc, "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    for line in filter(None, got):
+        cname, field, value = line.split()
+        cls = pm.Config if cname == "pnmix_config" else pm.Cache
+        want = ctypes.sizeof(cls) if field == "size" else getattr(cls, field).offset
+        assert int(value) == want, (cname, field)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_noalloc_entry_rejects_bad_arguments_before_any_cuda_call():
+    """Every rejection of the no-workspace decode happens on the host, before its scratch
+    address is looked up or its memset is enqueued (none of these calls reaches CUDA)."""
+    cfg = pm.Config.make(8, 2)
+    c = _fake_cache(cfg)
+    P = ctypes.c_void_p(1 << 41)
+    odd = ctypes.c_void_p((1 << 41) + 2)
+    f = pm._lib.pnmix_decode_attention_noalloc
+    assert f(None, P, ctypes.byref(c), 256, P, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), None, ctypes.byref(c), 256, P, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, None, 256, P, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, None, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), -1, P, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), odd, ctypes.byref(c), 256, P, None) == pm.ERR_ALIGNMENT
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, odd, None) == pm.ERR_ALIGNMENT
+    other = pm.Config.make(8, 2, n_salient_pairs=16)   # record size differs from the cache's
+    assert f(ctypes.byref(other), P, ctypes.byref(c), 256, P, None) == pm.ERR_INVALID_ARG
+    bad = pm.Cache.from_buffer_copy(c)
+    bad.capacity_tokens = -32
+    assert f(ctypes.byref(cfg), P, ctypes.byref(bad), 256, P, None) == pm.ERR_INVALID_ARG
+    unsupported = pm.Config.make(8, 2, key_bits_hi=8)
+    assert f(ctypes.byref(unsupported), P, ctypes.byref(c), 256, P, None) == pm.ERR_UNSUPPORTED
+    big_cfg = pm.Config.make(64, 8)                     # G = 8, 1024 units: > 4 MiB of partials
+    big = _fake_cache(big_cfg, B=128, cap=32)
+    assert pm.workspace_bytes(big_cfg, 128, 32) > (4 << 20)
+    assert f(ctypes.byref(big_cfg), P, ctypes.byref(big), 32, P, None) == pm.ERR_CAPACITY
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_stall_hook_rejects_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2)
+    c = _fake_cache(cfg)                    # 2 x 2 units
+    P = ctypes.c_void_p(1 << 41)
+    ws = pm.workspace_bytes(cfg, 2, 256)
+    f = pm._lib.pnmix_debug_decode_stall
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, P, ws, 4, 16, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, P, ws, -1, 16, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, P, ws, 0, 0, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, P, ws - 1, 0, 16, None) == pm.ERR_CAPACITY
+    assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, None, ws, 0, 16, None) == pm.ERR_INVALID_ARG
+    simt = pm.Config.make(8, 2, decode_kernel=pm.DECODE_SIMT)
+    assert f(ctypes.byref(simt), P, ctypes.byref(c), 256, P, P, ws, 0, 16, None) == pm.ERR_UNSUPPORTED

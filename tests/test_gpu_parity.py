@@ -42,21 +42,20 @@ def test_prefill_and_decode_shapes(B, Hq, Hkv, L, k, bhi, blo):
 
 
 # The library routes decode to one of two tensor-core kernels by the number of query heads
-# per KV head; each one is forced here on every shape (the variable is read per call).
-@pytest.mark.parametrize("kernel", ["mma", "ws"])
+# per KV head; each one, and the CUDA-core baseline, is forced here on every shape through
+# the configuration.
+@pytest.mark.parametrize("kernel", ["mma", "ws", "simt"])
 @pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo", SHAPES)
-def test_each_decode_kernel_on_every_shape(kernel, B, Hq, Hkv, L, k, bhi, blo, monkeypatch):
-    monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
-    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + k + 1)
+def test_each_decode_kernel_on_every_shape(kernel, B, Hq, Hkv, L, k, bhi, blo):
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + k + 1, kernel=kernel)
     c.prefill()
     got, want = c.attend(c.query(L))
     assert_close(got, want)
 
 
-@pytest.mark.parametrize("kernel", ["mma", "ws"])
-def test_each_decode_kernel_over_a_long_append_stream(kernel, monkeypatch):
-    monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
-    c = Case(2, 14, 2, 3000, extra_tokens=70, seed=11)
+@pytest.mark.parametrize("kernel", ["mma", "ws", "simt"])
+def test_each_decode_kernel_over_a_long_append_stream(kernel):
+    c = Case(2, 14, 2, 3000, extra_tokens=70, seed=11, kernel=kernel)
     c.prefill()
     for t in range(3000, 3070):
         c.append(t)
@@ -241,10 +240,8 @@ def test_saliency_statistics_select_like_the_oracle(score, B, Hq, Hkv, L, k, bhi
     (1, 28, 4, 1000, 1),   # one query equals the single-query call
     (2, 32, 8, 2047, 2),   # the step fills a group exactly
 ])
-def test_multi_query_decode_is_causal_like_the_oracle(kernel, B, Hq, Hkv, L, T, monkeypatch):
-    if kernel:
-        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
-    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + T)
+def test_multi_query_decode_is_causal_like_the_oracle(kernel, B, Hq, Hkv, L, T):
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + T, kernel=kernel)
     c.prefill()
     for t in range(L, L + T):
         c.append(t)
@@ -264,10 +261,8 @@ def test_multi_query_decode_is_causal_like_the_oracle(kernel, B, Hq, Hkv, L, T, 
     (2, 8, 2, 300, 26, 2),     # with two queries per sequence
     (1, 4, 1, 64, 63, 1),      # only pair 0 left
 ])
-def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T, monkeypatch):
-    if kernel:
-        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
-    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + n_prune, n_prune=n_prune)
+def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T):
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + n_prune, n_prune=n_prune, kernel=kernel)
     c.prefill()
     if T == 1:
         got, want = c.attend(c.query(L))
@@ -290,12 +285,9 @@ def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T
     (1, 8, 1, 64, 64, 4, 2),
     (1, 4, 1, 20, 8, 4, 2),     # no full group yet: only the residual window carries over
 ])
-def test_shrunk_cache_matches_the_oracle_and_decodes_like_it(kernel, B, Hq, Hkv, L, k, bhi, blo,
-                                                              monkeypatch):
-    if kernel:
-        monkeypatch.setenv("PNMIX_DECODE_KERNEL", kernel)
+def test_shrunk_cache_matches_the_oracle_and_decodes_like_it(kernel, B, Hq, Hkv, L, k, bhi, blo):
     extra = 40
-    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + 3 * k, extra_tokens=extra)
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, seed=L + 3 * k, extra_tokens=extra, kernel=kernel)
     c.prefill()
     small = c.cache.shrunk()
     want = c.ocache.shrunk()
@@ -378,3 +370,109 @@ def test_split_groups_and_two_precision_caches_match_the_oracle(B, Hq, Hkv, L, k
             np.testing.assert_array_equal(cache.resid("k").cpu().numpy().view(np.uint16)[:, :, :n % 32],
                                           part.resid_k[:, :, :n % 32])
         assert cache.read_error() == 0
+
+
+# Top-k ties on the GPU: integer inputs whose pair norms are integers (Pythagorean pairs)
+# make many pair scores exactly equal; every score is exact in binary32 (G * W = 4 divides
+# exactly), so the GPU scores must equal the exact rational scores and the selected pairs
+# must be the k best by (score descending, pair index ascending).
+PYTH = [(0, 0), (3, 4), (4, 3), (6, 8), (5, 12), (0, 7), (9, 12), (8, 15), (0, 1), (1, 0)]
+
+
+def _tie_inputs(rng, B, Hkv, G, W, L, n_key, n_query):
+    k = np.zeros((B, Hkv, L, 128), np.float32)
+    q = np.zeros((B, Hkv * G, W, 128), np.float32)
+    for b in range(B):
+        for h in range(Hkv):
+            for p in range(64):
+                ab = np.array(PYTH)[rng.integers(0, n_key, L)]
+                k[b, h, :, p] = ab[:, 0] * rng.choice([-1, 1], L)
+                k[b, h, :, p + 64] = ab[:, 1]
+        for hq in range(Hkv * G):
+            for p in range(64):
+                ab = np.array(PYTH)[rng.integers(0, n_query, W)]
+                q[b, hq, :, p] = ab[:, 0]
+                q[b, hq, :, p + 64] = -ab[:, 1]
+    bits = lambda a: (a.view(np.uint32) >> 16).astype(np.uint16)  # noqa: E731  (exact in bf16)
+    return bits(q), bits(k)
+
+
+def _exact_order(q, k):
+    """(score desc, p asc) order of the exact rational scores of one unit."""
+    import math
+    from fractions import Fraction
+    G, W, _ = q.shape
+    kf = (k.astype(np.uint32) << 16).view(np.float32).astype(np.int64)
+    qf = (q.astype(np.uint32) << 16).view(np.float32).astype(np.int64)
+    scores = []
+    for p in range(64):
+        kn = max(math.isqrt(int(a) ** 2 + int(b) ** 2) for a, b in zip(kf[:, p], kf[:, p + 64]))
+        qs = sum(math.isqrt(int(qf[h, t, p]) ** 2 + int(qf[h, t, p + 64]) ** 2) for h in range(G) for t in range(W))
+        scores.append(Fraction(qs, G * W) * kn)
+    return scores, sorted(range(64), key=lambda p: (-scores[p], p))
+
+
+@pytest.mark.parametrize("k", [8, 16, 32, 64])
+@pytest.mark.parametrize("L,n_key,n_query", [(3, 4, 5), (700, 4, 5), (40, 2, 2), (5, 1, 1)])
+def test_select_pairs_breaks_ties_by_the_lower_pair_index(k, L, n_key, n_query):
+    import decode_attention_prefill_b200 as pm
+    import oracle
+    rng = np.random.default_rng(1000 * k + L + n_key)
+    B, Hkv, G, W = 3, 2, 2, 2
+    q, kk = _tie_inputs(rng, B, Hkv, G, W, L, n_key, n_query)
+    cfg = pm.Config.make(Hkv * G, Hkv, 4, 2, k, W)
+    cache = pm.PNMixCache(cfg, B, (L + 31) // 32 * 32 + 32)
+    pm.pnmix_select_pairs(cfg, to_dev(q), to_dev(kk), L, cache)
+    torch.cuda.synchronize()
+    idx = cache.pair_idx().cpu().numpy()
+    mask = cache.pair_mask().cpu().numpy().view(np.uint64)
+    perm = cache.perm().cpu().numpy()
+    scores = cache.pair_scores().cpu().numpy()
+    n_tied = 0
+    for b in range(B):
+        for h in range(Hkv):
+            qu, ku = q[b, h * G:(h + 1) * G], kk[b, h]
+            exact, order = _exact_order(qu, ku)
+            np.testing.assert_array_equal(scores[b, h].astype(np.float64), [float(e) for e in exact])
+            want = sorted(order[:k])
+            assert list(idx[b, h, :k]) == want
+            assert int(mask[b, h]) == sum(1 << p for p in want)
+            s_o, idx_o, mask_o, perm_o = oracle.select_unit(qu, ku, k)
+            np.testing.assert_array_equal(scores[b, h].view(np.uint32), s_o.view(np.uint32))
+            np.testing.assert_array_equal(idx[b, h, :k], idx_o)
+            np.testing.assert_array_equal(perm[b, h], perm_o)
+            if 0 < k < 64:   # a tie straddles the cut when the k-th and (k+1)-th scores are equal
+                n_tied += exact[order[k - 1]] == exact[order[k]]
+    if n_key == 1 and k < 64:   # every key norm equal and every query norm equal: all scores tie
+        assert n_tied == B * Hkv
+
+
+# The bounded staging wait: the test hook never stages one unit's records and gives every
+# wait a short limit, so those waits run out.  The call must return, raise the timeout bit
+# of the error word, and leave the context, the cache and the workspace usable: the next
+# ordinary decode matches the oracle again.
+@pytest.mark.parametrize("kernel", ["mma", "ws"])
+@pytest.mark.parametrize("skip_unit", [0, 3])
+def test_staging_wait_that_runs_out_sets_the_error_word_and_returns(kernel, skip_unit):
+    import ctypes
+    import time
+    c = Case(2, 8, 2, 3000, seed=31, kernel=kernel)
+    c.prefill()
+    pm, q = c.pm, c.query(3000)
+    qd = to_dev(q)
+    out = torch.empty(2, 8, 128, dtype=torch.float32, device="cuda")
+    assert c.cache.read_error() == 0
+    ws = c.cache.workspace
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st = pm._lib.pnmix_debug_decode_stall(ctypes.byref(c.cfg), qd.data_ptr(), ctypes.byref(c.cache.c),
+                                          c.cache.max_context, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                          skip_unit, 256, torch.cuda.current_stream().cuda_stream)
+    assert st == pm.OK
+    torch.cuda.synchronize()
+    print(f"stalled decode returned after {time.perf_counter() - t0:.4f} s")
+    assert c.cache.read_error() & pm.DEVERR_TIMEOUT
+    assert c.cache.read_error() == 0          # cleared by the read
+    got, want = c.attend(q)
+    assert_close(got, want)
+    assert c.cache.read_error() == 0

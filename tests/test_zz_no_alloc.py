@@ -4,8 +4,9 @@ Callers that cannot allocate device memory -- a plugin whose host runtime owns
 every byte of device memory, or an interface with no slot for a workspace
 pointer -- use this call; its split-K scratch is a fixed 4 MiB array inside the
 library.  These checks call it through the C ABI and compare it with
-pnmix_decode_attention (caller workspace) on two calls in a row, with a call of
-another shape in between that leaves different contents in the shared array.
+pnmix_decode_attention (caller workspace) and with the CPU oracle on two calls in a
+row, with a call of another shape in between that leaves different contents in the
+shared array.
 """
 import ctypes
 
@@ -38,15 +39,18 @@ def test_noalloc_decode_matches_the_workspace_entry_point_twice():
     pm.pnmix_decode_attention(b.cfg, qb, b.cache, ref_b)
     torch.cuda.synchronize()
     ref_a, ref_b = ref_a.cpu().numpy().astype(np.float64), ref_b.cpu().numpy().astype(np.float64)
+    want_a, want_b = a.ocache.attend(a.query(300)), b.ocache.attend(b.query(700))
     for _ in range(2):
         out = torch.full((2, 8, 128), float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(pm, a.cfg, qa, a.cache, out) == pm.OK
         torch.cuda.synchronize()
         assert_close(out.cpu().numpy(), ref_a)
+        assert_close(out.cpu().numpy(), want_a)
         out_b = torch.full((3, 28, 128), float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(pm, b.cfg, qb, b.cache, out_b) == pm.OK
         torch.cuda.synchronize()
         assert_close(out_b.cpu().numpy(), ref_b)
+        assert_close(out_b.cpu().numpy(), want_b)
 
 
 def test_noalloc_rejects_a_workspace_beyond_its_scratch():
