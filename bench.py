@@ -284,6 +284,14 @@ def cpu_baseline(seed: int, budget_s: float, n_tokens: int):
                       f"{B}-sequence step"}
 
 
+def stream_config(world: int) -> dict:
+    """`config` of the stream_32k line (both arms)."""
+    return {"workload": "stream_32k", "batch_per_gpu": B, "n_q_heads": HQ, "n_kv_heads": HKV,
+            "head_dim": D, "context": CONTEXT, "prefill": PREFILL, "salient_pairs": K_SALIENT,
+            "key_bits": [BHI, BLO], "value_bits": 2, "key_code_bits": 2.25,
+            "parallelism": f"dp{world}", "l2": "inputs larger than L2 (419 MB cache read per step)"}
+
+
 def run_reference(args, world, rank):
     """Reference arm: the oracle on the host cores, same metric and workload."""
     if rank != 0:
@@ -310,18 +318,22 @@ def run_reference(args, world, rank):
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt * B * HKV)      # one unit -> a full 16-sequence step
-    total = sum(times)
-    value = B * len(times) / total
+    units = B * HKV
+    sampled_s = sum(times) / units          # wall time the sampled steps actually took
+    value = B * len(times) / sum(times)     # whole-step throughput: each step scaled by `units`
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * sampled_s / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "stream_32k", "batch": B, "n_q_heads": HQ, "n_kv_heads": HKV,
-                   "context": CONTEXT, "key_code_bits": 2.25},
+        "config": stream_config(world),
+        "sampled": {"units_per_step": 1, "units_per_full_step": units,
+                    "value_scale": f"each timed step is 1 of {units} (sequence, KV head) units; value "
+                                   f"divides {B} tokens per step by {units} x the sampled time",
+                    "ms_per_step": "wall time of the sampled step (one unit)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": "oracle append + decode attention of 1 of 128 (sequence, KV head) "
-                                   "units per step, scaled to a full 16-sequence step"},
+                         "sample": f"oracle append + decode attention of 1 of {units} (sequence, KV head) "
+                                   f"units per step, scaled to a full {B}-sequence step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -356,6 +368,68 @@ def timed_rotation(fns, reps: int, warmup: int) -> float:
     e1.record()
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def two_part_point(args, pm, wl, k_dev, v_dev, qwin_dev, q_dev, exact, peak, l2_bytes,
+                   k_hi=16, k_lo=8, percent=50):
+    """The mixed-precision point of the bit sweep: the prefill's 32-token groups ranked by
+    the saliency window's mean-query logit (pnmix_split_groups), the best `percent` kept with
+    k_hi salient pairs and the rest with k_lo, and decode attention over both parts
+    (pnmix_decode_attention_two).  Reports the split's time, the decode's, and the
+    relative L2 error against unquantized bf16 attention."""
+    import torch
+    Bw, Hq, Hkv, ctx = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.context
+    G = Hq // Hkv
+    cfg_hi = pm.Config.make(Hq, Hkv, 4, 2, k_hi, WINDOW)
+    cfg_lo = pm.Config.make(Hq, Hkv, 4, 2, k_lo, WINDOW)
+    L_hi, L_lo = pm.split_sizes(ctx, percent)
+    split = lambda: pm.pnmix_split_groups(cfg_hi, qwin_dev, k_dev, v_dev, ctx, percent)  # noqa: E731
+    for _ in range(2):
+        parts = split()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        parts = split()
+    e1.record()
+    torch.cuda.synchronize()
+    split_ms = e0.elapsed_time(e1) / 3
+
+    def build():
+        pair = []
+        for cfg, kp, vp, Lp in ((cfg_hi, parts["k_hi"], parts["v_hi"], L_hi), (cfg_lo, parts["k_lo"], parts["v_lo"], L_lo)):
+            c = pm.PNMixCache(cfg, Bw, ctx + 32, max_context=ctx)
+            pm.pnmix_select_pairs(cfg, qwin_dev, k_dev, ctx, c)
+            if Lp:
+                pm.pnmix_quantize_keys(cfg, kp, Lp, c)
+                pm.pnmix_quantize_values(cfg, vp, Lp, c)
+            pair.append(c)
+        return pair
+    first = build()
+    per_rep = sum(pm.cache_bytes(c.cfg, Bw, ctx + 32) for c in first)
+    n_rep = max(3, -(-3 * l2_bytes // per_rep))
+    reps = [first] + [build() for _ in range(n_rep - 1)]
+    out = torch.empty(Bw, Hq, D, dtype=torch.float32, device=q_dev.device)
+    fns = [(lambda a_=a_, b_=b_: pm.pnmix_decode_attention_two(a_, b_, q_dev, out)) for a_, b_ in reps]
+    t = timed_rotation(fns, max(args.steps, 3 * n_rep), args.warmup)
+    pm.pnmix_decode_attention_two(first[0], first[1], q_dev, out)
+    assert all(c.read_error() == 0 for pair in reps for c in pair)
+    units = Bw * Hkv
+    R_hi, R_lo = first[0].c.record_bytes, first[1].c.record_bytes
+    alg = decode_bytes(L_hi, units, G, R_hi) + decode_bytes(L_lo, units, G, R_lo) - units * G * D * (2 + 4)
+    bits = (L_hi * (2 + 0.5 * k_hi / 16) + L_lo * (2 + 0.5 * k_lo / 16)) / ctx
+    r = {"key_bits": [4, 2], "salient_pairs": [k_hi, k_lo], "two_precision_percent_high": percent,
+         "saliency_score": "pair-norm product", "pruned_query_pairs": 0, "shrunk_to_low_bits": False,
+         "key_code_bits": bits, "bytes_per_token_head": (L_hi * R_hi + L_lo * R_lo) / 32 / ctx,
+         "split_ms": split_ms, "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
+         "frac_of_8tbs": alg / t / 8e12, "tokens_per_s": Bw / t, "replicas": n_rep}
+    if exact is not None:
+        got = out.cpu().numpy().astype(np.float64)
+        num = sum(float(np.sum((got[b, h * G:(h + 1) * G] - e) ** 2)) for (b, h), e in exact.items())
+        den = sum(float(np.sum(e ** 2)) for e in exact.values())
+        r["rel_l2_vs_bf16_attention"] = (num / den) ** 0.5
+    del reps, first, parts
+    return r
 
 
 def run_decode_workload(args):
@@ -456,6 +530,8 @@ def run_decode_workload(args):
                 r["rel_l2_vs_bf16_attention"] = (num / den) ** 0.5
             results.append(r)
             del cache, replicas
+        if wl.sweep and not args.shrunk_only:
+            results.append(two_part_point(args, pm, wl, k_dev, v_dev, qwin_dev, q_dev, exact, peak, l2_bytes))
     line = {"workload": args.workload, "metric": "decode-attn GB/s (% of B200 HBM peak) + tokens/s",
             "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "data": "synthetic", "dtype": "f32",
@@ -864,10 +940,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "stream_32k", "batch_per_gpu": B, "n_q_heads": HQ, "n_kv_heads": HKV,
-                   "head_dim": D, "context": CONTEXT, "prefill": PREFILL, "salient_pairs": K_SALIENT,
-                   "key_bits": [BHI, BLO], "value_bits": 2, "key_code_bits": 2.25,
-                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (419 MB cache read per step)"},
+        "config": stream_config(world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": captured_traffic(sum(alg) / K),
                      "algorithmic_bytes": sum(alg) / K, "kernel": "pnmix decode attention",

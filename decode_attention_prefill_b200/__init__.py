@@ -44,7 +44,8 @@ EXPORTED = [
     "pnmix_workspace_bytes", "pnmix_decode_attention", "pnmix_read_error",
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
     "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi", "pnmix_shrink_keys",
-    "pnmix_split_groups", "pnmix_debug_decode_stall",
+    "pnmix_split_groups", "pnmix_debug_decode_stall", "pnmix_workspace_bytes_two",
+    "pnmix_decode_attention_two",
 ]
 
 
@@ -107,6 +108,8 @@ _SIGS = {
     "pnmix_split_groups": (_i, [_CP, _i, _vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp]),
     "pnmix_debug_decode_stall": (_i, [_CP, _vp, _KP, _i, _vp, _vp, _sz, _i, ctypes.c_uint32, _vp]),
+    "pnmix_workspace_bytes_two": (_sz, [_CP, _CP, _i, _i, _i]),
+    "pnmix_decode_attention_two": (_i, [_CP, _KP, _i, _CP, _KP, _i, _vp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -219,6 +222,28 @@ def pnmix_shrink_keys(cfg: Config, src: "PNMixCache", dst: "PNMixCache", stream=
     """src: a cache of cfg (b_hi = 2 b_lo, k > 0); dst: a cache of cfg with n_salient_pairs = 0."""
     _check(_lib.pnmix_shrink_keys(ctypes.byref(cfg), ctypes.byref(src.c), ctypes.byref(dst.c), _stream(stream)),
            "pnmix_shrink_keys")
+
+
+def workspace_bytes_two(cfg_a: Config, cfg_b: Config, batch: int, max_context_a: int, max_context_b: int) -> int:
+    return int(_lib.pnmix_workspace_bytes_two(ctypes.byref(cfg_a), ctypes.byref(cfg_b), batch, max_context_a,
+                                              max_context_b))
+
+
+def pnmix_decode_attention_two(cache_a: "PNMixCache", cache_b: "PNMixCache", q: torch.Tensor, out: torch.Tensor,
+                               workspace: torch.Tensor | None = None, stream=None):
+    """Attention of q bf16 [B][Hq][128] over the union of two caches' tokens -> out fp32 [B][Hq][128]."""
+    if workspace is None:
+        n = workspace_bytes_two(cache_a.cfg, cache_b.cfg, cache_a.batch, cache_a.max_context, cache_b.max_context)
+        workspace = getattr(cache_b, "_two_ws", None)
+        if workspace is None or workspace.numel() < n:
+            ws = torch.zeros(n + 256, dtype=torch.uint8, device=q.device)
+            off = (-ws.data_ptr()) % 256
+            workspace = cache_b._two_ws = ws[off:off + n]
+    _check(_lib.pnmix_decode_attention_two(ctypes.byref(cache_a.cfg), ctypes.byref(cache_a.c), cache_a.max_context,
+                                           ctypes.byref(cache_b.cfg), ctypes.byref(cache_b.c), cache_b.max_context,
+                                           _dev(q, torch.bfloat16, "q"), _dev(out, torch.float32, "out"),
+                                           _dev(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                           _stream(stream)), "pnmix_decode_attention_two")
 
 
 def split_sizes(L: int, hi_percent: int) -> tuple[int, int]:

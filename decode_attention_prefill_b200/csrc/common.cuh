@@ -52,15 +52,24 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
 
-// fp16 element index of key position j in the scale / zero arrays.
+// fp16 element index of key position j in the scale / zero arrays: one 16-byte chunk per
+// (tq, slice pair) holds (even slice e=0, odd slice e=0, even slice e=1, odd slice e=1).
 __host__ __device__ __forceinline__ int kscale_index(int j) {
   int sigma = j >> 4, e = (j >> 3) & 1, tq = (j >> 1) & 3, v = j & 1;
-  return ((tq * 8 + sigma) * 2 + e) * 2 + v;
+  return ((tq * 4 + (sigma >> 1)) * 4 + 2 * e + (sigma & 1)) * 2 + v;
 }
 
 // fp16 element index of the value scale of (token t, channel group jg).
 __host__ __device__ __forceinline__ int vscale_index(int t, int jg) {
   return ((t >> 1) * 4 + jg) * 2 + (t & 1);
+}
+
+// fp16 element index of the value zero point of (token t, channel group jg): the token
+// pair tp = t / 2 of group jg sits in the 16-byte chunk (tp % 4, jg) at slot
+// tp / 8 + 2 * ((tp / 4) % 2), i.e. the chunk holds tp, tp + 8, tp + 4, tp + 12.
+__host__ __device__ __forceinline__ int vzero_index(int t, int jg) {
+  const int tp = t >> 1;
+  return ((((tp & 3) * 4 + jg) * 4) + ((tp >> 3) & 1) + 2 * ((tp >> 2) & 1)) * 2 + (t & 1);
 }
 
 // Byte offset (inside the value-code area) of value word m of lane L.
@@ -189,7 +198,15 @@ pnmix_status check_decode_args(const pnmix_config* cfg, const uint16_t* q, const
                                int max_context, const float* out, Geometry* g);
 size_t decode_workspace_bytes(const Geometry& g, int max_context);
 size_t decode_ticket_offset(const Geometry& g, int max_context);
+// Optional log-sum-exp output and merge with an earlier attention over other tokens (the
+// two parts of a two-precision cache); see combine_segment in decode_common.cuh.
+struct DecodeMerge {
+  float* lse_out = nullptr;
+  const float* prior_out = nullptr;
+  const float* prior_lse = nullptr;
+};
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c,
-                          int max_context, float* out, void* ws, cudaStream_t s);
+                          int max_context, float* out, void* ws, cudaStream_t s,
+                          const DecodeMerge& merge = DecodeMerge());
 
 }  // namespace pnmix

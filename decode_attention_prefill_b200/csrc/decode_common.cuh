@@ -29,6 +29,11 @@ struct DecodeWs {
   float* part;         // [slots][G][kPartialStride]
   uint32_t* tickets;   // [units], zero between calls
   int N;               // CTAs of the launch
+  // Optional outputs / inputs of the final combine (all indexed like `out` by row_offset,
+  // one float per row for the log-sum-exps):
+  float* lse_out;            // if set: log2 sum_t 2^(logit_t) of every output row
+  const float* prior_out;    // if set: merge with an earlier attention over other tokens,
+  const float* prior_lse;    //   given by its normalised output and log-sum-exp
 };
 
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -121,9 +126,14 @@ __device__ __forceinline__ int visible_tokens(const Geometry& g, int len, int v)
 }
 
 // Called by every thread of the CTA after the segment's partials are in its slot: the
-// CTA that takes the unit's last ticket writes the unit's G = g.rows output rows.
-__device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G,
-                                                float* out, const Geometry& geo) {
+// CTA that takes the unit's last ticket writes the unit's G = g.rows output rows.  With
+// ws.lse_out it also writes each row's log-sum-exp L = m* + log2(sum_s l_s 2^(m_s - m*))
+// (log2 domain of the scaled logits; -inf for a row that sees no token).  With
+// ws.prior_out / prior_lse the row is merged with an attention over other tokens:
+//   out = (2^(L0 - M) o0 + 2^(L - M) o) / (2^(L0 - M) + 2^(L - M)),  M = max(L0, L),
+// and the log-sum-exp written is that of the union, M + log2(2^(L0 - M) + 2^(L - M)).
+__device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G, float* out,
+                                                const Geometry& geo) {
   __shared__ int is_last;
   __threadfence();
   __syncthreads();
@@ -136,9 +146,11 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
     // with independent loads
     __shared__ float wsh[kMaxG][kMaxCombineSegs];
     __shared__ float den_sh[kMaxG];
+    __shared__ float mix_sh[kMaxG][2];   // weights of the prior row and of this one
     const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;
     for (unsigned chunk = 0; chunk < nseg; chunk += kMaxCombineSegs) {
       const unsigned n = nseg - chunk < kMaxCombineSegs ? nseg - chunk : kMaxCombineSegs;
+      const bool last_chunk = chunk + n == nseg;
       if (threadIdx.x < G) {
         const int hh = threadIdx.x;
         float m = -INFINITY;
@@ -153,18 +165,42 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
           if (k >= chunk && k < chunk + n) wsh[hh][k - chunk] = f;
         }
         den_sh[hh] = den;
+        if (last_chunk && (ws.lse_out || ws.prior_out)) {
+          const size_t row = row_offset(geo, s.b, s.h, hh) / kHeadDim;
+          float L = den > 0.f ? m + log2f(den) : -INFINITY;
+          float w0 = 0.f, w1 = den > 0.f ? 1.f : 0.f;
+          if (ws.prior_out) {
+            const float L0 = ws.prior_lse[row];
+            const float M = fmaxf(L0, L);
+            w0 = L0 == -INFINITY ? 0.f : exp2f(L0 - M);
+            w1 = L == -INFINITY ? 0.f : exp2f(L - M);
+            const float t = w0 + w1;
+            L = t > 0.f ? M + log2f(t) : -INFINITY;
+            w0 = t > 0.f ? w0 / t : 0.f;
+            w1 = t > 0.f ? w1 / t : 0.f;
+          }
+          mix_sh[hh][0] = w0;
+          mix_sh[hh][1] = w1;
+          if (ws.lse_out) ws.lse_out[row] = L;
+        }
       }
       __syncthreads();
       for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
         const int hh = i / kHeadDim, c = i % kHeadDim;
-        float* out_row = out + row_offset(geo, s.b, s.h, hh);
+        const size_t off = row_offset(geo, s.b, s.h, hh);
+        float* out_row = out + off;
         float num = chunk == 0 ? 0.f : out_row[c];
 #pragma unroll 4
         for (unsigned k = 0; k < n; ++k)
           num = fmaf(__ldcg(base + (static_cast<size_t>(chunk + k) * G + hh) * kPartialStride + 2 + c),
                      wsh[hh][k], num);
-        const bool last_chunk = chunk + n == nseg;
-        out_row[c] = last_chunk ? (den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f) : num;
+        if (last_chunk) {
+          float o = den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f;
+          if (ws.prior_out) o = fmaf(mix_sh[hh][0], ws.prior_out[off + c], mix_sh[hh][1] * o);
+          out_row[c] = o;
+        } else {
+          out_row[c] = num;
+        }
       }
       __syncthreads();
     }

@@ -1,24 +1,31 @@
 // decode_mma.cu -- tensor-core decode attention over the packed cache, one role per warp.
 //
 // One CTA = one slice of the work partition (decode_common.cuh), 4 warps.  Every warp
-// owns whole 32-token group records (interleaved across the warps), stages them with TMA
-// bulk copies into its own shared-memory ring (6 slots when it takes its groups in pairs),
-// and keeps its own online softmax.  Per group:
+// takes a contiguous run of each segment's 32-token group records, stages them two
+// records per TMA bulk copy into its own shared-memory ring of record pairs, and keeps its
+// own online softmax.  Per group:
 //
 //   logits  q . k^_t = sum_p q_p (s_p code_{p,t} + z_p)
-//          = [codes (32 tok x 128 pos)] x [q_p s_p]  +  [z broadcast] x [q]
+//          = [codes (32 tok x 128 pos)] x [q_p s_p]  +  [z] x [q]
 //   The codes become exact fp16 A fragments in registers: an AND leaves them as fp16
 //   subnormals code * 2^(offset-24), which the tensor cores multiply exactly.  The bf16
 //   query is exact in fp16; the product q_p s_p (19 significant bits) is carried exactly
 //   by two interleaved B columns (head h -> columns 2h, 2h+1): fp16(q s) and its rounding
 //   error fma(q, s, -fp16(q s)).  One lane-uniform sequence b = fma(X, s, fp16(Y s)) with
 //   per-lane constants (X, Y) = (0, q) on even columns and (q, -q) on odd ones gives both.
-//   The zero-point term is one more MMA per slice with the z pairs broadcast over the
-//   rows and X as B (the pair of columns then sums to q).  The softmax scale is applied
-//   to the fp32 logits.
+//   The zero-point term is one more MMA per slice whose A operand is the 16-byte zero-point
+//   chunk of the slice pair exactly as loaded (rows 0-7 carry the even slice's zeros, rows
+//   8-15 the odd slice's, see the key scale order in include/pnmix.h) and whose B operand
+//   is X; the even slice's sum is read from rows 0-7 of one accumulator, the odd slice's
+//   from rows 8-15 of another.  The softmax scale is applied to the fp32 logits.
 //   out     sum_t p_t v^_t = sum_t (p_t s_{t,j}) code_{t,c} + sum_t p_t z_{t,j}
 //          = [codes^T (channels x tokens)] x [p s]  +  [z rows] x [p]
-//   with p rounded to fp16 once (fp32 accumulation).
+//   with p rounded to fp16 once (fp32 accumulation); the value zero-point chunk of a lane
+//   likewise serves both 16-token halves of a group from one load.
+//
+// The online softmax keeps a lazy reference m per head: a group pair only takes the
+// cross-lane max when one of its logits exceeds m, and then sets m = max + kHeadroom, so
+// p = 2^(logit - m) <= 1 and the accumulators are rescaled a few times per segment.
 //
 // The bit placement of the record (include/pnmix.h) is the fragment ownership of the
 // m16n8k16 tiles, so a lane's code words are exactly its A registers.  Splits merge
@@ -35,12 +42,13 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-// Staging ring per warp: 6 slots when the warp consumes its groups in pairs (G <= 4),
-// 3 when it takes them one at a time (G <= 8).
+// Headroom (log2 domain) the lazy softmax reference keeps above the largest logit seen.
+constexpr float kHeadroom = 4.f;
+// Staging ring per warp, in record pairs: 3 pairs (6 records) with one tile of query
+// columns (up to 4 rows, two CTAs per SM), 2 pairs with two tiles (three CTAs per SM).
 template <int NT>
-__host__ __device__ constexpr int stages_for() { return NT == 1 ? 6 : 3; }
-template <int NT>
-__host__ __device__ constexpr int groups_per_step() { return NT == 1 ? 2 : 1; }
+__host__ __device__ constexpr int pair_slots() { return NT == 1 ? 3 : 2; }
+
 // ------------------------------------------------------------------ shared memory map
 
 struct SmemMap {
@@ -49,14 +57,14 @@ struct SmemMap {
   int perm;      // 128 bytes
   int resid;     // fp32 [kMaxG][kPartialStride]: partial of the residual item
   int rrows;     // bf16 residual K rows [32][kResidKStride] then V rows [32][128]
-  int bars;      // uint64 [kWarps][stages] mbarriers
-  int stages;    // [kWarps][stages][R]
+  int bars;      // uint64 [kWarps][slots] mbarriers
+  int stages;    // [kWarps][slots][2 R]
   int part;      // fp32 [kWarps][kMaxG][kPartialStride], aliases the stages
   int total;
 };
 
 __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
-  const int nst = NT == 1 ? stages_for<1>() : stages_for<2>();
+  const int nsl = NT == 1 ? pair_slots<1>() : pair_slots<2>();
   SmemMap m;
   m.qsets = 0;
   m.qnat = NT * 2 * 4 * 32 * 16;
@@ -64,8 +72,8 @@ __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
   m.resid = m.perm + 128;
   m.rrows = m.resid + kMaxG * kPartialStride * 4;
   m.bars = m.rrows + kGroup * kResidKStride * 2 + kGroup * kHeadDim * 2;
-  m.stages = m.bars + ((kWarps * nst * 8 + 127) / 128) * 128;
-  int stage_bytes = kWarps * nst * R;
+  m.stages = m.bars + ((kWarps * nsl * 8 + 127) / 128) * 128;
+  int stage_bytes = kWarps * nsl * 2 * R;
   int part_bytes = kWarps * kMaxG * kPartialStride * 4;
   m.part = m.stages;
   m.total = m.stages + (stage_bytes > part_bytes ? stage_bytes : part_bytes);
@@ -76,131 +84,126 @@ __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
 
 template <int NT>
 struct WarpAcc {
-  float m[NT];          // running max (log2 domain) of head 4*nt + tq
+  float m[NT];          // lazy softmax reference (log2 domain) of head 4*nt + tq
   float l[NT];          // this lane's partial sum of 2^(logit - m)
   float pv[8][4];       // P.V accumulators: channels 16m + gq (+8), heads 2tq, 2tq+1
-  float bias[4];        // zero-point term: row gq = channel group, heads 2tq, 2tq+1
+  float bias[2][4];     // zero-point term: [0] rows 0-7 (first 16 tokens of each group),
+                        // [1] rows 8-15 (last 16); row gq = channel group, heads 2tq, 2tq+1
 };
 
-// NG group records at recs[0..NG) (shared memory, consecutive groups of this warp)
-// folded into the warp's state.  With NG = 2 the two groups' q.k^ chains interleave and
-// one online-softmax update covers both (64 tokens).
+// Logit scale factors: a row-u token's key products carry 2^(shift(u) - 24).
+template <int BHI, int BLO>
+struct RowScale {
+  float hi[4], lo[4];
+  __device__ __forceinline__ explicit RowScale(float qscale) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      hi[u] = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23) * qscale;
+      lo[u] = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23) * qscale;
+    }
+  }
+};
 
 // Key side of NG group records: the log2-domain logits lg[gi][nt][u] of head 4*nt + tq at
-// tokens gq + 8u of group gi.
+// tokens gq + 8u of group gi.  With NG = 2 the two groups' MMA chains interleave.
 template <int BHI, int BLO, int NT, int NHS, int NG, bool MQ>
 __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* const (&recs)[NG],
-                                             const QFrags<NT>& qf, float qscale, const int (&tok0)[NG],
-                                             int vis_base, float (&lg)[NG][NT][4]) {
+                                             const QFrags<NT>& qf, float qscale, const RowScale<BHI, BLO>& rs,
+                                             const int (&tok0)[NG], int vis_base, float (&lg)[NG][NT][4]) {
   constexpr int WH = NHS * BHI / 2;   // key-code words per lane of the salient block
-  constexpr int PAR = NG == 1 ? 2 : 1;   // accumulation chains per block (split by slice parity)
+  constexpr int kc = key_code_bytes<BHI, BLO, NHS>();
   const int lane = threadIdx.x & 31;
   const int tq = lane & 3;
-  const int kc = g.kc_bytes;
 
   // key-code products, kept apart per block because the two blocks' token-row bit
-  // offsets differ; the zero-point term separately (normal fp16 scale)
-  float acc_hi[NG][NT][2][4], acc_lo[NG][PAR][NT][2][4], dz[NG][PAR][NT][4];
+  // offsets differ; the zero-point term per slice parity (normal fp16 scale)
+  float acc_hi[NG][NT][2][4], acc_lo[NG][NT][2][4], dz[NG][NT][2][4];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc_hi[gi][nt][0][i] = 0.f;
-        acc_hi[gi][nt][1][i] = 0.f;
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int pr = 0; pr < PAR; ++pr) {
-          acc_lo[gi][pr][nt][0][i] = 0.f;
-          acc_lo[gi][pr][nt][1][i] = 0.f;
-          dz[gi][pr][nt][i] = 0.f;
+        for (int x = 0; x < 2; ++x) {
+          acc_hi[gi][nt][x][i] = 0.f;
+          acc_lo[gi][nt][x][i] = 0.f;
+          dz[gi][nt][x][i] = 0.f;
         }
-      }
 
-  uint4 s4[NG], z4[NG];
 #pragma unroll
-  for (int sigma = 0; sigma < 8; ++sigma) {
-    const int par = sigma & 1, pr = PAR == 2 ? par : 0;
-    if (par == 0) {
-      // key scales / zeros of this lane: fp16x2 index sigma*2 + e
-#pragma unroll
-      for (int gi = 0; gi < NG; ++gi) {
-        s4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + tq * 64)[sigma >> 1];
-        z4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + 256 + tq * 64)[sigma >> 1];
-      }
-    }
-    const bool hi = sigma < NHS;
+  for (int sp = 0; sp < 4; ++sp) {
+    // this lane's scale / zero chunk of slice pair sp: (even e=0, odd e=0, even e=1, odd e=1)
+    uint4 s4[NG], z4[NG];
 #pragma unroll
     for (int gi = 0; gi < NG; ++gi) {
-      // ---- A fragments of this slice (2 M-tiles x 4 registers)
-      const uint32_t* kw = reinterpret_cast<const uint32_t*>(recs[gi]);
-      uint32_t A[2][4];
-      if (hi) {
-        if constexpr (BHI == 4)
-          key_slice_frags<4>(kw[(2 * sigma) * 32 + lane], kw[(2 * sigma + 1) * 32 + lane], 0, A);
-        else
-          key_slice_frags<BHI>(kw[sigma * 32 + lane], 0u, 0, A);
-      } else {
-        const int sl = sigma - NHS;   // slice inside the lo block
-        if constexpr (BLO == 2)
-          key_slice_frags<2>(kw[(WH + sl) * 32 + lane], 0u, 0, A);
-        else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
-          key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, par, A);
-      }
-      // ---- B fragments: fp16(q s) on even columns, its rounding error on odd ones;
-      // X alone (q on odd columns) for the zero-point term
+      s4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + tq * 64)[sp];
+      z4[gi] = reinterpret_cast<const uint4*>(recs[gi] + kc + 256 + tq * 64)[sp];
+    }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint4& X = qf.x[nt][sigma >> 1];
-        const uint4& Y = qf.y[nt][sigma >> 1];
-        const uint32_t qx0 = par ? X.z : X.x, qx1 = par ? X.w : X.y;
-        const uint32_t qy0 = par ? Y.z : Y.x, qy1 = par ? Y.w : Y.y;
-        const uint32_t s0 = par ? s4[gi].z : s4[gi].x, s1 = par ? s4[gi].w : s4[gi].y;
-        const uint32_t b0 = hfma2(qx0, s0, hmul2(qy0, s0));
-        const uint32_t b1 = hfma2(qx1, s1, hmul2(qy1, s1));
+    for (int par = 0; par < 2; ++par) {
+      const int sigma = 2 * sp + par;
+      const bool hi = sigma < NHS;
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        // ---- A fragments of this slice (2 M-tiles x 4 registers)
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(recs[gi]);
+        uint32_t A[2][4];
         if (hi) {
-          mma16816(acc_hi[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-          mma16816(acc_hi[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+          if constexpr (BHI == 4)
+            key_slice_frags<4>(kw[(2 * sigma) * 32 + lane], kw[(2 * sigma + 1) * 32 + lane], 0, A);
+          else
+            key_slice_frags<BHI>(kw[sigma * 32 + lane], 0u, 0, A);
         } else {
-          mma16816(acc_lo[gi][pr][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
-          mma16816(acc_lo[gi][pr][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+          const int sl = sigma - NHS;   // slice inside the lo block
+          if constexpr (BLO == 2)
+            key_slice_frags<2>(kw[(WH + sl) * 32 + lane], 0u, 0, A);
+          else   // two slices per word; NHS is even, so sl % 2 == sigma % 2
+            key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, par, A);
         }
-        if constexpr (NG == 1) {
-          const uint32_t z0 = par ? z4[0].z : z4[0].x, z1 = par ? z4[0].w : z4[0].y;
-          mma16816(dz[0][pr][nt], z0, z0, z1, z1, qx0, qx1);
-        } else if (gi == NG - 1) {
-          // both groups' zero points in one product: rows 0-7 group 0, rows 8-15 group 1
-          const uint32_t za0 = par ? z4[0].z : z4[0].x, za1 = par ? z4[0].w : z4[0].y;
-          const uint32_t zb0 = par ? z4[1].z : z4[1].x, zb1 = par ? z4[1].w : z4[1].y;
-          mma16816(dz[0][pr][nt], za0, zb0, za1, zb1, qx0, qx1);
+        const uint32_t s0 = par ? s4[gi].y : s4[gi].x, s1 = par ? s4[gi].w : s4[gi].z;
+        // ---- B fragments: fp16(q s) on even columns, its rounding error on odd ones;
+        // X alone (q on odd columns) for the zero-point term
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4& X = qf.x[nt][sp];
+          const uint4& Y = qf.y[nt][sp];
+          const uint32_t qx0 = par ? X.z : X.x, qx1 = par ? X.w : X.y;
+          const uint32_t qy0 = par ? Y.z : Y.x, qy1 = par ? Y.w : Y.y;
+          const uint32_t b0 = hfma2(qx0, s0, hmul2(qy0, s0));
+          const uint32_t b1 = hfma2(qx1, s1, hmul2(qy1, s1));
+          if (hi) {
+            mma16816(acc_hi[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+            mma16816(acc_hi[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+          } else {
+            mma16816(acc_lo[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
+            mma16816(acc_lo[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
+          }
+          mma16816(dz[gi][nt][par], z4[gi].x, z4[gi].y, z4[gi].z, z4[gi].w, qx0, qx1);
         }
       }
     }
   }
 
-  // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3;
-  // the product of a row-u token carries 2^(shift(u) - 24)
+  // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3; the
+  // zero-point sum of the head is on its odd column (X is zero on even ones): rows 0-7 of
+  // the even-slice accumulator plus rows 8-15 of the odd-slice one
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      // zero-point term of this group: rows 0-7 (c0, c1) hold group 0, rows 8-15 (c2, c3)
-      // hold group 1 when two groups share the product
-      float zb = 0.f;
-#pragma unroll
-      for (int pr = 0; pr < PAR; ++pr)
-        zb += gi == 0 ? dz[0][pr][nt][0] + dz[0][pr][nt][1] : dz[0][pr][nt][2] + dz[0][pr][nt][3];
-      zb *= qscale;
+      const float zb = (dz[gi][nt][0][1] + dz[gi][nt][1][3]) * qscale;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int mt = u >> 1, r = 2 * (u & 1);
-        const float fh = __int_as_float((127 + 24 - key_row_shift<BHI>(u)) << 23) * qscale;
-        const float fl = __int_as_float((127 + 24 - key_row_shift<BLO>(u)) << 23) * qscale;
         const float vhi = acc_hi[gi][nt][mt][r] + acc_hi[gi][nt][mt][r + 1];
-        float vlo = 0.f;
-#pragma unroll
-        for (int pr = 0; pr < PAR; ++pr) vlo += acc_lo[gi][pr][nt][mt][r] + acc_lo[gi][pr][nt][mt][r + 1];
-        lg[gi][nt][u] = fmaf(vhi, fh, fmaf(vlo, fl, zb));
+        const float vlo = acc_lo[gi][nt][mt][r] + acc_lo[gi][nt][mt][r + 1];
+        if constexpr (NHS == 0)
+          lg[gi][nt][u] = fmaf(vlo, rs.lo[u], zb);
+        else if constexpr (NHS == 8)
+          lg[gi][nt][u] = fmaf(vhi, rs.hi[u], zb);
+        else
+          lg[gi][nt][u] = fmaf(vhi, rs.hi[u], fmaf(vlo, rs.lo[u], zb));
       }
     }
 
@@ -223,59 +226,71 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* c
   }
 }
 
-// Value side of NG group records with their logits: online softmax update, P as B
-// fragments, P x V into the warp's accumulators.
-template <int NT, int NG>
-__device__ __forceinline__ void group_softmax_values(const Geometry& g, const uint8_t* const (&recs)[NG],
-                                                     const float (&lg)[NG][NT][4], WarpAcc<NT>& st) {
+// Multiply the value-side accumulators by the per-head factors alpha (lane holds heads tq
+// and 4 + tq in alpha[0], alpha[1]; the accumulator columns are heads 2tq, 2tq+1).
+template <int NT>
+__device__ __forceinline__ void rescale_values(WarpAcc<NT>& st, const float (&alpha)[NT]) {
   const int lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
-  const int kc = g.kc_bytes;
+  const int h0 = 2 * tq, h1 = 2 * tq + 1;
+  float a0 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h0 & 3));
+  float a1 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h1 & 3));
+  if constexpr (NT == 2) {
+    const float b0 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h0 & 3));
+    const float b1 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h1 & 3));
+    if (h0 >= 4) a0 = b0;
+    if (h1 >= 4) a1 = b1;
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    st.pv[m][0] *= a0;
+    st.pv[m][1] *= a1;
+    st.pv[m][2] *= a0;
+    st.pv[m][3] *= a1;
+  }
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    st.bias[x][0] *= a0;
+    st.bias[x][1] *= a1;
+    st.bias[x][2] *= a0;
+    st.bias[x][3] *= a1;
+  }
+}
 
-  // ---- online softmax over the NG groups
-  float mnew[NT];
-  bool grow = false;
+// Value side of NG group records with their logits: lazy online softmax update, P as B
+// fragments, P x V into the warp's accumulators.
+template <int NT, int NG, bool MQ>
+__device__ __forceinline__ void group_softmax_values(const Geometry& g, const uint8_t* const (&recs)[NG],
+                                                     const float (&lg)[NG][NT][4], WarpAcc<NT>& st, int kc) {
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+
+  // ---- lazy reference: the cross-lane max only when a logit exceeds the reference
+  float mloc[NT];
+  bool raise = false;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float mx = -INFINITY;
 #pragma unroll
     for (int gi = 0; gi < NG; ++gi)
       mx = fmaxf(mx, fmaxf(fmaxf(lg[gi][nt][0], lg[gi][nt][1]), fmaxf(lg[gi][nt][2], lg[gi][nt][3])));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    mnew[nt] = fmaxf(st.m[nt], mx);
-    grow |= mnew[nt] > st.m[nt];
+    mloc[nt] = mx;
+    raise |= mx > st.m[nt];
   }
-  if (__any_sync(0xffffffffu, grow)) {
+  if (__any_sync(0xffffffffu, raise)) {
     float alpha[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      alpha[nt] = ex2(st.m[nt] - mnew[nt]);
+      float mx = mloc[nt];
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mnew = mx > st.m[nt] ? mx + kHeadroom : st.m[nt];
+      alpha[nt] = mnew == st.m[nt] ? 1.f : ex2(st.m[nt] - mnew);   // 0 from -inf
       st.l[nt] *= alpha[nt];
-      st.m[nt] = mnew[nt];
+      st.m[nt] = mnew;
     }
-    // P.V columns of this lane are heads 2tq and 2tq+1
-    const int h0 = 2 * tq, h1 = 2 * tq + 1;
-    float a0 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h0 & 3));
-    float a1 = __shfl_sync(0xffffffffu, alpha[0], gq * 4 + (h1 & 3));
-    if constexpr (NT == 2) {
-      const float b0 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h0 & 3));
-      const float b1 = __shfl_sync(0xffffffffu, alpha[1], gq * 4 + (h1 & 3));
-      if (h0 >= 4) a0 = b0;
-      if (h1 >= 4) a1 = b1;
-    }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      st.pv[m][0] *= a0;
-      st.pv[m][1] *= a1;
-      st.pv[m][2] *= a0;
-      st.pv[m][3] *= a1;
-    }
-    st.bias[0] *= a0;
-    st.bias[1] *= a1;
-    st.bias[2] *= a0;
-    st.bias[3] *= a1;
+    rescale_values<NT>(st, alpha);
   }
 
   const int srcA = (2 * tq) * 4 + (gq & 3), srcB = (2 * tq + 1) * 4 + (gq & 3);
@@ -289,7 +304,10 @@ __device__ __forceinline__ void group_softmax_values(const Geometry& g, const ui
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        p[nt][i] = ex2(lg[gi][nt][i] - st.m[nt]);
+        if constexpr (MQ)   // a head that sees no token yet keeps m = -inf: its masked logits give 0
+          p[nt][i] = lg[gi][nt][i] == -INFINITY ? 0.f : ex2(lg[gi][nt][i] - st.m[nt]);
+        else
+          p[nt][i] = ex2(lg[gi][nt][i] - st.m[nt]);
         st.l[nt] += p[nt][i];
       }
     }
@@ -315,7 +333,7 @@ __device__ __forceinline__ void group_softmax_values(const Geometry& g, const ui
 #pragma unroll
     for (int i = 0; i < 4; ++i) p16[i] = col_ok ? pack_f16x2(pa[i], pb[i]) : 0u;
 
-    // value scales: token pairs tp2 = tq + 4i, four channel groups each
+    // value scales: token pairs tq + 4i, four channel groups each
     const int vs_off = kc + 1536, vz_off = kc + 1792;
     uint32_t vsr[4][4];
 #pragma unroll
@@ -323,17 +341,14 @@ __device__ __forceinline__ void group_softmax_values(const Geometry& g, const ui
       const uint4 v = *reinterpret_cast<const uint4*>(rec + vs_off + (tq + 4 * i) * 16);
       vsr[i][0] = v.x; vsr[i][1] = v.y; vsr[i][2] = v.z; vsr[i][3] = v.w;
     }
-    // zero-point term: A rows = channel groups (rows 0..3), k = tokens
+    // zero-point term: A rows = channel groups (row gq holds group gq & 3; rows 4-7 repeat
+    // them and are not read), k = tokens.  The chunk (tq, j) holds the zero pairs of token
+    // pairs tq, tq + 8, tq + 4, tq + 12: as one A operand its rows 0-7 are the first 16
+    // tokens (with P of tokens 0-15) and its rows 8-15 the last 16 (with P of tokens 16-31).
     {
-      const int j = gq & 3;
-      uint32_t vz[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
-        vz[i] = gq < 4 ? v : 0u;
-      }
-      mma16816(st.bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
-      mma16816(st.bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
+      const uint4 zc = *reinterpret_cast<const uint4*>(rec + vz_off + (tq * 4 + (gq & 3)) * 16);
+      mma16816(st.bias[0], zc.x, zc.y, zc.z, zc.w, p16[0], p16[1]);
+      mma16816(st.bias[1], zc.x, zc.y, zc.z, zc.w, p16[2], p16[3]);
     }
     // value codes: words 0..7 of this lane (two 16-byte chunks).  Slot (r, p) of word m
     // sits at bits 8r + 2p; it is taken in place from w >> 8r, so token block p carries
@@ -363,11 +378,11 @@ __device__ __forceinline__ void group_softmax_values(const Geometry& g, const ui
 
 template <int BHI, int BLO, int NT, int NHS, int NG, bool MQ>
 __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t* const (&recs)[NG],
-                                               const QFrags<NT>& qf, float qscale, const int (&tok0)[NG],
-                                               int vis_base, WarpAcc<NT>& st) {
+                                               const QFrags<NT>& qf, float qscale, const RowScale<BHI, BLO>& rs,
+                                               const int (&tok0)[NG], int vis_base, WarpAcc<NT>& st) {
   float lg[NG][NT][4];
-  group_logits<BHI, BLO, NT, NHS, NG, MQ>(g, recs, qf, qscale, tok0, vis_base, lg);
-  group_softmax_values<NT, NG>(g, recs, lg, st);
+  group_logits<BHI, BLO, NT, NHS, NG, MQ>(g, recs, qf, qscale, rs, tok0, vis_base, lg);
+  group_softmax_values<NT, NG, MQ>(g, recs, lg, st, key_code_bytes<BHI, BLO, NHS>());
 }
 
 // MQ: several queries per sequence (rows = G * tq), with the causal mask on the newest
@@ -377,9 +392,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 3)
 decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
                   DecodeWs ws) {
   extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int R = record_bytes_of<BHI, BLO, NHS>();
+  constexpr int kSlots = pair_slots<NT>();
   const int G = g.rows;   // query rows per unit
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int R = g.record_bytes;
   const SmemMap sm = smem_map(NT, R);
   uint32_t* qsets = reinterpret_cast<uint32_t*>(smem + sm.qsets);
   float* qnat = reinterpret_cast<float*>(smem + sm.qnat);
@@ -388,61 +404,72 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
   uint16_t* rrk = reinterpret_cast<uint16_t*>(smem + sm.rrows);
   uint16_t* rrv = rrk + kGroup * kResidKStride;
   float* part = reinterpret_cast<float*>(smem + sm.part);
-  constexpr int kS = stages_for<NT>();
-  uint8_t* ring = smem + sm.stages + warp * kS * R;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm.bars) + warp * kS;
+  uint8_t* ring = smem + sm.stages + warp * kSlots * 2 * R;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm.bars) + warp * kSlots;
   if (lane == 0) {
-    for (int k = 0; k < kS; ++k) mbar_init(bars + k, 1);
+    for (int k = 0; k < kSlots; ++k) mbar_init(bars + k, 1);
     fence_mbar_init();
   }
   __syncwarp();
-  // A warp's staged groups are numbered in order across its segments: ordinal o lives in
-  // slot o % kS and completes phase (o / kS) & 1 of that slot's barrier.
-  uint32_t ord_base = 0;
+  // The ring is used in order across the warp's segments: pairs are issued into slot
+  // `iss_slot` and taken from slot `use_slot`, whose barrier completes phase `use_phase`.
+  int iss_slot = 0, use_slot = 0;
+  uint32_t use_phase = 0;
   bool failed = false;   // a staging wait ran out: stage and consume nothing more
+  const float qscale = g.scale * kLog2e;
+  const RowScale<BHI, BLO> rs(qscale);
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
     const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
-    // ---- this warp's groups of the segment; stage the first ones right away
+    // ---- this warp's contiguous run [g0, g0 + my_count) of the segment's groups, taken
+    // as pairs of consecutive records (a last single record when the count is odd)
     const int gend = seg.hi < seg.ng ? seg.hi : seg.ng;
-    const int my_first = seg.lo + warp;
-    const int my_count = my_first < gend ? (gend - my_first + kWarps - 1) / kWarps : 0;
+    const int n = gend > seg.lo ? gend - seg.lo : 0;
+    const int g0 = seg.lo + (n * warp) / kWarps;
+    const int my_count = seg.lo + (n * (warp + 1)) / kWarps - g0;
+    const int my_pairs = (my_count + 1) >> 1;
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
-    int issued = 0;     // groups of this segment handed to the copy engine
-    int consumed = 0;   // groups of this segment whose copies have landed and been taken
     const bool stage = unit != g.skip_unit;   // false only under the timeout test hook
-    // Issue the warp's groups [issued, upto) of this segment.  Ordinal j may only be
-    // issued while j - (first unconsumed ordinal) < kS, which the callers keep.
+    int issued = 0;     // pairs of this segment handed to the copy engine
+    int consumed = 0;   // pairs of this segment taken from the ring
+    // Issue the warp's pairs [issued, upto).  A pair may only be issued into a slot whose
+    // previous pair has been consumed, which the callers keep (upto <= consumed + kSlots).
     auto issue_upto = [&](int upto) {
-      const int last = upto < my_count ? upto : my_count;
+      const int last = upto < my_pairs ? upto : my_pairs;
       if (failed || !stage) return;
       for (; issued < last; ++issued) {
-        const uint32_t o = ord_base + issued, slot = o % kS;
-        stage_group(ring + slot * R, unit_rec + static_cast<size_t>(my_first + issued * kWarps) * R,
-                    static_cast<uint32_t>(R), bars + slot, lane == 0);
+        const int gi = 2 * issued;
+        const uint32_t bytes = static_cast<uint32_t>(gi + 1 < my_count ? 2 * R : R);
+        stage_group(ring + iss_slot * 2 * R, unit_rec + static_cast<size_t>(g0 + gi) * R, bytes, bars + iss_slot,
+                    lane == 0);
+        iss_slot = iss_slot + 1 == kSlots ? 0 : iss_slot + 1;
       }
     };
-    // wait until the group of ordinal ord_base + i has landed; returns its record
-    auto acquire = [&](int i) -> const uint8_t* {
-      const uint32_t o = ord_base + i, slot = o % kS, phase = (o / kS) & 1;
+    // wait until the next pair has landed; returns its slot (or nullptr after a timeout)
+    auto acquire = [&]() -> const uint8_t* {
       uint32_t spins = 0;
-      while (!failed && !mbar_try_wait(bars + slot, phase)) {
+      while (!failed && !mbar_try_wait(bars + use_slot, use_phase)) {
         if (++spins >= g.wait_limit) {
           failed = true;
           if (lane == 0) atomicOr(c.error, PNMIX_DEVERR_TIMEOUT);
         }
       }
       failed = __any_sync(0xffffffffu, failed);   // keep the warp's control flow uniform
-      if (!failed) consumed = i + 1;
-      return ring + slot * R;
+      if (failed) return nullptr;
+      const uint8_t* r = ring + use_slot * 2 * R;
+      if (++use_slot == kSlots) {
+        use_slot = 0;
+        use_phase ^= 1u;
+      }
+      ++consumed;
+      return r;
     };
-    issue_upto(kS - groups_per_step<NT>());
+    issue_upto(kSlots);
 
     // ---- query: unscaled fp32 in natural channel order, then the X / Y fp16 column sets
     // in position order
     perm[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid];
-    const float qscale = g.scale * kLog2e;
     for (int i = tid; i < kMaxG * kHeadDim; i += kThreads) {
       const int hh = i / kHeadDim;
       qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
@@ -517,33 +544,45 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 #pragma unroll
       for (int i = 0; i < 4; ++i) st.pv[m][i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) st.bias[i] = 0.f;
-
-    int i = 0;
-    if constexpr (groups_per_step<NT>() == 2) {
-      for (; i + 1 < my_count; i += 2) {
-        issue_upto(i + kS);
-        const uint8_t* const recs[2] = {acquire(i), acquire(i + 1)};
-        const int tok[2] = {(my_first + i * kWarps) * kGroup, (my_first + (i + 1) * kWarps) * kGroup};
-        if (!failed) process_groups<BHI, BLO, NT, NHS, 2, MQ>(g, recs, qf, qscale, tok, vis_base, st);
-        __syncwarp();
-      }
+    for (int i = 0; i < 4; ++i) {
+      st.bias[0][i] = 0.f;
+      st.bias[1][i] = 0.f;
     }
-    for (; i < my_count; ++i) {
-      issue_upto(i + kS);
-      const uint8_t* const recs[1] = {acquire(i)};
-      const int tok[1] = {(my_first + i * kWarps) * kGroup};
-      if (!failed) process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, recs, qf, qscale, tok, vis_base, st);
+
+    for (int i = 0; i < my_pairs; ++i) {
+      issue_upto(i + kSlots);
+      const uint8_t* slot = acquire();
+      if (slot == nullptr) break;   // warp-uniform
+      const int ga = g0 + 2 * i;
+      if (2 * i + 1 < my_count) {
+        const uint8_t* const recs[2] = {slot, slot + R};
+        const int tok[2] = {ga * kGroup, (ga + 1) * kGroup};
+        if constexpr (NT == 1) {
+          process_groups<BHI, BLO, NT, NHS, 2, MQ>(g, recs, qf, qscale, rs, tok, vis_base, st);
+        } else {   // two tiles of query columns: one group at a time
+          const uint8_t* const r0[1] = {recs[0]};
+          const uint8_t* const r1[1] = {recs[1]};
+          const int t0[1] = {tok[0]}, t1[1] = {tok[1]};
+          process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, r0, qf, qscale, rs, t0, vis_base, st);
+          process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, r1, qf, qscale, rs, t1, vis_base, st);
+        }
+      } else {
+        const uint8_t* const recs[1] = {slot};
+        const int tok[1] = {ga * kGroup};
+        process_groups<BHI, BLO, NT, NHS, 1, MQ>(g, recs, qf, qscale, rs, tok, vis_base, st);
+      }
       __syncwarp();
     }
-    if (failed) {   // let the copies issued and not yet taken land before the shared memory is reused
-      for (int k = consumed; k < issued; ++k) {
-        const uint32_t o = ord_base + k;
-        for (uint32_t spins = 0; spins < g.wait_limit && !mbar_try_wait(bars + o % kS, (o / kS) & 1); ++spins) {
+    if (failed) {   // let the pairs issued and not yet taken land before the shared memory is reused
+      for (; consumed < issued; ++consumed) {
+        for (uint32_t spins = 0; spins < g.wait_limit && !mbar_try_wait(bars + use_slot, use_phase); ++spins) {
+        }
+        if (++use_slot == kSlots) {
+          use_slot = 0;
+          use_phase ^= 1u;
         }
       }
     }
-    ord_base += my_count;
     __syncthreads();   // every ring is idle: the merge area may alias them
 
     // ---- warp partials into shared memory
@@ -559,22 +598,25 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
         lsum[nt] = v;
       }
       float* wp = part + warp * kMaxG * kPartialStride;
+      const bool any = consumed > 0;
       if (gq == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int hh = 4 * nt + tq;
           if (hh < G) {
-            wp[hh * kPartialStride + 0] = my_count ? st.m[nt] : -INFINITY;
-            wp[hh * kPartialStride + 1] = my_count ? lsum[nt] : 0.f;
+            wp[hh * kPartialStride + 0] = any ? st.m[nt] : -INFINITY;
+            wp[hh * kPartialStride + 1] = any ? lsum[nt] : 0.f;
           }
         }
       }
-      // zero-point term of channel group j for heads 2tq, 2tq+1 lives in lane (j, tq)
+      // zero-point term of channel group j for heads 2tq, 2tq+1: rows j (first 16 tokens)
+      // and 8 + j (last 16) of lane (j, tq)
+      const float zs0 = st.bias[0][0] + st.bias[1][2], zs1 = st.bias[0][1] + st.bias[1][3];
       float bz[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        bz[j][0] = __shfl_sync(0xffffffffu, st.bias[0], j * 4 + tq);
-        bz[j][1] = __shfl_sync(0xffffffffu, st.bias[1], j * 4 + tq);
+        bz[j][0] = __shfl_sync(0xffffffffu, zs0, j * 4 + tq);
+        bz[j][1] = __shfl_sync(0xffffffffu, zs1, j * 4 + tq);
       }
       const int h0 = 2 * tq, h1 = 2 * tq + 1;
       const float pv_scale = 4194304.0f;   // 2^22: the codes' 2^-24 and the pairs' 2^2
@@ -595,7 +637,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     __syncthreads();
 
     // ---- CTA merge (thread = channel) into the segment's partial slot
-    float* slot = partial_slot(ws, unit, G);
+    float* slotp = partial_slot(ws, unit, G);
     for (int hh = 0; hh < G; ++hh) {
       float m = rslot[hh * kPartialStride];
 #pragma unroll
@@ -611,7 +653,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
           a = fmaf(p[2 + tid], f, a);
         }
       }
-      float* o = slot + hh * kPartialStride;
+      float* o = slotp + hh * kPartialStride;
       if (tid == 0) {
         o[0] = m;
         o[1] = l;

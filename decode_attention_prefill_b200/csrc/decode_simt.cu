@@ -117,8 +117,8 @@ decode_simt_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, fl
         value_code_loc(t, ch, off, bit);
         uint32_t word = *reinterpret_cast<const uint32_t*>(vc + off);
         float code = static_cast<float>((word >> bit) & 3u);
-        int si = vscale_index(t, i);
-        return fmaf(code, __half2float(__ushort_as_half(vs[si])), __half2float(__ushort_as_half(vz[si])));
+        return fmaf(code, __half2float(__ushort_as_half(vs[vscale_index(t, i)])),
+                    __half2float(__ushort_as_half(vz[vzero_index(t, i)])));
       });
     }
 

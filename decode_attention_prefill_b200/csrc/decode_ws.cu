@@ -138,8 +138,9 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* r
       else
         key_slice_frags<1>(kw[(WH + (sl >> 1)) * 32 + lane], 0u, par, A);
     }
-    const uint32_t s0 = par ? s4.z : s4.x, s1 = par ? s4.w : s4.y;
-    const uint32_t z0 = par ? z4.z : z4.x, z1 = par ? z4.w : z4.y;
+    // scale / zero chunk of a slice pair: (even e=0, odd e=0, even e=1, odd e=1)
+    const uint32_t s0 = par ? s4.y : s4.x, s1 = par ? s4.w : s4.z;
+    const uint32_t z0 = par ? z4.y : z4.x, z1 = par ? z4.w : z4.z;
     uint32_t qxs[NT][2];   // this slice's X registers of each tile (for the zero-point term)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -229,13 +230,12 @@ __device__ __forceinline__ void group_values(const uint8_t* rec, const uint4& p4
     vsr[i][0] = v.x; vsr[i][1] = v.y; vsr[i][2] = v.z; vsr[i][3] = v.w;
   }
   {
+    // zero-point chunk (tq, j): token pairs tq, tq + 8, tq + 4, tq + 12 of channel group j
     const int j = gq & 3;
-    uint32_t vz[4];
+    const uint4 zc = *reinterpret_cast<const uint4*>(rec + vz_off + (tq * 4 + j) * 16);
+    uint32_t vz[4] = {zc.x, zc.z, zc.y, zc.w};   // token pairs tq + 4i
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(rec + vz_off + ((tq + 4 * i) * 4 + j) * 4);
-      vz[i] = gq < 4 ? v : 0u;
-    }
+    for (int i = 0; i < 4; ++i) vz[i] = gq < 4 ? vz[i] : 0u;
     mma16816_free(bias, vz[0], 0u, vz[1], 0u, p16[0], p16[1]);
     mma16816_free(bias, vz[2], 0u, vz[3], 0u, p16[2], p16[3]);
   }

@@ -16,29 +16,39 @@
 // others and the ragged tail the low-precision part; each part's K / V rows are gathered in
 // ascending token order into its own buffers, ready for the ordinary quantizers.
 //
-// route_kernel: one CTA of 256 threads per (sequence, KV head).  The token logits run one
-// token per thread (eight groups per pass, one warp per group), the group maxima one thread
-// per group over the staged logits, and the ranking one thread per group over all of the
-// unit's scores (ng^2 comparisons: a prefill-time cost).
+// score_kernel: grid (chunks, KV heads, sequences); a CTA rebuilds the unit's mean query
+// (the same sequential sums everywhere, so every CTA gets the same bits) and scores
+// kScoreGroups groups, one token per thread for the logits and one thread per group for
+// the maxima.
+// route_kernel: one CTA per (sequence, KV head).  The n_hi best groups are those whose key
+// (score, then lower index) is at least the n_hi-th largest key, found by a radix select
+// over the order-preserving bits of the score (four 8-bit digits, most significant
+// first) and then, among the groups whose score equals the threshold, the lowest
+// indices; a group's place inside its part is the count of earlier groups with the same
+// route (a block-wide prefix sum).  O(ng) work per pass instead of ng^2 comparisons.
 // split_kernel: one CTA per (group, KV head, sequence), plus one per unit for the tail.
 #include "common.cuh"
 
 namespace pnmix {
 namespace {
 
-constexpr int kRouteThreads = 256;
+constexpr int kScoreThreads = 256;
+constexpr int kScoreGroups = 64;       // groups scored by one CTA (2048 tokens)
+constexpr int kRouteThreads = 1024;
 constexpr int kSplitThreads = 128;
 
-__global__ void __launch_bounds__(kRouteThreads)
-route_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, const uint16_t* __restrict__ k,
-             int L, int ld, int n_hi, float* scores, uint8_t* route, int32_t* dest) {
+__global__ void __launch_bounds__(kScoreThreads)
+score_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, const uint16_t* __restrict__ k,
+             int L, int ld, float* scores) {
   __shared__ float qbar[kHeadDim];
-  __shared__ float logit[kRouteThreads];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  __shared__ float logit[kScoreThreads];
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int ng = L / kGroup;
+  const int gbeg = blockIdx.x * kScoreGroups;
+  const int gend = min(ng, gbeg + kScoreGroups);
   const size_t u = static_cast<size_t>(b) * Hkv + h;
 
-  // ---- mean query of the unit's saliency window
+  // ---- mean query of the unit's saliency window (heads outer, tokens inner)
   if (tid < kHeadDim) {
     float s = 0.f;
     for (int hh = 0; hh < G; ++hh) {
@@ -52,10 +62,10 @@ route_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
   // ---- group scores: 256 tokens (8 groups) per pass
   float* sc = scores + u * ng;
   const uint16_t* ku = k + u * static_cast<size_t>(ld) * kHeadDim;
-  for (int base = 0; base < ng * kGroup; base += kRouteThreads) {
+  for (int base = gbeg * kGroup; base < gend * kGroup; base += kScoreThreads) {
     const int t = base + tid;
     float acc = 0.f;
-    if (t < ng * kGroup) {
+    if (t < gend * kGroup) {
       const uint4* row = reinterpret_cast<const uint4*>(ku + static_cast<size_t>(t) * kHeadDim);
       for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
         const uint4 w = row[c8];
@@ -69,9 +79,9 @@ route_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
     }
     logit[tid] = acc;
     __syncthreads();
-    if (tid < kRouteThreads / kGroup) {
+    if (tid < kScoreThreads / kGroup) {
       const int g = base / kGroup + tid;
-      if (g < ng) {
+      if (g < gend) {
         float best = -INFINITY;
         for (int i = 0; i < kGroup; ++i) {
           const float x = logit[tid * kGroup + i];
@@ -82,24 +92,114 @@ route_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
     }
     __syncthreads();
   }
+}
 
-  // ---- rank and route (the block's own score writes are visible after the barrier)
-  for (int g = tid; g < ng; g += kRouteThreads) {
-    const float s = sc[g];
-    int r = 0;
-    for (int o = 0; o < ng; ++o) {
-      const float x = sc[o];
-      r += (x > s || (x == s && o < g)) ? 1 : 0;
+// Order-preserving unsigned image of a float; -0 and +0 map to the same value, as they
+// compare equal.
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  uint32_t v = __float_as_uint(x);
+  if (v == 0x80000000u) v = 0u;
+  return (v & 0x80000000u) ? ~v : (v | 0x80000000u);
+}
+
+// Block-wide exclusive prefix sum of `x` over the CTA's threads in thread order; returns
+// this thread's prefix and writes the block total.
+__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int v = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) warp_sums[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kRouteThreads >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
     }
-    route[u * ng + g] = r < n_hi ? 1 : 0;
+    warp_sums[lane] = w;   // inclusive prefix of the warp totals
   }
   __syncthreads();
-  // ---- place of each group inside its part: earlier groups with the same route
-  for (int g = tid; g < ng; g += kRouteThreads) {
-    const uint8_t mine = route[u * ng + g];
-    int d = 0;
-    for (int o = 0; o < g; ++o) d += route[u * ng + o] == mine ? 1 : 0;
-    dest[u * ng + g] = d;
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + v - x;
+  *total = warp_sums[(kRouteThreads >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_kernel(int Hkv, int L, int n_hi, const float* __restrict__ scores, uint8_t* route, int32_t* dest) {
+  __shared__ int hist[256];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t sel_prefix;
+  __shared__ int sel_rank;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int ng = L / kGroup;
+  const size_t u = static_cast<size_t>(b) * Hkv + h;
+  const float* sc = scores + u * ng;
+  uint8_t* ru = route + u * ng;
+  int32_t* du = dest + u * ng;
+
+  // ---- radix select of the n_hi-th largest score image: prefix/mask of the bits fixed
+  // so far; `rank` = how many of the keys sharing the prefix are still to be taken
+  uint32_t prefix = 0, mask = 0;
+  int rank = n_hi;   // 1-based rank of the threshold among the keys with the prefix
+  if (n_hi > 0 && n_hi < ng) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kRouteThreads) hist[i] = 0;
+      __syncthreads();
+      for (int g = tid; g < ng; g += kRouteThreads) {
+        const uint32_t v = ordered_bits(sc[g]);
+        if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {   // walk the digits from the top until the rank falls in one
+        int r = rank, d = 255;
+        for (; d > 0; --d) {
+          if (r <= hist[d]) break;
+          r -= hist[d];
+        }
+        sel_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+        sel_rank = r;
+      }
+      __syncthreads();
+      prefix = sel_prefix;
+      rank = sel_rank;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+  }
+  // threshold image T = prefix: groups above T are taken, and of the groups equal to T the
+  // `rank` lowest indices (rank = n_hi minus the count above T)
+  int eq_before = 0;   // groups equal to T with a lower index, over the earlier chunks
+  int hi_before = 0, lo_before = 0;
+  for (int base = 0; base < ng; base += kRouteThreads) {
+    const int g = base + tid;
+    uint32_t v = 0;
+    bool above = false, equal = false;
+    if (g < ng) {
+      v = ordered_bits(sc[g]);
+      if (n_hi >= ng) above = true;
+      else if (n_hi > 0) {
+        above = v > prefix;
+        equal = v == prefix;
+      }
+    }
+    int eq_total;
+    const int eq_rank = eq_before + block_exclusive_scan(equal ? 1 : 0, warp_sums, &eq_total);
+    eq_before += eq_total;
+    const bool r1 = above || (equal && eq_rank < rank);
+    int n_hi_chunk;
+    const int hi_rank = hi_before + block_exclusive_scan(r1 ? 1 : 0, warp_sums, &n_hi_chunk);
+    if (g < ng) {
+      ru[g] = r1 ? 1 : 0;
+      du[g] = r1 ? hi_rank : lo_before + (tid - (hi_rank - hi_before));
+    }
+    hi_before += n_hi_chunk;
+    lo_before += min(kRouteThreads, ng - base) - n_hi_chunk;
   }
 }
 
@@ -144,9 +244,13 @@ cudaError_t launch_split_groups(const Geometry& g, const uint16_t* q_window, int
   if (g.B == 0) return cudaSuccess;
   const int ng = L / kGroup;
   if (ng > 0) {
-    route_kernel<<<dim3(g.Hkv, g.B), kRouteThreads, 0, s>>>(g.G, g.Hq, g.Hkv, q_window, nw, k, L, ld, n_hi, scores,
-                                                           route, dest);
+    const int chunks = (ng + kScoreGroups - 1) / kScoreGroups;
+    score_kernel<<<dim3(chunks, g.Hkv, g.B), kScoreThreads, 0, s>>>(g.G, g.Hq, g.Hkv, q_window, nw, k, L, ld,
+                                                                     scores);
     cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    route_kernel<<<dim3(g.Hkv, g.B), kRouteThreads, 0, s>>>(g.Hkv, L, n_hi, scores, route, dest);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   split_kernel<<<dim3(ng + 1, g.Hkv, g.B), kSplitThreads, 0, s>>>(g.Hkv, k, v, L, ld, n_hi, route, dest, k_hi, v_hi,

@@ -124,12 +124,15 @@ pnmix_status check_decode_args(const pnmix_config* cfg, const uint16_t* q, const
 }
 
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int max_context,
-                          float* out, void* ws, cudaStream_t s) {
+                          float* out, void* ws, cudaStream_t s, const DecodeMerge& merge) {
   const int nmax = decode_max_ctas(g, max_context);
   DecodeWs w;
   w.part = static_cast<float*>(ws);
   w.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + decode_ticket_offset(g, max_context));
   w.N = nmax;
+  w.lse_out = merge.lse_out;
+  w.prior_out = merge.prior_out;
+  w.prior_lse = merge.prior_lse;
   switch (g.kernel) {
     case PNMIX_DECODE_SIMT: return launch_decode_simt(g, q, c, nmax, out, w, s);
     case PNMIX_DECODE_MMA: return launch_decode_mma(g, q, c, nmax, out, w, s);
@@ -282,6 +285,46 @@ pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
   if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
   return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+size_t pnmix_workspace_bytes_two(const pnmix_config* cfg_a, const pnmix_config* cfg_b, int batch,
+                                 int max_context_a, int max_context_b) {
+  Geometry ga, gb;
+  if (batch <= 0 || make_geometry(cfg_a, batch, 32, &ga) != PNMIX_OK || make_geometry(cfg_b, batch, 32, &gb) != PNMIX_OK)
+    return 0;
+  if (ga.Hq != gb.Hq || ga.Hkv != gb.Hkv || max_context_a < 0 || max_context_b < 0) return 0;
+  const size_t wa = decode_workspace_bytes(ga, max_context_a), wb = decode_workspace_bytes(gb, max_context_b);
+  const size_t rows = static_cast<size_t>(batch) * ga.Hq;
+  return align256(wa > wb ? wa : wb) + align256(rows * kHeadDim * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+pnmix_status pnmix_decode_attention_two(const pnmix_config* cfg_a, const pnmix_cache* cache_a, int max_context_a,
+                                        const pnmix_config* cfg_b, const pnmix_cache* cache_b, int max_context_b,
+                                        const uint16_t* q, float* out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  Geometry ga, gb;
+  pnmix_status st = check_decode_args(cfg_a, q, cache_a, max_context_a, out, &ga);
+  if (st != PNMIX_OK) return st;
+  if ((st = check_decode_args(cfg_b, q, cache_b, max_context_b, out, &gb)) != PNMIX_OK) return st;
+  if (ga.B != gb.B || ga.Hq != gb.Hq || ga.Hkv != gb.Hkv) return PNMIX_ERR_INVALID_ARG;
+  if (!workspace) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  const size_t wa = decode_workspace_bytes(ga, max_context_a), wb = decode_workspace_bytes(gb, max_context_b);
+  const size_t rows = static_cast<size_t>(ga.B) * ga.Hq;
+  const size_t split = align256(wa > wb ? wa : wb), tmp = align256(rows * kHeadDim * sizeof(float));
+  if (workspace_bytes < split + tmp + align256(rows * sizeof(float))) return PNMIX_ERR_CAPACITY;
+  char* w = static_cast<char*>(workspace);
+  float* part_out = reinterpret_cast<float*>(w + split);
+  float* part_lse = reinterpret_cast<float*>(w + split + tmp);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DecodeMerge first;
+  first.lse_out = part_lse;
+  cudaError_t e = launch_decode(ga, q, *cache_a, max_context_a, part_out, workspace, s, first);
+  if (e != cudaSuccess) return PNMIX_ERR_CUDA;
+  DecodeMerge second;
+  second.prior_out = part_out;
+  second.prior_lse = part_lse;
+  return cuda_status(launch_decode(gb, q, *cache_b, max_context_b, out, workspace, s, second));
 }
 
 pnmix_status pnmix_debug_decode_stall(const pnmix_config* cfg, const uint16_t* q, const pnmix_cache* cache,

@@ -148,7 +148,7 @@ __device__ void quantize_value_group(const Geometry& g, GroupSmem& sm, uint8_t* 
     uint16_t* vs = reinterpret_cast<uint16_t*>(rec + rec_vscale(g));
     uint16_t* vz = reinterpret_cast<uint16_t*>(rec + rec_vzero(g));
     vs[vscale_index(t, jg)] = q.s16;
-    vz[vscale_index(t, jg)] = q.z16;
+    vz[vzero_index(t, jg)] = q.z16;
   }
   __syncthreads();
   // word (m, L): slot q = 4r + p holds channel 16m + gq + 8r of tokens 2tq + 8p (+1)

@@ -108,7 +108,8 @@ shrink_kernel(Geometry gs, Geometry gd, pnmix_cache src, pnmix_cache dst) {
   for (int w = 0; w < 8; ++w)
     if (w < gs.wl) lw[w] = ws[(gs.wh + w) * 32 + L];
   // ---- scales (x (2^b + 1) where salient) and zero points: lane L holds the four fp16
-  //      entries 4L .. 4L + 3, all of 16-position slice L mod 8
+  //      entries 4L .. 4L + 3, i.e. the fp16x2 words 2L (slice 2 * ((L >> 1) & 3)) and
+  //      2L + 1 (the next slice)
   const uint2 sc = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(ws) + rec_kscale(gs) + 8 * L);
   const uint2 zr = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(ws) + rec_kzero(gs) + 8 * L);
   const uint4* vs = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(ws) + rec_vcode(gs));
@@ -124,10 +125,11 @@ shrink_kernel(Geometry gs, Geometry gd, pnmix_cache src, pnmix_cache dst) {
   for (int w = 0; w < 8; ++w)
     if (w < gs.wl) wd[(wh_d + w) * 32 + L] = lw[w];
   uint2 so = sc;
-  if ((L & 7) < gs.nhs) {
+  {
     const float mul = static_cast<float>((1 << B) + 1);
     uint32_t v[2] = {sc.x, sc.y};
     for (int i = 0; i < 2; ++i) {
+      if (2 * ((L >> 1) & 3) + i >= gs.nhs) continue;   // slice not salient: scale kept
       const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v[i]));
       const __half lo = __float2half_rn(__fmul_rn(f.x, mul)), hi = __float2half_rn(__fmul_rn(f.y, mul));
       v[i] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);

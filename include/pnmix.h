@@ -93,7 +93,9 @@
  *     Lane-local word w of lane L is stored at byte offset (w * 32 + L) * 4.
  *  2. Key scales, 128 fp16 (256 B): the scale of position
  *     j = 16*sigma + 8*e + 2*tq + v  (e, v in {0,1}) is fp16 element
- *     ((tq * 8 + sigma) * 2 + e) * 2 + v.
+ *     ((tq * 4 + sigma / 2) * 4 + 2 * e + sigma % 2) * 2 + v, so the 16 bytes of one
+ *     (tq, slice pair) hold the pairs (even slice e=0, odd slice e=0, even slice e=1,
+ *     odd slice e=1).
  *  3. Key zero points, 128 fp16 (256 B), same order as 2.
  *  4. Value codes, 1024 B, b_v = 2 bits.  A value SLOT is (m in {0..7},
  *     r in {0,1}, p in {0..3}); it names channel 16*m + gq + 8*r and the token
@@ -104,7 +106,10 @@
  *  5. Value scales, 64 fp16x2 (256 B): element (tp * 4 + jg) is the pair
  *     (scale of token 2*tp, scale of token 2*tp+1) of channel group jg
  *     (channels [32*jg, 32*jg + 32)), tp in [0,16).
- *  6. Value zero points, 256 B, same order as 5.
+ *  6. Value zero points, 64 fp16x2 (256 B): the pair (zero of token 2*tp, zero of
+ *     token 2*tp+1) of channel group jg is element
+ *     ((tp % 4) * 4 + jg) * 4 + (tp / 8) + 2 * ((tp / 4) % 2),
+ *     so the 16 bytes of one (tp % 4, jg) hold tp, tp + 8, tp + 4, tp + 12 in that order.
  * record_bytes = KC + 2048 (3200 B at b_hi=4, b_lo=2, k=8, i.e. 100 B/token).
  *
  * Other regions of the cache (all carved out of one caller-owned buffer by
@@ -424,6 +429,33 @@ PNMIX_API pnmix_status pnmix_split_groups(const pnmix_config* cfg, int batch, co
 PNMIX_API pnmix_status pnmix_decode_attention_noalloc(const pnmix_config* cfg, const uint16_t* q,
                                                       const pnmix_cache* cache, int max_context,
                                                       float* out, void* stream);
+
+/*
+ * Decode attention over a cache held in two parts (SemKV abstract, "SemKV: Semantic
+ * Mixed-Precision KV Cache Quantization Guided by the Quality Cliff for Long-Context LLM
+ * Inference": every token is kept, at one of two adjacent precisions).  Part a and part b
+ * are two caches of the same batch and head layout holding disjoint token sets, e.g. the
+ * high and the low precision parts that pnmix_split_groups prepares; each is read with its
+ * own configuration (cfg_a / cfg_b: bit widths and salient pairs may differ).  The result
+ * is the attention of every query row over the union of both parts' tokens:
+ *     out = sum over the tokens of both parts of softmax(q . k^ * scale) v^,
+ * computed as two decode launches: part a's normalised output and log-sum-exp go to the
+ * workspace, and part b's combine merges them with its own,
+ *     out = (2^(La - M) oa + 2^(Lb - M) ob) / (2^(La - M) + 2^(Lb - M)),  M = max(La, Lb)
+ * (log2-domain log-sum-exps; a part that holds no token of a sequence weighs nothing, and
+ * a sequence with no token in either part gets zeros).  q bf16 [B][Hq][128], out fp32
+ * [B][Hq][128].  max_context_a / _b bound the lengths of each part as in
+ * pnmix_decode_attention.  Workspace: pnmix_workspace_bytes_two bytes, 256-byte aligned,
+ * zero-filled before first use; it is left ready for the next call.  Errors as for
+ * pnmix_decode_attention, and INVALID_ARG when the parts' batch or head counts differ.
+ */
+PNMIX_API size_t pnmix_workspace_bytes_two(const pnmix_config* cfg_a, const pnmix_config* cfg_b, int batch,
+                                           int max_context_a, int max_context_b);
+PNMIX_API pnmix_status pnmix_decode_attention_two(const pnmix_config* cfg_a, const pnmix_cache* cache_a,
+                                                  int max_context_a, const pnmix_config* cfg_b,
+                                                  const pnmix_cache* cache_b, int max_context_b,
+                                                  const uint16_t* q, float* out, void* workspace,
+                                                  size_t workspace_bytes, void* stream);
 
 /*
  * Test hook of the bounded staging wait; the pages have no counterpart.  Runs

@@ -328,10 +328,22 @@ static void put16(uint8_t* p, uint16_t v) {
 }
 static uint16_t get16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
-/* fp16 element index of key position j in the scale (and zero) array. */
+/* fp16 element index of key position j in the scale (and zero) array: the 16 bytes of
+   (tq, slice pair) hold the pairs (even slice e=0, odd slice e=0, even slice e=1, odd
+   slice e=1). */
 static int orc_kscale_index(int j) {
   int sigma = j / 16, e = (j % 16) / 8, tq = (j % 8) / 2, v = j % 2;
-  return ((tq * 8 + sigma) * 2 + e) * 2 + v;
+  return ((tq * 4 + sigma / 2) * 4 + 2 * e + sigma % 2) * 2 + v;
+}
+
+/* fp16 element index of the value scale of (token t, channel group jg). */
+static int orc_vscale_index(int t, int jg) { return ((t / 2) * 4 + jg) * 2 + (t % 2); }
+
+/* fp16 element index of the value zero point of (token t, channel group jg): token pair
+   tp = t/2 sits in the 16 bytes of (tp mod 4, jg), which hold tp, tp+8, tp+4, tp+12. */
+static int orc_vzero_index(int t, int jg) {
+  int tp = t / 2;
+  return (((tp % 4) * 4 + jg) * 4 + tp / 8 + 2 * ((tp / 4) % 2)) * 2 + (t % 2);
 }
 
 /* Byte offset of the key-code word w (lane-local) of lane L. */
@@ -410,9 +422,8 @@ int orc_pack_record(int k, int bhi, int blo, const uint8_t* kcodes, const uint16
   uint8_t* vsb = rec + KC + 1536;
   for (int t = 0; t < 32; ++t) {
     for (int jg = 0; jg < 4; ++jg) {
-      int e = ((t / 2) * 4 + jg) * 2 + (t % 2);
-      put16(vsb + 2 * e, vs[t * 4 + jg]);
-      put16(vsb + 256 + 2 * e, vz[t * 4 + jg]);
+      put16(vsb + 2 * orc_vscale_index(t, jg), vs[t * 4 + jg]);
+      put16(vsb + 256 + 2 * orc_vzero_index(t, jg), vz[t * 4 + jg]);
     }
   }
   return 0;
@@ -449,9 +460,8 @@ int orc_unpack_record(int k, int bhi, int blo, const uint8_t* rec, uint8_t* kcod
   const uint8_t* vsb = rec + KC + 1536;
   for (int t = 0; t < 32; ++t) {
     for (int jg = 0; jg < 4; ++jg) {
-      int e = ((t / 2) * 4 + jg) * 2 + (t % 2);
-      vs[t * 4 + jg] = get16(vsb + 2 * e);
-      vz[t * 4 + jg] = get16(vsb + 256 + 2 * e);
+      vs[t * 4 + jg] = get16(vsb + 2 * orc_vscale_index(t, jg));
+      vz[t * 4 + jg] = get16(vsb + 256 + 2 * orc_vzero_index(t, jg));
     }
   }
   return 0;

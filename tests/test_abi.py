@@ -286,3 +286,24 @@ def test_stall_hook_rejects_bad_arguments_before_launching():
     assert f(ctypes.byref(cfg), P, ctypes.byref(c), 256, P, None, ws, 0, 16, None) == pm.ERR_INVALID_ARG
     simt = pm.Config.make(8, 2, decode_kernel=pm.DECODE_SIMT)
     assert f(ctypes.byref(simt), P, ctypes.byref(c), 256, P, P, ws, 0, 16, None) == pm.ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_two_part_decode_rejects_bad_arguments_before_launching():
+    hi, lo = pm.Config.make(8, 2, n_salient_pairs=16), pm.Config.make(8, 2, n_salient_pairs=8)
+    a, b = _fake_cache(hi), _fake_cache(lo)
+    P = ctypes.c_void_p(1 << 41)
+    odd = ctypes.c_void_p((1 << 41) + 16)
+    n = pm.workspace_bytes_two(hi, lo, 2, 256, 256)
+    assert n >= max(pm.workspace_bytes(hi, 2, 256), pm.workspace_bytes(lo, 2, 256)) + 2 * 8 * 128 * 4
+    assert pm.workspace_bytes_two(hi, pm.Config.make(8, 4), 2, 256, 256) == 0      # other head layout
+    f = pm._lib.pnmix_decode_attention_two
+    args = lambda cfg_a, ca, cfg_b, cb, ws, nb: (ctypes.byref(cfg_a), ctypes.byref(ca), 256, ctypes.byref(cfg_b),  # noqa: E731
+                                                 ctypes.byref(cb), 256, P, P, ws, nb, None)
+    assert f(*args(hi, a, lo, b, P, n - 1)) == pm.ERR_CAPACITY
+    assert f(*args(hi, a, lo, b, odd, n)) == pm.ERR_ALIGNMENT
+    assert f(*args(hi, a, lo, b, None, n)) == pm.ERR_INVALID_ARG
+    assert f(*args(lo, a, lo, b, P, n)) == pm.ERR_INVALID_ARG          # cache a laid out for another config
+    other = pm.Config.make(16, 4)
+    assert f(*args(hi, a, other, _fake_cache(other), P, n)) == pm.ERR_INVALID_ARG   # head counts differ

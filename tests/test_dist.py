@@ -81,3 +81,7 @@ def test_reference_arm_prints_one_contract_line(capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "stream_32k"
+    assert d["config"] == bench.stream_config(1)          # the GPU arm's config keys
+    assert d["sampled"]["units_per_full_step"] == bench.B * bench.HKV
+    # ms_per_step is the wall time actually spent per sampled step; value scales it to a step
+    assert abs(d["value"] - bench.B / (d["ms_per_step"] / 1e3 * bench.B * bench.HKV)) <= 1e-6 * d["value"]

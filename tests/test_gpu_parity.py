@@ -476,3 +476,79 @@ def test_staging_wait_that_runs_out_sets_the_error_word_and_returns(kernel, skip
     got, want = c.attend(q)
     assert_close(got, want)
     assert c.cache.read_error() == 0
+
+
+# Two-precision decode (the SemKV abstract's attention over tokens kept at two
+# precisions): the GPU attends over both caches of a split prefill, merging the parts by
+# their log-sum-exps, and must match the oracle's plain softmax over the union of tokens.
+def _two_part(B, Hq, Hkv, L, k_hi, k_lo, percent, seed, extra=0, bhi=4, blo=2, sample_units=None):
+    import decode_attention_prefill_b200 as pm
+    import oracle
+    import workload
+    G = Hq // Hkv
+    W = min(L, 64)
+    kin = workload.rows(seed, workload.K, B, Hkv, 0, L + extra)
+    vin = workload.rows(seed, workload.V, B, Hkv, 0, L + extra)
+    qwin = workload.rows(seed, workload.Q, B, Hq, L - W, W, group=G)
+    cap = (L + extra + 31) // 32 * 32 + 32
+    want = oracle.TwoPrecision(B, Hkv, cap, k_hi, k_lo, bhi, blo, percent)
+    want.prefill(qwin, kin, vin, L)
+    q_dev, k_dev, v_dev = to_dev(qwin), to_dev(kin), to_dev(vin)
+    cfg_hi = pm.Config.make(Hq, Hkv, bhi, blo, k_hi, 64)
+    cfg_lo = pm.Config.make(Hq, Hkv, bhi, blo, k_lo, 64)
+    parts = pm.pnmix_split_groups(cfg_hi, q_dev, k_dev, v_dev, L, percent)
+    L_hi, L_lo = pm.split_sizes(L, percent)
+    caches = []
+    for cfg, k_part, v_part, Lp in ((cfg_hi, parts["k_hi"], parts["v_hi"], L_hi),
+                                    (cfg_lo, parts["k_lo"], parts["v_lo"], L_lo)):
+        cache = pm.PNMixCache(cfg, B, cap)
+        pm.pnmix_select_pairs(cfg, q_dev, k_dev, L, cache)
+        if Lp > 0:
+            pm.pnmix_quantize_keys(cfg, k_part, Lp, cache)
+            pm.pnmix_quantize_values(cfg, v_part, Lp, cache)
+        caches.append(cache)
+    torch.cuda.synchronize()
+    return pm, caches, want, kin, vin, seed
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,k_hi,k_lo,percent", [
+    (2, 8, 2, 300, 16, 8, 50),
+    (1, 28, 4, 517, 32, 8, 25),
+    (2, 8, 2, 64, 16, 8, 100),    # every group high: the low part holds no token
+    (1, 4, 1, 100, 16, 8, 0),     # no group high: the high part holds no token
+    (2, 32, 8, 1000, 16, 0, 40),
+])
+def test_two_part_decode_matches_the_oracle_over_the_union(B, Hq, Hkv, L, k_hi, k_lo, percent):
+    import workload
+    extra = 40
+    pm, (c_hi, c_lo), want, kin, vin, seed = _two_part(B, Hq, Hkv, L, k_hi, k_lo, percent, L + 1, extra=extra)
+    G = Hq // Hkv
+    q = workload.rows(seed, workload.Q, B, Hq, L, 1, group=G)[:, :, 0]
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device="cuda")
+    pm.pnmix_decode_attention_two(c_hi, c_lo, to_dev(q), out)
+    torch.cuda.synchronize()
+    assert_close(out.cpu().numpy(), want.attend(q))
+    for t in range(L, L + extra):   # appended tokens go to the low part
+        kn, vn = np.ascontiguousarray(kin[:, :, t]), np.ascontiguousarray(vin[:, :, t])
+        c_lo.append(to_dev(kn), to_dev(vn))
+        want.append(kn, vn)
+    q = workload.rows(seed, workload.Q, B, Hq, L + extra - 1, 1, group=G)[:, :, 0]
+    pm.pnmix_decode_attention_two(c_hi, c_lo, to_dev(q), out)
+    torch.cuda.synchronize()
+    assert_close(out.cpu().numpy(), want.attend(q))
+    assert c_hi.read_error() == 0 and c_lo.read_error() == 0
+
+
+@pytest.mark.slow
+def test_two_part_decode_at_128k_context():
+    """The bit-sweep shape (2 x 28/4, 131072 tokens) split 50 / 50 between 16 and 8
+    salient pairs; two sampled units checked against the oracle."""
+    import workload
+    B, Hq, Hkv, L = 2, 28, 4, 131072
+    pm, (c_hi, c_lo), want, kin, vin, seed = _two_part(B, Hq, Hkv, L, 16, 8, 50, 5)
+    q = workload.rows(seed, workload.Q, B, Hq, L, 1, group=Hq // Hkv)[:, :, 0]
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device="cuda")
+    pm.pnmix_decode_attention_two(c_hi, c_lo, to_dev(q), out)
+    torch.cuda.synchronize()
+    units = [(0, 1), (1, 3)]
+    assert_close(out.cpu().numpy(), want.attend(q, heads=units), units=units, G=Hq // Hkv)

@@ -429,7 +429,9 @@ def test_pack_unpack_round_trip(k, bhi, blo):
 
 
 def test_scale_layout_puts_a_lanes_pairs_together():
-    """Scale of position j = 16*sigma + 8*e + 2*tq + v at fp16 index ((tq*8+sigma)*2+e)*2+v."""
+    """Scale of position j = 16*sigma + 8*e + 2*tq + v at fp16 index
+    ((tq*4 + sigma//2)*4 + 2e + sigma%2)*2 + v: the 16 bytes of one (tq, slice pair) hold
+    (even slice e=0, odd slice e=0, even slice e=1, odd slice e=1)."""
     ks = np.arange(128, dtype=np.uint16) + 1000
     zero8 = np.zeros((32, 128), np.uint8)
     zv = np.zeros((32, 4), np.uint16)
@@ -438,7 +440,34 @@ def test_scale_layout_puts_a_lanes_pairs_together():
     arr = rec[KC:KC + 256].view(np.uint16)
     for j in range(128):
         sigma, e, tq, v = j // 16, (j % 16) // 8, (j % 8) // 2, j % 2
-        assert arr[((tq * 8 + sigma) * 2 + e) * 2 + v] == 1000 + j
+        assert arr[((tq * 4 + sigma // 2) * 4 + 2 * e + sigma % 2) * 2 + v] == 1000 + j
+    assert sorted(arr.tolist()) == list(range(1000, 1128))    # every entry written once
+
+
+def test_value_scale_and_zero_layouts():
+    """Value scale of (token t, group jg) at fp16 index ((t//2)*4 + jg)*2 + t%2; value zero
+    of the token pair tp = t//2 in the 16-byte chunk (tp%4, jg) at slot tp//8 + 2*((tp//4)%2)
+    (the chunk holds tp, tp+8, tp+4, tp+12)."""
+    zero8 = np.zeros((32, 128), np.uint8)
+    z16 = np.zeros(128, np.uint16)
+    vs = (np.arange(128, dtype=np.uint16) + 3000).reshape(32, 4)
+    vz = (np.arange(128, dtype=np.uint16) + 5000).reshape(32, 4)
+    rec = oracle.pack_record(8, 4, 2, zero8, z16, z16, zero8, vs, vz)
+    KC = oracle.record_bytes(8, 4, 2) - 2048
+    sarr = rec[KC + 1536:KC + 1792].view(np.uint16)
+    zarr = rec[KC + 1792:KC + 2048].view(np.uint16)
+    for t in range(32):
+        for jg in range(4):
+            tp = t // 2
+            assert sarr[((t // 2) * 4 + jg) * 2 + t % 2] == vs[t, jg]
+            chunk, slot = (tp % 4) * 4 + jg, [tp // 8 + 2 * ((tp // 4) % 2)][0]
+            assert zarr[(chunk * 4 + slot) * 2 + t % 2] == vz[t, jg]
+    assert sorted(zarr.tolist()) == list(range(5000, 5128))
+    # one chunk: token pairs tp, tp + 8, tp + 4, tp + 12 of one channel group
+    for q4 in range(4):
+        for jg in range(4):
+            words = zarr[(q4 * 4 + jg) * 8:(q4 * 4 + jg) * 8 + 8:2]
+            assert [(int(w) - 5000) // 4 // 2 for w in words] == [q4, q4 + 8, q4 + 4, q4 + 12]
 
 
 # ------------------------------------------------------------------ append vs prefill
