@@ -68,6 +68,9 @@ def parse():
                          "prefill latencies and the extrapolated end-to-end tokens/s; verify_32k: "
                          "two new tokens per sequence attended at once at 32K; stream_full: the "
                          "whole 4096 -> 32768 stream, measured)")
+    ap.add_argument("--pipeline-sampled", action="store_true",
+                    help="pipeline_32l: time the decode phase at 8 contexts and integrate, instead of "
+                         "running all 28672 steps")
     ap.add_argument("--pipeline-layers-generated", type=int, default=4,
                     help="pipeline_32l: layers whose prefill inputs are generated (seed + layer); "
                          "the others reuse them cyclically")
@@ -626,8 +629,7 @@ def run_stream_full(args):
         cache.prefill(qwin_dev, k_dev, v_dev, PREFILL)
         e[1].record()
         for t in range(PREFILL, CONTEXT):
-            pm.pnmix_append(cfg, kn[t], vn[t], cache)
-            pm.pnmix_decode_attention(cfg, q_dev[(t - PREFILL) % n_q], cache, out)
+            pm.pnmix_append_decode(cfg, kn[t], vn[t], q_dev[(t - PREFILL) % n_q], cache, out)
         e[2].record()
         torch.cuda.synchronize()
     assert cache.read_error() == 0 and int(cache.lengths().min().item()) == CONTEXT
@@ -697,6 +699,8 @@ def run_pipeline(args):
     sal_ms = sum(ev[3 * l].elapsed_time(ev[3 * l + 1]) for l in range(NL))
     qnt_ms = sum(ev[3 * l + 1].elapsed_time(ev[3 * l + 2]) for l in range(NL))
     prefill_ms = ev[0].elapsed_time(ev[3 * NL - 1])
+    if not args.pipeline_sampled:
+        return run_pipeline_full(args, pm, wl, cfg, caches, sal_ms, qnt_ms, prefill_ms, n_gen)
     # ---- decode phase at sampled contexts
     reps = 8
     k_rep = inputs[0][1].repeat(1, 1, C // L, 1)           # [B][Hkv][C][128]
@@ -722,8 +726,7 @@ def run_pipeline(args):
                 if i == 2:
                     e0.record()
                 for l in range(NL):
-                    pm.pnmix_append(cfg, kn[i], vn[i], caches[l])
-                    pm.pnmix_decode_attention(cfg, qn[i], caches[l], out)
+                    pm.pnmix_append_decode(cfg, kn[i], vn[i], qn[i], caches[l], out)
             e1.record()
             torch.cuda.synchronize()
             step_ms = e0.elapsed_time(e1) / (reps - 2)
@@ -749,6 +752,57 @@ def run_pipeline(args):
                        "tokens_per_s_extrapolated": Bw * steps / (total_ms / 1e3)},
             "end_to_end": {"total_s_extrapolated": (total_ms + prefill_ms) / 1e3,
                            "tokens_per_s_extrapolated": Bw * steps / ((total_ms + prefill_ms) / 1e3)},
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_pipeline_full(args, pm, wl, cfg, caches, sal_ms, qnt_ms, prefill_ms, n_gen):
+    """pipeline_32l decode phase measured whole: after the prefill of every layer, all
+    C - L decode steps, each one pnmix_append_decode per layer, timed between two events.
+    The appended K / V rows and the queries of 1024 consecutive positions are reused
+    cyclically (the cost does not depend on their values)."""
+    import torch
+
+    import workload
+    Bw, Hq, Hkv, L, C, NL = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.prefill, wl.context, wl.layers
+    G = Hq // Hkv
+    dev = torch.device("cuda", 0)
+    pool = 1024
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a.transpose(2, 0, 1, 3))).view(torch.bfloat16).to(dev)  # noqa: E731
+    kn = to(workload.rows(args.seed, workload.K, Bw, Hkv, L, pool))
+    vn = to(workload.rows(args.seed, workload.V, Bw, Hkv, L, pool))
+    qn = to(workload.rows(args.seed, workload.Q, Bw, Hq, L, pool, group=G))
+    out = torch.empty(Bw, Hq, D, dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        e0.record()
+        for t in range(L, C):
+            i = (t - L) % pool
+            for l in range(NL):
+                pm.pnmix_append_decode(cfg, kn[i], vn[i], qn[i], caches[l], out)
+        e1.record()
+        torch.cuda.synchronize()
+    decode_s = e0.elapsed_time(e1) / 1e3
+    assert all(c.read_error() == 0 and int(c.lengths().min().item()) == C for c in caches)
+    steps = C - L
+    line = {"workload": "pipeline_32l", "metric": "end-to-end attention-path tokens/s",
+            "unit": "tokens/s", "n_gpus": 1, "data": "synthetic", "dtype": "f32",
+            "value": Bw * steps / (decode_s + prefill_ms / 1e3),
+            "config": {"layers": NL, "batch": Bw, "n_q_heads": Hq, "n_kv_heads": Hkv,
+                       "prefill": L, "context": C, "salient_pairs": K_SALIENT, "key_bits": [BHI, BLO],
+                       "prefill_inputs": f"seed + layer for {n_gen} generated layer(s), reused cyclically",
+                       "decode_inputs": f"K / V rows and queries of {pool} positions reused cyclically",
+                       "l2": "32 layers of cache between re-reads of a layer (>= 3 GB)"},
+            "prefill": {"saliency_ms_all_layers": sal_ms, "quantize_ms_all_layers": qnt_ms,
+                        "prefill_ms_all_layers": prefill_ms,
+                        "quantize_tokens_per_s": NL * Bw * L / (qnt_ms / 1e3)},
+            "decode": {"steps": steps, "launches": steps * NL, "total_s": decode_s,
+                       "mean_step_ms": 1e3 * decode_s / steps, "tokens_per_s": Bw * steps / decode_s},
+            "end_to_end": {"total_s": decode_s + prefill_ms / 1e3,
+                           "tokens_per_s": Bw * steps / (decode_s + prefill_ms / 1e3)},
+            "measured": "every step timed (not extrapolated)",
             "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     return 0
@@ -823,9 +877,9 @@ def main():
     torch.cuda.empty_cache()
 
     if args.profile_decode:
-        # decode-only launches at context T0 (for profiler captures)
+        # the bench's step (append + decode in one launch) from context T0, for profiler captures
         for i in range(W + K):
-            pm.pnmix_decode_attention(cfg, q_dev[0], cache, out)
+            pm.pnmix_append_decode(cfg, kn_dev[i], vn_dev[i], q_dev[i], cache, out)
         torch.cuda.synchronize()
         print(json.dumps({"profile_decode": True, "launches": W + K, "context": T0,
                           "error_word": cache.read_error()}), flush=True)
@@ -875,8 +929,7 @@ def main():
         comp_s.wait_event(ev_in[j])
         if used[j]:
             comp_s.wait_event(ev_out[j])     # the previous output of this buffer has left
-        pm.pnmix_append(cfg, bufs[j]["k"], bufs[j]["v"], cache)
-        pm.pnmix_decode_attention(cfg, bufs[j]["q"], cache, bufs[j]["out"])
+        pm.pnmix_append_decode(cfg, bufs[j]["k"], bufs[j]["v"], bufs[j]["q"], cache, bufs[j]["out"])
         ev_used[j].record(comp_s)
         d2h_s.wait_event(ev_used[j])
         with torch.cuda.stream(d2h_s):
@@ -892,18 +945,16 @@ def main():
     # ---- device-resident steps, two passes of W + K steps each.  Pass 1 (the bench value):
     # K whole steps between two events.  Pass 2 (the kernel roofline): the next steps with
     # an event around every launch (those records cost a little time between launches,
-    # so they stay out of pass 1).  The last step brings the context to CONTEXT.
+    # so they stay out of pass 1).  The last step brings the context to CONTEXT.  A step is
+    # one pnmix_append_decode call: the append runs inside the decode launch.
     def run_steps(first, n, events=None):
         for i in range(n):
             t = first + i
             if events:
                 events[0][i].record()
-            pm.pnmix_append(cfg, kn_dev[t - T0], vn_dev[t - T0], cache)
+            pm.pnmix_append_decode(cfg, kn_dev[t - T0], vn_dev[t - T0], q_dev[t - T0], cache, out)
             if events:
                 events[1][i].record()
-            pm.pnmix_decode_attention(cfg, q_dev[t - T0], cache, out)
-            if events:
-                events[2][i].record()
 
     base = T0 + n_e2e
     run_steps(base, W)
@@ -917,21 +968,21 @@ def main():
         torch.cuda.synchronize()
     total_ms = e0.elapsed_time(e1)
     base2 = base + W + K
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(K)] for _ in range(3)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(K)] for _ in range(2)]
     run_steps(base2, W)
     torch.cuda.synchronize()
     run_steps(base2 + W, K, ev)
     torch.cuda.synchronize()
-    dec_ms = [ev[1][i].elapsed_time(ev[2][i]) for i in range(K)]
-    app_ms = [ev[0][i].elapsed_time(ev[1][i]) for i in range(K)]
+    dec_ms = [ev[0][i].elapsed_time(ev[1][i]) for i in range(K)]
     total_ms = max_over_ranks(total_ms, pg, dev)
     err = cache.read_error()
     lens = cache.lengths().cpu().numpy()
     assert err == 0 and int(lens.min()) == CONTEXT, (err, lens)
 
-    # algorithmic bytes of the timed decode launches (context after each append)
+    # algorithmic bytes of the timed launches (context after each append): the decode's,
+    # plus the append's new rows (read, and stored into the residual window)
     units, G = B * HKV, HQ // HKV
-    alg = [decode_bytes(base2 + W + i + 1, units, G, rec_bytes) for i in range(K)]
+    alg = [decode_bytes(base2 + W + i + 1, units, G, rec_bytes) + units * 2 * 2 * D * 2 for i in range(K)]
     avg_dec_s = sum(dec_ms) / K / 1e3
     achieved = sum(alg) / K / avg_dec_s / 1e9
     peak, peak_kind = measured_peaks()
@@ -943,17 +994,17 @@ def main():
         "config": stream_config(world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": captured_traffic(sum(alg) / K),
-                     "algorithmic_bytes": sum(alg) / K, "kernel": "pnmix decode attention",
+                     "algorithmic_bytes": sum(alg) / K, "kernel": "pnmix append + decode attention (one launch)",
                      "peak_source": peak_kind, "frac_of_8tbs": achieved / 8000.0},
         "decode_kernel_us": 1e3 * sum(dec_ms) / K,
-        "append_kernel_us": 1e3 * sum(app_ms) / K,
+        "append_fused": True,
         "prefill": {"tokens": PREFILL, "saliency_ms": saliency_ms, "quantize_ms": quant_ms,
                     "quantize_tokens_per_s": B * PREFILL / (quant_ms / 1e3)},
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(q_host[0].numel() * 2 + kn_host[0].numel() * 2 * 2),
                 "d2h_bytes_per_step": int(out_host[0].numel() * 4),
                 "overlap": "inputs of step i+1 and the output of step i-1 copy during step i"},
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clocks.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

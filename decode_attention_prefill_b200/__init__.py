@@ -45,7 +45,7 @@ EXPORTED = [
     "pnmix_status_string", "pnmix_version", "pnmix_decode_attention_noalloc",
     "pnmix_workspace_bytes_multi", "pnmix_decode_attention_multi", "pnmix_shrink_keys",
     "pnmix_split_groups", "pnmix_debug_decode_stall", "pnmix_workspace_bytes_two",
-    "pnmix_decode_attention_two",
+    "pnmix_decode_attention_two", "pnmix_append_decode",
 ]
 
 
@@ -110,6 +110,7 @@ _SIGS = {
     "pnmix_debug_decode_stall": (_i, [_CP, _vp, _KP, _i, _vp, _vp, _sz, _i, ctypes.c_uint32, _vp]),
     "pnmix_workspace_bytes_two": (_sz, [_CP, _CP, _i, _i, _i]),
     "pnmix_decode_attention_two": (_i, [_CP, _KP, _i, _CP, _KP, _i, _vp, _vp, _vp, _sz, _vp]),
+    "pnmix_append_decode": (_i, [_CP, _vp, _vp, _vp, _KP, _i, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -200,6 +201,20 @@ def pnmix_decode_attention(cfg: Config, q: torch.Tensor, cache: "PNMixCache", ou
                                        ctypes.byref(cache.c), mc, _dev(out, torch.float32, "out"),
                                        _dev(ws, torch.uint8, "workspace"), ws.numel(),
                                        _stream(stream)), "pnmix_decode_attention")
+
+
+def pnmix_append_decode(cfg: Config, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                        cache: "PNMixCache", out: torch.Tensor, workspace: torch.Tensor | None = None,
+                        max_context: int | None = None, stream=None):
+    """One decode step: append k_new, v_new bf16 [B][Hkv][128], then attend q bf16 [B][Hq][128]
+    over the cache including the new token -> out fp32 [B][Hq][128]."""
+    ws = cache.workspace if workspace is None else workspace
+    mc = cache.max_context if max_context is None else max_context
+    _check(_lib.pnmix_append_decode(ctypes.byref(cfg), _dev(k_new, torch.bfloat16, "k_new"),
+                                    _dev(v_new, torch.bfloat16, "v_new"), _dev(q, torch.bfloat16, "q"),
+                                    ctypes.byref(cache.c), mc, _dev(out, torch.float32, "out"),
+                                    _dev(ws, torch.uint8, "workspace"), ws.numel(), _stream(stream)),
+           "pnmix_append_decode")
 
 
 def workspace_bytes_multi(cfg: Config, batch: int, max_context: int, n_queries: int) -> int:

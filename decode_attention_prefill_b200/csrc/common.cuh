@@ -34,6 +34,7 @@ struct Geometry {
   int kernel;     // decode kernel, PNMIX_DECODE_*
   uint32_t wait_limit;   // decode: try_wait rounds before a staging wait gives up
   int skip_unit;         // decode test hook: the unit whose records are never staged (-1: none)
+  int append;            // decode: the launch first appends one K/V row per sequence (fused)
 };
 
 // try_wait rounds before a decode staging wait gives up (each round may suspend the warp
@@ -176,8 +177,12 @@ __host__ __device__ __forceinline__ size_t scratch_append_ticket_offset(int B, i
 __host__ __device__ __forceinline__ size_t scratch_range_offset(int B, int Hkv) {
   return static_cast<size_t>(B) * Hkv * 65 + B;
 }
-__host__ __device__ __forceinline__ size_t scratch_words(int B, int Hkv) {
+// one word: the grid ticket of a fused append + decode launch (its last CTA advances len)
+__host__ __device__ __forceinline__ size_t scratch_fused_ticket_offset(int B, int Hkv) {
   return static_cast<size_t>(B) * Hkv * (65 + 256) + B;
+}
+__host__ __device__ __forceinline__ size_t scratch_words(int B, int Hkv) {
+  return static_cast<size_t>(B) * Hkv * (65 + 256) + B + 1;
 }
 
 // Launchers (one translation unit each).
@@ -198,12 +203,15 @@ pnmix_status check_decode_args(const pnmix_config* cfg, const uint16_t* q, const
                                int max_context, const float* out, Geometry* g);
 size_t decode_workspace_bytes(const Geometry& g, int max_context);
 size_t decode_ticket_offset(const Geometry& g, int max_context);
-// Optional log-sum-exp output and merge with an earlier attention over other tokens (the
-// two parts of a two-precision cache); see combine_segment in decode_common.cuh.
+// Optional parts of a decode launch: the log-sum-exp output and the merge with an earlier
+// attention over other tokens (the two parts of a two-precision cache; see combine_segment
+// in decode_common.cuh), and the rows of a fused append (Geometry::append).
 struct DecodeMerge {
   float* lse_out = nullptr;
   const float* prior_out = nullptr;
   const float* prior_lse = nullptr;
+  const uint16_t* k_new = nullptr;
+  const uint16_t* v_new = nullptr;
 };
 cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cache& c,
                           int max_context, float* out, void* ws, cudaStream_t s,

@@ -34,6 +34,9 @@ struct DecodeWs {
   float* lse_out;            // if set: log2 sum_t 2^(logit_t) of every output row
   const float* prior_out;    // if set: merge with an earlier attention over other tokens,
   const float* prior_lse;    //   given by its normalised output and log-sum-exp
+  // fused append (Geometry::append): the new K / V rows, bf16 [B][Hkv][128]
+  const uint16_t* k_new;
+  const uint16_t* v_new;
 };
 
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -47,11 +50,18 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int N) {
   return static_cast<int>(((x + 1) * N - 1) / T);
 }
 
+// Whether a fused append adds a token to a sequence holding `raw` tokens (as pnmix_append:
+// only while there is room).
+__device__ __forceinline__ bool appends(const Geometry& g, int raw) {
+  return g.append && raw >= 0 && raw < g.capacity;
+}
+
 // Length of sequence b as the partition uses it: len[b] clamped to [0, capacity], so a
 // length array holding anything else (stale memory, a caller's ordering mistake) cannot
-// send a record read outside the cache.
+// send a record read outside the cache; plus the token a fused append adds.
 __device__ __forceinline__ int seq_len(const Geometry& g, const int32_t* len, int b) {
-  return min(max(len[b], 0), g.capacity);
+  const int raw = len[b];
+  return min(max(raw, 0), g.capacity) + (appends(g, raw) ? 1 : 0);
 }
 
 __device__ __forceinline__ long long total_items(const Geometry& g, const int32_t* len) {
@@ -65,6 +75,8 @@ struct Segment {
   int lo, hi;          // items [lo, hi) of the unit; item len/32 is the residual item
   int ng, nr;          // full groups and residual tokens of the unit
   int first, last;     // CTAs covering the unit
+  int app_slot;        // fused append: residual slot of the new token (31: it completes
+                       // group ng - 1), or -1 when nothing is appended
 };
 
 // Calls fn(seg) for every segment of this CTA, in item order.  All threads of the CTA
@@ -101,6 +113,7 @@ __device__ __forceinline__ void for_each_segment(const Geometry& g, const int32_
     s.hi = static_cast<int>((uend < e ? uend : e) - ustart);
     s.ng = lb / kGroup;
     s.nr = lb % kGroup;
+    s.app_slot = appends(g, len[b]) ? (lb - 1) % kGroup : -1;
     s.first = cta_of(ustart, T, N);
     s.last = cta_of(uend - 1, T, N);
     fn(s);

@@ -140,10 +140,12 @@ __device__ __forceinline__ void key_slice_frags(uint32_t w0, uint32_t w1, int pa
 }
 
 // The query constants of one lane, per slice pair c (entries 2*sigma + e of the pair):
-// X = (0 | q) and Y = (q | -q) on (even | odd) B columns, fp16x2.
+// X = (0 | q) and Y = (q | -q) on (even | odd) B columns, fp16x2; z: the B operand of the
+// pair's zero-point product where a kernel uses one (see decode_mma.cu).
 template <int NT>
 struct QFrags {
   uint4 x[NT][4], y[NT][4];
+  uint2 z[NT][4];
 };
 
 // Dynamic query-channel pruning of the unit's query rows in shared memory (qnat, fp32
@@ -192,9 +194,9 @@ __device__ __forceinline__ void prune_query_rows(const Geometry& g, float* qnat,
 // per head into `slot`.
 __device__ __noinline__ void residual_partial(const Geometry& g, const uint16_t* rk, const uint16_t* rv,
                                               int nr, const float* qnat, float qscale, float* slot, int h0,
-                                              int hstep, int tok0, int vis_base) {
+                                              int hstep, int tok0, int vis_base, int kstride = kResidKStride) {
   const int lane = threadIdx.x & 31;
-  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kResidKStride);
+  const uint4* row = reinterpret_cast<const uint4*>(rk + (lane < nr ? lane : 0) * kstride);
 #pragma unroll 1
   for (int hh = h0; hh < g.rows; hh += hstep) {
     // residual row `lane` is token tok0 + lane; row hh sees tokens below vis_base + hh / G

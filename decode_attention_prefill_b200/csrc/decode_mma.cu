@@ -13,11 +13,12 @@
 //   by two interleaved B columns (head h -> columns 2h, 2h+1): fp16(q s) and its rounding
 //   error fma(q, s, -fp16(q s)).  One lane-uniform sequence b = fma(X, s, fp16(Y s)) with
 //   per-lane constants (X, Y) = (0, q) on even columns and (q, -q) on odd ones gives both.
-//   The zero-point term is one more MMA per slice whose A operand is the 16-byte zero-point
-//   chunk of the slice pair exactly as loaded (rows 0-7 carry the even slice's zeros, rows
-//   8-15 the odd slice's, see the key scale order in include/pnmix.h) and whose B operand
-//   is X; the even slice's sum is read from rows 0-7 of one accumulator, the odd slice's
-//   from rows 8-15 of another.  The softmax scale is applied to the fp32 logits.
+//   The zero-point term is one more MMA per slice PAIR whose A operand is the 16-byte
+//   zero-point chunk of the pair exactly as loaded (rows 0-7 carry the even slice's zeros,
+//   rows 8-15 the odd slice's, see the key scale order in include/pnmix.h) and whose B
+//   operand carries q of the even slice on the odd columns and q of the odd slice on the
+//   even columns: rows 0-7 of a head's odd column and rows 8-15 of its even column are the
+//   two slices' sums.  The softmax scale is applied to the fp32 logits.
 //   out     sum_t p_t v^_t = sum_t (p_t s_{t,j}) code_{t,c} + sum_t p_t z_{t,j}
 //          = [codes^T (channels x tokens)] x [p s]  +  [z rows] x [p]
 //   with p rounded to fp16 once (fp32 accumulation); the value zero-point chunk of a lane
@@ -36,6 +37,7 @@
 #include "common.cuh"
 #include "decode_common.cuh"
 #include "decode_frag.cuh"
+#include "quantize_group.cuh"
 
 namespace pnmix {
 namespace {
@@ -44,10 +46,11 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 // Headroom (log2 domain) the lazy softmax reference keeps above the largest logit seen.
 constexpr float kHeadroom = 4.f;
-// Staging ring per warp, in record pairs: 3 pairs (6 records) with one tile of query
-// columns (up to 4 rows, two CTAs per SM), 2 pairs with two tiles (three CTAs per SM).
+// Fused append, flush step: the quantizers' staging tile sits in the (then idle) ring.
+static_assert(sizeof(GroupSmem) <= 4 * 2 * 2 * 3072, "the quantizers' tile must fit the staging ring");
+// Staging ring per warp: 2 record pairs (4 records), three CTAs per SM.
 template <int NT>
-__host__ __device__ constexpr int pair_slots() { return NT == 1 ? 3 : 2; }
+__host__ __device__ constexpr int pair_slots() { return 2; }
 
 // ------------------------------------------------------------------ shared memory map
 
@@ -56,7 +59,6 @@ struct SmemMap {
   int qnat;      // fp32 [kMaxG][128], natural channel order, unscaled
   int perm;      // 128 bytes
   int resid;     // fp32 [kMaxG][kPartialStride]: partial of the residual item
-  int rrows;     // bf16 residual K rows [32][kResidKStride] then V rows [32][128]
   int bars;      // uint64 [kWarps][slots] mbarriers
   int stages;    // [kWarps][slots][2 R]
   int part;      // fp32 [kWarps][kMaxG][kPartialStride], aliases the stages
@@ -70,8 +72,7 @@ __host__ __device__ __forceinline__ SmemMap smem_map(int NT, int R) {
   m.qnat = NT * 2 * 4 * 32 * 16;
   m.perm = m.qnat + kMaxG * kHeadDim * 4;
   m.resid = m.perm + 128;
-  m.rrows = m.resid + kMaxG * kPartialStride * 4;
-  m.bars = m.rrows + kGroup * kResidKStride * 2 + kGroup * kHeadDim * 2;
+  m.bars = m.resid + kMaxG * kPartialStride * 4;
   m.stages = m.bars + ((kWarps * nsl * 8 + 127) / 128) * 128;
   int stage_bytes = kWarps * nsl * 2 * R;
   int part_bytes = kWarps * kMaxG * kPartialStride * 4;
@@ -116,20 +117,21 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* c
   const int tq = lane & 3;
 
   // key-code products, kept apart per block because the two blocks' token-row bit
-  // offsets differ; the zero-point term per slice parity (normal fp16 scale)
-  float acc_hi[NG][NT][2][4], acc_lo[NG][NT][2][4], dz[NG][NT][2][4];
+  // offsets differ; the zero-point term (normal fp16 scale), one product per slice pair
+  float acc_hi[NG][NT][2][4], acc_lo[NG][NT][2][4], dz[NG][NT][4];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        dz[gi][nt][i] = 0.f;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           acc_hi[gi][nt][x][i] = 0.f;
           acc_lo[gi][nt][x][i] = 0.f;
-          dz[gi][nt][x][i] = 0.f;
         }
+      }
 
 #pragma unroll
   for (int sp = 0; sp < 4; ++sp) {
@@ -179,20 +181,20 @@ __device__ __forceinline__ void group_logits(const Geometry& g, const uint8_t* c
             mma16816(acc_lo[gi][nt][0], A[0][0], A[0][1], A[0][2], A[0][3], b0, b1);
             mma16816(acc_lo[gi][nt][1], A[1][0], A[1][1], A[1][2], A[1][3], b0, b1);
           }
-          mma16816(dz[gi][nt][par], z4[gi].x, z4[gi].y, z4[gi].z, z4[gi].w, qx0, qx1);
+          if (par == 0) mma16816(dz[gi][nt], z4[gi].x, z4[gi].y, z4[gi].z, z4[gi].w, qf.z[nt][sp].x, qf.z[nt][sp].y);
         }
       }
     }
   }
 
   // ---- logits (log2 domain): lane holds head 4*nt + tq at tokens gq + 8*u, u = 0..3; the
-  // zero-point sum of the head is on its odd column (X is zero on even ones): rows 0-7 of
-  // the even-slice accumulator plus rows 8-15 of the odd-slice one
+  // zero-point sum of the head: rows 0-7 (even slices) of its odd column plus rows 8-15
+  // (odd slices) of its even column
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const float zb = (dz[gi][nt][0][1] + dz[gi][nt][1][3]) * qscale;
+      const float zb = (dz[gi][nt][1] + dz[gi][nt][2]) * qscale;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int mt = u >> 1, r = 2 * (u & 1);
@@ -388,7 +390,7 @@ __device__ __forceinline__ void process_groups(const Geometry& g, const uint8_t*
 // MQ: several queries per sequence (rows = G * tq), with the causal mask on the newest
 // tokens; a separate instance so the one-query kernel carries none of it.
 template <int BHI, int BLO, int NT, int NHS, bool MQ>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, 3)
 decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out,
                   DecodeWs ws) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -401,8 +403,6 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
   float* qnat = reinterpret_cast<float*>(smem + sm.qnat);
   uint8_t* perm = smem + sm.perm;
   float* rslot = reinterpret_cast<float*>(smem + sm.resid);
-  uint16_t* rrk = reinterpret_cast<uint16_t*>(smem + sm.rrows);
-  uint16_t* rrv = rrk + kGroup * kResidKStride;
   float* part = reinterpret_cast<float*>(smem + sm.part);
   uint8_t* ring = smem + sm.stages + warp * kSlots * 2 * R;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm.bars) + warp * kSlots;
@@ -424,6 +424,11 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
     // ---- this warp's contiguous run [g0, g0 + my_count) of the segment's groups, taken
     // as pairs of consecutive records (a last single record when the count is odd)
+    // fused append: on a flush step the new token completes group seg.ng - 1, whose record
+    // this launch builds; the CTA owning that item quantizes it first (staging tile in the
+    // idle ring), stores it, and then stages it like every other record
+    const int gf = seg.ng - 1;
+    const bool own_flush = seg.app_slot == kGroup - 1 && gf >= seg.lo && gf < seg.hi;
     const int gend = seg.hi < seg.ng ? seg.hi : seg.ng;
     const int n = gend > seg.lo ? gend - seg.lo : 0;
     const int g0 = seg.lo + (n * warp) / kWarps;
@@ -465,6 +470,39 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       ++consumed;
       return r;
     };
+    // ---- fused append, flush step: quantize the 31 residual rows and the new row into the
+    // record of group gf and store it (the bit-exact quantizers of quantize_group.cuh, the
+    // staging tile in this CTA's ring, idle between segments), before any copy is issued
+    if (own_flush) {
+      __syncthreads();   // every warp of the CTA is past its previous segment's ring use
+      GroupSmem& gs = *reinterpret_cast<GroupSmem*>(smem + sm.stages);
+      gs.perm[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid] & (kHeadDim - 1);
+      const uint16_t* rows[2] = {c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim,
+                                 c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim};
+      const uint16_t* fresh[2] = {ws.k_new + static_cast<size_t>(unit) * kHeadDim,
+                                  ws.v_new + static_cast<size_t>(unit) * kHeadDim};
+      uint8_t* frec = record_ptr(g, c.records, b, h, gf);
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {
+        for (int i = tid; i < kGroup * 16; i += kThreads) {
+          const int r = i >> 4, cc = i & 15;
+          const uint4* src = r == kGroup - 1 ? reinterpret_cast<const uint4*>(fresh[part]) + cc
+                                             : reinterpret_cast<const uint4*>(rows[part]) + i;
+          *reinterpret_cast<uint4*>(&gs.tile[r][cc * 8]) = __ldg(src);
+        }
+        __syncthreads();
+        if (part == 0)
+          quantize_key_group(g, gs, frec);
+        else
+          quantize_value_group(g, gs, frec);
+        __syncthreads();
+      }
+      // the record was written through the generic proxy; the bulk copy that stages it
+      // reads through the async proxy
+      __threadfence();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncthreads();
+    }
     issue_upto(kSlots);
 
     // ---- query: unscaled fp32 in natural channel order, then the X / Y fp16 column sets
@@ -475,14 +513,16 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
     }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
-    if (seg_resid) {   // residual K and V rows into shared memory, 16-byte loads
-      const uint4* gk = reinterpret_cast<const uint4*>(c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim);
-      const uint4* gv = reinterpret_cast<const uint4*>(c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim);
-      for (int i = tid; i < seg.nr * 16; i += kThreads) {
-        const int r = i >> 4, cc = i & 15;
-        reinterpret_cast<uint4*>(rrk + r * kResidKStride)[cc] = __ldg(gk + i);
-        reinterpret_cast<uint4*>(rrv)[i] = __ldg(gv + i);
-      }
+    uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
+    uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
+    if (seg_resid && seg.app_slot >= 0 && tid < 32) {
+      // fused append: the new row goes into residual slot app_slot (< 31) of the cache;
+      // the residual partial below reads the window from there (plain loads, after the
+      // barrier)
+      const int cc = tid & 15;
+      const uint16_t* src = (tid < 16 ? ws.k_new : ws.v_new) + static_cast<size_t>(unit) * kHeadDim;
+      uint16_t* dst = (tid < 16 ? rk : rv) + seg.app_slot * kHeadDim;
+      reinterpret_cast<uint4*>(dst)[cc] = __ldg(reinterpret_cast<const uint4*>(src) + cc);
     }
     if (g.n_prune > 0) {   // dynamic query-channel pruning of the staged query rows
       __syncthreads();
@@ -516,9 +556,9 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     }
     __syncthreads();
 
-    // ---- the residual item (CUDA cores): warp w takes heads w, w + 4
+    // ---- the residual item (CUDA cores, rows read from the cache): warp w takes heads w, w + 4
     if (seg_resid) {
-      residual_partial(g, rrk, rrv, seg.nr, qnat, qscale, rslot, warp, kWarps, seg.ng * kGroup, vis_base);
+      residual_partial(g, rk, rv, seg.nr, qnat, qscale, rslot, warp, kWarps, seg.ng * kGroup, vis_base, kHeadDim);
     } else if (warp == 0 && lane < G) {
       rslot[lane * kPartialStride + 0] = -INFINITY;
       rslot[lane * kPartialStride + 1] = 0.f;
@@ -532,6 +572,10 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       for (int cp = 0; cp < 4; ++cp) {
         qf.x[nt][cp] = reinterpret_cast<const uint4*>(qsets)[((nt * 2 + 0) * 4 + cp) * 32 + lane];
         qf.y[nt][cp] = reinterpret_cast<const uint4*>(qsets)[((nt * 2 + 1) * 4 + cp) * 32 + lane];
+        // zero-point B operand of slice pair cp: q of the even slice on odd columns (X), q of
+        // the odd slice on even columns (Y holds q there)
+        const bool odd_col = (lane >> 2) & 1;
+        qf.z[nt][cp] = odd_col ? make_uint2(qf.x[nt][cp].x, qf.x[nt][cp].y) : make_uint2(qf.y[nt][cp].z, qf.y[nt][cp].w);
       }
     WarpAcc<NT> st;
 #pragma unroll
@@ -662,6 +706,30 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
     }
     combine_segment(ws, seg, G, out, g);
   });
+
+  // ---- fused append: the grid's last CTA (every CTA has read len[] by now) advances the
+  // lengths, as pnmix_append does; a full sequence keeps its length and raises the error bit
+  if (g.append) {
+    __shared__ int last_cta;
+    uint32_t* ticket = c.scratch + scratch_fused_ticket_offset(g.B, g.Hkv);
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      last_cta = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (last_cta) {
+      __threadfence();
+      for (int bb = tid; bb < g.B; bb += kThreads) {
+        const int raw = c.len[bb];
+        if (appends(g, raw))
+          c.len[bb] = raw + 1;
+        else
+          atomicOr(c.error, PNMIX_DEVERR_APPEND_FULL);
+      }
+      if (tid == 0) *ticket = 0u;
+    }
+  }
 }
 
 // Resident CTAs of one full wave of a kernel instance, per device: the shared-memory

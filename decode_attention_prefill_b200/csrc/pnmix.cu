@@ -57,6 +57,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->kernel = cfg->decode_kernel;
   g->wait_limit = kDecodeWaitLimit;
   g->skip_unit = -1;
+  g->append = 0;
   return PNMIX_OK;
 }
 
@@ -133,6 +134,8 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   w.lse_out = merge.lse_out;
   w.prior_out = merge.prior_out;
   w.prior_lse = merge.prior_lse;
+  w.k_new = merge.k_new;
+  w.v_new = merge.v_new;
   switch (g.kernel) {
     case PNMIX_DECODE_SIMT: return launch_decode_simt(g, q, c, nmax, out, w, s);
     case PNMIX_DECODE_MMA: return launch_decode_mma(g, q, c, nmax, out, w, s);
@@ -285,6 +288,31 @@ pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uint16_t* q,
   if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
   return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+pnmix_status pnmix_append_decode(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
+                                 const uint16_t* q, pnmix_cache* cache, int max_context, float* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  Geometry g;
+  pnmix_status st = check_decode_args(cfg, q, cache, max_context, out, &g);
+  if (st != PNMIX_OK) return st;
+  if (!k_new || !v_new || !workspace) return PNMIX_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
+  if (workspace_bytes < decode_workspace_bytes(g, max_context)) return PNMIX_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the one-role tensor-core kernel appends inside the decode launch; the others take the
+  // append kernel first
+  const bool fused = g.kernel == PNMIX_DECODE_MMA || (g.kernel == PNMIX_DECODE_AUTO && g.rows <= 4);
+  if (!fused) {
+    const cudaError_t e = launch_append(g, k_new, v_new, *cache, s);
+    if (e != cudaSuccess) return PNMIX_ERR_CUDA;
+    return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace, s));
+  }
+  g.append = 1;
+  DecodeMerge rows;
+  rows.k_new = k_new;
+  rows.v_new = v_new;
+  return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace, s, rows));
 }
 
 size_t pnmix_workspace_bytes_two(const pnmix_config* cfg_a, const pnmix_config* cfg_b, int batch,

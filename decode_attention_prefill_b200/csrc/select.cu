@@ -23,10 +23,8 @@ constexpr int kRowsPerIter = kThreads / 8;   // 8 threads per 128-channel row
 // Pair norms of 8 consecutive pairs p = 8*c .. 8*c+7 of one row, from the two 16-byte
 // chunks (channels 8c..8c+7 and 64+8c..64+8c+7); with RANGE also the 16 channel values.
 template <bool RANGE = false>
-__device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float out[8],
-                                               float* mn = nullptr, float* mx = nullptr) {
-  uint4 lo = __ldg(reinterpret_cast<const uint4*>(row) + c);
-  uint4 hi = __ldg(reinterpret_cast<const uint4*>(row) + 8 + c);
+__device__ __forceinline__ void chunk_pair_norm2(const uint4& lo, const uint4& hi, float out[8],
+                                                 float* mn = nullptr, float* mx = nullptr) {
   const uint16_t* a = reinterpret_cast<const uint16_t*>(&lo);
   const uint16_t* b = reinterpret_cast<const uint16_t*>(&hi);
 #pragma unroll
@@ -41,6 +39,15 @@ __device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float
     }
   }
 }
+template <bool RANGE = false>
+__device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float out[8],
+                                               float* mn = nullptr, float* mx = nullptr) {
+  const uint4 lo = __ldg(reinterpret_cast<const uint4*>(row) + c);
+  const uint4 hi = __ldg(reinterpret_cast<const uint4*>(row) + 8 + c);
+  chunk_pair_norm2<RANGE>(lo, hi, out, mn, mx);
+}
+
+constexpr int kRowUnroll = 4;   // rows per thread per pass: 8 independent 16-byte loads in flight
 
 // Order-preserving map of non-NaN floats to unsigned integers (and back), so that
 // integer atomics compute float min / max.
@@ -90,11 +97,26 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
       mx16[i] = -INFINITY;
     }
   }
-  for (int t = t0 + rsub; t < t1; t += kRowsPerIter) {
-    float n2[8];
-    row_pair_norm2<RANGE>(kbase + static_cast<size_t>(t) * kHeadDim, cidx, n2, mn16, mx16);
+  for (int t = t0 + rsub; t < t1; t += kRowUnroll * kRowsPerIter) {
+    uint4 lo[kRowUnroll], hi[kRowUnroll];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], n2[i]);
+    for (int u = 0; u < kRowUnroll; ++u) {   // all loads of the pass first
+      const int tt = t + u * kRowsPerIter;
+      if (tt < t1) {
+        const uint4* row = reinterpret_cast<const uint4*>(kbase + static_cast<size_t>(tt) * kHeadDim);
+        lo[u] = __ldg(row + cidx);
+        hi[u] = __ldg(row + 8 + cidx);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      if (t + u * kRowsPerIter < t1) {
+        float n2[8];
+        chunk_pair_norm2<RANGE>(lo[u], hi[u], n2, mn16, mx16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], n2[i]);
+      }
+    }
   }
   // lanes with the same cidx: xor 8, 16
 #pragma unroll
@@ -238,9 +260,10 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
     e = cudaMemset2DAsync(cm + 128, 1024, 0x00, 512, units, s);
     if (e != cudaSuccess) return e;
   }
-  // about eight CTAs per SM so the max pass balances, with >= 128 tokens per CTA
+  // about eight CTAs per SM so the max pass balances, with >= 256 tokens per CTA (two
+  // passes of kRowUnroll rows per thread)
   int want = (8 * 148 + units - 1) / units;
-  int max_split = (L + 127) / 128;
+  int max_split = (L + 255) / 256;
   int nsplit = want < max_split ? want : max_split;
   if (nsplit < 1) nsplit = 1;
   if (nsplit > 512) nsplit = 512;

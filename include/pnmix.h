@@ -329,6 +329,23 @@ PNMIX_API pnmix_status pnmix_decode_attention(const pnmix_config* cfg, const uin
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * One decode step in one call: pnmix_append of k_new, v_new (bf16 [B][Hkv][128]) followed
+ * by pnmix_decode_attention of q (bf16 [B][Hq][128]) over the cache that includes the new
+ * token; out fp32 [B][Hq][128].  The result, the cache contents and the error bits are
+ * those of the two calls in sequence.  With the one-role tensor-core kernel (the automatic
+ * choice for up to 4 query heads per KV head, or PNMIX_DECODE_MMA) the append runs inside
+ * the decode launch: the CTA that attends over a unit's residual window stores the new row
+ * there, on a step that completes a 32-token group the CTA owning that group quantizes it
+ * (the same quantizers, bit-exact) and stores its record, and the launch's last CTA
+ * advances len[].  Other kernels take an append launch first.  max_context bounds the
+ * lengths after the append; workspace as for pnmix_decode_attention.  Errors as for
+ * pnmix_decode_attention and pnmix_append.
+ */
+PNMIX_API pnmix_status pnmix_append_decode(const pnmix_config* cfg, const uint16_t* k_new, const uint16_t* v_new,
+                                           const uint16_t* q, pnmix_cache* cache, int max_context, float* out,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Workspace bytes pnmix_decode_attention_multi needs for n_queries queries per
  * sequence (n_queries = 1 gives pnmix_workspace_bytes); 0 if unsupported.
  */

@@ -307,3 +307,18 @@ def test_two_part_decode_rejects_bad_arguments_before_launching():
     assert f(*args(lo, a, lo, b, P, n)) == pm.ERR_INVALID_ARG          # cache a laid out for another config
     other = pm.Config.make(16, 4)
     assert f(*args(hi, a, other, _fake_cache(other), P, n)) == pm.ERR_INVALID_ARG   # head counts differ
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses fake device pointers; runs only where no kernel can launch")
+def test_append_decode_rejects_bad_arguments_before_launching():
+    cfg = pm.Config.make(8, 2)
+    c = _fake_cache(cfg)
+    P = ctypes.c_void_p(1 << 41)
+    odd = ctypes.c_void_p((1 << 41) + 2)
+    ws = pm.workspace_bytes(cfg, 2, 256)
+    f = pm._lib.pnmix_append_decode
+    assert f(ctypes.byref(cfg), None, P, P, ctypes.byref(c), 256, P, P, ws, None) == pm.ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), P, odd, P, ctypes.byref(c), 256, P, P, ws, None) == pm.ERR_ALIGNMENT
+    assert f(ctypes.byref(cfg), P, P, P, ctypes.byref(c), 256, P, P, ws - 1, None) == pm.ERR_CAPACITY
+    assert f(ctypes.byref(cfg), P, P, P, ctypes.byref(c), -1, P, P, ws, None) == pm.ERR_INVALID_ARG

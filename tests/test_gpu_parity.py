@@ -552,3 +552,48 @@ def test_two_part_decode_at_128k_context():
     torch.cuda.synchronize()
     units = [(0, 1), (1, 3)]
     assert_close(out.cpu().numpy(), want.attend(q, heads=units), units=units, G=Hq // Hkv)
+
+
+# One call per decode step (pnmix_append_decode): with the one-role tensor-core kernel the
+# append runs inside the decode launch (residual row store, the flush of a completed group,
+# the length update); the outputs and the cache bytes must equal append-then-attend in the
+# oracle at every step, across flush boundaries.
+@pytest.mark.parametrize("kernel", [None, "mma", "ws", "simt"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,steps", [
+    (2, 8, 2, 40, 70),       # crosses two flushes
+    (1, 4, 1, 31, 3),        # the first step completes the first group
+    (3, 32, 8, 250, 40),
+    (2, 28, 4, 95, 34),
+])
+def test_fused_append_decode_step_matches_append_then_attend(kernel, B, Hq, Hkv, L, steps):
+    import decode_attention_prefill_b200 as pm
+    c = Case(B, Hq, Hkv, L, extra_tokens=steps, seed=L + steps, kernel=kernel)
+    c.prefill()
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device="cuda")
+    for t in range(L, L + steps):
+        kn = np.ascontiguousarray(c.kin[:, :, t])
+        vn = np.ascontiguousarray(c.vin[:, :, t])
+        q = c.query(t)
+        pm.pnmix_append_decode(c.cfg, to_dev(kn), to_dev(vn), to_dev(q), c.cache, out)
+        c.ocache.append(kn, vn)
+        if t % 7 == 0 or t % 32 == 31 or t == L + steps - 1:
+            torch.cuda.synchronize()
+            assert_close(out.cpu().numpy(), c.ocache.attend(q))
+    c.check_state()
+    assert c.cache.read_error() == 0
+
+
+def test_fused_append_decode_on_a_full_cache_raises_the_error_bit():
+    import decode_attention_prefill_b200 as pm
+    c = Case(1, 4, 1, 64, capacity=64)
+    c.prefill()
+    out = torch.empty(1, 4, 128, dtype=torch.float32, device="cuda")
+    before = c.cache.records().clone()
+    q = c.query(64)
+    pm.pnmix_append_decode(c.cfg, to_dev(c.kin[:, :, 0].copy()), to_dev(c.vin[:, :, 0].copy()), to_dev(q),
+                           c.cache, out)
+    torch.cuda.synchronize()
+    assert c.cache.read_error() == 0x1
+    assert int(c.cache.lengths()[0]) == 64
+    assert torch.equal(before, c.cache.records())
+    assert_close(out.cpu().numpy(), c.ocache.attend(q))     # attends over the 64 cached tokens
