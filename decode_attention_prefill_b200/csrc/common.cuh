@@ -35,6 +35,9 @@ struct Geometry {
   uint32_t wait_limit;   // decode: try_wait rounds before a staging wait gives up
   int skip_unit;         // decode test hook: the unit whose records are never staged (-1: none)
   int append;            // decode: the launch first appends one K/V row per sequence (fused)
+  int lead;              // decode partition: work items counted at the start of every unit for
+                         // its fixed cost (setup, merge, combine), with no work of their own
+  int resid_w;           // decode partition: items the residual window counts for (>= 1)
 };
 
 // try_wait rounds before a decode staging wait gives up (each round may suspend the warp

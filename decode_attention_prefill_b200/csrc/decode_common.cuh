@@ -64,15 +64,23 @@ __device__ __forceinline__ int seq_len(const Geometry& g, const int32_t* len, in
   return min(max(raw, 0), g.capacity) + (appends(g, raw) ? 1 : 0);
 }
 
+// Work items of a unit holding lb tokens: g.lead items for its fixed cost (a CTA whose slice
+// starts a unit takes fewer groups), its lb / 32 groups, and for the residual window
+// g.resid_w items (one when it is empty), taken whole by the CTA whose slice holds the first.
+__device__ __forceinline__ long long unit_items(const Geometry& g, int lb) {
+  return static_cast<long long>(g.lead) + lb / kGroup + (lb % kGroup ? g.resid_w : 1);
+}
+
 __device__ __forceinline__ long long total_items(const Geometry& g, const int32_t* len) {
   long long T = 0;
-  for (int b = 0; b < g.B; ++b) T += static_cast<long long>(g.Hkv) * (seq_len(g, len, b) / kGroup + 1);
+  for (int b = 0; b < g.B; ++b) T += static_cast<long long>(g.Hkv) * unit_items(g, seq_len(g, len, b));
   return T;
 }
 
 struct Segment {
   int b, h, unit;
-  int lo, hi;          // items [lo, hi) of the unit; item len/32 is the residual item
+  int lo, hi;          // groups [lo, min(hi, ng)) of the unit; hi > ng: with the residual
+                       // window; lo >= hi: nothing (a slice of lead items only)
   int ng, nr;          // full groups and residual tokens of the unit
   int first, last;     // CTAs covering the unit
   int app_slot;        // fused append: residual slot of the new token (31: it completes
@@ -94,30 +102,33 @@ __device__ __forceinline__ void for_each_segment(const Geometry& g, const int32_
   long long x = a;
   while (x < e) {
     int lb = seq_len(g, len, b);
-    long long per_b = static_cast<long long>(g.Hkv) * (lb / kGroup + 1);
+    long long per_b = static_cast<long long>(g.Hkv) * unit_items(g, lb);
     while (b < g.B - 1 && cum + per_b <= x) {
       cum += per_b;
       ++b;
       lb = seq_len(g, len, b);
-      per_b = static_cast<long long>(g.Hkv) * (lb / kGroup + 1);
+      per_b = static_cast<long long>(g.Hkv) * unit_items(g, lb);
     }
-    const int items = lb / kGroup + 1;
+    const long long items = unit_items(g, lb);
     const int h = static_cast<int>((x - cum) / items);
     const long long ustart = cum + static_cast<long long>(h) * items;
     const long long uend = ustart + items;
+    const long long x_lo = x - ustart, x_hi = (uend < e ? uend : e) - ustart;   // unit-local items
+    const long long ng = lb / kGroup, rfirst = g.lead + ng;                    // first residual item
     Segment s;
     s.b = b;
     s.h = h;
     s.unit = b * g.Hkv + h;
-    s.lo = static_cast<int>(x - ustart);
-    s.hi = static_cast<int>((uend < e ? uend : e) - ustart);
+    s.lo = static_cast<int>(min(max(x_lo - g.lead, 0ll), ng));
+    s.hi = (x_lo <= rfirst && x_hi > rfirst) ? static_cast<int>(ng) + 1
+                                              : static_cast<int>(min(max(x_hi - g.lead, 0ll), ng));
     s.ng = lb / kGroup;
     s.nr = lb % kGroup;
     s.app_slot = appends(g, len[b]) ? (lb - 1) % kGroup : -1;
     s.first = cta_of(ustart, T, N);
     s.last = cta_of(uend - 1, T, N);
     fn(s);
-    x = ustart + s.hi;
+    x = ustart + x_hi;
   }
 }
 
@@ -155,30 +166,49 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
   __syncthreads();
   if (is_last) {
     __threadfence();
-    // weights first (one thread per (head, segment)), then every thread sums its channels
-    // with independent loads
+    // (1) per head, one warp: every lane loads the (m, l) pairs of its segments once (one
+    // round), the largest reference m* and the denominator follow by shuffles and the
+    // weights 2^(m_s - m*) of the first chunk go to shared memory; (2) per chunk of up to 32
+    // segments, every thread sums its (head, channel) pairs with four loads in flight
     __shared__ float wsh[kMaxG][kMaxCombineSegs];
-    __shared__ float den_sh[kMaxG];
+    __shared__ float mstar_sh[kMaxG], den_sh[kMaxG];
     __shared__ float mix_sh[kMaxG][2];   // weights of the prior row and of this one
+    constexpr int kLaneSegs = 4;         // segments per lane held in registers (128 per head)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;
-    for (unsigned chunk = 0; chunk < nseg; chunk += kMaxCombineSegs) {
-      const unsigned n = nseg - chunk < kMaxCombineSegs ? nseg - chunk : kMaxCombineSegs;
-      const bool last_chunk = chunk + n == nseg;
-      if (threadIdx.x < G) {
-        const int hh = threadIdx.x;
-        float m = -INFINITY;
-        for (unsigned k = 0; k < nseg; ++k)
-          m = fmaxf(m, __ldcg(base + (static_cast<size_t>(k) * G + hh) * kPartialStride));
-        float den = 0.f;
-        for (unsigned k = 0; k < nseg; ++k) {
-          const float* p = base + (static_cast<size_t>(k) * G + hh) * kPartialStride;
-          const float ms = __ldcg(p);
-          const float f = (ms == -INFINITY || m == -INFINITY) ? 0.f : exp2f(ms - m);
-          den = fmaf(__ldcg(p + 1), f, den);
-          if (k >= chunk && k < chunk + n) wsh[hh][k - chunk] = f;
-        }
+    const size_t seg_stride = static_cast<size_t>(G) * kPartialStride;
+    for (int hh = warp; hh < G; hh += nwarps) {
+      float2 ml[kLaneSegs];
+#pragma unroll
+      for (int r = 0; r < kLaneSegs; ++r) {
+        const unsigned k = lane + 32u * r;
+        ml[r] = k < nseg ? __ldcg(reinterpret_cast<const float2*>(base + k * seg_stride + hh * kPartialStride))
+                         : make_float2(-INFINITY, 0.f);
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kLaneSegs; ++r) m = fmaxf(m, ml[r].x);
+      for (unsigned k = lane + 32u * kLaneSegs; k < nseg; k += 32)   // beyond 128 segments: reload
+        m = fmaxf(m, __ldcg(base + k * seg_stride + hh * kPartialStride));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float den = 0.f;
+#pragma unroll
+      for (int r = 0; r < kLaneSegs; ++r) {
+        const float f = (ml[r].x == -INFINITY || m == -INFINITY) ? 0.f : exp2f(ml[r].x - m);
+        den = fmaf(ml[r].y, f, den);
+        if (r == 0 && static_cast<unsigned>(lane) < nseg) wsh[hh][lane] = f;
+      }
+      for (unsigned k = lane + 32u * kLaneSegs; k < nseg; k += 32) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(base + k * seg_stride + hh * kPartialStride));
+        den = fmaf(v.y, (v.x == -INFINITY || m == -INFINITY) ? 0.f : exp2f(v.x - m), den);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane == 0) {
+        mstar_sh[hh] = m;
         den_sh[hh] = den;
-        if (last_chunk && (ws.lse_out || ws.prior_out)) {
+        if (ws.lse_out || ws.prior_out) {
           const size_t row = row_offset(geo, s.b, s.h, hh) / kHeadDim;
           float L = den > 0.f ? m + log2f(den) : -INFINITY;
           float w0 = 0.f, w1 = den > 0.f ? 1.f : 0.f;
@@ -197,16 +227,37 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
           if (ws.lse_out) ws.lse_out[row] = L;
         }
       }
-      __syncthreads();
+    }
+    __syncthreads();
+    for (unsigned chunk = 0; chunk < nseg; chunk += kMaxCombineSegs) {
+      const unsigned n = nseg - chunk < kMaxCombineSegs ? nseg - chunk : kMaxCombineSegs;
+      const bool last_chunk = chunk + n == nseg;
+      if (chunk > 0) {   // the weights of a later chunk
+        for (int hh = warp; hh < G; hh += nwarps) {
+          if (static_cast<unsigned>(lane) < n) {
+            const float ms = __ldcg(base + (chunk + lane) * seg_stride + hh * kPartialStride);
+            const float m = mstar_sh[hh];
+            wsh[hh][lane] = (ms == -INFINITY || m == -INFINITY) ? 0.f : exp2f(ms - m);
+          }
+        }
+        __syncthreads();
+      }
       for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
         const int hh = i / kHeadDim, c = i % kHeadDim;
         const size_t off = row_offset(geo, s.b, s.h, hh);
         float* out_row = out + off;
+        const float* col = base + static_cast<size_t>(hh) * kPartialStride + 2 + c;
         float num = chunk == 0 ? 0.f : out_row[c];
-#pragma unroll 4
-        for (unsigned k = 0; k < n; ++k)
-          num = fmaf(__ldcg(base + (static_cast<size_t>(chunk + k) * G + hh) * kPartialStride + 2 + c),
-                     wsh[hh][k], num);
+        unsigned k = 0;
+        for (; k + 4 <= n; k += 4) {   // four segments' values in flight
+          const float a0 = __ldcg(col + (chunk + k) * seg_stride), a1 = __ldcg(col + (chunk + k + 1) * seg_stride);
+          const float a2 = __ldcg(col + (chunk + k + 2) * seg_stride), a3 = __ldcg(col + (chunk + k + 3) * seg_stride);
+          num = fmaf(a0, wsh[hh][k], num);
+          num = fmaf(a1, wsh[hh][k + 1], num);
+          num = fmaf(a2, wsh[hh][k + 2], num);
+          num = fmaf(a3, wsh[hh][k + 3], num);
+        }
+        for (; k < n; ++k) num = fmaf(__ldcg(col + (chunk + k) * seg_stride), wsh[hh][k], num);
         if (last_chunk) {
           float o = den_sh[hh] > 0.f ? num / den_sh[hh] : 0.f;
           if (ws.prior_out) o = fmaf(mix_sh[hh][0], ws.prior_out[off + c], mix_sh[hh][1] * o);

@@ -148,6 +148,27 @@ struct QFrags {
   uint2 z[NT][4];
 };
 
+// The unit's query rows (unscaled fp32, natural channel order, rows >= g.rows zero) and
+// its position order into shared memory, every load of the CTA issued in one round:
+// thread i < 128 takes 16-byte chunk i (row i / 16), threads < 8 the order.  Needs a CTA
+// of at least 128 threads.
+__device__ __forceinline__ void load_query_rows(const Geometry& g, const uint16_t* q, const uint8_t* cperm, int b,
+                                                int h, int unit, float* qnat, uint8_t* perm, int tid) {
+  static_assert(kMaxG * (kHeadDim / 8) == 128, "one 16-byte chunk per thread");
+  const int hh = tid >> 4;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u), pv = make_uint4(0u, 0u, 0u, 0u);
+  if (tid < 128 && hh < g.rows) v = __ldg(reinterpret_cast<const uint4*>(q + row_offset(g, b, h, hh)) + (tid & 15));
+  if (tid < kHeadDim / 16) pv = __ldg(reinterpret_cast<const uint4*>(cperm + static_cast<size_t>(unit) * kHeadDim) + tid);
+  if (tid < 128) {
+    float4* dst = reinterpret_cast<float4*>(qnat + tid * 8);
+    dst[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+    dst[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
+                         __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+  }
+  if (tid < kHeadDim / 16) reinterpret_cast<uint4*>(perm)[tid] = pv;
+}
+
 // Dynamic query-channel pruning of the unit's query rows in shared memory (qnat, fp32
 // [kMaxG][128], natural channel order): row v drops the g.n_prune pairs of smallest
 // squared pair norm fl(fl(a*a) + fl(b*b)), never pair 0, the higher pair index first among

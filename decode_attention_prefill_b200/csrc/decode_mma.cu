@@ -46,6 +46,10 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 // Headroom (log2 domain) the lazy softmax reference keeps above the largest logit seen.
 constexpr float kHeadroom = 4.f;
+// Work-partition weights (decode_common.cuh, unit_items), in group items: the fixed cost of
+// a unit's segment and the residual window's CUDA-core pass.
+constexpr int kLeadItems = 40;
+constexpr int kResidItems = 8;
 // Fused append, flush step: the quantizers' staging tile sits in the (then idle) ring.
 static_assert(sizeof(GroupSmem) <= 4 * 2 * 2 * 3072, "the quantizers' tile must fit the staging ring");
 // Staging ring per warp: 2 record pairs (4 records), three CTAs per SM.
@@ -421,6 +425,18 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
+    if (seg.lo >= seg.hi) {   // a slice of lead items only: an empty partial for the combine
+      float* o = partial_slot(ws, unit, G);
+      for (int hh = 0; hh < G; ++hh) {
+        if (tid == 0) {
+          o[hh * kPartialStride] = -INFINITY;
+          o[hh * kPartialStride + 1] = 0.f;
+        }
+        o[hh * kPartialStride + 2 + tid] = 0.f;
+      }
+      combine_segment(ws, seg, G, out, g);
+      return;
+    }
     const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
     // ---- this warp's contiguous run [g0, g0 + my_count) of the segment's groups, taken
     // as pairs of consecutive records (a last single record when the count is odd)
@@ -507,11 +523,7 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
 
     // ---- query: unscaled fp32 in natural channel order, then the X / Y fp16 column sets
     // in position order
-    perm[tid] = c.perm[static_cast<size_t>(unit) * kHeadDim + tid];
-    for (int i = tid; i < kMaxG * kHeadDim; i += kThreads) {
-      const int hh = i / kHeadDim;
-      qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
-    }
+    load_query_rows(g, q, c.perm, b, h, unit, qnat, perm, tid);
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
     uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
@@ -762,7 +774,12 @@ cudaError_t launch_mma_t(const Geometry& g, const uint16_t* q, const pnmix_cache
     if (cacheable) wave_cache[dev].store(wave, std::memory_order_relaxed);
   }
   ws.N = wave < nmax ? wave : nmax;
-  kern<<<ws.N, kThreads, sm.total, s>>>(g, q, c, out, ws);
+  // partition weights: a unit's fixed cost (query setup, merge, combine) and its residual
+  // window (CUDA cores, rows read from L2), in 32-token group items, measured on B200 at 32K
+  Geometry gw = g;
+  gw.lead = kLeadItems;
+  gw.resid_w = kResidItems;
+  kern<<<ws.N, kThreads, sm.total, s>>>(gw, q, c, out, ws);
   return cudaGetLastError();
 }
 

@@ -331,12 +331,8 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     }
 
     // ---- query (unscaled fp32, natural order), residual rows, then the X / Y sets
-    perm[tid & 127] = c.perm[static_cast<size_t>(unit) * kHeadDim + (tid & 127)];
+    load_query_rows(g, q, c.perm, b, h, unit, qnat, perm, tid);
     const float qscale = g.scale * kLog2e;
-    for (int i = tid; i < kMaxG * kHeadDim; i += kWsThreads) {
-      const int hh = i / kHeadDim;
-      qnat[i] = hh < G ? bf16_bits_to_float(q[row_offset(g, b, h, hh) + (i & (kHeadDim - 1))]) : 0.f;
-    }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     if (seg_resid) {
       const uint4* gk = reinterpret_cast<const uint4*>(c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim);

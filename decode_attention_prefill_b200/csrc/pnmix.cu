@@ -58,6 +58,8 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->wait_limit = kDecodeWaitLimit;
   g->skip_unit = -1;
   g->append = 0;
+  g->lead = 0;
+  g->resid_w = 1;
   return PNMIX_OK;
 }
 
