@@ -547,20 +547,24 @@ def run_decode_workload(args):
 
 
 def run_verify(args):
-    """verify_32k: the stream_32k shape (16 x 32/8 heads, 32768 tokens) with T = 2 new
-    tokens per sequence attended at once (pnmix_decode_attention_multi after two appends),
-    against one single-query decode of the same cache.  The 419 MB cache exceeds L2."""
+    """verify_32k: the stream_32k shape (16 x 32/8 heads, 32768 tokens) with T new tokens
+    per sequence attended at once (pnmix_decode_attention_multi after T appends), for
+    T = 1, 2, 4, 8 and 16 (4 to 64 query rows per KV head), each against the roofline of
+    the bytes it must read.  The 419 MB cache exceeds L2.  Besides the algorithmic bytes,
+    each point reports the tensor-core work per launch (the key- and value-side products
+    of every row with every cached token)."""
     import torch
 
     import decode_attention_prefill_b200 as pm
-    T = 2
+    Ts = [1, 2, 4, 8, 16]
+    Tmax = max(Ts)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    n0 = CONTEXT - T
+    n0 = CONTEXT - Tmax
     kin, vin, qwin, _ = gen_inputs(args.seed, CONTEXT, [])
-    qm = workload_rows_q(args.seed, CONTEXT - T, T)                      # [B][T][Hq][128]
+    qm = workload_rows_q(args.seed, CONTEXT - Tmax, Tmax)                # [B][Tmax][Hq][128]
     cfg = pm.Config.make(HQ, HKV, BHI, BLO, K_SALIENT, WINDOW)
-    cache = pm.PNMixCache(cfg, B, CONTEXT + 32, max_context=CONTEXT, max_queries=T)
+    cache = pm.PNMixCache(cfg, B, CONTEXT + 32, max_context=CONTEXT, max_queries=Tmax)
     k_dev = torch.from_numpy(kin).view(torch.bfloat16).to(dev)
     v_dev = torch.from_numpy(vin).view(torch.bfloat16).to(dev)
     pm.pnmix_select_pairs(cfg, torch.from_numpy(qwin).view(torch.bfloat16).to(dev), k_dev, PREFILL, cache)
@@ -569,31 +573,33 @@ def run_verify(args):
     for t in range(n0, CONTEXT):
         pm.pnmix_append(cfg, k_dev[:, :, t].contiguous(), v_dev[:, :, t].contiguous(), cache)
     del k_dev, v_dev
-    q_dev = torch.from_numpy(qm).view(torch.bfloat16).to(dev)
-    out_m = torch.empty(B, T, HQ, D, dtype=torch.float32, device=dev)
-    out_1 = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
-    q1 = q_dev[:, T - 1].contiguous()
-    with ClockSampler(0) as clocks:
-        t_multi = timed_rotation([lambda: pm.pnmix_decode_attention_multi(cfg, q_dev, cache, out_m)],
-                                 args.steps, args.warmup)
-        t_single = timed_rotation([lambda: pm.pnmix_decode_attention(cfg, q1, cache, out_1)],
-                                  args.steps, args.warmup)
-    assert cache.read_error() == 0
+    q_all = torch.from_numpy(qm).view(torch.bfloat16).to(dev)
     G = HQ // HKV
     rec = cache.c.record_bytes
-    alg_m = decode_bytes(CONTEXT, B * HKV, G * T, rec)
-    alg_1 = decode_bytes(CONTEXT, B * HKV, G, rec)
     peak, peak_kind = measured_peaks()
+    points = []
+    with ClockSampler(0) as clocks:
+        for T in Ts:
+            q_dev = q_all[:, Tmax - T:].contiguous()   # the last T queries: the newest T tokens
+            out = torch.empty(B, T, HQ, D, dtype=torch.float32, device=dev)
+            if T == 1:
+                q1 = q_dev[:, 0].contiguous()
+                o1 = out[:, 0]
+                fn = lambda: pm.pnmix_decode_attention(cfg, q1, cache, o1)   # noqa: E731
+            else:
+                fn = lambda q_=q_dev, o_=out: pm.pnmix_decode_attention_multi(cfg, q_, cache, o_)   # noqa: E731
+            t = timed_rotation([fn], args.steps, args.warmup)
+            alg = decode_bytes(CONTEXT, B * HKV, G * T, rec)
+            flops = 2 * 2 * B * HQ * T * CONTEXT * D     # q.k and p.v per row and token
+            points.append({"queries_per_sequence": T, "rows_per_kv_head": G * T, "decode_us": t * 1e6,
+                           "tokens_per_s": B * T / t, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
+                           "tensor_tflops": flops / t / 1e12})
+    assert cache.read_error() == 0
     line = {"workload": "verify_32k", "metric": "multi-token decode attention at 32K", "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic", "dtype": "f32",
             "config": {"batch": B, "n_q_heads": HQ, "n_kv_heads": HKV, "context": CONTEXT,
-                       "queries_per_sequence": T, "key_code_bits": 2.25,
-                       "l2": "inputs larger than L2 (419 MB cache per launch)"},
-            "multi": {"decode_us": t_multi * 1e6, "tokens_per_s": B * T / t_multi,
-                      "decode_gbs": alg_m / t_multi / 1e9, "frac": alg_m / t_multi / 1e9 / peak},
-            "single": {"decode_us": t_single * 1e6, "tokens_per_s": B / t_single,
-                       "decode_gbs": alg_1 / t_single / 1e9, "frac": alg_1 / t_single / 1e9 / peak},
-            "peak": peak, "peak_source": peak_kind, "clocks": clocks.summary()}
+                       "key_code_bits": 2.25, "l2": "inputs larger than L2 (419 MB cache per launch)"},
+            "points": points, "peak": peak, "peak_source": peak_kind, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     return 0
 

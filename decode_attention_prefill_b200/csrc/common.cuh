@@ -13,6 +13,7 @@ namespace pnmix {
 constexpr int kHeadDim = 128;
 constexpr int kGroup = 32;      // tokens per key group / value records
 constexpr int kMaxG = 8;        // query heads per KV head
+constexpr int kMaxRows = 64;    // query rows per KV head in one decode launch (G x queries)
 
 // Geometry derived from a validated pnmix_config (host computes, kernels read by value).
 struct Geometry {

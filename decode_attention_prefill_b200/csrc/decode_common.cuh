@@ -156,6 +156,7 @@ __device__ __forceinline__ int visible_tokens(const Geometry& g, int len, int v)
 // ws.prior_out / prior_lse the row is merged with an attention over other tokens:
 //   out = (2^(L0 - M) o0 + 2^(L - M) o) / (2^(L0 - M) + 2^(L - M)),  M = max(L0, L),
 // and the log-sum-exp written is that of the union, M + log2(2^(L0 - M) + 2^(L - M)).
+template <int MAXR = kMaxG>   // the most rows a launch has (G <= MAXR)
 __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G, float* out,
                                                 const Geometry& geo) {
   __shared__ int is_last;
@@ -170,9 +171,9 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
     // round), the largest reference m* and the denominator follow by shuffles and the
     // weights 2^(m_s - m*) of the first chunk go to shared memory; (2) per chunk of up to 32
     // segments, every thread sums its (head, channel) pairs with four loads in flight
-    __shared__ float wsh[kMaxG][kMaxCombineSegs];
-    __shared__ float mstar_sh[kMaxG], den_sh[kMaxG];
-    __shared__ float mix_sh[kMaxG][2];   // weights of the prior row and of this one
+    __shared__ float wsh[MAXR][kMaxCombineSegs];
+    __shared__ float mstar_sh[MAXR], den_sh[MAXR];
+    __shared__ float mix_sh[MAXR][2];   // weights of the prior row and of this one
     constexpr int kLaneSegs = 4;         // segments per lane held in registers (128 per head)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;
@@ -288,5 +289,7 @@ cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_
                               float* out, DecodeWs ws, cudaStream_t s);
 cudaError_t launch_decode_ws(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                              float* out, DecodeWs ws, cudaStream_t s);
+cudaError_t launch_decode_rows(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
+                               float* out, DecodeWs ws, cudaStream_t s);
 
 }  // namespace pnmix

@@ -138,6 +138,7 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   w.prior_lse = merge.prior_lse;
   w.k_new = merge.k_new;
   w.v_new = merge.v_new;
+  if (g.rows > kMaxG) return launch_decode_rows(g, q, c, nmax, out, w, s);   // 9 .. 64 query rows
   switch (g.kernel) {
     case PNMIX_DECODE_SIMT: return launch_decode_simt(g, q, c, nmax, out, w, s);
     case PNMIX_DECODE_MMA: return launch_decode_mma(g, q, c, nmax, out, w, s);
@@ -375,7 +376,7 @@ pnmix_status pnmix_debug_decode_stall(const pnmix_config* cfg, const uint16_t* q
 size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch, int max_context, int n_queries) {
   Geometry g;
   if (batch <= 0 || n_queries < 1 || make_geometry(cfg, batch, 32, &g) != PNMIX_OK) return 0;
-  if (g.G * n_queries > kMaxG) return 0;
+  if (g.G * n_queries > kMaxRows) return 0;
   g.tq = n_queries;
   g.rows = g.G * n_queries;
   return decode_workspace_bytes(g, max_context);
@@ -390,7 +391,7 @@ pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_
   if (st != PNMIX_OK) return st;
   if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
   if (!q || !out || !workspace || max_context < 0 || n_queries < 1) return PNMIX_ERR_INVALID_ARG;
-  if (g.G * n_queries > kMaxG) return PNMIX_ERR_UNSUPPORTED;
+  if (g.G * n_queries > kMaxRows) return PNMIX_ERR_UNSUPPORTED;
   if (g.kernel == PNMIX_DECODE_SIMT && n_queries > 1) return PNMIX_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
   g.tq = n_queries;

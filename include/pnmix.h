@@ -359,8 +359,11 @@ PNMIX_API size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch,
  * Query j (0-based) of sequence b attends causally over the first len[b] - T + 1 + j
  * cached tokens: the cache before the step plus the new tokens up to its own.  The
  * pages have no such call; it is the multi-token neighbour of pnmix_decode_attention
- * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 8 (PNMIX_ERR_UNSUPPORTED
- * otherwise).  A query that sees no token gets zeros.  Workspace from
+ * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 64 (PNMIX_ERR_UNSUPPORTED
+ * otherwise; PNMIX_DECODE_SIMT takes T = 1 only).  Up to 8 query rows per KV head (G * T)
+ * run on the single-query kernels; 9 to 64 rows on a kernel whose warps each hold 8 rows
+ * and share one staging of the packed records, so the cache is read once for all T
+ * queries.  A query that sees no token gets zeros.  Workspace from
  * pnmix_workspace_bytes_multi with the same T.
  */
 PNMIX_API pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_t* q,

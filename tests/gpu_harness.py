@@ -21,7 +21,7 @@ class Case:
     """One workload instance: inputs on host and device, a GPU cache and an oracle cache."""
 
     def __init__(self, B, Hq, Hkv, L, k=8, bhi=4, blo=2, capacity=None, seed=0, W=64,
-                 max_context=None, extra_tokens=0, score=0, n_prune=0, kernel=None):
+                 max_context=None, extra_tokens=0, score=0, n_prune=0, kernel=None, max_queries=None):
         import decode_attention_prefill_b200 as pm
         self.pm = pm
         self.B, self.Hq, self.Hkv, self.G, self.L = B, Hq, Hkv, Hq // Hkv, L
@@ -36,7 +36,7 @@ class Case:
         self.qwin = workload.rows(seed, workload.Q, B, Hq, L - self.W, max(self.W, 1), group=self.G) \
             if L > 0 else None
         self.cache = pm.PNMixCache(self.cfg, B, self.capacity, max_context=max_context,
-                                   max_queries=max(1, 8 // self.G))
+                                   max_queries=max_queries or max(1, 8 // self.G))
         self.ocache = oracle.Cache(B, Hkv, self.capacity, k, bhi, blo, score=score, n_prune=n_prune)
         self.k_dev = to_dev(self.kin)
         self.v_dev = to_dev(self.vin)

@@ -124,7 +124,9 @@ def test_multi_query_workspace_follows_the_rows():
     one = pm.workspace_bytes(cfg, 2, 256)
     assert pm.workspace_bytes_multi(cfg, 2, 256, 1) == one
     assert pm.workspace_bytes_multi(cfg, 2, 256, 2) > one
-    assert pm.workspace_bytes_multi(cfg, 2, 256, 3) == 0   # 12 rows per KV head: unsupported
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 3) > pm.workspace_bytes_multi(cfg, 2, 256, 2)   # 12 rows
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 16) > 0       # 64 rows per KV head: the most
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 17) == 0      # 68 rows: unsupported
     assert pm.workspace_bytes_multi(cfg, 2, 256, 0) == 0
 
 
@@ -136,7 +138,12 @@ def test_multi_query_entry_rejects_bad_arguments_before_launching():
     P = ctypes.c_void_p(1 << 41)
     L = pm._lib
     ws = pm.workspace_bytes_multi(cfg, 2, 256, 2)
+    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 17, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_UNSUPPORTED      # 68 rows per KV head
     assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 3, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_CAPACITY         # a 12-row workspace is larger
+    simt = pm.Config.make(8, 2, decode_kernel=pm.DECODE_SIMT)
+    assert L.pnmix_decode_attention_multi(ctypes.byref(simt), P, 2, ctypes.byref(c), 256, P, P, ws,
                                           None) == pm.ERR_UNSUPPORTED
     assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 0, ctypes.byref(c), 256, P, P, ws,
                                           None) == pm.ERR_INVALID_ARG

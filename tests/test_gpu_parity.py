@@ -597,3 +597,24 @@ def test_fused_append_decode_on_a_full_cache_raises_the_error_bit():
     assert int(c.cache.lengths()[0]) == 64
     assert torch.equal(before, c.cache.records())
     assert_close(out.cpu().numpy(), c.ocache.attend(q))     # attends over the 64 cached tokens
+
+
+# Many query rows per KV head (9 to 64 = G x T): warps holding 8 rows each share one staging
+# of the records; every row must match the oracle's causal attention.
+@pytest.mark.parametrize("B,Hq,Hkv,L,T,n_prune", [
+    (2, 8, 2, 300, 4, 0),       # 16 rows
+    (1, 32, 8, 1000, 16, 0),    # 64 rows: the most
+    (2, 28, 4, 517, 9, 0),      # 63 rows, G = 7
+    (1, 4, 1, 40, 12, 0),       # 48 rows; the step crosses a flush, new tokens in the residual
+    (2, 8, 1, 64, 3, 0),        # 24 rows, G = 8, the step starts a new group
+    (2, 8, 2, 300, 6, 26),      # 24 rows with query-channel pruning
+    (1, 16, 4, 2500, 5, 0),     # 20 rows, several split-K segments per unit
+])
+def test_many_query_rows_per_kv_head_like_the_oracle(B, Hq, Hkv, L, T, n_prune):
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + 5 * T, n_prune=n_prune, max_queries=T)
+    c.prefill()
+    for t in range(L, L + T):
+        c.append(t)
+    got, want = c.attend_multi(c.query_multi(L, T))
+    assert_close(got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128))
+    assert c.cache.read_error() == 0
