@@ -63,6 +63,8 @@ def lib():
                 "orc_ers": (ctypes.c_uint32, [ctypes.c_uint32, i]),
                 "orc_shrink_record": (i, [i, i, i, vp, vp]),
                 "orc_prune_queries": (None, [i, vp, i, vp]),
+                "orc_pruned_slices": (ctypes.c_uint32, [i, vp, vp, i, i]),
+                "orc_prune_query_slices": (None, [i, vp, vp, i, i, vp]),
                 "orc_topk": (None, [vp, i, vp, vp]),
                 "orc_position_order": (i, [ctypes.c_uint64, vp]),
                 "orc_minmax_quant": (None, [vp, i, i, vp, vp, vp]),
@@ -141,6 +143,26 @@ def prune_queries(q: np.ndarray, n_prune: int) -> np.ndarray:
         out[...] = q
         return out
     lib().orc_prune_queries(q.size // 128, _p(q), n_prune, _p(out))
+    return out
+
+
+def pruned_slices(q_rows: np.ndarray, perm: np.ndarray, k: int, n_prune: int) -> int:
+    """Mask of the position slices one unit's query rows (bf16 [rows][128]) prune, see
+    orc_pruned_slices."""
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.uint16).reshape(-1, 128)
+    perm = np.ascontiguousarray(perm, dtype=np.uint8)
+    return int(lib().orc_pruned_slices(q_rows.shape[0], _p(q_rows), _p(perm), k, n_prune))
+
+
+def prune_query_slices(q_rows: np.ndarray, perm: np.ndarray, k: int, n_prune: int) -> np.ndarray:
+    """bf16 [rows][128] query rows of one unit with the channels of its pruned slices zeroed."""
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.uint16)
+    out = np.empty_like(q_rows)
+    if n_prune <= 0:
+        out[...] = q_rows
+        return out
+    perm = np.ascontiguousarray(perm, dtype=np.uint8)
+    lib().orc_prune_query_slices(q_rows.size // 128, _p(q_rows), _p(perm), k, n_prune, _p(out))
     return out
 
 
@@ -255,11 +277,13 @@ def unpack_record(k, bhi, blo, rec):
 class Cache:
     """Host image of the cache regions the tests compare with the device."""
 
-    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2, score=SCORE_PNMIX, n_prune=0):
+    def __init__(self, batch, n_kv, capacity, k, bhi, blo, bv=2, score=SCORE_PNMIX, n_prune=0,
+                 n_prune_slices=0):
         self.batch, self.n_kv, self.capacity = batch, n_kv, capacity
         self.k, self.bhi, self.blo, self.bv = k, bhi, blo, bv
         self.score = score
         self.n_prune = n_prune   # query pairs each decode row drops (0: none)
+        self.n_prune_slices = n_prune_slices   # low-precision key slices each unit drops
         self.R = record_bytes(k, bhi, blo)
         if not self.R:
             raise ValueError("unsupported bit point")
@@ -311,7 +335,7 @@ class Cache:
 
     def attend_unit(self, q: np.ndarray, b: int, h: int, scale: float | None = None) -> np.ndarray:
         """q bf16 [G][128] of KV head h of sequence b -> fp64 [G][128]."""
-        q = prune_queries(q, self.n_prune)
+        q = prune_query_slices(prune_queries(q, self.n_prune), self.perm[b, h], self.k, self.n_prune_slices)
         G = q.shape[0]
         n = int(self.len[b])
         out = np.zeros((G, 128), np.float64)
@@ -326,7 +350,7 @@ class Cache:
         """The cache with its salient key positions shrunk from b_hi to b_lo = b_hi / 2 bits
         (orc_shrink_record on every full group): a k = 0 cache in the same position order."""
         out = Cache(self.batch, self.n_kv, self.capacity, 0, self.bhi, self.blo, self.bv,
-                    self.score, self.n_prune)
+                    self.score, self.n_prune, self.n_prune_slices)
         out.perm[:] = self.perm
         out.scores[:] = self.scores
         out.len[:] = self.len
@@ -343,7 +367,7 @@ class Cache:
     def attend_rows(self, q: np.ndarray, n_visible, b: int, h: int, scale: float | None = None) -> np.ndarray:
         """q bf16 [rows][128] of KV head h of sequence b, row r over the first n_visible[r]
         cached tokens -> fp64 [rows][128]."""
-        q = prune_queries(q, self.n_prune)
+        q = prune_query_slices(prune_queries(q, self.n_prune), self.perm[b, h], self.k, self.n_prune_slices)
         nv = np.ascontiguousarray(n_visible, dtype=np.int32)
         n = int(self.len[b])
         out = np.zeros((q.shape[0], 128), np.float64)

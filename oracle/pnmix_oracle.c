@@ -38,7 +38,9 @@
  * the 16-bit pass-through reducing to plain softmax attention; for the two-
  * precision mixing: exact means of identical rows, exact integer group scores,
  * the route against a stable sort, and the union of two equal-precision parts
- * against one cache.
+ * against one cache; for query-channel pruning: the pruned pairs and the pruned
+ * key slices against sorts of exact integer norms and energies, the channel-0 rule,
+ * and pruned key channels that can hold anything without changing the output.
  */
 #include <math.h>
 #include <stdint.h>
@@ -737,6 +739,67 @@ void orc_prune_queries(int rows, const uint16_t* q, int n_prune, uint16_t* out) 
     for (int c = 0; c < 128; ++c)
       out[(size_t)r * 128 + c] = ((mask >> (c & 63)) & 1ull) ? 0 : q[(size_t)r * 128 + c];
   }
+}
+
+/*
+ * Key-slice pruning (the Dual-QK abstract's query-channel pruning, taken at the
+ * granularity the packed record reads keys in, so that a pruned block of channels is a
+ * block of key codes left unread).  The unit is one (sequence, KV head) and all `rows`
+ * query rows that attend it (bf16 [rows][128]): they read the same key codes, so they
+ * share one decision.  Candidates are the position slices of the low-precision block
+ * (sigma in [2k/16, 8), positions 16*sigma .. 16*sigma+15 of the order perm) that hold
+ * neither channel 0 nor channel 64 (the abstract's channel-0 protection, kept for the
+ * RoPE pair 0).  The energy of a slice is
+ *     E_sigma = sum over rows v (ascending) of e_{sigma,v},
+ *     e_{sigma,v} = sum over its 16 positions j (ascending) of q_v[perm[j]]^2,
+ * every square and every partial sum rounded to fp32.  The n_prune candidates of least
+ * energy are pruned (all candidates when there are fewer), the higher slice first among
+ * equal energies.  Returns the mask of pruned slices (bit sigma).
+ */
+uint32_t orc_pruned_slices(int rows, const uint16_t* q, const uint8_t* perm, int k, int n_prune) {
+  const int nhs = 2 * k / 16;
+  float E[8];
+  int cand[8];
+  for (int sigma = 0; sigma < 8; ++sigma) {
+    E[sigma] = 0.0f;
+    cand[sigma] = sigma >= nhs;
+    for (int j = 16 * sigma; j < 16 * sigma + 16; ++j)
+      if ((perm[j] & 63) == 0) cand[sigma] = 0;
+    if (!cand[sigma]) continue;
+    for (int v = 0; v < rows; ++v) {
+      float e = 0.0f;
+      for (int j = 16 * sigma; j < 16 * sigma + 16; ++j) {
+        const float x = orc_f32_from_bf16(q[(size_t)v * 128 + perm[j]]);
+        const float sq = x * x;
+        e = e + sq;
+      }
+      E[sigma] = E[sigma] + e;
+    }
+  }
+  uint32_t mask = 0;
+  for (int i = 0; i < n_prune; ++i) {
+    int best = -1;
+    for (int sigma = 7; sigma >= 0; --sigma) {   /* high to low: ties keep the higher slice */
+      if (!cand[sigma] || ((mask >> sigma) & 1u)) continue;
+      if (best < 0 || E[sigma] < E[best]) best = sigma;
+    }
+    if (best < 0) break;
+    mask |= 1u << best;
+  }
+  return mask;
+}
+
+/* Copy of the unit's query rows with the channels of its pruned slices
+ * (orc_pruned_slices) set to zero in every row. */
+void orc_prune_query_slices(int rows, const uint16_t* q, const uint8_t* perm, int k, int n_prune,
+                            uint16_t* out) {
+  const uint32_t mask = orc_pruned_slices(rows, q, perm, k, n_prune);
+  int pruned[128] = {0};
+  for (int j = 0; j < 128; ++j)
+    if ((mask >> (j / 16)) & 1u) pruned[perm[j]] = 1;
+  for (int v = 0; v < rows; ++v)
+    for (int c = 0; c < 128; ++c)
+      out[(size_t)v * 128 + c] = pruned[c] ? 0 : q[(size_t)v * 128 + c];
 }
 
 /* Plain softmax attention over unquantized bf16 K and V ([n][128]). */

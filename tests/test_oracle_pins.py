@@ -736,6 +736,100 @@ def test_pruned_key_channels_do_not_change_the_pruned_attention():
     assert np.abs(outs["orig", 0] - outs["changed", 0]).max() > 1e-3
 
 
+def _salient_mask(rng, k, with_pair0=None):
+    pairs = list(rng.choice(64, k, replace=False)) if k else []
+    if with_pair0 is True and 0 not in pairs:
+        pairs[0] = 0
+    if with_pair0 is False and 0 in pairs:
+        pairs[pairs.index(0)] = next(p for p in range(1, 64) if p not in pairs)
+    return sum(1 << int(p) for p in pairs)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_pruned_slices_match_a_sort_of_exact_integer_energies(seed):
+    """Key-slice pruning on integer queries (every energy an exact integer, many ties):
+    the pruned set is the first n candidates - low-precision slices of the unit's position
+    order holding neither channel 0 nor 64 - sorted by (sum of q^2 over every row and the
+    slice's channels, higher slice first)."""
+    rng = np.random.default_rng(300 + seed)
+    k = [0, 8, 16, 32, 8, 0][seed]
+    rows = [1, 4, 8, 3, 2, 5][seed]
+    perm, nhi = oracle.position_order(_salient_mask(rng, k, with_pair0=(seed % 2 == 0) and k > 0))
+    assert nhi == 2 * k
+    q = rng.integers(-3, 4, (rows, 128)).astype(np.float32)
+    qb = bf16_bits(q)
+    qi = q.astype(np.int64)
+    energy = {s: int(sum(qi[v, perm[j]] ** 2 for v in range(rows) for j in range(16 * s, 16 * s + 16)))
+              for s in range(8)}
+    cands = [s for s in range(2 * k // 16, 8)
+             if all(int(perm[j]) % 64 != 0 for j in range(16 * s, 16 * s + 16))]
+    order = sorted(cands, key=lambda s: (energy[s], -s))
+    for n in range(0, 9):
+        want = sum(1 << s for s in order[:n])
+        assert oracle.pruned_slices(qb, perm, k, n) == want, (n, order, energy)
+
+
+def test_pruned_slices_keep_the_channel_0_and_64_slices():
+    """The slices holding channels 0 and 64 are never pruned, even with the least energy;
+    once pair 0 is salient (high-precision block), every low-precision slice is a candidate."""
+    rng = np.random.default_rng(7)
+    q = np.full((2, 128), 3.0, np.float32)
+    for k, with0 in ((8, False), (0, False), (8, True)):
+        perm, _ = oracle.position_order(_salient_mask(rng, k, with_pair0=with0))
+        qq = q.copy()
+        slice_of = {int(perm[j]): j // 16 for j in range(128)}
+        for c in (0, 64):   # empty the slices of channels 0 and 64
+            s = slice_of[c]
+            qq[:, perm[16 * s:16 * s + 16]] = 0.0
+        mask = oracle.pruned_slices(bf16_bits(qq), perm, k, 8)
+        lo = set(range(2 * k // 16, 8))
+        if with0:
+            assert mask == sum(1 << s for s in lo)
+        else:
+            assert mask == sum(1 << s for s in lo - {slice_of[0], slice_of[64]})
+
+
+def test_pruned_slices_are_decided_by_all_rows_of_the_unit():
+    """One row alone prunes its own quietest slice; with a second row whose energy sits
+    there, the shared decision moves to the slice both rows leave quiet."""
+    perm, _ = oracle.position_order(0)   # k = 0: slices 0 (channel 0) and 4 (channel 64) kept
+    a = np.full(128, 2.0, np.float32)
+    a[perm[16 * 2:16 * 3]] = 0.0         # row a: slice 2 silent, slice 5 weak
+    a[perm[16 * 5:16 * 6]] = 1.0
+    b = np.full(128, 1.0, np.float32)
+    b[perm[16 * 2:16 * 3]] = 4.0         # row b: loud in slice 2
+    assert oracle.pruned_slices(bf16_bits(a[None]), perm, 0, 1) == 1 << 2
+    assert oracle.pruned_slices(bf16_bits(np.stack([a, b])), perm, 0, 1) == 1 << 5
+
+
+def test_pruned_slice_channels_do_not_change_the_pruned_attention():
+    """The pruned slices' key channels can hold anything: with slice pruning the output is
+    the same to the last bit, without pruning it changes."""
+    rng = np.random.default_rng(11)
+    n = 3 * 32 + 7
+    kf = rng.integers(-6, 7, (n, 128)).astype(np.float32) / 2
+    vf = _grid_rows(rng, n)
+    qf = rng.integers(-4, 5, (4, 128)).astype(np.float32)
+    qb = bf16_bits(qf)
+    perm, _ = oracle.position_order(0xFF)
+    mask = oracle.pruned_slices(qb, perm, 8, 3)
+    assert bin(mask).count("1") == 3
+    kf2 = kf.copy()
+    for j in range(128):
+        if (mask >> (j // 16)) & 1:   # token-dependent changes (a constant would cancel in softmax)
+            kf2[:, perm[j]] += rng.integers(-4, 5, n) * 1.5
+    outs = {}
+    for name, kk in (("orig", kf), ("changed", kf2)):
+        for prune in (0, 3):
+            c = oracle.Cache(1, 1, 128, 8, 4, 2, n_prune_slices=prune)
+            c.perm[0, 0] = perm
+            c.mask[0, 0] = 0xFF
+            c.prefill(bf16_bits(kk)[None, None], bf16_bits(vf)[None, None], n)
+            outs[name, prune] = c.attend_unit(qb, 0, 0)
+    np.testing.assert_array_equal(outs["orig", 3], outs["changed", 3])
+    assert np.abs(outs["orig", 0] - outs["changed", 0]).max() > 1e-3
+
+
 @pytest.mark.parametrize("b", [1, 2, 4, 8])
 def test_equivalent_right_shift_is_round_of_the_division_exhaustively(b):
     """The shift formula equals round(X / (2^b + 1)) for every 2b-bit X (no value sits
