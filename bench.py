@@ -41,12 +41,14 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one decode launch from the committed ncu capture (profiles/
 # decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
 # of the decode sources it was taken on.  Reported only while the sources still match.
-DECODE_CAPTURE = {"sources_sha256_16": "f44445064588b350", "traffic_bytes": 424529664,
+DECODE_CAPTURE = {"sources_sha256_16": "3a122affbc792698", "traffic_bytes": 425706752,
                   "algorithmic_bytes": 420855808}
 DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
                   "decode_attention_prefill_b200/csrc/decode_common.cuh",
                   "decode_attention_prefill_b200/csrc/common.cuh",
-                  "decode_attention_prefill_b200/csrc/decode_frag.cuh"]
+                  "decode_attention_prefill_b200/csrc/decode_frag.cuh",
+                  "decode_attention_prefill_b200/csrc/decode_group.cuh",
+                  "decode_attention_prefill_b200/csrc/quantize_group.cuh"]
 
 
 def parse():

@@ -1,8 +1,8 @@
 // decode_simt.cu -- plain CUDA-core decode attention over the packed cache.
 //
 // The straightforward formulation, kept as the readable baseline of the tensor-core
-// kernel in decode_mma.cu (selected with PNMIX_DECODE_KERNEL=simt): lane = token for
-// q.k^, lane = channel for p.v^, fp32 online softmax per warp.  Same work partition and
+// kernel in decode_mma.cu (selected with decode_kernel = PNMIX_DECODE_SIMT in the
+// config): lane = token for q.k^, lane = channel for p.v^, fp32 online softmax per warp.  Same work partition and
 // fused combine as the tensor-core kernel (decode_common.cuh).
 #include "common.cuh"
 #include "decode_common.cuh"

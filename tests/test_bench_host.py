@@ -9,8 +9,11 @@ def test_decode_bytes_of_the_profiled_launch_equal_the_recorded_algorithmic_byte
     # 128 units (16 x 8) at 32758 tokens: 1023 records of 3200 B and 22 residual rows each,
     # plus 4 query rows (bf16) and 4 output rows (fp32) per unit
     assert bench.decode_bytes(32758, 128, 4, 3200) == 128 * (1023 * 3200 + 22 * 512 + 4 * 256 + 4 * 512)
-    assert bench.decode_bytes(32758, 128, 4, 3200) == bench.DECODE_CAPTURE["algorithmic_bytes"]
     assert bench.decode_bytes(0, 3, 7, 3200) == 3 * (7 * 256 + 7 * 512)
+    # the captured launch: the third append + decode step of --profile-decode --steps 3
+    # --warmup 2, from 32768 - 15 cached tokens to 32756, plus each unit's new K and V row
+    ctx = 32768 - 3 * (3 + 2) + 3
+    assert bench.decode_bytes(ctx, 128, 4, 3200) + 128 * 2 * 2 * 128 * 2 == bench.DECODE_CAPTURE["algorithmic_bytes"]
 
 
 def test_captured_traffic_scales_with_the_launch_or_is_withheld(monkeypatch):
