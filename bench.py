@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one decode launch from the committed ncu capture (profiles/
 # decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
 # of the decode sources it was taken on.  Reported only while the sources still match.
-DECODE_CAPTURE = {"sources_sha256_16": "3a122affbc792698", "traffic_bytes": 425706752,
+DECODE_CAPTURE = {"sources_sha256_16": "4e1d5f381b88ffcd", "traffic_bytes": 425009152,
                   "algorithmic_bytes": 420855808}
 DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
                   "decode_attention_prefill_b200/csrc/decode_common.cuh",
@@ -451,18 +451,23 @@ def run_decode_workload(args):
     wl = workload.WORKLOADS[args.workload]
     Bw, Hq, Hkv, ctx = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.context
     G = Hq // Hkv
-    # (bit point, saliency statistic, pruned query pairs, shrunk): the sweep adds the
-    # key-only (1) and key-range x query (2) statistics at two bit points, 40 % dynamic
-    # query-channel pruning (26 of 64 pairs) at 2.25 bits, and two caches whose salient
-    # keys were shrunk to the low bit width after quantization (pnmix_shrink_keys)
-    points = [(bp, 0, 0, False) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
+    # (bit point, saliency statistic, pruned query pairs, shrunk, pruned key slices): the
+    # sweep adds the key-only (1) and key-range x query (2) statistics at two bit points,
+    # 40 % dynamic query-channel pruning (26 of 64 pairs) at 2.25 bits, key-slice pruning
+    # (3 of the 7 low-precision slices, 48 of 128 channels), and two caches whose salient
+    # keys were shrunk to the low bit width after quantization (pnmix_shrink_keys); the
+    # llama3_8b shape adds key-slice pruning of 2, 3 and 4 slices (the cost of the decision)
+    p42 = workload.BitPoint(4, 2, 8)
+    points = [(bp, 0, 0, False, 0) for bp in (wl.sweep if wl.sweep else (wl.bits,))]
     if wl.sweep:
-        points += [(workload.BitPoint(4, 2, 8), 1, 0, False), (workload.BitPoint(4, 2, 8), 2, 0, False),
-                   (workload.BitPoint(2, 1, 16), 1, 0, False), (workload.BitPoint(2, 1, 16), 2, 0, False),
-                   (workload.BitPoint(4, 2, 8), 0, 26, False),
-                   (workload.BitPoint(4, 2, 8), 0, 0, True), (workload.BitPoint(2, 1, 16), 0, 0, True)]
+        points += [(p42, 1, 0, False, 0), (p42, 2, 0, False, 0),
+                   (workload.BitPoint(2, 1, 16), 1, 0, False, 0), (workload.BitPoint(2, 1, 16), 2, 0, False, 0),
+                   (p42, 0, 26, False, 0), (p42, 0, 0, False, 3),
+                   (p42, 0, 0, True, 0), (workload.BitPoint(2, 1, 16), 0, 0, True, 0)]
         if args.shrunk_only:
             points = [p_ for p_ in points if p_[3]]
+    elif wl.bits.key_bits_lo == 2:
+        points += [(wl.bits, 0, 0, False, n) for n in (2, 3, 4)]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     kin = workload.rows(args.seed, workload.K, Bw, Hkv, 0, ctx)
@@ -481,9 +486,9 @@ def run_decode_workload(args):
                  for b in range(Bw) for h in range(Hkv)}
     results = []
     with ClockSampler(0) as clocks:
-        for bp, score, prune, shrink in points:
+        for bp, score, prune, shrink, slices in points:
             qcfg = pm.Config.make(Hq, Hkv, bp.key_bits_hi, bp.key_bits_lo, bp.n_salient_pairs, WINDOW,
-                                  saliency_score=score, n_pruned_pairs=prune)
+                                  saliency_score=score, n_pruned_pairs=prune, n_pruned_slices=slices)
             cfg = qcfg.without_salient() if shrink else qcfg
             src = pm.PNMixCache(qcfg, Bw, ctx + 32, max_context=ctx)
             src.prefill(qwin_dev, k_dev, v_dev, ctx)
@@ -519,11 +524,11 @@ def run_decode_workload(args):
             t = timed_rotation(fns, max(args.steps, 3 * n_rep), args.warmup)
             pm.pnmix_decode_attention(cfg, q_dev, cache, out)
             assert all(c_.read_error() == 0 for c_ in replicas)
-            alg = decode_bytes(ctx, Bw * Hkv, G, cache.c.record_bytes)
+            alg = decode_bytes(ctx, Bw * Hkv, G, cache.c.record_bytes)   # records are read whole
             r = {"key_bits": [bp.key_bits_hi, bp.key_bits_lo], "salient_pairs": bp.n_salient_pairs,
                  "saliency_score": ["pair-norm product", "key only", "key range x query"][score],
-                 "pruned_query_pairs": prune, "shrunk_to_low_bits": shrink, "shrink_us": shrink_us,
-                 "shrink_gbs": shrink_gbs,
+                 "pruned_query_pairs": prune, "pruned_key_slices": slices, "shrunk_to_low_bits": shrink,
+                 "shrink_us": shrink_us, "shrink_gbs": shrink_gbs,
                  "key_code_bits": bp.key_bits_lo if shrink else bp.key_code_bits,
                  "bytes_per_token_head": cache.c.record_bytes / 32,
                  "decode_us": t * 1e6, "decode_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / peak,

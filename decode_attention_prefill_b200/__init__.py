@@ -54,14 +54,17 @@ class Config(ctypes.Structure):
         "head_dim", "n_q_heads", "n_kv_heads", "group_tokens", "residual_tokens", "key_bits_hi",
         "key_bits_lo", "n_salient_pairs", "value_bits", "value_group", "saliency_window")] + [
         ("softmax_scale", ctypes.c_float), ("saliency_score", ctypes.c_int32),
-        ("n_pruned_pairs", ctypes.c_int32), ("decode_kernel", ctypes.c_int32)]
+        ("n_pruned_pairs", ctypes.c_int32), ("decode_kernel", ctypes.c_int32),
+        ("n_pruned_slices", ctypes.c_int32)]
 
     @classmethod
     def make(cls, n_q_heads: int, n_kv_heads: int, key_bits_hi: int = 4, key_bits_lo: int = 2,
              n_salient_pairs: int = 8, saliency_window: int = 64, softmax_scale: float = 0.0,
-             saliency_score: int = 0, n_pruned_pairs: int = 0, decode_kernel: int = 0):
+             saliency_score: int = 0, n_pruned_pairs: int = 0, decode_kernel: int = 0,
+             n_pruned_slices: int = 0):
         return cls(128, n_q_heads, n_kv_heads, 32, 32, key_bits_hi, key_bits_lo, n_salient_pairs,
-                   2, 32, saliency_window, softmax_scale, saliency_score, n_pruned_pairs, decode_kernel)
+                   2, 32, saliency_window, softmax_scale, saliency_score, n_pruned_pairs, decode_kernel,
+                   n_pruned_slices)
 
     @property
     def group(self) -> int:

@@ -40,17 +40,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in sources():
-        obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            sys.stderr.write(res.stdout + res.stderr)
-            raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
-        if verbose:
-            sys.stderr.write(res.stderr)
-        objs.append(obj)
+    objs = [os.path.join(objdir, os.path.basename(src) + ".o") for src in sources()]
+    # one nvcc process per translation unit, all at once (each is single-threaded)
+    procs = [subprocess.Popen([nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj],
+                              stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+             for src, obj in zip(sources(), objs)]
+    failed = []
+    for src, p in zip(sources(), procs):
+        out, err = p.communicate()
+        if p.returncode != 0:
+            sys.stderr.write(out + err)
+            failed.append(os.path.basename(src))
+        elif verbose:
+            sys.stderr.write(err)
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, "-shared", "-cudart", "static", "-gencode", "arch=compute_100a,code=sm_100a",
            "-o", tmp, *objs]

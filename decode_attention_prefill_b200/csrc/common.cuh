@@ -30,6 +30,7 @@ struct Geometry {
   float scale;    // softmax scale
   int score;      // saliency statistic, PNMIX_SCORE_*
   int n_prune;    // decode: query pairs each query row drops (0: none)
+  int n_prune_slices;   // decode: low-precision key slices each unit drops (0: none)
   int tq;         // decode queries per sequence (1, or T of a multi-query step)
   int rows;       // query rows per (b, KV head) in decode: G * tq (row v = query v / G, head v % G)
   int kernel;     // decode kernel, PNMIX_DECODE_*

@@ -209,6 +209,65 @@ __device__ __forceinline__ void prune_query_rows(const Geometry& g, float* qnat,
   }
 }
 
+// Key-slice pruning of a unit's query rows (qnat fp32 [g.rows][128], natural channel order;
+// perm the unit's position order): the g.n_prune_slices slices of the low-precision block of
+// least energy sum_v sum_{j in slice} q_v[perm[j]]^2 (rows ascending, positions ascending,
+// each square and partial sum rounded to fp32), among those holding neither channel 0 nor
+// channel 64, the higher slice first among equal energies.  Every warp computes the decision
+// (the same one) with lane = 4 * slice + row-in-block; the caller zeroes the channels with
+// zero_pruned_slices after a barrier.  Returns the pruned-slice mask (bit sigma).
+__device__ __forceinline__ uint32_t pruned_slices(const Geometry& g, const float* qnat, const uint8_t* perm) {
+  const int lane = threadIdx.x & 31;
+  const int sl = lane >> 2, rl = lane & 3;
+  const int nls = 8 - g.nhs, sigma = g.nhs + sl;
+  const bool live = sl < nls;
+  int chan[16];
+  bool protect = false;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    chan[j] = live ? (perm[16 * sigma + j] & (kHeadDim - 1)) : 0;
+    protect |= (chan[j] & 63) == 0;
+  }
+  float E = 0.f;   // lanes rl == 0: the slice's energy, rows in order
+  for (int v0 = 0; v0 < g.rows; v0 += 4) {
+    const int v = v0 + rl;
+    float e = 0.f;
+    if (live && v < g.rows) {
+      const float* row = qnat + v * kHeadDim;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) e = __fadd_rn(e, __fmul_rn(row[chan[j]], row[chan[j]]));
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float er = __shfl_sync(0xffffffffu, e, (lane & ~3) | r);
+      if (v0 + r < g.rows) E = __fadd_rn(E, er);
+    }
+  }
+  const bool cand = live && !protect;
+  int before = 0;   // candidates pruned ahead of this slice: (energy, higher slice first)
+#pragma unroll
+  for (int o = 0; o < 8; ++o) {
+    const float Eo = __shfl_sync(0xffffffffu, E, 4 * o);
+    const bool co = __shfl_sync(0xffffffffu, cand, 4 * o);
+    before += (co && o != sl && (Eo < E || (Eo == E && o > sl))) ? 1 : 0;
+  }
+  const uint32_t ball = __ballot_sync(0xffffffffu, cand && before < g.n_prune_slices && rl == 0);
+  uint32_t mask = 0;
+#pragma unroll
+  for (int o = 0; o < 8; ++o)
+    if ((ball >> (4 * o)) & 1u) mask |= 1u << (g.nhs + o);
+  return mask;
+}
+
+// Zero the channels of the pruned slices (mask from pruned_slices) in every query row.
+__device__ __forceinline__ void zero_pruned_slices(const Geometry& g, float* qnat, const uint8_t* perm, uint32_t mask,
+                                                   int tid, int nthreads) {
+  for (int i = tid; i < g.rows * kHeadDim; i += nthreads) {
+    const int j = i & (kHeadDim - 1);
+    if ((mask >> (j >> 4)) & 1u) qnat[(i >> 7) * kHeadDim + (perm[j] & (kHeadDim - 1))] = 0.f;
+  }
+}
+
 // The residual item: up to 31 bf16 tokens staged in shared memory, with CUDA cores, heads
 // h0, h0 + hstep, ... one at a time (few registers).  Lane = token for the logit (its K
 // row, q in natural channel order), lane = channel for the values.  Writes one partial

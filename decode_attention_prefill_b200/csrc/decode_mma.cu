@@ -233,6 +233,12 @@ decode_mma_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, flo
       __syncthreads();
       prune_query_rows(g, qnat, warp, kWarps);
     }
+    if (g.n_prune_slices > 0) {   // key-slice pruning of the staged query rows
+      __syncthreads();
+      const uint32_t pmask = pruned_slices(g, qnat, perm);
+      __syncthreads();
+      zero_pruned_slices(g, qnat, perm, pmask, tid, kThreads);
+    }
     __syncthreads();
     {
       const int L = lane, chunk = warp;   // entries 4*chunk .. 4*chunk+3 (= sigma*2 + e)

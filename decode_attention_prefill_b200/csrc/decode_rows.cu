@@ -192,6 +192,12 @@ decode_rows_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, fl
       prune_query_rows(g, qnat, warp, nwarps);
       __syncthreads();
     }
+    if (g.n_prune_slices > 0) {   // key-slice pruning of the staged query rows
+      const uint32_t pmask = pruned_slices(g, qnat, perm);
+      __syncthreads();
+      zero_pruned_slices(g, qnat, perm, pmask, tid, blockDim.x);
+      __syncthreads();
+    }
     const bool seg_resid = seg.hi > seg.ng && seg.nr > 0;
     if (seg_resid) {   // the residual window on CUDA cores, rows spread over the warps
       residual_partial(g, c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim,

@@ -347,6 +347,12 @@ decode_ws_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       __syncthreads();
       prune_query_rows(g, qnat, warp, kWsWarps);
     }
+    if (g.n_prune_slices > 0) {   // key-slice pruning of the staged query rows
+      __syncthreads();
+      const uint32_t pmask = pruned_slices(g, qnat, perm);
+      __syncthreads();
+      zero_pruned_slices(g, qnat, perm, pmask, tid, kWsThreads);
+    }
     __syncthreads();
     if (is_qk) {   // QK warp w builds slice pair w of the sets
       const int tq = lane & 3, gq = lane >> 2, chunk = warp;

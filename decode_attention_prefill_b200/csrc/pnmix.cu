@@ -32,7 +32,10 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   if (cfg->n_pruned_pairs < 0 || cfg->n_pruned_pairs > 63) return PNMIX_ERR_UNSUPPORTED;
   if (cfg->decode_kernel < PNMIX_DECODE_AUTO || cfg->decode_kernel > PNMIX_DECODE_PAIRS)
     return PNMIX_ERR_UNSUPPORTED;
-  if (cfg->decode_kernel == PNMIX_DECODE_SIMT && cfg->n_pruned_pairs > 0) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->n_pruned_slices < 0 || cfg->n_pruned_slices > 8) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->n_pruned_pairs > 0 && cfg->n_pruned_slices > 0) return PNMIX_ERR_UNSUPPORTED;
+  if (cfg->decode_kernel == PNMIX_DECODE_SIMT && (cfg->n_pruned_pairs > 0 || cfg->n_pruned_slices > 0))
+    return PNMIX_ERR_UNSUPPORTED;
   g->B = batch;
   g->Hq = cfg->n_q_heads;
   g->Hkv = cfg->n_kv_heads;
@@ -52,6 +55,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   g->scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale : 1.0f / sqrtf(128.0f);
   g->score = cfg->saliency_score;
   g->n_prune = cfg->n_pruned_pairs;
+  g->n_prune_slices = cfg->n_pruned_slices;
   g->tq = 1;
   g->rows = G;
   g->kernel = cfg->decode_kernel;
@@ -338,6 +342,7 @@ pnmix_status pnmix_decode_attention_two(const pnmix_config* cfg_a, const pnmix_c
   if (st != PNMIX_OK) return st;
   if ((st = check_decode_args(cfg_b, q, cache_b, max_context_b, out, &gb)) != PNMIX_OK) return st;
   if (ga.B != gb.B || ga.Hq != gb.Hq || ga.Hkv != gb.Hkv) return PNMIX_ERR_INVALID_ARG;
+  if (ga.n_prune_slices > 0 || gb.n_prune_slices > 0) return PNMIX_ERR_UNSUPPORTED;
   if (!workspace) return PNMIX_ERR_INVALID_ARG;
   if (!aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
   const size_t wa = decode_workspace_bytes(ga, max_context_a), wb = decode_workspace_bytes(gb, max_context_b);

@@ -160,7 +160,7 @@ typedef enum {
  *   G = n_q_heads / n_kv_heads in [1, 8];
  *   saliency_window W in [1, 1024];
  *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*);
- *   n_pruned_pairs in [0, 63];
+ *   n_pruned_pairs in [0, 63]; n_pruned_slices in [0, 8]; not both non-zero;
  *   decode_kernel in {0, 1, 2, 3} (PNMIX_DECODE_*).
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
  *
@@ -171,6 +171,21 @@ typedef enum {
  * abstract's channel-0 protection), the higher pair index first among equal norms.  A
  * dropped pair contributes nothing to that row's logits (its query channels count as
  * zero).  The packed records are still read whole; what changes is the arithmetic.
+ *
+ * Key-slice pruning (n_pruned_slices > 0; the same abstract's query-channel pruning taken
+ * at the granularity the records store keys in): in every decode call, per (sequence, KV
+ * head) unit and for all query rows that attend it together,
+ * the n_pruned_slices position slices of the low-precision block (sigma in [2k/16, 8)) with
+ * the least energy  E_sigma = sum over rows v of sum over the slice's 16 positions j of
+ * q_v[perm[j]]^2  are dropped: rows in order, positions in order, every square and partial
+ * sum rounded to fp32; slices holding channel 0 or 64 are never dropped (channel-0
+ * protection); the higher slice goes first among equal energies; when fewer slices are
+ * candidates, all of them are dropped.  A dropped slice's channels count as zero in every
+ * row's query (packed and residual tokens alike).  The records are still read whole: at
+ * b_lo = 2 a dropped slice is one 128-byte row of each record, and leaving those rows
+ * unread (one copy per run of kept rows) or skipping their products (a branch per slice in
+ * the unrolled group loop) measured slower on B200 than reading and multiplying them.
+ * Not available in pnmix_decode_attention_two (its two parts order positions differently).
  */
 typedef struct {
   int32_t head_dim;
@@ -188,6 +203,7 @@ typedef struct {
   int32_t saliency_score;   /* statistic that ranks the pairs, PNMIX_SCORE_* (0 = PN-Mix) */
   int32_t n_pruned_pairs;   /* decode: query pairs each query row drops, 0..63 (0 = none) */
   int32_t decode_kernel;    /* decode: which kernel runs, PNMIX_DECODE_* (0 = automatic) */
+  int32_t n_pruned_slices;  /* decode: low-precision key slices each unit drops, 0..8 (0 = none) */
 } pnmix_config;
 
 /*
@@ -467,7 +483,8 @@ PNMIX_API pnmix_status pnmix_decode_attention_noalloc(const pnmix_config* cfg, c
  * [B][Hq][128].  max_context_a / _b bound the lengths of each part as in
  * pnmix_decode_attention.  Workspace: pnmix_workspace_bytes_two bytes, 256-byte aligned,
  * zero-filled before first use; it is left ready for the next call.  Errors as for
- * pnmix_decode_attention, and INVALID_ARG when the parts' batch or head counts differ.
+ * pnmix_decode_attention, INVALID_ARG when the parts' batch or head counts differ, and
+ * UNSUPPORTED when either configuration asks for key-slice pruning.
  */
 PNMIX_API size_t pnmix_workspace_bytes_two(const pnmix_config* cfg_a, const pnmix_config* cfg_b, int batch,
                                            int max_context_a, int max_context_b);

@@ -19,13 +19,13 @@
  *  - Saliency from the query-key pair-norm product, chosen once at prefill and
  *    reused through decode: "PN-Mix: Pair-Norm Guided Mixed-Precision Key Cache
  *    Quantization for Efficient Long-Output LLM Inference", abstract, and the
- *    same page's transcript ("pairs where the product of query and key pair
- *    norms is large").  The exact statistic (mean query pair-norm over the
+ *    same page's transcript (the pairs whose query and key pair norms have a
+ *    large product are the salient ones).  The exact statistic (mean query pair-norm over the
  *    last W prefill queries of the group, max key pair-norm over the prefill
  *    tokens), k, W and the half-split pairing are this library's fixed
  *    parameters.
  *  - Mixed-precision per-channel keys: PN-Mix abstract; MixKVQ abstract
- *    ("channel-level mixed-precision quantization policy").
+ *    (precision chosen per key channel).
  *  - Per-token values: "MixKVQ: Query-Aware Mixed-Precision KV Cache
  *    Quantization for Long-Context Reasoning", abstract.
  *  - Asymmetric min-max quantizer with a float zero point (KIVI-style, as

@@ -21,7 +21,8 @@ class Case:
     """One workload instance: inputs on host and device, a GPU cache and an oracle cache."""
 
     def __init__(self, B, Hq, Hkv, L, k=8, bhi=4, blo=2, capacity=None, seed=0, W=64,
-                 max_context=None, extra_tokens=0, score=0, n_prune=0, kernel=None, max_queries=None):
+                 max_context=None, extra_tokens=0, score=0, n_prune=0, kernel=None, max_queries=None,
+                 n_prune_slices=0):
         import decode_attention_prefill_b200 as pm
         self.pm = pm
         self.B, self.Hq, self.Hkv, self.G, self.L = B, Hq, Hkv, Hq // Hkv, L
@@ -30,14 +31,16 @@ class Case:
         total = L + extra_tokens
         self.capacity = capacity or ((total + 31) // 32 * 32 + 32)
         self.cfg = pm.Config.make(Hq, Hkv, bhi, blo, k, W, saliency_score=score, n_pruned_pairs=n_prune,
-                                  decode_kernel=pm.DECODE_KERNELS[kernel or "auto"])
+                                  decode_kernel=pm.DECODE_KERNELS[kernel or "auto"],
+                                  n_pruned_slices=n_prune_slices)
         self.kin = workload.rows(seed, workload.K, B, Hkv, 0, max(total, 1))
         self.vin = workload.rows(seed, workload.V, B, Hkv, 0, max(total, 1))
         self.qwin = workload.rows(seed, workload.Q, B, Hq, L - self.W, max(self.W, 1), group=self.G) \
             if L > 0 else None
         self.cache = pm.PNMixCache(self.cfg, B, self.capacity, max_context=max_context,
                                    max_queries=max_queries or max(1, 8 // self.G))
-        self.ocache = oracle.Cache(B, Hkv, self.capacity, k, bhi, blo, score=score, n_prune=n_prune)
+        self.ocache = oracle.Cache(B, Hkv, self.capacity, k, bhi, blo, score=score, n_prune=n_prune,
+                                   n_prune_slices=n_prune_slices)
         self.k_dev = to_dev(self.kin)
         self.v_dev = to_dev(self.vin)
 

@@ -56,6 +56,10 @@ def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
     (dict(decode_kernel=4), pm.ERR_UNSUPPORTED),
     (dict(decode_kernel=-1), pm.ERR_UNSUPPORTED),
     (dict(decode_kernel=pm.DECODE_SIMT, n_pruned_pairs=5), pm.ERR_UNSUPPORTED),   # simt has no pruning
+    (dict(n_pruned_slices=9), pm.ERR_UNSUPPORTED),
+    (dict(n_pruned_slices=-1), pm.ERR_UNSUPPORTED),
+    (dict(n_pruned_slices=3, n_pruned_pairs=5), pm.ERR_UNSUPPORTED),   # one pruning at a time
+    (dict(decode_kernel=pm.DECODE_SIMT, n_pruned_slices=2), pm.ERR_UNSUPPORTED),
 ])
 def test_config_validation(change, status):
     cfg = pm.Config.make(32, 8)
@@ -314,6 +318,8 @@ def test_two_part_decode_rejects_bad_arguments_before_launching():
     assert f(*args(lo, a, lo, b, P, n)) == pm.ERR_INVALID_ARG          # cache a laid out for another config
     other = pm.Config.make(16, 4)
     assert f(*args(hi, a, other, _fake_cache(other), P, n)) == pm.ERR_INVALID_ARG   # head counts differ
+    pruned = pm.Config.make(8, 2, n_salient_pairs=8, n_pruned_slices=2)
+    assert f(*args(hi, a, pruned, b, P, n)) == pm.ERR_UNSUPPORTED      # no key-slice pruning across parts
 
 
 @pytest.mark.skipif(torch.cuda.is_available(),

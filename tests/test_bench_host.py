@@ -45,3 +45,4 @@ def test_clock_summary_names_every_reason_seen_and_the_median_clock():
 def test_whole_job_value_counts_every_rank():
     ms = 2.0
     assert bench.whole_job_tokens_per_s(1, 10, ms) * 4 == bench.whole_job_tokens_per_s(4, 10, ms)
+

@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from gpu_harness import Case, assert_close, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -272,6 +273,81 @@ def test_query_channel_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, n_prune, T
         got, want = c.attend_multi(c.query_multi(L, T))
         got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
     assert_close(got, want)
+
+
+# Key-slice pruning (all query rows of a unit drop the low-precision key slices of least
+# energy): every kernel and shape must match the oracle's pruned attention.
+@pytest.mark.parametrize("kernel", [None, "mma", "ws"])
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo,n,T", [
+    (2, 8, 2, 1000, 8, 4, 2, 3, 1),     # G = 4: the one-role kernel
+    (1, 1, 1, 77, 8, 4, 2, 2, 1),       # one row
+    (2, 32, 8, 2100, 8, 4, 2, 8, 1),    # every candidate pruned
+    (2, 28, 4, 517, 0, 4, 2, 4, 1),     # k = 0, G = 7
+    (2, 16, 2, 1200, 16, 2, 1, 3, 1),   # 1-bit low block: two slices per code word
+    (2, 8, 2, 700, 0, 2, 1, 4, 1),
+    (1, 8, 1, 300, 64, 4, 2, 3, 1),     # k = 64: no low-precision slice, nothing pruned
+    (2, 8, 2, 300, 8, 4, 2, 3, 2),      # two queries per sequence: 8 rows share the decision
+    (2, 8, 2, 300, 8, 4, 2, 3, 4),      # 16 rows (the many-rows kernel)
+])
+def test_key_slice_pruning_like_the_oracle(kernel, B, Hq, Hkv, L, k, bhi, blo, n, T):
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, extra_tokens=T, seed=L + 11 * n + T, kernel=kernel,
+             n_prune_slices=n, max_queries=T)
+    c.prefill()
+    if T == 1:
+        got, want = c.attend(c.query(L))
+    else:
+        for t in range(L, L + T):
+            c.append(t)
+        got, want = c.attend_multi(c.query_multi(L, T))
+        got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
+    assert_close(got, want)
+    assert c.cache.read_error() == 0
+
+
+@pytest.mark.parametrize("kernel", [None, "ws"])
+def test_pruned_key_code_rows_are_not_used(kernel):
+    """Overwriting the key codes of every unit's pruned slices leaves the output bit for bit
+    unchanged: no kernel takes anything from them."""
+    B, Hq, Hkv, L = 2, 8, 2, 1500
+    c = Case(B, Hq, Hkv, L, seed=91, kernel=kernel, n_prune_slices=3)
+    c.prefill()
+    q = c.query(L)
+    before, want = c.attend(q)
+    assert_close(before, want)
+    rec = c.cache.records()
+    perm = c.cache.perm().cpu().numpy()
+    G, nhs = Hq // Hkv, 2 * c.k // 16
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    for b in range(B):
+        for h in range(Hkv):
+            mask = oracle.pruned_slices(q[b, h * G:(h + 1) * G], perm[b, h], c.k, 3)
+            assert bin(mask).count("1") == 3
+            for sigma in range(nhs, 8):
+                if (mask >> sigma) & 1:   # 2-bit low block: row 2 * nhs + (sigma - nhs) of 128 bytes
+                    row = 2 * nhs + (sigma - nhs)
+                    rec[b, h, :, 128 * row:128 * row + 128] = torch.randint(
+                        0, 256, (rec.shape[2], 128), dtype=torch.uint8, device="cuda", generator=gen)
+    after = c.cache.attend(to_dev(q)).cpu().numpy()
+    np.testing.assert_array_equal(after, before)
+
+
+@pytest.mark.parametrize("kernel", [None, "ws"])
+def test_fused_append_decode_with_key_slice_pruning(kernel):
+    import decode_attention_prefill_b200 as pm
+    B, Hq, Hkv, L, steps = 2, 8, 2, 90, 40     # crosses two flushes
+    c = Case(B, Hq, Hkv, L, extra_tokens=steps, seed=17, kernel=kernel, n_prune_slices=3)
+    c.prefill()
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device="cuda")
+    for t in range(L, L + steps):
+        kn = np.ascontiguousarray(c.kin[:, :, t])
+        vn = np.ascontiguousarray(c.vin[:, :, t])
+        q = c.query(t)
+        pm.pnmix_append_decode(c.cfg, to_dev(kn), to_dev(vn), to_dev(q), c.cache, out)
+        c.ocache.append(kn, vn)
+        torch.cuda.synchronize()
+        assert_close(out.cpu().numpy(), c.ocache.attend(q))
+    c.check_state()
+    assert c.cache.read_error() == 0
 
 
 # Bit-width shrinking of the salient keys (the PM-KVQ review page's equivalent right shift):
