@@ -18,8 +18,8 @@
 //
 // score_kernel: grid (chunks, KV heads, sequences); a CTA rebuilds the unit's mean query
 // (the same sequential sums everywhere, so every CTA gets the same bits) and scores
-// kScoreGroups groups, one token per thread for the logits and one thread per group for
-// the maxima.
+// kScoreGroups groups, one token per thread for the logits (rows staged through shared
+// memory by coalesced loads) and one thread per group for the maxima.
 // route_kernel: one CTA per (sequence, KV head).  The n_hi best groups are those whose key
 // (score, then lower index) is at least the n_hi-th largest key, found by a radix select
 // over the order-preserving bits of the score (four 8-bit digits, most significant
@@ -32,8 +32,9 @@
 namespace pnmix {
 namespace {
 
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 128;
 constexpr int kScoreGroups = 64;       // groups scored by one CTA (2048 tokens)
+constexpr int kStageRow = 272;         // bytes per staged key row (256 + 16 of padding)
 constexpr int kRouteThreads = 1024;
 constexpr int kSplitThreads = 128;
 
@@ -42,33 +43,61 @@ score_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
              int L, int ld, float* scores) {
   __shared__ float qbar[kHeadDim];
   __shared__ float logit[kScoreThreads];
+  __shared__ __align__(16) uint8_t stage[kScoreThreads * kStageRow];
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int ng = L / kGroup;
   const int gbeg = blockIdx.x * kScoreGroups;
   const int gend = min(ng, gbeg + kScoreGroups);
   const size_t u = static_cast<size_t>(b) * Hkv + h;
 
-  // ---- mean query of the unit's saliency window (heads outer, tokens inner)
+  // ---- mean query of the unit's saliency window (heads outer, tokens inner).  The G
+  // heads' windows are consecutive rows, so row r = head r / nw, token r % nw; sixteen
+  // rows' loads are issued before their sequential sum
   if (tid < kHeadDim) {
+    const int rows = G * nw;
+    const uint16_t* col = qwin + (static_cast<size_t>(b) * Hq + h * G) * nw * kHeadDim + tid;
     float s = 0.f;
-    for (int hh = 0; hh < G; ++hh) {
-      const uint16_t* col = qwin + ((static_cast<size_t>(b) * Hq + h * G + hh) * nw) * kHeadDim + tid;
-      for (int t = 0; t < nw; ++t) s = __fadd_rn(s, bf16_bits_to_float(col[static_cast<size_t>(t) * kHeadDim]));
+    for (int r0 = 0; r0 < rows; r0 += 16) {
+      uint16_t x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = r0 + i < rows ? __ldg(col + static_cast<size_t>(r0 + i) * kHeadDim) : 0;
+      asm volatile("" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (r0 + i < rows) s = __fadd_rn(s, bf16_bits_to_float(x[i]));
     }
-    qbar[tid] = __fdiv_rn(s, static_cast<float>(G * nw));
+    qbar[tid] = __fdiv_rn(s, static_cast<float>(rows));
   }
   __syncthreads();
 
-  // ---- group scores: 256 tokens (8 groups) per pass
+  // ---- group scores: 128 tokens (4 groups) per pass, warp w taking tokens 32w .. 32w+31
+  // of the pass.  The warp stages its 32 rows (8 KB) in shared memory with coalesced
+  // 16-byte loads (one 512-byte stretch per instruction), rows padded to 272 bytes so that
+  // the row-per-lane reads below hit distinct banks; lane l then sums row l in channel
+  // order.
   float* sc = scores + u * ng;
   const uint16_t* ku = k + u * static_cast<size_t>(ld) * kHeadDim;
+  const int lane = tid & 31, warp = tid >> 5;
+  uint8_t* wst = stage + warp * 32 * kStageRow;
   for (int base = gbeg * kGroup; base < gend * kGroup; base += kScoreThreads) {
-    const int t = base + tid;
+    const int t0 = base + 32 * warp, tend = gend * kGroup;
+    uint4 ld16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {   // rows 2i + (lane >> 4), chunk lane & 15
+      const int r = 2 * i + (lane >> 4), t = t0 + r;
+      ld16[i] = t < tend ? __ldg(reinterpret_cast<const uint4*>(ku + static_cast<size_t>(t) * kHeadDim) + (lane & 15))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      *reinterpret_cast<uint4*>(wst + (2 * i + (lane >> 4)) * kStageRow + (lane & 15) * 16) = ld16[i];
+    __syncwarp();
     float acc = 0.f;
-    if (t < gend * kGroup) {
-      const uint4* row = reinterpret_cast<const uint4*>(ku + static_cast<size_t>(t) * kHeadDim);
+    if (t0 + lane < tend) {
+      const uint8_t* row = wst + lane * kStageRow;
+#pragma unroll
       for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
-        const uint4 w = row[c8];
+        const uint4 w = *reinterpret_cast<const uint4*>(row + c8 * 16);
         const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {   // channel c8*8 + 2e in the low half, + 1 in the high half
@@ -77,6 +106,7 @@ score_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
         }
       }
     }
+    __syncwarp();   // the warp's stage is free for the next pass
     logit[tid] = acc;
     __syncthreads();
     if (tid < kScoreThreads / kGroup) {

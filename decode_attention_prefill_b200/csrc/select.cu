@@ -12,6 +12,8 @@
 //   G x W window, sums them sequentially in the reference order (heads outer, tokens
 //   inner), builds the scores of the configured statistic and selects the top k with
 //   warp shuffles.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace pnmix {
@@ -226,21 +228,54 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
     unsigned sel_lo = __ballot_sync(0xffffffffu, rank0 < g.k);
     unsigned sel_hi = __ballot_sync(0xffffffffu, rank1 < g.k);
     unsigned long long mask = (static_cast<unsigned long long>(sel_hi) << 32) | sel_lo;
-    if (lane == 0) {
-      c.pair_mask[unit] = mask;
-      uint8_t* idx = c.pair_idx + static_cast<size_t>(unit) * 64;
-      int n = 0;
-      for (int p = 0; p < 64; ++p)
-        if ((mask >> p) & 1ull) idx[n++] = static_cast<uint8_t>(p);
-      for (; n < 64; ++n) idx[n] = 0;
-      uint8_t* perm = c.perm + static_cast<size_t>(unit) * 128;
-      n = 0;
-      for (int ch = 0; ch < 128; ++ch)
-        if ((mask >> (ch & 63)) & 1ull) perm[n++] = static_cast<uint8_t>(ch);
-      for (int ch = 0; ch < 128; ++ch)
-        if (!((mask >> (ch & 63)) & 1ull)) perm[n++] = static_cast<uint8_t>(ch);
+    if (lane == 0) c.pair_mask[unit] = mask;
+    // pair indices (salient pairs ascending, then zeros) and the position order (salient
+    // channels ascending, then the others ascending): every lane places its own entries,
+    // the position of each from a population count of the mask below it
+    uint8_t* idx = c.pair_idx + static_cast<size_t>(unit) * 64;
+    uint8_t* perm = c.perm + static_cast<size_t>(unit) * 128;
+    const int k = __popcll(mask);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int p = lane + 32 * e;
+      const int below = __popcll(mask & ((1ull << p) - 1ull));   // salient pairs below p
+      if ((mask >> p) & 1ull) idx[below] = static_cast<uint8_t>(p);
+      if (p >= k) idx[p] = 0;   // entries k..63: zero (none of them is a salient slot)
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int ch = lane + 32 * e, p = ch & 63;
+      const int below = __popcll(mask & ((1ull << p) - 1ull)) + (ch >= 64 ? k : 0);   // salient channels below ch
+      const int pos = ((mask >> p) & 1ull) ? below : 2 * k + (ch - below);
+      perm[pos] = static_cast<uint8_t>(ch);
     }
   }
+}
+
+// Resident CTAs of one full wave of a select instance on the current device (the occupancy
+// query runs once per instance and device).
+template <typename K>
+cudaError_t resident_ctas(K kern, int* out) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[3][kMaxDevices];
+  const int which = kern == select_pairs_kernel<PNMIX_SCORE_KEY_ONLY> ? 1
+                    : kern == select_pairs_kernel<PNMIX_SCORE_RANGE_QUERY> ? 2 : 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  int v = cacheable ? cache[which][dev].load(std::memory_order_relaxed) : 0;
+  if (v == 0) {
+    int sms = 0, occ = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    v = sms * (occ > 0 ? occ : 1);
+    if (cacheable) cache[which][dev].store(v, std::memory_order_relaxed);
+  }
+  *out = v;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -260,24 +295,22 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
     e = cudaMemset2DAsync(cm + 128, 1024, 0x00, 512, units, s);
     if (e != cudaSuccess) return e;
   }
-  // about eight CTAs per SM so the max pass balances, with >= 256 tokens per CTA (two
-  // passes of kRowUnroll rows per thread)
-  int want = (8 * 148 + units - 1) / units;
+  // one wave: as many token splits per unit as the resident CTAs allow (the max pass then
+  // ends together on every SM), with >= 256 tokens per CTA (two passes of kRowUnroll rows
+  // per thread)
+  auto kern = select_pairs_kernel<PNMIX_SCORE_PNMIX>;
+  if (g.score == PNMIX_SCORE_KEY_ONLY) kern = select_pairs_kernel<PNMIX_SCORE_KEY_ONLY>;
+  if (g.score == PNMIX_SCORE_RANGE_QUERY) kern = select_pairs_kernel<PNMIX_SCORE_RANGE_QUERY>;
+  int resident = 0;
+  e = resident_ctas(kern, &resident);
+  if (e != cudaSuccess) return e;
+  int want = resident / units;
   int max_split = (L + 255) / 256;
   int nsplit = want < max_split ? want : max_split;
   if (nsplit < 1) nsplit = 1;
   if (nsplit > 512) nsplit = 512;
   dim3 grid(nsplit, units);
-  switch (g.score) {
-    case PNMIX_SCORE_KEY_ONLY:
-      select_pairs_kernel<PNMIX_SCORE_KEY_ONLY><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
-      break;
-    case PNMIX_SCORE_RANGE_QUERY:
-      select_pairs_kernel<PNMIX_SCORE_RANGE_QUERY><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
-      break;
-    default:
-      select_pairs_kernel<PNMIX_SCORE_PNMIX><<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
-  }
+  kern<<<grid, kThreads, 0, s>>>(g, q_window, n_window, k, L, ld, c);
   return cudaGetLastError();
 }
 
