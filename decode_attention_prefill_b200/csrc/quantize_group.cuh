@@ -22,12 +22,20 @@ struct GroupSmem {
   uint8_t perm[kHeadDim];
 };
 
-// Stage 32 rows of 128 bf16 (row stride `ld_elems`) into shared memory.
+// Stage 32 rows of 128 bf16 (row stride `ld_elems`) into shared memory: every thread's
+// four 16-byte loads are issued before their stores.
 __device__ __forceinline__ void load_tile(GroupSmem& sm, const uint16_t* src, size_t ld_elems) {
-  for (int i = threadIdx.x; i < kGroup * 16; i += kQuantThreads) {
-    int r = i >> 4, c = i & 15;
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(src + r * ld_elems) + c);
-    *reinterpret_cast<uint4*>(&sm.tile[r][c * 8]) = v;
+  constexpr int kPer = kGroup * 16 / kQuantThreads;
+  uint4 v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int i = threadIdx.x + k * kQuantThreads, r = i >> 4, c = i & 15;
+    v[k] = __ldg(reinterpret_cast<const uint4*>(src + r * ld_elems) + c);
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int i = threadIdx.x + k * kQuantThreads, r = i >> 4, c = i & 15;
+    *reinterpret_cast<uint4*>(&sm.tile[r][c * 8]) = v[k];
   }
 }
 
