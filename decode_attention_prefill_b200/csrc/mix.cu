@@ -17,9 +17,9 @@
 // ascending token order into its own buffers, ready for the ordinary quantizers.
 //
 // score_kernel: grid (chunks, KV heads, sequences); a CTA rebuilds the unit's mean query
-// (the same sequential sums everywhere, so every CTA gets the same bits) and scores
-// kScoreGroups groups, one token per thread for the logits (rows staged through shared
-// memory by coalesced loads) and one thread per group for the maxima.
+// (the same sequential sums everywhere, so every CTA gets the same bits) and scores a run
+// of groups (one wave of CTAs in all), one token per thread for the logits (rows staged
+// through shared memory by coalesced loads) and one thread per group for the maxima.
 // route_kernel: one CTA per (sequence, KV head).  The n_hi best groups are those whose key
 // (score, then lower index) is at least the n_hi-th largest key, found by a radix select
 // over the order-preserving bits of the score (four 8-bit digits, most significant
@@ -27,86 +27,116 @@
 // indices; a group's place inside its part is the count of earlier groups with the same
 // route (a block-wide prefix sum).  O(ng) work per pass instead of ng^2 comparisons.
 // split_kernel: one CTA per (group, KV head, sequence), plus one per unit for the tail.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace pnmix {
 namespace {
 
 constexpr int kScoreThreads = 128;
-constexpr int kScoreGroups = 64;       // groups scored by one CTA (2048 tokens)
+constexpr int kScoreMinGroups = 4;     // groups scored by one CTA at least (one pass)
 constexpr int kStageRow = 272;         // bytes per staged key row (256 + 16 of padding)
 constexpr int kRouteThreads = 1024;
 constexpr int kSplitThreads = 128;
 
+constexpr int kScoreStageBytes = (kScoreThreads / 32) * 2 * 32 * kStageRow;   // two stages per warp
+static_assert(kScoreThreads == kHeadDim, "one score thread per channel for the mean query");
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, const uint16_t* __restrict__ k,
-             int L, int ld, float* scores) {
-  __shared__ float qbar[kHeadDim];
+             int L, int ld, int gpc, float* scores) {
+  __shared__ __align__(16) float qbar[kHeadDim];
   __shared__ float logit[kScoreThreads];
-  __shared__ __align__(16) uint8_t stage[kScoreThreads * kStageRow];
+  extern __shared__ __align__(16) uint8_t stage[];   // [warps][2][32 rows][kStageRow]
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int ng = L / kGroup;
-  const int gbeg = blockIdx.x * kScoreGroups;
-  const int gend = min(ng, gbeg + kScoreGroups);
+  const int gbeg = blockIdx.x * gpc;
+  const int gend = min(ng, gbeg + gpc);
   const size_t u = static_cast<size_t>(b) * Hkv + h;
+  float* sc = scores + u * ng;
+  const uint16_t* ku = k + u * static_cast<size_t>(ld) * kHeadDim;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int first = gbeg * kGroup, tend = gend * kGroup;
 
-  // ---- mean query of the unit's saliency window (heads outer, tokens inner).  The G
-  // heads' windows are consecutive rows, so row r = head r / nw, token r % nw; sixteen
-  // rows' loads are issued before their sequential sum
-  if (tid < kHeadDim) {
+  // ---- key rows, 128 tokens (4 groups) per pass, warp w taking tokens 32w .. 32w+31 of the
+  // pass: the warp copies its 32 rows (8 KB) into shared memory with coalesced 16-byte
+  // asynchronous copies (one 512-byte stretch per instruction; rows past the end are
+  // zero-filled), rows padded to 272 bytes so that the row-per-lane reads hit distinct
+  // banks.  Two stages: the next pass's rows are in flight while this pass is summed.
+  uint8_t* wst = stage + warp * 2 * 32 * kStageRow;
+  auto issue = [&](int base, int buf) {
+    const int t0 = base + 32 * warp;
+    uint8_t* dst = wst + buf * 32 * kStageRow;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {   // rows 2i + (lane >> 4), chunk lane & 15
+      const int r = 2 * i + (lane >> 4), t = t0 + r;
+      const bool ok = t < tend;
+      cp_async16(dst + r * kStageRow + (lane & 15) * 16,
+                 ku + static_cast<size_t>(ok ? t : first) * kHeadDim + (lane & 15) * 8, ok ? 16 : 0);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // ---- mean query of the unit's saliency window (heads outer, tokens inner).  The G heads'
+  // windows are consecutive rows (row r = head r / nw, token r % nw); they are copied into
+  // the stage in rounds of as many rows as it holds (coalesced 16-byte copies), and thread c
+  // sums column c over each round in row order
+  {
     const int rows = G * nw;
-    const uint16_t* col = qwin + (static_cast<size_t>(b) * Hq + h * G) * nw * kHeadDim + tid;
+    const uint16_t* qbase = qwin + (static_cast<size_t>(b) * Hq + h * G) * nw * kHeadDim;
+    constexpr int kCap = kScoreStageBytes / (kHeadDim * 2);   // window rows per round
     float s = 0.f;
-    for (int r0 = 0; r0 < rows; r0 += 16) {
-      uint16_t x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = r0 + i < rows ? __ldg(col + static_cast<size_t>(r0 + i) * kHeadDim) : 0;
-      asm volatile("" ::: "memory");
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (r0 + i < rows) s = __fadd_rn(s, bf16_bits_to_float(x[i]));
+    for (int r0 = 0; r0 < rows; r0 += kCap) {
+      const int nr = min(kCap, rows - r0);
+      for (int i = tid; i < nr * 16; i += kScoreThreads)
+        cp_async16(stage + i * 16, qbase + static_cast<size_t>(r0) * kHeadDim + i * 8, 16);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      const uint16_t* col = reinterpret_cast<const uint16_t*>(stage) + tid;
+#pragma unroll 16
+      for (int r = 0; r < nr; ++r) s = __fadd_rn(s, bf16_bits_to_float(col[r * kHeadDim]));
+      __syncthreads();
     }
     qbar[tid] = __fdiv_rn(s, static_cast<float>(rows));
   }
   __syncthreads();
+  if (first < tend) issue(first, 0);
 
-  // ---- group scores: 128 tokens (4 groups) per pass, warp w taking tokens 32w .. 32w+31
-  // of the pass.  The warp stages its 32 rows (8 KB) in shared memory with coalesced
-  // 16-byte loads (one 512-byte stretch per instruction), rows padded to 272 bytes so that
-  // the row-per-lane reads below hit distinct banks; lane l then sums row l in channel
-  // order.
-  float* sc = scores + u * ng;
-  const uint16_t* ku = k + u * static_cast<size_t>(ld) * kHeadDim;
-  const int lane = tid & 31, warp = tid >> 5;
-  uint8_t* wst = stage + warp * 32 * kStageRow;
-  for (int base = gbeg * kGroup; base < gend * kGroup; base += kScoreThreads) {
-    const int t0 = base + 32 * warp, tend = gend * kGroup;
-    uint4 ld16[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {   // rows 2i + (lane >> 4), chunk lane & 15
-      const int r = 2 * i + (lane >> 4), t = t0 + r;
-      ld16[i] = t < tend ? __ldg(reinterpret_cast<const uint4*>(ku + static_cast<size_t>(t) * kHeadDim) + (lane & 15))
-                         : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      *reinterpret_cast<uint4*>(wst + (2 * i + (lane >> 4)) * kStageRow + (lane & 15) * 16) = ld16[i];
+  // ---- group scores: lane l sums row l of its warp's stage in channel order
+  const float4* qbar4 = reinterpret_cast<const float4*>(qbar);
+  int buf = 0;
+  for (int base = first; base < tend; base += kScoreThreads, buf ^= 1) {
+    if (base + kScoreThreads < tend)
+      issue(base + kScoreThreads, buf ^ 1);
+    else
+      asm volatile("cp.async.commit_group;" ::: "memory");   // an empty group keeps the count
+    asm volatile("cp.async.wait_group 1;" ::: "memory");     // this pass's rows have landed
     __syncwarp();
+    const int t0 = base + 32 * warp;
     float acc = 0.f;
     if (t0 + lane < tend) {
-      const uint8_t* row = wst + lane * kStageRow;
+      const uint8_t* row = wst + buf * 32 * kStageRow + lane * kStageRow;
 #pragma unroll
       for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
         const uint4 w = *reinterpret_cast<const uint4*>(row + c8 * 16);
+        const float4 qa = qbar4[2 * c8], qb = qbar4[2 * c8 + 1];
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {   // channel c8*8 + 2e in the low half, + 1 in the high half
-          acc = __fadd_rn(acc, __fmul_rn(qbar[c8 * 8 + 2 * e], __uint_as_float(wv[e] << 16)));
-          acc = __fadd_rn(acc, __fmul_rn(qbar[c8 * 8 + 2 * e + 1], __uint_as_float(wv[e] & 0xFFFF0000u)));
+          acc = __fadd_rn(acc, __fmul_rn(qv[2 * e], __uint_as_float(wv[e] << 16)));
+          acc = __fadd_rn(acc, __fmul_rn(qv[2 * e + 1], __uint_as_float(wv[e] & 0xFFFF0000u)));
         }
       }
     }
-    __syncwarp();   // the warp's stage is free for the next pass
+    __syncwarp();   // this stage is free for the copies two passes on
     logit[tid] = acc;
     __syncthreads();
     if (tid < kScoreThreads / kGroup) {
@@ -122,6 +152,7 @@ score_kernel(int G, int Hq, int Hkv, const uint16_t* __restrict__ qwin, int nw, 
     }
     __syncthreads();
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Order-preserving unsigned image of a float; -0 and +0 map to the same value, as they
@@ -265,6 +296,30 @@ split_kernel(int Hkv, const uint16_t* __restrict__ k, const uint16_t* __restrict
   }
 }
 
+// Resident score CTAs of one full wave on the current device (queried once per device).
+cudaError_t score_resident_ctas(int* out) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  int v = cacheable ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (v == 0) {
+    int sms = 0, occ = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreStageBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score_kernel, kScoreThreads, kScoreStageBytes);
+    if (e != cudaSuccess) return e;
+    v = sms * (occ > 0 ? occ : 1);
+    if (cacheable) cache[dev].store(v, std::memory_order_relaxed);
+  }
+  *out = v;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_split_groups(const Geometry& g, const uint16_t* q_window, int nw, const uint16_t* k,
@@ -274,10 +329,20 @@ cudaError_t launch_split_groups(const Geometry& g, const uint16_t* q_window, int
   if (g.B == 0) return cudaSuccess;
   const int ng = L / kGroup;
   if (ng > 0) {
-    const int chunks = (ng + kScoreGroups - 1) / kScoreGroups;
-    score_kernel<<<dim3(chunks, g.Hkv, g.B), kScoreThreads, 0, s>>>(g.G, g.Hq, g.Hkv, q_window, nw, k, L, ld,
-                                                                     scores);
-    cudaError_t e = cudaGetLastError();
+    // one wave of CTAs: the key rows are read with enough loads in flight only when every
+    // resident slot holds a CTA
+    int resident = 0;
+    cudaError_t e = score_resident_ctas(&resident);
+    if (e != cudaSuccess) return e;
+    const long long units = static_cast<long long>(g.B) * g.Hkv;
+    long long per_unit = resident / units;
+    if (per_unit < 1) per_unit = 1;
+    int gpc = static_cast<int>((ng + per_unit - 1) / per_unit);
+    if (gpc < kScoreMinGroups) gpc = kScoreMinGroups;
+    const int chunks = (ng + gpc - 1) / gpc;
+    score_kernel<<<dim3(chunks, g.Hkv, g.B), kScoreThreads, kScoreStageBytes, s>>>(g.G, g.Hq, g.Hkv, q_window, nw,
+                                                                                    k, L, ld, gpc, scores);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     route_kernel<<<dim3(g.Hkv, g.B), kRouteThreads, 0, s>>>(g.Hkv, L, n_hi, scores, route, dest);
     e = cudaGetLastError();
