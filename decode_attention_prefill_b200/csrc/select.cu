@@ -41,15 +41,8 @@ __device__ __forceinline__ void chunk_pair_norm2(const uint4& lo, const uint4& h
     }
   }
 }
-template <bool RANGE = false>
-__device__ __forceinline__ void row_pair_norm2(const uint16_t* row, int c, float out[8],
-                                               float* mn = nullptr, float* mx = nullptr) {
-  const uint4 lo = __ldg(reinterpret_cast<const uint4*>(row) + c);
-  const uint4 hi = __ldg(reinterpret_cast<const uint4*>(row) + 8 + c);
-  chunk_pair_norm2<RANGE>(lo, hi, out, mn, mx);
-}
-
 constexpr int kRowUnroll = 4;   // rows per thread per pass: 8 independent 16-byte loads in flight
+constexpr int kQnRows = 3 * kRowsPerIter;   // query-window rows per round of the last CTA
 
 // Order-preserving map of non-NaN floats to unsigned integers (and back), so that
 // integer atomics compute float min / max.
@@ -74,7 +67,7 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
   const int rsub = tid >> 3;         // row within an iteration
 
   __shared__ float red[kThreads / 32][64];
-  __shared__ float qn[kRowsPerIter][64];
+  __shared__ float qn[kQnRows][64];
   __shared__ float score_s[64];
   __shared__ float rmin[RANGE ? kThreads / 32 : 1][128], rmax[RANGE ? kThreads / 32 : 1][128];
   __shared__ int is_last;
@@ -172,23 +165,36 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
   if (!is_last) return;
   __threadfence();
 
-  // ---- query pair norms, summed in the reference order
+  // ---- query pair norms, summed in the reference order: kQnRows window rows per round,
+  // all of a round's loads issued together (the G heads' windows are consecutive rows:
+  // row i = head i / n_window, token i % n_window)
   float qsum = 0.0f;   // meaningful for tid < 64
-  const int rows = g.G * n_window;   // row i = head (i / n_window), token (i % n_window)
-  for (int r0 = 0; r0 < rows; r0 += kRowsPerIter) {
-    int r = r0 + rsub;
-    if (r < rows) {
-      int hh = r / n_window, tt = r % n_window;
-      const uint16_t* row =
-          q_window + ((static_cast<size_t>(b) * g.Hq + h * g.G + hh) * n_window + tt) * kHeadDim;
-      float n2[8];
-      row_pair_norm2(row, cidx, n2);
+  const int rows = g.G * n_window;
+  const uint16_t* qrows = q_window + (static_cast<size_t>(b) * g.Hq + h * g.G) * n_window * kHeadDim;
+  for (int r0 = 0; r0 < rows; r0 += kQnRows) {
+    uint4 lo[kQnRows / kRowsPerIter], hi[kQnRows / kRowsPerIter];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) qn[rsub][8 * cidx + i] = __fsqrt_rn(n2[i]);
+    for (int u = 0; u < kQnRows / kRowsPerIter; ++u) {
+      const int r = r0 + rsub + u * kRowsPerIter;
+      if (r < rows) {
+        const uint4* row = reinterpret_cast<const uint4*>(qrows + static_cast<size_t>(r) * kHeadDim);
+        lo[u] = __ldg(row + cidx);
+        hi[u] = __ldg(row + 8 + cidx);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQnRows / kRowsPerIter; ++u) {
+      if (r0 + rsub + u * kRowsPerIter < rows) {
+        float n2[8];
+        chunk_pair_norm2(lo[u], hi[u], n2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qn[rsub + u * kRowsPerIter][8 * cidx + i] = __fsqrt_rn(n2[i]);
+      }
     }
     __syncthreads();
     if (tid < 64) {
-      int nr = min(kRowsPerIter, rows - r0);
+      const int nr = min(kQnRows, rows - r0);
+#pragma unroll 8
       for (int i = 0; i < nr; ++i) qsum = __fadd_rn(qsum, qn[i][tid]);
     }
     __syncthreads();
