@@ -7,11 +7,13 @@
 //   loads and merges it into a per-unit scratch array with atomicMax on the float bits
 //   (non-negative floats order like their bit patterns, and max is order-free, so the
 //   split is exact); for the range statistic it also reduces every channel's min and max
-//   (atomicMin / atomicMax on an order-preserving integer image of the float);
+//   (atomicMax on an order-preserving integer image of the float, and on its complement
+//   for the minimum, so that zero means "no value" for both);
 //   the last CTA of a unit (atomic ticket, no waiting) forms the query pair norms of the
 //   G x W window, sums them sequentially in the reference order (heads outer, tokens
-//   inner), builds the scores of the configured statistic and selects the top k with
-//   warp shuffles.
+//   inner), builds the scores of the configured statistic, selects the top k with warp
+//   shuffles and sets the unit's accumulators and ticket back to zero, so a call needs no
+//   clearing beforehand (the cache starts zero-filled).
 #include <atomic>
 
 #include "common.cuh"
@@ -154,7 +156,7 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
         lo = fminf(lo, rmin[w][tid]);
         hi = fmaxf(hi, rmax[w][tid]);
       }
-      atomicMin(cmin + tid, ordered_key(lo));
+      atomicMax(cmin + tid, ~ordered_key(lo));   // the complement: zero is "no value yet"
       atomicMax(cmax + tid, ordered_key(hi));
     }
   }
@@ -206,8 +208,8 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
     if constexpr (SCORE == PNMIX_SCORE_KEY_ONLY) {
       s = kp;
     } else if constexpr (RANGE) {
-      const float r0 = __fsub_rn(ordered_value(__ldcg(cmax + tid)), ordered_value(__ldcg(cmin + tid)));
-      const float r1 = __fsub_rn(ordered_value(__ldcg(cmax + 64 + tid)), ordered_value(__ldcg(cmin + 64 + tid)));
+      const float r0 = __fsub_rn(ordered_value(__ldcg(cmax + tid)), ordered_value(~__ldcg(cmin + tid)));
+      const float r1 = __fsub_rn(ordered_value(__ldcg(cmax + 64 + tid)), ordered_value(~__ldcg(cmin + 64 + tid)));
       s = __fmul_rn(qp, __fsqrt_rn(__fadd_rn(__fmul_rn(r0, r0), __fmul_rn(r1, r1))));
     } else {
       s = __fmul_rn(qp, kp);
@@ -216,6 +218,13 @@ select_pairs_kernel(Geometry g, const uint16_t* __restrict__ q_window, int n_win
     c.pair_scores[static_cast<size_t>(unit) * 64 + tid] = s;
   }
   __syncthreads();
+  // leave the unit's accumulators and ticket at zero for the next call (every CTA of the
+  // unit has added to them, and the scores above have read them)
+  if (tid < 64) kmax[tid] = 0u;
+  if constexpr (RANGE) {
+    cmin[tid] = 0u;   // 256 threads: 128 minima then 128 maxima
+  }
+  if (tid == 0) *ticket = 0u;
 
   // ---- top k by (score desc, pair asc): rank of every pair, by warp shuffles
   if (warp == 0) {
@@ -290,17 +299,6 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
                                 const uint16_t* k, int L, int ld, const pnmix_cache& c,
                                 cudaStream_t s) {
   const int units = g.B * g.Hkv;
-  // scratch (max-norm accumulators and tickets) starts at zero for every call; the range
-  // statistic's channel minima start at the largest key, maxima at the smallest
-  cudaError_t e = cudaMemsetAsync(c.scratch, 0, sizeof(uint32_t) * static_cast<size_t>(units) * 65, s);
-  if (e != cudaSuccess) return e;
-  if (g.score == PNMIX_SCORE_RANGE_QUERY) {
-    uint32_t* cm = c.scratch + scratch_range_offset(g.B, g.Hkv);
-    e = cudaMemset2DAsync(cm, 1024, 0xFF, 512, units, s);
-    if (e != cudaSuccess) return e;
-    e = cudaMemset2DAsync(cm + 128, 1024, 0x00, 512, units, s);
-    if (e != cudaSuccess) return e;
-  }
   // one wave: as many token splits per unit as the resident CTAs allow (the max pass then
   // ends together on every SM), with >= 256 tokens per CTA (two passes of kRowUnroll rows
   // per thread)
@@ -308,7 +306,7 @@ cudaError_t launch_select_pairs(const Geometry& g, const uint16_t* q_window, int
   if (g.score == PNMIX_SCORE_KEY_ONLY) kern = select_pairs_kernel<PNMIX_SCORE_KEY_ONLY>;
   if (g.score == PNMIX_SCORE_RANGE_QUERY) kern = select_pairs_kernel<PNMIX_SCORE_RANGE_QUERY>;
   int resident = 0;
-  e = resident_ctas(kern, &resident);
+  cudaError_t e = resident_ctas(kern, &resident);
   if (e != cudaSuccess) return e;
   int want = resident / units;
   int max_split = (L + 255) / 256;

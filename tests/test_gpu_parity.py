@@ -232,6 +232,25 @@ def test_saliency_statistics_select_like_the_oracle(score, B, Hq, Hkv, L, k, bhi
     assert_close(got, want)
 
 
+@pytest.mark.parametrize("score", [0, 1, 2])
+def test_select_called_again_on_the_same_cache_starts_clean(score):
+    """The selection's accumulators and tickets are left at zero by each call: three calls
+    on one cache with different inputs (and a shorter prefill in between) each give the
+    oracle's scores, pairs and permutation bit for bit."""
+    import decode_attention_prefill_b200 as pm
+    B, Hq, Hkv = 2, 8, 2
+    c = Case(B, Hq, Hkv, 900, 8, 4, 2, seed=3, score=score)
+    for seed, L in ((3, 900), (4, 300), (5, 900)):
+        d = Case(B, Hq, Hkv, L, 8, 4, 2, seed=seed, score=score)
+        pm.pnmix_select_pairs(c.cfg, to_dev(d.qwin), d.k_dev, L, c.cache)
+        d.ocache.select(d.qwin, d.kin, L)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(c.cache.pair_scores().cpu().numpy().view(np.uint32),
+                                      d.ocache.scores.view(np.uint32))
+        np.testing.assert_array_equal(c.cache.perm().cpu().numpy(), d.ocache.perm)
+        np.testing.assert_array_equal(c.cache.pair_mask().cpu().numpy().view(np.uint64), d.ocache.mask)
+
+
 @pytest.mark.parametrize("kernel", [None, "mma", "ws"])
 @pytest.mark.parametrize("B,Hq,Hkv,L,T", [
     (1, 1, 1, 40, 3),      # all new tokens in the residual
