@@ -47,7 +47,7 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 // Work-partition weights (decode_common.cuh, unit_items), in group items: the fixed cost of
 // a unit's segment and the residual window's CUDA-core pass.
-constexpr int kLeadItems = 40;
+constexpr int kLeadItems = 28;
 constexpr int kResidItems = 8;
 // Fused append, flush step: the quantizers' staging tile sits in the (then idle) ring.
 static_assert(sizeof(GroupSmem) <= 4 * 2 * 2 * 3072, "the quantizers' tile must fit the staging ring");
