@@ -35,8 +35,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_ALIGNMENT, ERR
 DEVERR_APPEND_FULL = 0x1
 DEVERR_TIMEOUT = 0x2
 # decode kernels (Config.decode_kernel)
-DECODE_AUTO, DECODE_SIMT, DECODE_MMA, DECODE_PAIRS = range(4)
-DECODE_KERNELS = {"auto": DECODE_AUTO, "simt": DECODE_SIMT, "mma": DECODE_MMA, "ws": DECODE_PAIRS}
+DECODE_AUTO, DECODE_SIMT, DECODE_MMA, DECODE_PAIRS, DECODE_TC = range(5)
+DECODE_KERNELS = {"auto": DECODE_AUTO, "simt": DECODE_SIMT, "mma": DECODE_MMA, "ws": DECODE_PAIRS, "tc": DECODE_TC}
 
 EXPORTED = [
     "pnmix_record_bytes", "pnmix_cache_bytes", "pnmix_cache_init", "pnmix_cache_reset",

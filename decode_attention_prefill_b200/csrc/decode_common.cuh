@@ -289,6 +289,8 @@ cudaError_t launch_decode_mma(const Geometry& g, const uint16_t* q, const pnmix_
                               float* out, DecodeWs ws, cudaStream_t s);
 cudaError_t launch_decode_ws(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                              float* out, DecodeWs ws, cudaStream_t s);
+cudaError_t launch_decode_tc(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
+                             float* out, DecodeWs ws, cudaStream_t s);
 cudaError_t launch_decode_rows(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                                float* out, DecodeWs ws, cudaStream_t s);
 

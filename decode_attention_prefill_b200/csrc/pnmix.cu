@@ -30,7 +30,7 @@ static pnmix_status make_geometry(const pnmix_config* cfg, int batch, int capaci
   if (cfg->saliency_score < PNMIX_SCORE_PNMIX || cfg->saliency_score > PNMIX_SCORE_RANGE_QUERY)
     return PNMIX_ERR_UNSUPPORTED;
   if (cfg->n_pruned_pairs < 0 || cfg->n_pruned_pairs > 63) return PNMIX_ERR_UNSUPPORTED;
-  if (cfg->decode_kernel < PNMIX_DECODE_AUTO || cfg->decode_kernel > PNMIX_DECODE_PAIRS)
+  if (cfg->decode_kernel < PNMIX_DECODE_AUTO || cfg->decode_kernel > PNMIX_DECODE_TC)
     return PNMIX_ERR_UNSUPPORTED;
   if (cfg->n_pruned_slices < 0 || cfg->n_pruned_slices > 8) return PNMIX_ERR_UNSUPPORTED;
   if (cfg->n_pruned_pairs > 0 && cfg->n_pruned_slices > 0) return PNMIX_ERR_UNSUPPORTED;
@@ -142,6 +142,7 @@ cudaError_t launch_decode(const Geometry& g, const uint16_t* q, const pnmix_cach
   w.prior_lse = merge.prior_lse;
   w.k_new = merge.k_new;
   w.v_new = merge.v_new;
+  if (g.kernel == PNMIX_DECODE_TC) return launch_decode_tc(g, q, c, nmax, out, w, s);
   if (g.rows > kMaxG) return launch_decode_rows(g, q, c, nmax, out, w, s);   // 9 .. 64 query rows
   switch (g.kernel) {
     case PNMIX_DECODE_SIMT: return launch_decode_simt(g, q, c, nmax, out, w, s);

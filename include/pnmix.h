@@ -161,7 +161,7 @@ typedef enum {
  *   saliency_window W in [1, 1024];
  *   saliency_score in {0, 1, 2} (PNMIX_SCORE_*);
  *   n_pruned_pairs in [0, 63]; n_pruned_slices in [0, 8]; not both non-zero;
- *   decode_kernel in {0, 1, 2, 3} (PNMIX_DECODE_*).
+ *   decode_kernel in {0, 1, 2, 3, 4} (PNMIX_DECODE_*).
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
  *
  * Dynamic query-channel pruning (n_pruned_pairs > 0; the query-channel pruning of the
@@ -216,11 +216,15 @@ typedef struct {
  *                       pruning (PNMIX_ERR_UNSUPPORTED otherwise).
  *   PNMIX_DECODE_MMA    tensor cores, every warp scores and accumulates its own groups.
  *   PNMIX_DECODE_PAIRS  tensor cores, a key-side and a value-side warp per group stream.
+ *   PNMIX_DECODE_TC     5th-generation tensor cores (tcgen05, accumulators in TMEM): each
+ *                       group's keys and values dequantized once into shared memory for all
+ *                       of a unit's query rows (up to 64); meant for multi-token steps.
  */
 #define PNMIX_DECODE_AUTO 0
 #define PNMIX_DECODE_SIMT 1
 #define PNMIX_DECODE_MMA 2
 #define PNMIX_DECODE_PAIRS 3
+#define PNMIX_DECODE_TC 4
 
 /*
  * Pair statistics pnmix_select_pairs can rank by (all per (b, kv head), fp32, one

@@ -53,7 +53,7 @@ def test_record_bytes_agree_with_the_layout_definition(k, bhi, blo):
     (dict(saliency_score=-1), pm.ERR_UNSUPPORTED),
     (dict(n_pruned_pairs=64), pm.ERR_UNSUPPORTED),
     (dict(n_pruned_pairs=-1), pm.ERR_UNSUPPORTED),
-    (dict(decode_kernel=4), pm.ERR_UNSUPPORTED),
+    (dict(decode_kernel=5), pm.ERR_UNSUPPORTED),
     (dict(decode_kernel=-1), pm.ERR_UNSUPPORTED),
     (dict(decode_kernel=pm.DECODE_SIMT, n_pruned_pairs=5), pm.ERR_UNSUPPORTED),   # simt has no pruning
     (dict(n_pruned_slices=9), pm.ERR_UNSUPPORTED),

@@ -546,7 +546,7 @@ def test_select_pairs_breaks_ties_by_the_lower_pair_index(k, L, n_key, n_query):
 # wait a short limit, so those waits run out.  The call must return, raise the timeout bit
 # of the error word, and leave the context, the cache and the workspace usable: the next
 # ordinary decode matches the oracle again.
-@pytest.mark.parametrize("kernel", ["mma", "ws"])
+@pytest.mark.parametrize("kernel", ["mma", "ws", "tc"])
 @pytest.mark.parametrize("skip_unit", [0, 3])
 def test_staging_wait_that_runs_out_sets_the_error_word_and_returns(kernel, skip_unit):
     import ctypes
@@ -762,3 +762,44 @@ def test_random_configurations_like_the_oracle(seed):
         got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
     assert_close(got, want)
     assert c.cache.read_error() == 0
+
+
+# The tcgen05 kernel (cfg->decode_kernel = PNMIX_DECODE_TC, accumulators in TMEM), forced on
+# single- and multi-query shapes, every bit point, pruning, and many segments per unit.
+@pytest.mark.parametrize("B,Hq,Hkv,L,k,bhi,blo,T,prune,slices", [
+    (1, 4, 1, 100, 8, 4, 2, 1, 0, 0),      # 4 rows, one group and the residual window
+    (1, 4, 1, 64, 8, 4, 2, 1, 0, 0),       # whole groups only
+    (2, 8, 2, 300, 8, 4, 2, 2, 0, 0),      # 8 rows
+    (2, 8, 2, 300, 8, 4, 2, 4, 0, 0),      # 16 rows
+    (1, 32, 8, 1000, 8, 4, 2, 16, 0, 0),   # 64 rows
+    (2, 28, 4, 517, 0, 4, 2, 9, 0, 0),     # 63 rows, k = 0
+    (2, 16, 2, 700, 16, 2, 1, 3, 0, 0),    # 1-bit low block
+    (1, 8, 1, 64, 64, 4, 2, 3, 0, 0),      # k = 64
+    (5, 4, 1, 1000, 8, 4, 2, 2, 0, 0),     # more slices than SMs: CTAs with several groups
+    (1, 16, 4, 2500, 8, 4, 2, 5, 26, 0),   # pair pruning, several segments per unit
+    (2, 8, 2, 600, 8, 4, 2, 4, 0, 3),      # key-slice pruning
+])
+def test_tcgen05_decode_like_the_oracle(B, Hq, Hkv, L, k, bhi, blo, T, prune, slices):
+    c = Case(B, Hq, Hkv, L, k, bhi, blo, extra_tokens=T, seed=L + T + prune, kernel="tc", max_queries=max(T, 2),
+             n_prune=prune, n_prune_slices=slices)
+    c.prefill()
+    if T == 1:
+        got, want = c.attend(c.query(L))
+    else:
+        for t in range(L, L + T):
+            c.append(t)
+        got, want = c.attend_multi(c.query_multi(L, T))
+        got, want = got.reshape(B, T * Hq, 128), want.reshape(B, T * Hq, 128)
+    assert_close(got, want)
+    assert c.cache.read_error() == 0
+
+
+def test_tcgen05_decode_is_repeatable():
+    c = Case(2, 8, 2, 700, extra_tokens=4, seed=3, kernel="tc", max_queries=4)
+    c.prefill()
+    for t in range(700, 704):
+        c.append(t)
+    q = to_dev(c.query_multi(700, 4))
+    a = c.cache.attend_multi(q).clone()
+    b = c.cache.attend_multi(q)
+    assert torch.equal(a, b)
