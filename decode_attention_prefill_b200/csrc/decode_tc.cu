@@ -4,28 +4,45 @@
 //
 // One CTA (one warpgroup, 128 threads) per slice of the work partition (decode_common.cuh);
 // thread r owns query row r, which is TMEM lane r of every accumulator (rows >= G are
-// zero).  Per 32-token group record:
+// zero).  A dequantised key is k = c * s + z (code c, fp16 scale s and zero z of its group
+// and position), a value v = c * s_v + z_v.  Per 32-token group record:
 //
-//   logits  S = Q x K^T:  A = the unit's query rows, fp16 (exact from bf16), 128 x 128
-//           positions, written once per segment; B = the group's keys as two fp16 tiles,
-//           hi = fp16(x) and lo = fp16(x - hi) of x = code * s + z in fp32 (32 tokens x
-//           128 positions), so that hi + lo carries x to 22 bits; 16 MMAs of K = 16
-//           (8 slices x hi, lo) accumulate the 128 x 32 fp32 logits in TMEM.
-//   softmax each thread loads its row's 32 logits (tcgen05.ld), applies the softmax scale
-//           and the causal mask, and keeps a lazy online reference m per row (raised to
-//           max + 4 only when a logit exceeds it, so p = 2^(logit - m) <= 1); a raise
-//           rescales the row's value accumulator in TMEM (load, scale, store).
-//   values  O += P x V:  A = P (fp16, 128 rows x 32 tokens), B = the dequantized values as
-//           hi / lo fp16 tiles (128 channels x 32 tokens); 4 MMAs of K = 16 accumulate the
-//           128 x 128 fp32 output rows in TMEM.
+//   logits  S = Q x K^T = Q x (C s)^T + Q x z:  A = the unit's query rows, fp16 (exact from
+//           bf16), 128 rows x 128 positions, written once per segment.  c * s has at most
+//           15 significant bits, so it is exactly the sum of two fp16 numbers, hi = fp16(c s)
+//           (one half-precision multiply) and lo = c s - hi (one half-precision fma, whose
+//           result is exact).  B is one tile of 80 rows x 128 positions: row 0 the zero
+//           points z (the term Q z is the same for the group's 32 tokens), rows 1..15 zero,
+//           rows 16..47 the hi and rows 48..79 the lo parts of the 32 tokens; 8 MMAs of
+//           K = 16 (N = 80) accumulate the three sums of every row in TMEM, fp32, and the
+//           logit of token t is D[16 + t] + D[48 + t] + D[0].
+//   softmax the query rows are repeated in A rows 64..127, so TMEM lane r and r + 64 hold the
+//           same row; lane r takes tokens 0..15 of every group and lane r + 64 tokens 16..31,
+//           as two independent partials merged at the segment's end.  Each thread loads its
+//           16 logits and the zero term (tcgen05.ld), applies the softmax scale and the causal
+//           mask, and keeps a reference m (the first visible maximum, moved only when a logit
+//           would give p = 2^(logit - m) above 2^14, which fp16 still holds; a move rescales
+//           the lane's accumulators in TMEM).  The denominator is the product of P with a row
+//           of ones in the value tile, so it sums the same fp16 p as the outputs.
+//   values  O += P x (C_v s_v)^T + P x z_v:  A = P (fp16, 128 rows x 32 tokens), B = one
+//           tile of 144 rows x 32 tokens: rows 0..3 the zero points of the four 32-channel
+//           groups, rows 4..15 zero, rows 16..143 fp16(c s_v) of the 128 channels (one
+//           rounding, exact for codes 0 .. 2: the value side's precision in every decode
+//           kernel); 2 MMAs (N = 144) accumulate the zero terms and the outputs in TMEM.  A
+//           row's result is O[ch] plus the zero term of ch's channel group.
 //
-// The bf16 residual window takes the same path as one more group (its keys and values
-// split into hi / lo exactly, the tokens past it masked).  One thread issues every MMA
-// (tcgen05.mma, operands from shared memory, K-major, no swizzle) and commits each batch
-// to an mbarrier; the records arrive by TMA bulk copy (no multicast) into a ring of three.
-// Every wait is bounded.  At the end of a segment each thread writes its row's partial
-// (m, l, O) for the fused combine.
+// Pipeline of one group: build the key tiles; one thread issues the key products and commits
+// them to an mbarrier; meanwhile every thread builds the value tiles (two buffers); after the
+// commit (which also covers every earlier product, so TMEM, P and the value buffer two
+// groups back are idle) the softmax writes P; one thread issues the value products without
+// waiting for them.  The bf16 residual window takes the same path as one more group (its
+// keys split into hi / lo, its values rounded to fp16, zero tiles empty, the tokens past it
+// masked).  The
+// records arrive by TMA bulk copy (no multicast) into a ring of four.  Every wait is
+// bounded.  At the end of a segment each thread writes its row's partial (m, l, O) for the
+// fused combine.  Needs |c s| below 65504 (keys and values whose group range fits fp16).
 #include <atomic>
+#include <string.h>
 
 #include "common.cuh"
 #include "decode_common.cuh"
@@ -35,9 +52,15 @@ namespace pnmix {
 namespace {
 
 constexpr int kTcThreads = 128;   // one warpgroup: TMEM lanes 0 .. 127
-constexpr int kTcSlots = 3;       // record ring
-constexpr int kTmemCols = 256;    // logits in columns 0 .. 31, outputs in 128 .. 255
-constexpr int kTmemOut = 128;
+constexpr int kTcSlots = 4;       // record ring
+constexpr int kTmemCols = 256;    // TMEM columns per CTA (two CTAs per SM)
+// TMEM columns: key products 0 .. 79 (zero term in 0, hi in 16 .. 47, lo in 48 .. 79), value
+// products 112 .. 255 (zero terms in 112 .. 115, outputs in 128 .. 255)
+constexpr int kTmemKz = 0, kTmemKhi = 16, kTmemKlo = 48;
+constexpr int kTmemV = 112, kTmemZv = 112, kTmemOut = 128;
+constexpr int kKRows = 80;    // key B tile rows
+constexpr float kRefSlack = 14.f;   // largest log2 of p before the row's reference moves
+constexpr int kVRows = 144;   // value B tile rows
 
 // Byte offset of element (row r, k) of an operand tile of `rows` rows in the K-major
 // no-swizzle layout: K = 16 steps of rows x 32 bytes; inside a step, 8-row core matrices of
@@ -70,10 +93,10 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective; no wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -82,7 +105,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld1_nowait(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32_nowait(taddr, r);
+  tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -103,6 +145,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ __half2 bits_h2(uint32_t x) {
+  __half2 h;
+  memcpy(&h, &x, 4);
+  return h;
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  uint32_t x;
+  memcpy(&x, &h, 4);
+  return x;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo_elem, float hi_elem) {
+  return h2_bits(__floats2half2_rn(lo_elem, hi_elem));
+}
 
 // x split into two fp16 whose sum is x to 22 bits, packed (hi, lo) for two adjacent K.
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
@@ -112,30 +176,49 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
 }
 
+// Four code pairs of one 32-bit code word (both halves: two adjacent K of one tile row),
+// the pair u at bit BITS * u of `w` in each half: the hi / lo parts of c * s for the scale
+// pair `s2`, stored `step` bytes apart.  1024 + c is an fp16 with c in its low mantissa bits,
+// so one subtraction gives c exactly; hi = fp16(c s) and lo = fma(c, s, -hi) are exact.
+template <int BITS>
+__device__ __forceinline__ void cs_pairs4(uint32_t w, uint32_t s2, uint8_t* dh, uint8_t* dl, int step) {
+  constexpr uint32_t kMask = ((1u << BITS) - 1u) * 0x10001u;
+  const __half2 s = bits_h2(s2);
+  const __half2 k1024 = __float2half2_rn(1024.f);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const __half2 c = __hsub2(bits_h2(((w >> (BITS * u)) & kMask) | 0x64006400u), k1024);
+    const __half2 hi = __hmul2(c, s);
+    const __half2 lo = __hfma2(c, s, __hneg2(hi));
+    *reinterpret_cast<uint32_t*>(dh + u * step) = h2_bits(hi);
+    *reinterpret_cast<uint32_t*>(dl + u * step) = h2_bits(lo);
+  }
+}
+
 struct TcSmem {
   int aq;      // fp16 [128 rows][128 positions]
-  int bk_hi;   // fp16 [32 tokens][128 positions]
-  int bk_lo;
+  int bk;      // fp16 [80 rows][128 positions] (zero row, hi, lo)
   int ap;      // fp16 [128 rows][32 tokens]
-  int bv_hi;   // fp16 [128 channels][32 tokens]
-  int bv_lo;
-  int qnat;    // fp32 [64 rows][128], aliases bk_hi .. bv_lo (segment setup only)
+  int bv;      // two buffers of fp16 [144 rows][32 tokens] (zero rows, values)
+  int qnat;    // fp32 [64 rows][128], aliases bk, ap and the start of the first value buffer
   int ring;    // [kTcSlots][R]
   int perm;    // 128 bytes
   int bars;    // uint64 full[kTcSlots], mma_k, mma_v; uint32 TMEM address
   int total;
 };
 
+constexpr int kStepK = kKRows * 32;     // bytes of one K = 16 step of the key tile
+constexpr int kStepV = kVRows * 32;     // of the value tile
+constexpr int kVBuf = 2 * kStepV;
+
 __host__ __device__ __forceinline__ TcSmem tc_smem(int R) {
   TcSmem m;
   m.aq = 0;
-  m.bk_hi = m.aq + 128 * 128 * 2;
-  m.bk_lo = m.bk_hi + 32 * 128 * 2;
-  m.ap = m.bk_lo + 32 * 128 * 2;
-  m.bv_hi = m.ap + 128 * 32 * 2;
-  m.bv_lo = m.bv_hi + 128 * 32 * 2;
-  m.qnat = m.bk_hi;   // 32 KB inside the 40 KB of tiles
-  m.ring = m.bv_lo + 128 * 32 * 2;
+  m.bk = m.aq + 128 * 128 * 2;
+  m.ap = m.bk + 8 * kStepK;
+  m.bv = m.ap + 128 * 32 * 2;
+  m.qnat = m.bk;   // 32 KB: bk (20 KB), ap (8 KB), the first 4 KB of value buffer 0
+  m.ring = m.bv + 2 * kVBuf;
   m.perm = m.ring + kTcSlots * ((R + 127) / 128 * 128);
   m.bars = m.perm + 128;
   m.total = m.bars + 128;
@@ -148,17 +231,14 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int R = record_bytes_of<BHI, BLO, NHS>();
   constexpr int WH = NHS * BHI / 2;                   // key-code words per lane, salient block
-  constexpr int NW = WH + (8 - NHS) * BLO / 2;        // key-code words per lane
   constexpr int KC = key_code_bytes<BHI, BLO, NHS>();
   const TcSmem sm = tc_smem(R);
   const int G = g.rows;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tq = lane & 3;
   uint8_t* aq = smem + sm.aq;
-  uint8_t* bkh = smem + sm.bk_hi;
-  uint8_t* bkl = smem + sm.bk_lo;
+  uint8_t* bk = smem + sm.bk;
   uint8_t* ap = smem + sm.ap;
-  uint8_t* bvh = smem + sm.bv_hi;
-  uint8_t* bvl = smem + sm.bv_lo;
   float* qnat = reinterpret_cast<float*>(smem + sm.qnat);
   uint8_t* perm = smem + sm.perm;
   constexpr int kSlotBytes = (R + 127) / 128 * 128;
@@ -187,16 +267,20 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;   // this warp's TMEM lanes
-  const uint32_t t_logit = tmem + lane_base, t_out = tmem + lane_base + kTmemOut;
+  const uint32_t t_row = tmem + lane_base;
   volatile int* fail = &fail_sh;
   const float qscale = g.scale * kLog2e;
-  constexpr uint32_t kIdescK = mma_idesc(32), kIdescV = mma_idesc(128);
-  // records staged so far / taken so far (ring position), MMA batches committed so far
+  constexpr uint32_t kIdescK = mma_idesc(kKRows), kIdescV = mma_idesc(kVRows);
+  // operand descriptors of the first K step of each tile (a step further is a fixed offset)
+  const uint64_t dq0 = tile_desc(aq), dk0 = tile_desc(bk), dp0 = tile_desc(ap), dv0 = tile_desc(smem + sm.bv);
+  // TMEM lane tid holds query row rr = tid % 64 for the tokens [16 kc, 16 kc + 16) of every
+  // group: the two copies of a row are independent partials, merged at the segment's end
+  const int kc = warp >> 1, rr = tid & 63;
+  // records staged so far / taken so far (ring position), commits to bar_k / bar_v so far
   uint32_t nis = 0, ncons = 0, nk = 0, nv = 0;
   // bounded wait for phase `parity` of `bar`; gives up (error bit, CTA-wide stop) after
   // `limit` rounds: g.wait_limit for the staged records, kDecodeWaitLimit for the tensor
-  // cores' commits (they always arrive; the bound only guards against a hang, and a product
-  // still in flight must not outlive the TMEM it writes)
+  // cores' commits (they always arrive; the bound only guards against a hang)
   auto wait_bar = [&](uint64_t* bar, uint32_t parity, uint32_t limit) -> bool {
     uint32_t spins = 0;
     while (!mbar_try_wait(bar, parity)) {
@@ -218,9 +302,10 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
     const bool stage = unit != g.skip_unit;   // false only under the timeout test hook
     int issued = 0;
+    bool mma_issued = false;   // thread 0: a product of this segment may still be in flight
     // thread 0: stage the segment's next record into its slot (the slot's previous record
-    // has been consumed: records are taken in order and a slot is refilled after its
-    // record's tiles were built)
+    // has been consumed: records are taken in order and a slot is refilled once the tiles of
+    // its record were built)
     auto issue_next = [&]() {
       if (*fail || !stage || issued >= ngr) return;
       const uint32_t slot = nis % kTcSlots;
@@ -256,208 +341,266 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       zero_pruned_slices(g, qnat, perm, pmask, tid, kTcThreads);
       __syncthreads();
     }
-    // A = Q (row tid, positions in order; bf16 -> fp16 is exact in fp16's normal range)
-    {
-      const int r = tid;
-#pragma unroll 4
-      for (int j = 0; j < kHeadDim; j += 2) {
-        const float x0 = r < G ? qnat[r * kHeadDim + (perm[j] & (kHeadDim - 1))] : 0.f;
-        const float x1 = r < G ? qnat[r * kHeadDim + (perm[j + 1] & (kHeadDim - 1))] : 0.f;
-        const uint32_t w = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(x0))) |
-                           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(x1))) << 16);
-        *reinterpret_cast<uint32_t*>(aq + tile_off(128, r, j)) = w;
+    // A = Q (positions in order; bf16 -> fp16 is exact in fp16's normal range), one 16-byte
+    // chunk of 8 positions per item; rows 64..127 repeat rows 0..63; rows >= G are zero
+    for (int item = tid; item < 128 * 16; item += kTcThreads) {
+      const int r = item >> 4, c8 = item & 15, src = r & 63;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (src < G) {
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const int j = 8 * c8 + 2 * k2;
+          w[k2] = pack_f16(qnat[src * kHeadDim + (perm[j] & (kHeadDim - 1))],
+                           qnat[src * kHeadDim + (perm[j + 1] & (kHeadDim - 1))]);
+        }
       }
+      *reinterpret_cast<uint4*>(aq + tile_off(128, r, 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    __syncthreads();   // qnat is dead: the fixed rows of the tiles it overlapped
+    // rows 0..15 of the key tile's 8 steps and of both value buffers' 2 steps: zero, except
+    // row 4 of the value tiles, all ones (its product is the row's softmax denominator)
+    for (int i = tid; i < 12 * 32; i += kTcThreads) {
+      const int step = i >> 5, j = i & 31;
+      uint8_t* base = step < 8 ? bk + step * kStepK : smem + sm.bv + (step - 8) * kStepV;
+      const uint32_t fill = (step >= 8 && (j == 4 || j == 12)) ? 0x3C003C00u : 0u;
+      reinterpret_cast<uint4*>(base)[j] = make_uint4(fill, fill, fill, fill);
+    }
+    // this lane's P row outside its tokens stays zero
+#pragma unroll
+    for (int c8 = 0; c8 < 2; ++c8)
+      *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * (1 - kc) + 8 * c8)) = make_uint4(0u, 0u, 0u, 0u);
     proxy_fence();
-    __syncthreads();   // qnat (aliasing the tiles) is no longer needed
+    if (tid == 0 && ngr > 0 && !*fail) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
+    // the first record is in (or the CTA stops: a decision every thread takes alike, from a
+    // barrier's reduction, since a wait that runs out sets the flag at any time)
+    const bool stop0 = __syncthreads_or(*fail);
 
-    float m_row = -INFINITY, l_row = 0.f;
-    bool out_live = false;   // the TMEM output rows hold a value MMA's result
+    float m_row = -INFINITY;
+    bool out_live = false;   // the TMEM output rows hold a value product's result
     const int nitems = ngr + (seg_resid ? 1 : 0);
-    for (int it = 0; it < nitems && !*fail; ++it) {
-      const bool resid_item = it == ngr;
-      const int tok0 = resid_item ? seg.ng * kGroup : (seg.lo + it) * kGroup;
-      const int ntok = resid_item ? seg.nr : kGroup;
-      const uint8_t* rec = nullptr;
-      if (!resid_item) {
-        if (tid == 0) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
-        __syncthreads();
-        if (*fail) break;
-        rec = ring + (ncons % kTcSlots) * kSlotBytes;
-      }
-      // ---- key tiles: x = code * s + z (or the bf16 residual key), split hi / lo
-      if (!resid_item) {
-        const uint16_t* ks = reinterpret_cast<const uint16_t*>(rec + KC);
-        const uint16_t* kz = reinterpret_cast<const uint16_t*>(rec + KC + 256);
-        for (int item = tid; item < NW * 32; item += kTcThreads) {
-          const int w = item >> 5, L = item & 31, gq = L >> 2, tq = L & 3;
-          const bool hiw = w < WH;
-          constexpr int kBitsHi = BHI, kBitsLo = BLO;
-          const int bits = hiw ? kBitsHi : kBitsLo, mslots = 16 / bits, cmask = (1 << bits) - 1;
-          const uint32_t word = reinterpret_cast<const uint32_t*>(rec)[w * 32 + L];
-          const int n0 = (hiw ? w : w - WH) * mslots;
-          for (int i = 0; i < mslots; ++i) {
-            const int n = n0 + i, u = n & 3, cc = (n >> 2) & 1;
-            const int sigma = (n >> 3) + (hiw ? 0 : NHS);
-            const int p0 = 16 * sigma + 2 * tq + 8 * cc, tau = gq + 8 * u;
-            const float c0 = static_cast<float>((word >> (bits * i)) & cmask);
-            const float c1 = static_cast<float>((word >> (16 + bits * i)) & cmask);
-            const int si = kscale_index(p0);   // p0 + 1 is element si + 1
-            const float x0 = fmaf(c0, __half2float(__ushort_as_half(ks[si])), __half2float(__ushort_as_half(kz[si])));
-            const float x1 =
-                fmaf(c1, __half2float(__ushort_as_half(ks[si + 1])), __half2float(__ushort_as_half(kz[si + 1])));
-            uint32_t hi, lo;
-            split_pair(x0, x1, hi, lo);
-            *reinterpret_cast<uint32_t*>(bkh + tile_off(32, tau, p0)) = hi;
-            *reinterpret_cast<uint32_t*>(bkl + tile_off(32, tau, p0)) = lo;
+    // ---- key tile of item i (a record in `rec`, or the residual window): hi / lo of c * s
+    // and the zero row
+    auto build_keys = [&](int i, const uint8_t* rec) {
+      if (i < ngr) {
+        const uint32_t* recw = reinterpret_cast<const uint32_t*>(rec);
+        const uint32_t* ks2 = reinterpret_cast<const uint32_t*>(rec + KC);
+        // unit j = 4 warp + jj: code slots n = 4 j' .. 4 j' + 3 of its block (j' = j, or j - 2 NHS
+        // in the low block), i.e. slice j / 2, half j % 2, tokens gq + 8 u
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = 4 * warp + jj, sigma = j >> 1, cc = j & 1;
+          const uint32_t s2 = ks2[(tq * 4 + (sigma >> 1)) * 4 + 2 * cc + (sigma & 1)];
+          uint8_t* dh = bk + sigma * kStepK + 2 * 256 + cc * 128 + 4 * lane;   // row 16 + tau
+          uint8_t* dl = dh + 4 * 256;                                           // row 48 + tau
+          if (j < 2 * NHS) {
+            constexpr int m = 16 / BHI;
+            const uint32_t w = recw[((4 * j) / m) * 32 + lane] >> (BHI * ((4 * j) % m));
+            cs_pairs4<BHI>(w, s2, dh, dl, 256);
+          } else {
+            constexpr int m = 16 / BLO;
+            const int jl = j - 2 * NHS;
+            const uint32_t w = recw[(WH + (4 * jl) / m) * 32 + lane] >> (BLO * ((4 * jl) % m));
+            cs_pairs4<BLO>(w, s2, dh, dl, 256);
           }
+        }
+        if (tid >= 64) {   // zero row: positions 2i, 2i + 1
+          const int p0 = 2 * (tid - 64);
+          const uint32_t z2 = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kscale_index(p0) >> 1];
+          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 0, p0)) = z2;
         }
       } else {
         const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
         for (int item = tid; item < kGroup * (kHeadDim / 2); item += kTcThreads) {
           const int tau = item >> 6, p0 = 2 * (item & 63);
           float x0 = 0.f, x1 = 0.f;
-          if (tau < ntok) {
+          if (tau < seg.nr) {
             x0 = bf16_bits_to_float(rk[tau * kHeadDim + (perm[p0] & (kHeadDim - 1))]);
             x1 = bf16_bits_to_float(rk[tau * kHeadDim + (perm[p0 + 1] & (kHeadDim - 1))]);
           }
           uint32_t hi, lo;
           split_pair(x0, x1, hi, lo);
-          *reinterpret_cast<uint32_t*>(bkh + tile_off(32, tau, p0)) = hi;
-          *reinterpret_cast<uint32_t*>(bkl + tile_off(32, tau, p0)) = lo;
+          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 16 + tau, p0)) = hi;
+          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 48 + tau, p0)) = lo;
         }
+        if (tid >= 64) *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 0, 2 * (tid - 64))) = 0u;
       }
-      proxy_fence();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int s = 0; s < kHeadDim / 16; ++s) {
-          const uint64_t da = tile_desc(aq + s * 128 * 32);
-          tc_mma(tmem, da, tile_desc(bkh + s * 32 * 32), kIdescK, s > 0);
-          tc_mma(tmem, da, tile_desc(bkl + s * 32 * 32), kIdescK, true);
-        }
-        tc_commit(bar_k);
-      }
-      // ---- logits of this thread's row
-      if (tid == 0) wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
-      ++nk;
-      __syncthreads();
-      if (*fail) break;
-      tc_fence_after();
-      float lg[32];
-      tmem_ld32(t_logit, lg);
-      const int r = tid;
-      const int lim = r < G ? vis_base + r / g.G : 0;   // tokens this row sees
-      float mx = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const bool vis = t < ntok && tok0 + t < lim;
-        lg[t] = vis ? lg[t] * qscale : -INFINITY;
-        mx = fmaxf(mx, lg[t]);
-      }
-      // ---- the previous group's value products are done with P, V and the outputs
-      if (nv > 0) {
-        if (tid == 0) wait_bar(bar_v, (nv - 1) & 1u, kDecodeWaitLimit);
-        __syncthreads();
-        if (*fail) break;
-        tc_fence_after();
-      }
-      // lazy reference: raise it to max + 4 when a logit exceeds it, rescaling the row
-      const bool raise = mx > m_row;
-      float alpha = 1.f;
-      if (raise) {
-        const float mnew = mx + 4.f;
-        alpha = m_row == -INFINITY ? 0.f : ex2(m_row - mnew);
-        l_row *= alpha;
-        m_row = mnew;
-      }
-      if (out_live && __any_sync(0xffffffffu, raise && alpha != 1.f)) {   // warp-collective TMEM traffic
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float o[32];
-          tmem_ld32(t_out + 32 * c4, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(t_out + 32 * c4, o);
-        }
-      }
-      // P row (fp16) for the value product
-#pragma unroll
-      for (int t = 0; t < 32; t += 2) {
-        const float p0 = lg[t] == -INFINITY ? 0.f : ex2(lg[t] - m_row);
-        const float p1 = lg[t + 1] == -INFINITY ? 0.f : ex2(lg[t + 1] - m_row);
-        l_row += p0 + p1;
-        const uint32_t w = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(p0))) |
-                           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(p1))) << 16);
-        *reinterpret_cast<uint32_t*>(ap + tile_off(128, r, t)) = w;
-      }
-      // ---- value tiles: v = code * s_v + z_v (or the bf16 residual value), split hi / lo
-      if (!resid_item) {
+    };
+    // ---- value tile of item i into buffer i % 2: fp16(c * s_v) and the zero rows
+    auto build_values = [&](int i, const uint8_t* rec) {
+      uint8_t* bv = smem + sm.bv + (i & 1) * kVBuf;
+      if (i < ngr) {
         const uint8_t* vc = rec + KC + 512;
-        const uint16_t* vs = reinterpret_cast<const uint16_t*>(rec + KC + 1536);
-        const uint16_t* vz = reinterpret_cast<const uint16_t*>(rec + KC + 1792);
-        for (int item = tid; item < 8 * 32; item += kTcThreads) {
-          const int mw = item >> 5, L = item & 31, gq = L >> 2, tq = L & 3;
-          const uint32_t word = *reinterpret_cast<const uint32_t*>(vc + vword_offset(mw, L));
+        const uint32_t* vs2 = reinterpret_cast<const uint32_t*>(rec + KC + 1536);
+        // warp w: code words m = 2w, 2w + 1 (channels 16 m + gq + 8 r), channel group w; the
+        // scale pair of tokens (8 p + 2 tq, + 1)
+        uint32_t s2[4];
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr)
+        for (int p = 0; p < 4; ++p) s2[p] = vs2[(4 * p + tq) * 4 + warp];
+        const uint2 wv = *reinterpret_cast<const uint2*>(vc + vword_offset(2 * warp, lane));   // m = 2w, 2w + 1
 #pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-              const int qq = rr * 4 + pp, ch = 16 * mw + gq + 8 * rr, jg = ch >> 5;
-              const int t0 = 2 * tq + 8 * pp;
-              const float c0 = static_cast<float>((word >> (2 * qq)) & 3u);
-              const float c1 = static_cast<float>((word >> (16 + 2 * qq)) & 3u);
-              const float x0 = fmaf(c0, __half2float(__ushort_as_half(vs[vscale_index(t0, jg)])),
-                                    __half2float(__ushort_as_half(vz[vzero_index(t0, jg)])));
-              const float x1 = fmaf(c1, __half2float(__ushort_as_half(vs[vscale_index(t0 + 1, jg)])),
-                                    __half2float(__ushort_as_half(vz[vzero_index(t0 + 1, jg)])));
-              uint32_t hi, lo;
-              split_pair(x0, x1, hi, lo);
-              *reinterpret_cast<uint32_t*>(bvh + tile_off(128, ch, t0)) = hi;
-              *reinterpret_cast<uint32_t*>(bvl + tile_off(128, ch, t0)) = lo;
+        for (int mm = 0; mm < 2; ++mm) {
+          const int m = 2 * warp + mm;
+          const uint32_t w = mm ? wv.y : wv.x;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            uint8_t* dh = bv + (2 + 2 * m + r) * 256 + 4 * lane;   // row 16 + channel
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const __half2 cv = __hsub2(bits_h2(((w >> (2 * (4 * r + p))) & 0x00030003u) | 0x64006400u),
+                                         __float2half2_rn(1024.f));
+              *reinterpret_cast<uint32_t*>(dh + (p >> 1) * kStepV + (p & 1) * 128) =
+                  h2_bits(__hmul2(cv, bits_h2(s2[p])));
             }
+          }
+        }
+        if (tid < 64) {   // zero rows: channel group jg, tokens 2 tp, 2 tp + 1
+          const int jg = tid >> 4, tp = tid & 15, t0 = 2 * tp;
+          const uint32_t z2 = reinterpret_cast<const uint32_t*>(rec + KC + 1792)[vzero_index(t0, jg) >> 1];
+          *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, jg, t0)) = z2;
         }
       } else {
         const uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
         for (int item = tid; item < kHeadDim * (kGroup / 2); item += kTcThreads) {
           const int ch = item >> 4, t0 = 2 * (item & 15);
-          const float x0 = t0 < ntok ? bf16_bits_to_float(rv[t0 * kHeadDim + ch]) : 0.f;
-          const float x1 = t0 + 1 < ntok ? bf16_bits_to_float(rv[(t0 + 1) * kHeadDim + ch]) : 0.f;
-          uint32_t hi, lo;
-          split_pair(x0, x1, hi, lo);
-          *reinterpret_cast<uint32_t*>(bvh + tile_off(128, ch, t0)) = hi;
-          *reinterpret_cast<uint32_t*>(bvl + tile_off(128, ch, t0)) = lo;
+          const float x0 = t0 < seg.nr ? bf16_bits_to_float(rv[t0 * kHeadDim + ch]) : 0.f;
+          const float x1 = t0 + 1 < seg.nr ? bf16_bits_to_float(rv[(t0 + 1) * kHeadDim + ch]) : 0.f;
+          *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, 16 + ch, t0)) = pack_f16(x0, x1);
         }
+        if (tid < 64) *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, tid >> 4, 2 * (tid & 15))) = 0u;
+      }
+    };
+    auto issue_keys = [&]() {   // thread 0: the key products of the tile just built
+#pragma unroll
+      for (int s = 0; s < kHeadDim / 16; ++s)
+        tc_mma(tmem + kTmemKz, dq0 + s * (128 * 32 >> 4), dk0 + s * (kStepK >> 4), kIdescK, s > 0);
+      tc_commit(bar_k);
+      mma_issued = true;
+    };
+
+    // Pipeline: item i's value tile is built while its key products run; after their commit
+    // (which covers every earlier product) the softmax of item i and the key tile of item
+    // i + 1 are written; then one thread issues the value products of i and the key products
+    // of i + 1 together.
+    if (nitems > 0 && !stop0) {
+      build_keys(0, ring + (ncons % kTcSlots) * kSlotBytes);
+      proxy_fence();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        issue_keys();
+      }
+    }
+    for (int it = 0; it < nitems && !stop0; ++it) {
+      const bool resid_item = it == ngr;
+      const int tok0 = resid_item ? seg.ng * kGroup : (seg.lo + it) * kGroup;
+      const int ntok = resid_item ? seg.nr : kGroup;
+      // ---- value tile (this buffer's last reader, the value products two items back,
+      // completed before the previous key commit)
+      build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);   // (the ring is not read for the residual)
+      // ---- every thread: the key products (and with them every earlier product) are done
+      wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
+      ++nk;
+      if (!resid_item) ++ncons;   // the ring position names the next record's slot
+      tc_fence_after();
+      // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
+      float sv[16];
+      float zk;
+      {
+        uint32_t rh[16], rl[16], zraw;
+        tmem_ld16_nowait(t_row + kTmemKhi + 16 * kc, rh);
+        tmem_ld16_nowait(t_row + kTmemKlo + 16 * kc, rl);
+        tmem_ld1_nowait(t_row + kTmemKz, zraw);
+        tmem_wait_ld();
+        zk = __uint_as_float(zraw);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
+      }
+      // tokens 16 kc + t of the group this row sees: t < nvis
+      const int lim = rr < G ? vis_base + rr / g.G : 0;
+      const int nvis = min(ntok, lim - tok0) - 16 * kc;
+      if (nvis < 16) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          if (t >= nvis) sv[t] = -INFINITY;
+      }
+      float mxr = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) mxr = fmaxf(mxr, sv[t]);
+      const float mx = (mxr + zk) * qscale;   // -inf when no token is visible
+      // reference m of the row: the first visible logit's group maximum, moved up only when a
+      // logit would give p above 2^kRefSlack (fp16 holds p up to 65504; the accumulators are
+      // fp32), so the accumulators in TMEM are rescaled almost never; a row that has seen no
+      // token has zero accumulators and needs no rescale
+      bool rescale = false;
+      float alpha = 1.f;
+      if (mx > m_row + kRefSlack) {
+        rescale = m_row != -INFINITY;
+        if (rescale) alpha = ex2(m_row - mx);
+        m_row = mx;
+      }
+      if (out_live && __any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM traffic
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float o[32];
+          tmem_ld32(t_row + kTmemOut + 32 * c4, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_row + kTmemOut + 32 * c4, o);
+        }
+        uint32_t zr[8];
+        tmem_ld8_nowait(t_row + kTmemZv, zr);   // zero terms and the denominator
+        tmem_wait_ld();
+        float zf[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zf[i] = __uint_as_float(zr[i]) * alpha;
+        tmem_st8(t_row + kTmemZv, zf);
+      }
+      // P (fp16): p = 2^(logit * scale - m), 0 for a hidden token (and for all while the row
+      // has seen none), 8 tokens per 16-byte store
+      const float off = m_row == -INFINITY ? -INFINITY : zk * qscale - m_row;
+#pragma unroll
+      for (int c8 = 0; c8 < 2; ++c8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const int t = 8 * c8 + 2 * k2;
+          w[k2] = pack_f16(ex2(fmaf(sv[t], qscale, off)), ex2(fmaf(sv[t + 1], qscale, off)));
+        }
+        *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // ---- the next item's key tile (this item's key products have completed; every thread
+      // waits for the record itself)
+      const bool next = it + 1 < nitems;
+      if (next) {
+        if (it + 1 < ngr) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
+        build_keys(it + 1, ring + (ncons % kTcSlots) * kSlotBytes);
       }
       proxy_fence();
       tc_fence_before();
-      __syncthreads();   // the record's slot is free again; tiles and rescales are in place
-      if (!resid_item) ++ncons;   // every thread: the ring position names the next record's slot
+      // P, the value tile, any rescale and the next key tile are in place; every thread is done
+      // with this item's record
+      if (__syncthreads_or(*fail)) break;
       if (tid == 0) {
         tc_fence_after();
         if (!resid_item) issue_next();
-#pragma unroll 1
-        for (int s = 0; s < kGroup / 16; ++s) {
-          const uint64_t da = tile_desc(ap + s * 128 * 32);
-          tc_mma(tmem + kTmemOut, da, tile_desc(bvh + s * 128 * 32), kIdescV, out_live || s > 0);
-          tc_mma(tmem + kTmemOut, da, tile_desc(bvl + s * 128 * 32), kIdescV, true);
-        }
-        tc_commit(bar_v);
+        const uint64_t dv = dv0 + (it & 1) * (kVBuf >> 4);
+#pragma unroll
+        for (int s = 0; s < kGroup / 16; ++s)
+          tc_mma(tmem + kTmemV, dp0 + s * (128 * 32 >> 4), dv + s * (kStepV >> 4), kIdescV, out_live || s > 0);
+        if (next) issue_keys();
       }
-      ++nv;
       out_live = true;
     }
-    // ---- the segment's last value products (waited for even after a stop: TMEM and the
-    // tiles must be idle before they are read or reused), then this row's partial
-    if (nv > 0) {
-      if (tid == 0)
-        for (uint32_t spins = 0; spins < kDecodeWaitLimit && !mbar_try_wait(bar_v, (nv - 1) & 1u); ++spins) {
-        }
-      __syncthreads();
-      tc_fence_after();
+    // ---- every product of the segment completes (waited for even after a stop: TMEM and
+    // the tiles must be idle before they are read or reused), then this row's partial
+    if (tid == 0 && mma_issued) {
+      tc_commit(bar_v);
+      for (uint32_t spins = 0; spins < kDecodeWaitLimit && !mbar_try_wait(bar_v, nv & 1u); ++spins) {
+      }
     }
+    if (__syncthreads_or(tid == 0 && mma_issued)) ++nv;
+    tc_fence_after();
     if (*fail && tid == 0) {   // let staged copies land before the shared memory is reused
       for (; ncons < nis; ++ncons) {
         const uint32_t slot = ncons % kTcSlots;
@@ -466,21 +609,63 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         }
       }
     }
+    // merge the two copies of each row (shared memory of the idle A and key tiles):
+    // M = max(m0, m1), weights f = 2^(m - M), partial (M, f0 l0 + f1 l1, f0 O0 + f1 O1) with
+    // O = the outputs plus the zero term of their channel group and l = the ones-row product
     {
-      float* o = partial_slot(ws, unit, G) + tid * kPartialStride;
-      const bool live = tid < G && out_live && m_row != -INFINITY && !*fail;
+      constexpr int kXRow = kHeadDim + 4;
+      float* xch = reinterpret_cast<float*>(smem);          // [64][kXRow]: copy 1's weighted (l, O)
+      float* msh = xch + 64 * kXRow;                         // [128]: every lane's m
+      const bool live = out_live && !*fail;
+      const float m_me = live ? m_row : -INFINITY;
+      msh[tid] = m_me;
+      __syncthreads();
+      const float M = fmaxf(msh[rr], msh[rr + 64]);
+      const float f = m_me == -INFINITY ? 0.f : ex2(m_me - M);
+      float zv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) zv[i] = 0.f;
+      if (out_live) {
+        uint32_t zr[8];
+        tmem_ld8_nowait(t_row + kTmemZv, zr);   // warp-collective
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zv[i] = __uint_as_float(zr[i]);
+      }
+      float* mine = xch + rr * kXRow;
+      if (kc == 1) mine[0] = f * zv[4];
 #pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
-        if (out_live) tmem_ld32(t_out + 32 * c4, v);   // warp-collective
-        if (tid < G) {
+        if (out_live) {
+          tmem_ld32(t_row + kTmemOut + 32 * c4, v);   // warp-collective
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[2 + 32 * c4 + i] = live ? v[i] : 0.f;
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-      }
-      if (tid < G) {
-        o[0] = live ? m_row : -INFINITY;
-        o[1] = live ? l_row : 0.f;
+        if (kc == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(mine + 4 + 32 * c4 + i) =
+                make_float4(f * (v[i] + zv[c4]), f * (v[i + 1] + zv[c4]), f * (v[i + 2] + zv[c4]),
+                            f * (v[i + 3] + zv[c4]));
+        }
+        __syncthreads();
+        if (kc == 0 && rr < G) {
+          float* o = partial_slot(ws, unit, G) + rr * kPartialStride;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(mine + 4 + 32 * c4 + i);
+            o[2 + 32 * c4 + i] = f * (v[i] + zv[c4]) + x.x;
+            o[3 + 32 * c4 + i] = f * (v[i + 1] + zv[c4]) + x.y;
+            o[4 + 32 * c4 + i] = f * (v[i + 2] + zv[c4]) + x.z;
+            o[5 + 32 * c4 + i] = f * (v[i + 3] + zv[c4]) + x.w;
+          }
+          if (c4 == 3) {
+            o[0] = M;
+            o[1] = f * zv[4] + mine[0];
+          }
+        }
       }
     }
     tc_fence_before();
@@ -509,13 +694,23 @@ cudaError_t launch_tc_t(const Geometry& g, const uint16_t* q, const pnmix_cache&
   if (wave == 0) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm.total);
     if (e != cudaSuccess) return e;
-    int sms = 148, occ = 1;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // two CTAs per SM need the largest shared-memory carveout
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTcThreads, sm.total);
-    if (e != cudaSuccess) return e;
-    // TMEM: kTmemCols columns per CTA, 512 per SM
-    if (occ > 512 / kTmemCols) occ = 512 / kTmemCols;
+    // CTAs per SM: what TMEM (512 columns per SM), shared memory and registers allow.  (The
+    // runtime's occupancy query answers one for this kernel; two are resident, measured.)
+    int sms = 148, smem_sm = 0, reserved = 0;
+    cudaFuncAttributes fa;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess ||
+        (e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
+      return e;
+    const int per_block = sm.total + static_cast<int>(fa.sharedSizeBytes) + reserved;
+    const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+    int occ = 512 / kTmemCols;
+    occ = min(occ, smem_sm / per_block);
+    occ = min(occ, 65536 / (regs_warp * (kTcThreads / 32)));
     wave = sms * (occ > 0 ? occ : 1);
     if (cacheable) wave_cache[dev].store(wave, std::memory_order_relaxed);
   }

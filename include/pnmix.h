@@ -211,14 +211,18 @@ typedef struct {
  * above; they differ in speed.  The choice is part of the configuration, so it costs no
  * host work per call.
  *   PNMIX_DECODE_AUTO   the faster tensor-core kernel for the shape (one role per warp for
- *                       up to 4 query rows per KV head, warp pairs above).
+ *                       up to 4 query rows per KV head, warp pairs up to 8, warps of 8 rows
+ *                       up to 32, PNMIX_DECODE_TC from 33 rows on).
  *   PNMIX_DECODE_SIMT   CUDA cores only (a baseline): one query per sequence and no query
  *                       pruning (PNMIX_ERR_UNSUPPORTED otherwise).
  *   PNMIX_DECODE_MMA    tensor cores, every warp scores and accumulates its own groups.
  *   PNMIX_DECODE_PAIRS  tensor cores, a key-side and a value-side warp per group stream.
  *   PNMIX_DECODE_TC     5th-generation tensor cores (tcgen05, accumulators in TMEM): each
  *                       group's keys and values dequantized once into shared memory for all
- *                       of a unit's query rows (up to 64); meant for multi-token steps.
+ *                       of a unit's query rows (up to 64); its cost per group hardly depends
+ *                       on the rows, so it is the multi-token kernel.  Keys and values whose
+ *                       32-token group range exceeds 65504 are outside its domain (c * s must
+ *                       be a finite fp16).
  */
 #define PNMIX_DECODE_AUTO 0
 #define PNMIX_DECODE_SIMT 1
@@ -381,10 +385,10 @@ PNMIX_API size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch,
  * pages have no such call; it is the multi-token neighbour of pnmix_decode_attention
  * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 64 (PNMIX_ERR_UNSUPPORTED
  * otherwise; PNMIX_DECODE_SIMT takes T = 1 only).  Up to 8 query rows per KV head (G * T)
- * run on the single-query kernels; 9 to 64 rows on a kernel whose warps each hold 8 rows
- * and share one staging of the packed records, so the cache is read once for all T
- * queries.  A query that sees no token gets zeros.  Workspace from
- * pnmix_workspace_bytes_multi with the same T.
+ * run on the single-query kernels; 9 to 32 rows on a kernel whose warps each hold 8 rows
+ * and share one staging of the packed records, and from 33 rows on the tcgen05 kernel
+ * (PNMIX_DECODE_TC), so the cache is read once for all T queries.  A query that sees no
+ * token gets zeros.  Workspace from pnmix_workspace_bytes_multi with the same T.
  */
 PNMIX_API pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_t* q,
                                                     int n_queries, const pnmix_cache* cache,

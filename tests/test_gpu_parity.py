@@ -695,7 +695,8 @@ def test_fused_append_decode_on_a_full_cache_raises_the_error_bit():
 
 
 # Many query rows per KV head (9 to 64 = G x T): warps holding 8 rows each share one staging
-# of the records; every row must match the oracle's causal attention.
+# of the records (and from 33 rows the automatic choice, the tcgen05 kernel); every row must
+# match the oracle's causal attention.
 @pytest.mark.parametrize("B,Hq,Hkv,L,T,n_prune", [
     (2, 8, 2, 300, 4, 0),       # 16 rows
     (1, 32, 8, 1000, 16, 0),    # 64 rows: the most
@@ -705,8 +706,9 @@ def test_fused_append_decode_on_a_full_cache_raises_the_error_bit():
     (2, 8, 2, 300, 6, 26),      # 24 rows with query-channel pruning
     (1, 16, 4, 2500, 5, 0),     # 20 rows, several split-K segments per unit
 ])
-def test_many_query_rows_per_kv_head_like_the_oracle(B, Hq, Hkv, L, T, n_prune):
-    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + 5 * T, n_prune=n_prune, max_queries=T)
+@pytest.mark.parametrize("kernel", [None, "mma"])   # automatic (tcgen05 from 33 rows), 8-row warps
+def test_many_query_rows_per_kv_head_like_the_oracle(kernel, B, Hq, Hkv, L, T, n_prune):
+    c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + 5 * T, n_prune=n_prune, max_queries=T, kernel=kernel)
     c.prefill()
     for t in range(L, L + T):
         c.append(t)
@@ -727,7 +729,7 @@ def _random_case(seed):
     B = int(rng.integers(1, 4))
     L = int(rng.integers(1, 2500))
     T = int(rng.choice([1, 1, 2, 3])) if G * 3 <= 64 else 1
-    kernel = str(rng.choice(["auto", "mma", "ws"]))
+    kernel = str(rng.choice(["auto", "mma", "ws", "tc"]))
     prune = int(rng.choice([0, 0, 20]))
     slices = 0 if prune else int(rng.choice([0, 0, 2, 4]))
     fused = T == 1 and bool(rng.integers(2))
@@ -778,6 +780,7 @@ def test_random_configurations_like_the_oracle(seed):
     (5, 4, 1, 1000, 8, 4, 2, 2, 0, 0),     # more slices than SMs: CTAs with several groups
     (1, 16, 4, 2500, 8, 4, 2, 5, 26, 0),   # pair pruning, several segments per unit
     (2, 8, 2, 600, 8, 4, 2, 4, 0, 3),      # key-slice pruning
+    (1, 32, 8, 8192, 8, 4, 2, 16, 0, 0),   # 64 rows at 8K: many groups and segments per CTA
 ])
 def test_tcgen05_decode_like_the_oracle(B, Hq, Hkv, L, k, bhi, blo, T, prune, slices):
     c = Case(B, Hq, Hkv, L, k, bhi, blo, extra_tokens=T, seed=L + T + prune, kernel="tc", max_queries=max(T, 2),
