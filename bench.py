@@ -580,6 +580,7 @@ def run_verify(args):
     for t in range(n0, CONTEXT):
         pm.pnmix_append(cfg, k_dev[:, :, t].contiguous(), v_dev[:, :, t].contiguous(), cache)
     del k_dev, v_dev
+    torch.cuda.empty_cache()
     q_all = torch.from_numpy(qm).view(torch.bfloat16).to(dev)
     G = HQ // HKV
     rec = cache.c.record_bytes
