@@ -293,6 +293,40 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     return true;
   };
 
+  // per-thread constants of the tile builds: word, scale and zero offsets inside a record,
+  // destinations inside the tiles.  Key unit j = 4 warp + jj: code slots n = 4 j' .. 4 j' + 3
+  // of its block (j' = j, or j - 2 NHS in the low block), i.e. slice j / 2, half j % 2,
+  // tokens gq + 8 u.  Values: warp w takes code words m = 2w, 2w + 1 (channels 16 m + gq +
+  // 8 r) of channel group w, tokens 8 p + 2 tq, + 1.
+  int k_src[4], k_shift[4], k_s2[4], k_dst[4];
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 4 * warp + jj, sigma = j >> 1, cc = j & 1;
+    k_s2[jj] = (tq * 4 + (sigma >> 1)) * 4 + 2 * cc + (sigma & 1);
+    k_dst[jj] = sigma * kStepK + 2 * 256 + cc * 128 + 4 * lane;   // row 16 + tau
+    if (j < 2 * NHS) {
+      constexpr int m = 16 / BHI;
+      k_src[jj] = ((4 * j) / m) * 32 + lane;
+      k_shift[jj] = BHI * ((4 * j) % m);
+    } else {
+      constexpr int m = 16 / BLO;
+      const int jl = j - 2 * NHS;
+      k_src[jj] = (WH + (4 * jl) / m) * 32 + lane;
+      k_shift[jj] = BLO * ((4 * jl) % m);
+    }
+  }
+  const int kz_src = tid >= 64 ? kscale_index(2 * (tid - 64)) >> 1 : 0;   // zero row: positions 2i, 2i + 1
+  const int kz_dst = tid >= 64 ? tile_off(kKRows, 0, 2 * (tid - 64)) : 0;
+  int v_s2[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) v_s2[p] = (4 * p + tq) * 4 + warp;
+  const int v_src = vword_offset(2 * warp, lane);
+  const int v_dst = (2 + 4 * warp) * 256 + 4 * lane;   // row 16 + channel of m = 2 warp, r = 0
+  // value zero rows: channel group jg = tid / 16, tokens 2 tp, 2 tp + 1 (tp = tid % 16)
+  const int vz_src = tid < 64 ? vzero_index(2 * (tid & 15), tid >> 4) >> 1 : 0;
+  const int vz_dst = tid < 64 ? tile_off(kVRows, tid >> 4, 2 * (tid & 15)) : 0;
+  const int row_query = rr < G ? rr / g.G : -1;   // the query of this lane's row
+
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
     const int b = seg.b, h = seg.h, unit = seg.unit;
     const int vis_base = seg.ng * kGroup + seg.nr - g.tq + 1;   // tokens row 0 sees
@@ -384,30 +418,18 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       if (i < ngr) {
         const uint32_t* recw = reinterpret_cast<const uint32_t*>(rec);
         const uint32_t* ks2 = reinterpret_cast<const uint32_t*>(rec + KC);
-        // unit j = 4 warp + jj: code slots n = 4 j' .. 4 j' + 3 of its block (j' = j, or j - 2 NHS
-        // in the low block), i.e. slice j / 2, half j % 2, tokens gq + 8 u
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          const int j = 4 * warp + jj, sigma = j >> 1, cc = j & 1;
-          const uint32_t s2 = ks2[(tq * 4 + (sigma >> 1)) * 4 + 2 * cc + (sigma & 1)];
-          uint8_t* dh = bk + sigma * kStepK + 2 * 256 + cc * 128 + 4 * lane;   // row 16 + tau
-          uint8_t* dl = dh + 4 * 256;                                           // row 48 + tau
-          if (j < 2 * NHS) {
-            constexpr int m = 16 / BHI;
-            const uint32_t w = recw[((4 * j) / m) * 32 + lane] >> (BHI * ((4 * j) % m));
-            cs_pairs4<BHI>(w, s2, dh, dl, 256);
-          } else {
-            constexpr int m = 16 / BLO;
-            const int jl = j - 2 * NHS;
-            const uint32_t w = recw[(WH + (4 * jl) / m) * 32 + lane] >> (BLO * ((4 * jl) % m));
-            cs_pairs4<BLO>(w, s2, dh, dl, 256);
-          }
+          const uint32_t s2 = ks2[k_s2[jj]];
+          const uint32_t w = recw[k_src[jj]] >> k_shift[jj];
+          uint8_t* dh = bk + k_dst[jj];
+          if (4 * warp + jj < 2 * NHS)
+            cs_pairs4<BHI>(w, s2, dh, dh + 4 * 256, 256);   // hi in row 16 + tau, lo in 48 + tau
+          else
+            cs_pairs4<BLO>(w, s2, dh, dh + 4 * 256, 256);
         }
-        if (tid >= 64) {   // zero row: positions 2i, 2i + 1
-          const int p0 = 2 * (tid - 64);
-          const uint32_t z2 = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kscale_index(p0) >> 1];
-          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 0, p0)) = z2;
-        }
+        if (tid >= 64)
+          *reinterpret_cast<uint32_t*>(bk + kz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kz_src];
       } else {
         const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
         for (int item = tid; item < kGroup * (kHeadDim / 2); item += kTcThreads) {
@@ -422,28 +444,24 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 16 + tau, p0)) = hi;
           *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 48 + tau, p0)) = lo;
         }
-        if (tid >= 64) *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 0, 2 * (tid - 64))) = 0u;
+        if (tid >= 64) *reinterpret_cast<uint32_t*>(bk + kz_dst) = 0u;
       }
     };
     // ---- value tile of item i into buffer i % 2: fp16(c * s_v) and the zero rows
     auto build_values = [&](int i, const uint8_t* rec) {
       uint8_t* bv = smem + sm.bv + (i & 1) * kVBuf;
       if (i < ngr) {
-        const uint8_t* vc = rec + KC + 512;
         const uint32_t* vs2 = reinterpret_cast<const uint32_t*>(rec + KC + 1536);
-        // warp w: code words m = 2w, 2w + 1 (channels 16 m + gq + 8 r), channel group w; the
-        // scale pair of tokens (8 p + 2 tq, + 1)
         uint32_t s2[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) s2[p] = vs2[(4 * p + tq) * 4 + warp];
-        const uint2 wv = *reinterpret_cast<const uint2*>(vc + vword_offset(2 * warp, lane));   // m = 2w, 2w + 1
+        for (int p = 0; p < 4; ++p) s2[p] = vs2[v_s2[p]];
+        const uint2 wv = *reinterpret_cast<const uint2*>(rec + KC + 512 + v_src);   // m = 2w, 2w + 1
 #pragma unroll
         for (int mm = 0; mm < 2; ++mm) {
-          const int m = 2 * warp + mm;
           const uint32_t w = mm ? wv.y : wv.x;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            uint8_t* dh = bv + (2 + 2 * m + r) * 256 + 4 * lane;   // row 16 + channel
+            uint8_t* dh = bv + v_dst + (2 * mm + r) * 256;
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
               const __half2 cv = __hsub2(bits_h2(((w >> (2 * (4 * r + p))) & 0x00030003u) | 0x64006400u),
@@ -453,11 +471,8 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
             }
           }
         }
-        if (tid < 64) {   // zero rows: channel group jg, tokens 2 tp, 2 tp + 1
-          const int jg = tid >> 4, tp = tid & 15, t0 = 2 * tp;
-          const uint32_t z2 = reinterpret_cast<const uint32_t*>(rec + KC + 1792)[vzero_index(t0, jg) >> 1];
-          *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, jg, t0)) = z2;
-        }
+        if (tid < 64)
+          *reinterpret_cast<uint32_t*>(bv + vz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 1792)[vz_src];
       } else {
         const uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
         for (int item = tid; item < kHeadDim * (kGroup / 2); item += kTcThreads) {
@@ -466,7 +481,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           const float x1 = t0 + 1 < seg.nr ? bf16_bits_to_float(rv[(t0 + 1) * kHeadDim + ch]) : 0.f;
           *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, 16 + ch, t0)) = pack_f16(x0, x1);
         }
-        if (tid < 64) *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, tid >> 4, 2 * (tid & 15))) = 0u;
+        if (tid < 64) *reinterpret_cast<uint32_t*>(bv + vz_dst) = 0u;
       }
     };
     auto issue_keys = [&]() {   // thread 0: the key products of the tile just built
@@ -517,7 +532,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
       }
       // tokens 16 kc + t of the group this row sees: t < nvis
-      const int lim = rr < G ? vis_base + rr / g.G : 0;
+      const int lim = row_query >= 0 ? vis_base + row_query : 0;
       const int nvis = min(ntok, lim - tok0) - 16 * kc;
       if (nvis < 16) {
 #pragma unroll
