@@ -81,6 +81,9 @@ def parse():
     ap.add_argument("--profile-decode", action="store_true",
                     help="build the 32K state, then run only --warmup + --steps decode launches "
                          "(small device footprint, for profiler captures); prints no bench line")
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "simt", "mma", "ws", "tc"],
+                    help="with --profile-decode: the decode kernel those launches run (default: the "
+                         "automatic choice, the one the bench times)")
     return ap.parse_args()
 
 
@@ -859,6 +862,8 @@ def main():
     kin, vin, qwin, qs = gen_inputs(seed, CONTEXT, positions)
 
     cfg = pm.Config.make(HQ, HKV, BHI, BLO, K_SALIENT, WINDOW)
+    if args.profile_decode:
+        cfg.decode_kernel = pm.DECODE_KERNELS[args.decode_kernel]
     cache = pm.PNMixCache(cfg, B, CONTEXT + 32, max_context=CONTEXT)
     dev = torch.device("cuda", local)
     out = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)

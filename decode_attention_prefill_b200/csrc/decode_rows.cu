@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kRowsPerWarp = 8;
 constexpr int kRowWarps = kMaxRows / kRowsPerWarp;   // at most 8 warps
-constexpr int kRowSlots = 6;                          // ring of record pairs
+constexpr int kRowSlots = 4;                          // ring of record pairs
 
 // Shared memory of a launch with `nrows` rows per unit (rounded up to whole warps of 8), so
 // that small launches fit several CTAs per SM.
