@@ -2,10 +2,11 @@
 // many query rows per KV head: a multi-token step (speculative verify, chunked decode) with
 // up to 64 rows = G * T.
 //
-// One CTA (one warpgroup, 128 threads) per slice of the work partition (decode_common.cuh);
-// thread r owns query row r, which is TMEM lane r of every accumulator (rows >= G are
-// zero).  A dequantised key is k = c * s + z (code c, fp16 scale s and zero z of its group
-// and position), a value v = c * s_v + z_v.  Per 32-token group record:
+// One CTA of 8 warps per slice of the work partition (decode_common.cuh), two CTAs per SM.
+// Warps 0..3 run the softmax: query row r is TMEM lane r of every accumulator (rows >= G are
+// zero).  Warps 4..7 build the operand tiles from the staged records.  A dequantised key
+// is k = c * s + z (code c, fp16 scale s and zero z of its group and position), a value
+// v = c * s_v + z_v.  Per 32-token group record:
 //
 //   logits  S = Q x K^T = Q x (C s)^T + Q x z:  A = the unit's query rows, fp16 (exact from
 //           bf16), 128 rows x 128 positions, written once per segment.  c * s has at most
@@ -26,21 +27,22 @@
 //           of ones in the value tile, so it sums the same fp16 p as the outputs.
 //   values  O += P x (C_v s_v)^T + P x z_v:  A = P (fp16, 128 rows x 32 tokens), B = one
 //           tile of 144 rows x 32 tokens: rows 0..3 the zero points of the four 32-channel
-//           groups, rows 4..15 zero, rows 16..143 fp16(c s_v) of the 128 channels (one
-//           rounding, exact for codes 0 .. 2: the value side's precision in every decode
-//           kernel); 2 MMAs (N = 144) accumulate the zero terms and the outputs in TMEM.  A
-//           row's result is O[ch] plus the zero term of ch's channel group.
+//           groups, row 4 all ones, rows 5..15 zero, rows 16..143 fp16(c s_v) of the 128
+//           channels (one rounding, exact for codes 0 .. 2: the value side's precision in
+//           every decode kernel); 2 MMAs (N = 144) accumulate the zero terms, the denominator
+//           and the outputs in TMEM.  A row's result is O[ch] plus the zero term of ch's
+//           channel group.
 //
-// Pipeline of one group: build the key tiles; one thread issues the key products and commits
-// them to an mbarrier; meanwhile every thread builds the value tiles (two buffers); after the
-// commit (which also covers every earlier product, so TMEM, P and the value buffer two
-// groups back are idle) the softmax writes P; one thread issues the value products without
-// waiting for them.  The bf16 residual window takes the same path as one more group (its
-// keys split into hi / lo, its values rounded to fp16, zero tiles empty, the tokens past it
-// masked).  The
-// records arrive by TMA bulk copy (no multicast) into a ring of four.  Every wait is
-// bounded.  At the end of a segment each thread writes its row's partial (m, l, O) for the
-// fused combine.  Needs |c s| below 65504 (keys and values whose group range fits fp16).
+// Pipeline of one group: while its key products run, the builder warps write its value tile
+// (two buffers); after the key commit (which also covers every earlier product, so TMEM, P
+// and the value buffer two groups back are idle) the softmax warps write P and the builders
+// the next group's key tile; after one barrier a single thread issues this group's value
+// products and the next group's key products.  The bf16 residual window takes the same
+// path as one more group (its keys split into hi / lo, its values rounded to fp16, zero
+// tiles empty, the tokens past it masked).  The records arrive by TMA bulk copy (no
+// multicast) into a ring of four.  Every wait is bounded.  At the end of a segment the
+// softmax threads write each row's partial (m, l, O) for the fused combine.  Needs |c s|
+// below 65504 (keys and values whose group range fits fp16).
 #include <atomic>
 #include <string.h>
 
@@ -51,7 +53,8 @@
 namespace pnmix {
 namespace {
 
-constexpr int kTcThreads = 128;   // one warpgroup: TMEM lanes 0 .. 127
+constexpr int kTcThreads = 256;   // warps 0..3: softmax (TMEM lanes 0..127); warps 4..7: tile building
+constexpr int kTcHalf = 128;      // threads of one role
 constexpr int kTcSlots = 4;       // record ring
 constexpr int kTmemCols = 256;    // TMEM columns per CTA (two CTAs per SM)
 // TMEM columns: key products 0 .. 79 (zero term in 0, hi in 16 .. 47, lo in 48 .. 79), value
@@ -266,7 +269,11 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;   // this warp's TMEM lanes
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;   // this warp's TMEM lanes
+  // roles: the softmax warps own the TMEM lanes (query rows); the builder warps turn each
+  // record into the key and value tiles; bt / bw are a builder's thread / warp index
+  const bool builder = warp >= 4;
+  const int bt = tid & (kTcHalf - 1), bw = warp & 3;
   const uint32_t t_row = tmem + lane_base;
   volatile int* fail = &fail_sh;
   const float qscale = g.scale * kLog2e;
@@ -275,7 +282,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   const uint64_t dq0 = tile_desc(aq), dk0 = tile_desc(bk), dp0 = tile_desc(ap), dv0 = tile_desc(smem + sm.bv);
   // TMEM lane tid holds query row rr = tid % 64 for the tokens [16 kc, 16 kc + 16) of every
   // group: the two copies of a row are independent partials, merged at the segment's end
-  const int kc = warp >> 1, rr = tid & 63;
+  const int kc = (warp & 3) >> 1, rr = tid & 63;
   // records staged so far / taken so far (ring position), commits to bar_k / bar_v so far
   uint32_t nis = 0, ncons = 0, nk = 0, nv = 0;
   // bounded wait for phase `parity` of `bar`; gives up (error bit, CTA-wide stop) after
@@ -294,14 +301,14 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   };
 
   // per-thread constants of the tile builds: word, scale and zero offsets inside a record,
-  // destinations inside the tiles.  Key unit j = 4 warp + jj: code slots n = 4 j' .. 4 j' + 3
+  // destinations inside the tiles.  Key unit j = 4 bw + jj: code slots n = 4 j' .. 4 j' + 3
   // of its block (j' = j, or j - 2 NHS in the low block), i.e. slice j / 2, half j % 2,
-  // tokens gq + 8 u.  Values: warp w takes code words m = 2w, 2w + 1 (channels 16 m + gq +
-  // 8 r) of channel group w, tokens 8 p + 2 tq, + 1.
+  // tokens gq + 8 u.  Values: builder warp bw takes code words m = 2 bw, 2 bw + 1 (channels
+  // 16 m + gq + 8 r) of channel group bw, tokens 8 p + 2 tq, + 1.
   int k_src[4], k_shift[4], k_s2[4], k_dst[4];
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
-    const int j = 4 * warp + jj, sigma = j >> 1, cc = j & 1;
+    const int j = 4 * bw + jj, sigma = j >> 1, cc = j & 1;
     k_s2[jj] = (tq * 4 + (sigma >> 1)) * 4 + 2 * cc + (sigma & 1);
     k_dst[jj] = sigma * kStepK + 2 * 256 + cc * 128 + 4 * lane;   // row 16 + tau
     if (j < 2 * NHS) {
@@ -315,16 +322,16 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       k_shift[jj] = BLO * ((4 * jl) % m);
     }
   }
-  const int kz_src = tid >= 64 ? kscale_index(2 * (tid - 64)) >> 1 : 0;   // zero row: positions 2i, 2i + 1
-  const int kz_dst = tid >= 64 ? tile_off(kKRows, 0, 2 * (tid - 64)) : 0;
+  const int kz_src = bt >= 64 ? kscale_index(2 * (bt - 64)) >> 1 : 0;   // zero row: positions 2i, 2i + 1
+  const int kz_dst = bt >= 64 ? tile_off(kKRows, 0, 2 * (bt - 64)) : 0;
   int v_s2[4];
 #pragma unroll
-  for (int p = 0; p < 4; ++p) v_s2[p] = (4 * p + tq) * 4 + warp;
-  const int v_src = vword_offset(2 * warp, lane);
-  const int v_dst = (2 + 4 * warp) * 256 + 4 * lane;   // row 16 + channel of m = 2 warp, r = 0
-  // value zero rows: channel group jg = tid / 16, tokens 2 tp, 2 tp + 1 (tp = tid % 16)
-  const int vz_src = tid < 64 ? vzero_index(2 * (tid & 15), tid >> 4) >> 1 : 0;
-  const int vz_dst = tid < 64 ? tile_off(kVRows, tid >> 4, 2 * (tid & 15)) : 0;
+  for (int p = 0; p < 4; ++p) v_s2[p] = (4 * p + tq) * 4 + bw;
+  const int v_src = vword_offset(2 * bw, lane);
+  const int v_dst = (2 + 4 * bw) * 256 + 4 * lane;   // row 16 + channel of m = 2 bw, r = 0
+  // value zero rows: channel group jg = bt / 16, tokens 2 tp, 2 tp + 1 (tp = bt % 16)
+  const int vz_src = bt < 64 ? vzero_index(2 * (bt & 15), bt >> 4) >> 1 : 0;
+  const int vz_dst = bt < 64 ? tile_off(kVRows, bt >> 4, 2 * (bt & 15)) : 0;
   const int row_query = rr < G ? rr / g.G : -1;   // the query of this lane's row
 
   for_each_segment(g, c.len, ws.N, [&](const Segment& seg) {
@@ -400,9 +407,11 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       reinterpret_cast<uint4*>(base)[j] = make_uint4(fill, fill, fill, fill);
     }
     // this lane's P row outside its tokens stays zero
+    if (!builder) {
 #pragma unroll
-    for (int c8 = 0; c8 < 2; ++c8)
-      *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * (1 - kc) + 8 * c8)) = make_uint4(0u, 0u, 0u, 0u);
+      for (int c8 = 0; c8 < 2; ++c8)
+        *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * (1 - kc) + 8 * c8)) = make_uint4(0u, 0u, 0u, 0u);
+    }
     proxy_fence();
     if (tid == 0 && ngr > 0 && !*fail) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
     // the first record is in (or the CTA stops: a decision every thread takes alike, from a
@@ -423,16 +432,16 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           const uint32_t s2 = ks2[k_s2[jj]];
           const uint32_t w = recw[k_src[jj]] >> k_shift[jj];
           uint8_t* dh = bk + k_dst[jj];
-          if (4 * warp + jj < 2 * NHS)
+          if (4 * bw + jj < 2 * NHS)
             cs_pairs4<BHI>(w, s2, dh, dh + 4 * 256, 256);   // hi in row 16 + tau, lo in 48 + tau
           else
             cs_pairs4<BLO>(w, s2, dh, dh + 4 * 256, 256);
         }
-        if (tid >= 64)
+        if (bt >= 64)
           *reinterpret_cast<uint32_t*>(bk + kz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kz_src];
       } else {
         const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
-        for (int item = tid; item < kGroup * (kHeadDim / 2); item += kTcThreads) {
+        for (int item = bt; item < kGroup * (kHeadDim / 2); item += kTcHalf) {
           const int tau = item >> 6, p0 = 2 * (item & 63);
           float x0 = 0.f, x1 = 0.f;
           if (tau < seg.nr) {
@@ -444,7 +453,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 16 + tau, p0)) = hi;
           *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 48 + tau, p0)) = lo;
         }
-        if (tid >= 64) *reinterpret_cast<uint32_t*>(bk + kz_dst) = 0u;
+        if (bt >= 64) *reinterpret_cast<uint32_t*>(bk + kz_dst) = 0u;
       }
     };
     // ---- value tile of item i into buffer i % 2: fp16(c * s_v) and the zero rows
@@ -471,17 +480,17 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
             }
           }
         }
-        if (tid < 64)
+        if (bt < 64)
           *reinterpret_cast<uint32_t*>(bv + vz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 1792)[vz_src];
       } else {
         const uint16_t* rv = c.v_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
-        for (int item = tid; item < kHeadDim * (kGroup / 2); item += kTcThreads) {
+        for (int item = bt; item < kHeadDim * (kGroup / 2); item += kTcHalf) {
           const int ch = item >> 4, t0 = 2 * (item & 15);
           const float x0 = t0 < seg.nr ? bf16_bits_to_float(rv[t0 * kHeadDim + ch]) : 0.f;
           const float x1 = t0 + 1 < seg.nr ? bf16_bits_to_float(rv[(t0 + 1) * kHeadDim + ch]) : 0.f;
           *reinterpret_cast<uint32_t*>(bv + tile_off(kVRows, 16 + ch, t0)) = pack_f16(x0, x1);
         }
-        if (tid < 64) *reinterpret_cast<uint32_t*>(bv + vz_dst) = 0u;
+        if (bt < 64) *reinterpret_cast<uint32_t*>(bv + vz_dst) = 0u;
       }
     };
     auto issue_keys = [&]() {   // thread 0: the key products of the tile just built
@@ -492,12 +501,12 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       mma_issued = true;
     };
 
-    // Pipeline: item i's value tile is built while its key products run; after their commit
-    // (which covers every earlier product) the softmax of item i and the key tile of item
-    // i + 1 are written; then one thread issues the value products of i and the key products
-    // of i + 1 together.
+    // Pipeline: the builders write item i's value tile while its key products run; after
+    // their commit (which covers every earlier product) the softmax warps write P of item i
+    // and the builders the key tile of item i + 1, at the same time; then one thread issues
+    // the value products of i and the key products of i + 1 together.
     if (nitems > 0 && !stop0) {
-      build_keys(0, ring + (ncons % kTcSlots) * kSlotBytes);
+      if (builder) build_keys(0, ring + (ncons % kTcSlots) * kSlotBytes);
       proxy_fence();
       tc_fence_before();
       __syncthreads();
@@ -512,82 +521,83 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       const int ntok = resid_item ? seg.nr : kGroup;
       // ---- value tile (this buffer's last reader, the value products two items back,
       // completed before the previous key commit)
-      build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);   // (the ring is not read for the residual)
+      if (builder) build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);   // (not read for the residual)
       // ---- every thread: the key products (and with them every earlier product) are done
       wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
       ++nk;
       if (!resid_item) ++ncons;   // the ring position names the next record's slot
       tc_fence_after();
-      // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
-      float sv[16];
-      float zk;
-      {
-        uint32_t rh[16], rl[16], zraw;
-        tmem_ld16_nowait(t_row + kTmemKhi + 16 * kc, rh);
-        tmem_ld16_nowait(t_row + kTmemKlo + 16 * kc, rl);
-        tmem_ld1_nowait(t_row + kTmemKz, zraw);
-        tmem_wait_ld();
-        zk = __uint_as_float(zraw);
-#pragma unroll
-        for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
-      }
-      // tokens 16 kc + t of the group this row sees: t < nvis
-      const int lim = row_query >= 0 ? vis_base + row_query : 0;
-      const int nvis = min(ntok, lim - tok0) - 16 * kc;
-      if (nvis < 16) {
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          if (t >= nvis) sv[t] = -INFINITY;
-      }
-      float mxr = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 16; ++t) mxr = fmaxf(mxr, sv[t]);
-      const float mx = (mxr + zk) * qscale;   // -inf when no token is visible
-      // reference m of the row: the first visible logit's group maximum, moved up only when a
-      // logit would give p above 2^kRefSlack (fp16 holds p up to 65504; the accumulators are
-      // fp32), so the accumulators in TMEM are rescaled almost never; a row that has seen no
-      // token has zero accumulators and needs no rescale
-      bool rescale = false;
-      float alpha = 1.f;
-      if (mx > m_row + kRefSlack) {
-        rescale = m_row != -INFINITY;
-        if (rescale) alpha = ex2(m_row - mx);
-        m_row = mx;
-      }
-      if (out_live && __any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM traffic
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float o[32];
-          tmem_ld32(t_row + kTmemOut + 32 * c4, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(t_row + kTmemOut + 32 * c4, o);
-        }
-        uint32_t zr[8];
-        tmem_ld8_nowait(t_row + kTmemZv, zr);   // zero terms and the denominator
-        tmem_wait_ld();
-        float zf[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) zf[i] = __uint_as_float(zr[i]) * alpha;
-        tmem_st8(t_row + kTmemZv, zf);
-      }
-      // P (fp16): p = 2^(logit * scale - m), 0 for a hidden token (and for all while the row
-      // has seen none), 8 tokens per 16-byte store
-      const float off = m_row == -INFINITY ? -INFINITY : zk * qscale - m_row;
-#pragma unroll
-      for (int c8 = 0; c8 < 2; ++c8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
-          const int t = 8 * c8 + 2 * k2;
-          w[k2] = pack_f16(ex2(fmaf(sv[t], qscale, off)), ex2(fmaf(sv[t + 1], qscale, off)));
-        }
-        *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      // ---- the next item's key tile (this item's key products have completed; every thread
-      // waits for the record itself)
       const bool next = it + 1 < nitems;
-      if (next) {
+      if (!builder) {
+        // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
+        float sv[16];
+        float zk;
+        {
+          uint32_t rh[16], rl[16], zraw;
+          tmem_ld16_nowait(t_row + kTmemKhi + 16 * kc, rh);
+          tmem_ld16_nowait(t_row + kTmemKlo + 16 * kc, rl);
+          tmem_ld1_nowait(t_row + kTmemKz, zraw);
+          tmem_wait_ld();
+          zk = __uint_as_float(zraw);
+#pragma unroll
+          for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
+        }
+        // tokens 16 kc + t of the group this row sees: t < nvis
+        const int lim = row_query >= 0 ? vis_base + row_query : 0;
+        const int nvis = min(ntok, lim - tok0) - 16 * kc;
+        if (nvis < 16) {
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (t >= nvis) sv[t] = -INFINITY;
+        }
+        float mxr = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) mxr = fmaxf(mxr, sv[t]);
+        const float mx = (mxr + zk) * qscale;   // -inf when no token is visible
+        // reference m of the row: the first visible logit's group maximum, moved up only when a
+        // logit would give p above 2^kRefSlack (fp16 holds p up to 65504; the accumulators are
+        // fp32), so the accumulators in TMEM are rescaled almost never; a row that has seen no
+        // token has zero accumulators and needs no rescale
+        bool rescale = false;
+        float alpha = 1.f;
+        if (mx > m_row + kRefSlack) {
+          rescale = m_row != -INFINITY;
+          if (rescale) alpha = ex2(m_row - mx);
+          m_row = mx;
+        }
+        if (out_live && __any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM traffic
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float o[32];
+            tmem_ld32(t_row + kTmemOut + 32 * c4, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(t_row + kTmemOut + 32 * c4, o);
+          }
+          uint32_t zr[8];
+          tmem_ld8_nowait(t_row + kTmemZv, zr);   // zero terms and the denominator
+          tmem_wait_ld();
+          float zf[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) zf[i] = __uint_as_float(zr[i]) * alpha;
+          tmem_st8(t_row + kTmemZv, zf);
+        }
+        // P (fp16): p = 2^(logit * scale - m), 0 for a hidden token (and for all while the row
+        // has seen none), 8 tokens per 16-byte store
+        const float off = m_row == -INFINITY ? -INFINITY : zk * qscale - m_row;
+#pragma unroll
+        for (int c8 = 0; c8 < 2; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const int t = 8 * c8 + 2 * k2;
+            w[k2] = pack_f16(ex2(fmaf(sv[t], qscale, off)), ex2(fmaf(sv[t + 1], qscale, off)));
+          }
+          *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else if (next) {
+        // ---- the next item's key tile (this item's key products have completed; every
+        // builder waits for the record itself)
         if (it + 1 < ngr) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
         build_keys(it + 1, ring + (ncons % kTcSlots) * kSlotBytes);
       }
@@ -633,14 +643,14 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       float* msh = xch + 64 * kXRow;                         // [128]: every lane's m
       const bool live = out_live && !*fail;
       const float m_me = live ? m_row : -INFINITY;
-      msh[tid] = m_me;
+      if (!builder) msh[tid] = m_me;
       __syncthreads();
       const float M = fmaxf(msh[rr], msh[rr + 64]);
       const float f = m_me == -INFINITY ? 0.f : ex2(m_me - M);
       float zv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) zv[i] = 0.f;
-      if (out_live) {
+      if (!builder && out_live) {
         uint32_t zr[8];
         tmem_ld8_nowait(t_row + kTmemZv, zr);   // warp-collective
         tmem_wait_ld();
@@ -648,17 +658,17 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         for (int i = 0; i < 8; ++i) zv[i] = __uint_as_float(zr[i]);
       }
       float* mine = xch + rr * kXRow;
-      if (kc == 1) mine[0] = f * zv[4];
+      if (!builder && kc == 1) mine[0] = f * zv[4];
 #pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
-        if (out_live) {
+        if (!builder && out_live) {
           tmem_ld32(t_row + kTmemOut + 32 * c4, v);   // warp-collective
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-        if (kc == 1) {
+        if (!builder && kc == 1) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(mine + 4 + 32 * c4 + i) =
@@ -666,7 +676,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
                             f * (v[i + 3] + zv[c4]));
         }
         __syncthreads();
-        if (kc == 0 && rr < G) {
+        if (!builder && kc == 0 && rr < G) {
           float* o = partial_slot(ws, unit, G) + rr * kPartialStride;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
