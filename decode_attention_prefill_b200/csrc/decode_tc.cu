@@ -157,6 +157,12 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Named barrier ID of the 128 threads of one role (barrier 0 is __syncthreads).
+template <int ID>
+__device__ __forceinline__ void role_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(128) : "memory");
+}
+
 __device__ __forceinline__ __half2 bits_h2(uint32_t x) {
   __half2 h;
   memcpy(&h, &x, 4);
@@ -522,12 +528,22 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       // ---- value tile (this buffer's last reader, the value products two items back,
       // completed before the previous key commit)
       if (builder) build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);   // (not read for the residual)
-      // ---- every thread: the key products (and with them every earlier product) are done
-      wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
+      // ---- the key products (and with them every earlier product) are done, and for the
+      // builders the next record is in: one thread of each role polls, the role's warps meet
+      // at its named barrier (waiting there issues nothing)
+      const bool next = it + 1 < nitems;
+      if (bt == 0) {
+        wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
+        if (builder && it + 1 < ngr)
+          wait_bar(full + ((ncons + 1) % kTcSlots), ((ncons + 1) / kTcSlots) & 1u, g.wait_limit);
+      }
+      if (builder)
+        role_sync<2>();
+      else
+        role_sync<1>();
       ++nk;
       if (!resid_item) ++ncons;   // the ring position names the next record's slot
       tc_fence_after();
-      const bool next = it + 1 < nitems;
       if (!builder) {
         // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
         float sv[16];
@@ -596,9 +612,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else if (next) {
-        // ---- the next item's key tile (this item's key products have completed; every
-        // builder waits for the record itself)
-        if (it + 1 < ngr) wait_bar(full + (ncons % kTcSlots), (ncons / kTcSlots) & 1u, g.wait_limit);
+        // ---- the next item's key tile (this item's key products have completed)
         build_keys(it + 1, ring + (ncons % kTcSlots) * kSlotBytes);
       }
       proxy_fence();
