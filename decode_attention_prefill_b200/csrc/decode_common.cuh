@@ -156,10 +156,33 @@ __device__ __forceinline__ int visible_tokens(const Geometry& g, int len, int v)
 // ws.prior_out / prior_lse the row is merged with an attention over other tokens:
 //   out = (2^(L0 - M) o0 + 2^(L - M) o) / (2^(L0 - M) + 2^(L - M)),  M = max(L0, L),
 // and the log-sum-exp written is that of the union, M + log2(2^(L0 - M) + 2^(L - M)).
-template <int MAXR = kMaxG>   // the most rows a launch has (G <= MAXR)
+// Shared memory of the combine: the weights of a chunk of segments per row, each row's m*
+// and denominator, the mixing weights of a merge with a prior part, the ticket verdict.
+template <int MAXR>
+struct CombineScratch {
+  float w[MAXR][kMaxCombineSegs];
+  float mstar[MAXR], den[MAXR];
+  float mix[MAXR][2];   // weights of the prior row and of this one
+  int is_last;
+};
+
+// EXT: the caller passes the scratch (a region of its dynamic shared memory that is idle
+// while the combine runs) instead of the combine declaring it statically.
+template <int MAXR = kMaxG, bool EXT = false>   // the most rows a launch has (G <= MAXR)
 __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segment& s, int G, float* out,
-                                                const Geometry& geo) {
-  __shared__ int is_last;
+                                                const Geometry& geo, CombineScratch<MAXR>* ext = nullptr) {
+  CombineScratch<MAXR>* sc;
+  if constexpr (EXT) {
+    sc = ext;
+  } else {
+    __shared__ CombineScratch<MAXR> own;
+    sc = &own;
+  }
+  auto& wsh = sc->w;
+  auto& mstar_sh = sc->mstar;
+  auto& den_sh = sc->den;
+  auto& mix_sh = sc->mix;
+  int& is_last = sc->is_last;
   __threadfence();
   __syncthreads();
   const unsigned nseg = static_cast<unsigned>(s.last - s.first + 1);
@@ -171,9 +194,6 @@ __device__ __forceinline__ void combine_segment(const DecodeWs& ws, const Segmen
     // round), the largest reference m* and the denominator follow by shuffles and the
     // weights 2^(m_s - m*) of the first chunk go to shared memory; (2) per chunk of up to 32
     // segments, every thread sums its (head, channel) pairs with four loads in flight
-    __shared__ float wsh[MAXR][kMaxCombineSegs];
-    __shared__ float mstar_sh[MAXR], den_sh[MAXR];
-    __shared__ float mix_sh[MAXR][2];   // weights of the prior row and of this one
     constexpr int kLaneSegs = 4;         // segments per lane held in registers (128 per head)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const float* base = ws.part + static_cast<size_t>(s.first + s.unit) * G * kPartialStride;

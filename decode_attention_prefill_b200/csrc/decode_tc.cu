@@ -40,7 +40,7 @@
 // products and the next group's key products.  The bf16 residual window takes the same
 // path as one more group (its keys split into hi / lo, its values rounded to fp16, zero
 // tiles empty, the tokens past it masked).  The records arrive by TMA bulk copy (no
-// multicast) into a ring of four.  Every wait is bounded.  At the end of a segment the
+// multicast) into a ring of three.  Every wait is bounded.  At the end of a segment the
 // softmax threads write each row's partial (m, l, O) for the fused combine.  Needs |c s|
 // below 65504 (keys and values whose group range fits fp16).
 #include <atomic>
@@ -55,7 +55,7 @@ namespace {
 
 constexpr int kTcThreads = 256;   // warps 0..3: softmax (TMEM lanes 0..127); warps 4..7: tile building
 constexpr int kTcHalf = 128;      // threads of one role
-constexpr int kTcSlots = 4;       // record ring
+constexpr int kTcSlots = 3;       // record ring
 constexpr int kTmemCols = 256;    // TMEM columns per CTA (two CTAs per SM)
 // TMEM columns: key products 0 .. 79 (zero term in 0, hi in 16 .. 47, lo in 48 .. 79), value
 // products 112 .. 255 (zero terms in 112 .. 115, outputs in 128 .. 255)
@@ -157,6 +157,10 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Named barrier ID of the 128 threads of one role (barrier 0 is __syncthreads).
 template <int ID>
 __device__ __forceinline__ void role_sync() {
@@ -206,27 +210,28 @@ __device__ __forceinline__ void cs_pairs4(uint32_t w, uint32_t s2, uint8_t* dh, 
 
 struct TcSmem {
   int aq;      // fp16 [128 rows][128 positions]
-  int bk;      // fp16 [80 rows][128 positions] (zero row, hi, lo)
+  int bk;      // two buffers of fp16 [80 rows][128 positions] (zero row, hi, lo)
   int ap;      // fp16 [128 rows][32 tokens]
   int bv;      // two buffers of fp16 [144 rows][32 tokens] (zero rows, values)
-  int qnat;    // fp32 [64 rows][128], aliases bk, ap and the start of the first value buffer
+  int qnat;    // fp32 [64 rows][128], aliases the key tiles
   int ring;    // [kTcSlots][R]
   int perm;    // 128 bytes
-  int bars;    // uint64 full[kTcSlots], mma_k, mma_v; uint32 TMEM address
+  int bars;    // uint64 full[kTcSlots], mma_k, mma_v, logits read; uint32 TMEM address
   int total;
 };
 
 constexpr int kStepK = kKRows * 32;     // bytes of one K = 16 step of the key tile
 constexpr int kStepV = kVRows * 32;     // of the value tile
 constexpr int kVBuf = 2 * kStepV;
+constexpr int kBkBuf = 8 * kStepK;      // one key tile (8 K steps)
 
 __host__ __device__ __forceinline__ TcSmem tc_smem(int R) {
   TcSmem m;
   m.aq = 0;
   m.bk = m.aq + 128 * 128 * 2;
-  m.ap = m.bk + 8 * kStepK;
+  m.ap = m.bk + 2 * kBkBuf;
   m.bv = m.ap + 128 * 32 * 2;
-  m.qnat = m.bk;   // 32 KB: bk (20 KB), ap (8 KB), the first 4 KB of value buffer 0
+  m.qnat = m.bk;   // 32 KB of the 40 KB of key tiles
   m.ring = m.bv + 2 * kVBuf;
   m.perm = m.ring + kTcSlots * ((R + 127) / 128 * 128);
   m.bars = m.perm + 128;
@@ -255,7 +260,8 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sm.bars);
   uint64_t* bar_k = full + kTcSlots;
   uint64_t* bar_v = bar_k + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_v + 1);
+  uint64_t* bar_l = bar_v + 1;   // every softmax thread has read this item's logits
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_l + 1);
   __shared__ int fail_sh;
 
   if (tid == 0) {
@@ -263,6 +269,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     for (int k = 0; k < kTcSlots; ++k) mbar_init(full + k, 1);
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
+    mbar_init(bar_l, kTcHalf);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -289,8 +296,8 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   // TMEM lane tid holds query row rr = tid % 64 for the tokens [16 kc, 16 kc + 16) of every
   // group: the two copies of a row are independent partials, merged at the segment's end
   const int kc = (warp & 3) >> 1, rr = tid & 63;
-  // records staged so far / taken so far (ring position), commits to bar_k / bar_v so far
-  uint32_t nis = 0, ncons = 0, nk = 0, nv = 0;
+  // records staged so far / taken so far (ring position); product commits and waits
+  uint32_t nis = 0, ncons = 0, nk = 0, nv = 0, ck = 0, cv = 0, nl = 0;
   // bounded wait for phase `parity` of `bar`; gives up (error bit, CTA-wide stop) after
   // `limit` rounds: g.wait_limit for the staged records, kDecodeWaitLimit for the tensor
   // cores' commits (they always arrive; the bound only guards against a hang)
@@ -349,7 +356,6 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     const uint8_t* unit_rec = record_ptr(g, c.records, b, h, 0);
     const bool stage = unit != g.skip_unit;   // false only under the timeout test hook
     int issued = 0;
-    bool mma_issued = false;   // thread 0: a product of this segment may still be in flight
     // thread 0: stage the segment's next record into its slot (the slot's previous record
     // has been consumed: records are taken in order and a slot is refilled once the tiles of
     // its record were built)
@@ -404,12 +410,12 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       *reinterpret_cast<uint4*>(aq + tile_off(128, r, 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     __syncthreads();   // qnat is dead: the fixed rows of the tiles it overlapped
-    // rows 0..15 of the key tile's 8 steps and of both value buffers' 2 steps: zero, except
+    // rows 0..15 of both key tiles' 8 steps and of both value buffers' 2 steps: zero, except
     // row 4 of the value tiles, all ones (its product is the row's softmax denominator)
-    for (int i = tid; i < 12 * 32; i += kTcThreads) {
+    for (int i = tid; i < 20 * 32; i += kTcThreads) {
       const int step = i >> 5, j = i & 31;
-      uint8_t* base = step < 8 ? bk + step * kStepK : smem + sm.bv + (step - 8) * kStepV;
-      const uint32_t fill = (step >= 8 && (j == 4 || j == 12)) ? 0x3C003C00u : 0u;
+      uint8_t* base = step < 16 ? bk + step * kStepK : smem + sm.bv + (step - 16) * kStepV;
+      const uint32_t fill = (step >= 16 && (j == 4 || j == 12)) ? 0x3C003C00u : 0u;
       reinterpret_cast<uint4*>(base)[j] = make_uint4(fill, fill, fill, fill);
     }
     // this lane's P row outside its tokens stays zero
@@ -430,6 +436,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     // ---- key tile of item i (a record in `rec`, or the residual window): hi / lo of c * s
     // and the zero row
     auto build_keys = [&](int i, const uint8_t* rec) {
+      uint8_t* bkb = bk + (i & 1) * kBkBuf;
       if (i < ngr) {
         const uint32_t* recw = reinterpret_cast<const uint32_t*>(rec);
         const uint32_t* ks2 = reinterpret_cast<const uint32_t*>(rec + KC);
@@ -437,14 +444,14 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         for (int jj = 0; jj < 4; ++jj) {
           const uint32_t s2 = ks2[k_s2[jj]];
           const uint32_t w = recw[k_src[jj]] >> k_shift[jj];
-          uint8_t* dh = bk + k_dst[jj];
+          uint8_t* dh = bkb + k_dst[jj];
           if (4 * bw + jj < 2 * NHS)
             cs_pairs4<BHI>(w, s2, dh, dh + 4 * 256, 256);   // hi in row 16 + tau, lo in 48 + tau
           else
             cs_pairs4<BLO>(w, s2, dh, dh + 4 * 256, 256);
         }
         if (bt >= 64)
-          *reinterpret_cast<uint32_t*>(bk + kz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kz_src];
+          *reinterpret_cast<uint32_t*>(bkb + kz_dst) = reinterpret_cast<const uint32_t*>(rec + KC + 256)[kz_src];
       } else {
         const uint16_t* rk = c.k_resid + static_cast<size_t>(unit) * kGroup * kHeadDim;
         for (int item = bt; item < kGroup * (kHeadDim / 2); item += kTcHalf) {
@@ -456,10 +463,10 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           }
           uint32_t hi, lo;
           split_pair(x0, x1, hi, lo);
-          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 16 + tau, p0)) = hi;
-          *reinterpret_cast<uint32_t*>(bk + tile_off(kKRows, 48 + tau, p0)) = lo;
+          *reinterpret_cast<uint32_t*>(bkb + tile_off(kKRows, 16 + tau, p0)) = hi;
+          *reinterpret_cast<uint32_t*>(bkb + tile_off(kKRows, 48 + tau, p0)) = lo;
         }
-        if (bt >= 64) *reinterpret_cast<uint32_t*>(bk + kz_dst) = 0u;
+        if (bt >= 64) *reinterpret_cast<uint32_t*>(bkb + kz_dst) = 0u;
       }
     };
     // ---- value tile of item i into buffer i % 2: fp16(c * s_v) and the zero rows
@@ -499,18 +506,23 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         if (bt < 64) *reinterpret_cast<uint32_t*>(bv + vz_dst) = 0u;
       }
     };
-    auto issue_keys = [&]() {   // thread 0: the key products of the tile just built
+    auto issue_keys = [&](int i) {   // one thread: the key products of item i's tile
+      const uint64_t dk = dk0 + (i & 1) * (kBkBuf >> 4);
 #pragma unroll
       for (int s = 0; s < kHeadDim / 16; ++s)
-        tc_mma(tmem + kTmemKz, dq0 + s * (128 * 32 >> 4), dk0 + s * (kStepK >> 4), kIdescK, s > 0);
+        tc_mma(tmem + kTmemKz, dq0 + s * (128 * 32 >> 4), dk + s * (kStepK >> 4), kIdescK, s > 0);
       tc_commit(bar_k);
-      mma_issued = true;
     };
 
-    // Pipeline: the builders write item i's value tile while its key products run; after
-    // their commit (which covers every earlier product) the softmax warps write P of item i
-    // and the builders the key tile of item i + 1, at the same time; then one thread issues
-    // the value products of i and the key products of i + 1 together.
+    // Pipeline (item i): the builders write the key tile of item i + 1 (the other of two
+    // buffers) while the key products of item i run; once every softmax thread has read
+    // item i's logits (bar_l), one builder issues the key products of item i + 1 (they
+    // overlap the rest of the softmax and the value tile of item i, which the builders write
+    // next); the softmax warps wait for the value products of item i - 1 and write P of item
+    // i; after one barrier thread 0 issues the value products of item i.  Every product is
+    // committed to an mbarrier by the thread that issued it (keys: bar_k, values: bar_v);
+    // ck / cv count the commits, nk / nv / nl the phases waited for (all threads count
+    // alike).
     if (nitems > 0 && !stop0) {
       if (builder) build_keys(0, ring + (ncons % kTcSlots) * kSlotBytes);
       proxy_fence();
@@ -518,33 +530,40 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       __syncthreads();
       if (tid == 0) {
         tc_fence_after();
-        issue_keys();
+        issue_keys(0);
       }
+      ++ck;
     }
     for (int it = 0; it < nitems && !stop0; ++it) {
       const bool resid_item = it == ngr;
       const int tok0 = resid_item ? seg.ng * kGroup : (seg.lo + it) * kGroup;
       const int ntok = resid_item ? seg.nr : kGroup;
-      // ---- value tile (this buffer's last reader, the value products two items back,
-      // completed before the previous key commit)
-      if (builder) build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);   // (not read for the residual)
-      // ---- the key products (and with them every earlier product) are done, and for the
-      // builders the next record is in: one thread of each role polls, the role's warps meet
-      // at its named barrier (waiting there issues nothing)
       const bool next = it + 1 < nitems;
-      if (bt == 0) {
-        wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
-        if (builder && it + 1 < ngr)
-          wait_bar(full + ((ncons + 1) % kTcSlots), ((ncons + 1) / kTcSlots) & 1u, g.wait_limit);
-      }
-      if (builder)
-        role_sync<2>();
-      else
+      if (builder) {
+        if (next) {
+          // the next record is in (one poller); its key tile goes to the other buffer, whose
+          // last reader (the key products of item i - 1) completed before the last barrier
+          if (bt == 0 && it + 1 < ngr)
+            wait_bar(full + ((ncons + 1) % kTcSlots), ((ncons + 1) / kTcSlots) & 1u, g.wait_limit);
+          role_sync<2>();
+          build_keys(it + 1, ring + ((ncons + 1) % kTcSlots) * kSlotBytes);
+          proxy_fence();
+          role_sync<2>();   // the key tile is complete
+          if (bt == 0) {   // item i's logits are read: the key accumulators may be overwritten
+            wait_bar(bar_l, nl & 1u, kDecodeWaitLimit);
+            tc_fence_after();
+            issue_keys(it + 1);
+          }
+        }
+        // this item's value tile (its buffer's last reader, the value products of item i - 2,
+        // completed before the last barrier; the ring is not read for the residual)
+        build_values(it, ring + (ncons % kTcSlots) * kSlotBytes);
+      } else {
+        // ---- the key products of this item are done: one poller, the role meets at its
+        // barrier (waiting there issues nothing)
+        if (bt == 0) wait_bar(bar_k, nk & 1u, kDecodeWaitLimit);
         role_sync<1>();
-      ++nk;
-      if (!resid_item) ++ncons;   // the ring position names the next record's slot
-      tc_fence_after();
-      if (!builder) {
+        tc_fence_after();
         // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
         float sv[16];
         float zk;
@@ -558,6 +577,11 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
 #pragma unroll
           for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
         }
+        tc_fence_before();
+        if (next) mbar_arrive(bar_l);   // this thread's logits are read
+        if (tid == 0 && it > 0) wait_bar(bar_v, nv & 1u, kDecodeWaitLimit);   // value products of item i - 1
+        role_sync<1>();   // P and the value accumulators are free
+        tc_fence_after();
         // tokens 16 kc + t of the group this row sees: t < nvis
         const int lim = row_query >= 0 ? vis_base + row_query : 0;
         const int nvis = min(ntok, lim - tok0) - 16 * kc;
@@ -611,15 +635,19 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
           }
           *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-      } else if (next) {
-        // ---- the next item's key tile (this item's key products have completed)
-        build_keys(it + 1, ring + (ncons % kTcSlots) * kSlotBytes);
       }
+      ++nk;
+      if (next) {
+        ++ck;
+        ++nl;
+      }
+      if (it > 0) ++nv;
       proxy_fence();
       tc_fence_before();
       // P, the value tile, any rescale and the next key tile are in place; every thread is done
       // with this item's record
       if (__syncthreads_or(*fail)) break;
+      if (!resid_item) ++ncons;   // the ring position names the next record's slot
       if (tid == 0) {
         tc_fence_after();
         if (!resid_item) issue_next();
@@ -627,18 +655,25 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
 #pragma unroll
         for (int s = 0; s < kGroup / 16; ++s)
           tc_mma(tmem + kTmemV, dp0 + s * (128 * 32 >> 4), dv + s * (kStepV >> 4), kIdescV, out_live || s > 0);
-        if (next) issue_keys();
+        tc_commit(bar_v);
       }
+      ++cv;
       out_live = true;
     }
     // ---- every product of the segment completes (waited for even after a stop: TMEM and
-    // the tiles must be idle before they are read or reused), then this row's partial
-    if (tid == 0 && mma_issued) {
-      tc_commit(bar_v);
-      for (uint32_t spins = 0; spins < kDecodeWaitLimit && !mbar_try_wait(bar_v, nv & 1u); ++spins) {
-      }
+    // the tiles must be idle before they are read or reused): the latest commit of each
+    // barrier covers every earlier product
+    if (tid == 0) {
+      if (ck > 0)
+        for (uint32_t spins = 0; spins < kDecodeWaitLimit && !mbar_try_wait(bar_k, (ck - 1) & 1u); ++spins) {
+        }
+      if (cv > 0)
+        for (uint32_t spins = 0; spins < kDecodeWaitLimit && !mbar_try_wait(bar_v, (cv - 1) & 1u); ++spins) {
+        }
     }
-    if (__syncthreads_or(tid == 0 && mma_issued)) ++nv;
+    __syncthreads();
+    nk = ck;
+    nv = cv;
     tc_fence_after();
     if (*fail && tid == 0) {   // let staged copies land before the shared memory is reused
       for (; ncons < nis; ++ncons) {
@@ -708,7 +743,8 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       }
     }
     tc_fence_before();
-    combine_segment<kMaxRows>(ws, seg, G, out, g);
+    // the combine's scratch: the A tile, idle until the next segment's setup
+    combine_segment<kMaxRows, true>(ws, seg, G, out, g, reinterpret_cast<CombineScratch<kMaxRows>*>(smem + sm.aq));
   });
   tc_fence_before();
   __syncthreads();
