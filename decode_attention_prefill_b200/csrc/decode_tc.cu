@@ -293,8 +293,9 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   constexpr uint32_t kIdescK = mma_idesc(kKRows), kIdescV = mma_idesc(kVRows);
   // operand descriptors of the first K step of each tile (a step further is a fixed offset)
   const uint64_t dq0 = tile_desc(aq), dk0 = tile_desc(bk), dp0 = tile_desc(ap), dv0 = tile_desc(smem + sm.bv);
-  // TMEM lane tid holds query row rr = tid % 64 for the tokens [16 kc, 16 kc + 16) of every
-  // group: the two copies of a row are independent partials, merged at the segment's end
+  // softmax thread tid (TMEM lane tid) holds query row rr = tid % 64 for the tokens
+  // [16 kc, 16 kc + 16) of every group: the two copies of a row are independent partials,
+  // merged at the segment's end
   const int kc = (warp & 3) >> 1, rr = tid & 63;
   // records staged so far / taken so far (ring position); product commits and waits
   uint32_t nis = 0, ncons = 0, nk = 0, nv = 0, ck = 0, cv = 0, nl = 0;
