@@ -63,3 +63,44 @@ def test_append_and_decode_replay_from_a_cuda_graph():
     np.testing.assert_array_equal(graphed.lengths().cpu().numpy(), eager.lengths().cpu().numpy())
     np.testing.assert_array_equal(graphed.records().cpu().numpy(), eager.records().cpu().numpy())
     np.testing.assert_array_equal(graphed.resid("k").cpu().numpy(), eager.resid("k").cpu().numpy())
+
+
+def test_multi_token_decode_replays_from_a_cuda_graph():
+    """A verify step of 16 new tokens per sequence (64 query rows per KV head: the tcgen05
+    kernel) captured once and replayed with fresh queries gives the eager call's output
+    bit for bit."""
+    import decode_attention_prefill_b200 as pm
+    B, Hq, Hkv, L, T = 2, 32, 8, 700, 16
+    G = Hq // Hkv
+    kin = workload.rows(5, workload.K, B, Hkv, 0, L + T)
+    vin = workload.rows(5, workload.V, B, Hkv, 0, L + T)
+    qwin = workload.rows(5, workload.Q, B, Hq, L - 64, 64, group=G)
+    cfg = pm.Config.make(Hq, Hkv)
+    cache = pm.PNMixCache(cfg, B, (L + T + 31) // 32 * 32 + 32, max_queries=T)
+    cache.prefill(to_dev(qwin), to_dev(kin), to_dev(vin), L)
+    for t in range(L, L + T):
+        cache.append(to_dev(np.ascontiguousarray(kin[:, :, t])), to_dev(np.ascontiguousarray(vin[:, :, t])))
+
+    def queries(seed):
+        q = workload.rows(seed, workload.Q, B, Hq, L, T, group=G)
+        return to_dev(np.ascontiguousarray(q.transpose(0, 2, 1, 3)))
+
+    q_in = torch.empty(B, T, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    out_g = torch.empty(B, T, Hq, 128, dtype=torch.float32, device="cuda")
+    out_e = torch.empty_like(out_g)
+    q_in.copy_(queries(0))
+    cache.attend_multi(q_in, out_g)   # eager first call: caches the launch geometry
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        cache.attend_multi(q_in, out_g, stream=stream)
+    for seed in (1, 2, 3):
+        q = queries(seed)
+        q_in.copy_(q)
+        graph.replay()
+        cache.attend_multi(q, out_e)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(out_g.cpu().numpy(), out_e.cpu().numpy())
+    assert cache.read_error() == 0
