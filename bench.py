@@ -559,14 +559,14 @@ def run_decode_workload(args):
 def run_verify(args):
     """verify_32k: the stream_32k shape (16 x 32/8 heads, 32768 tokens) with T new tokens
     per sequence attended at once (pnmix_decode_attention_multi after T appends), for
-    T = 1, 2, 4, 8 and 16 (4 to 64 query rows per KV head), each against the roofline of
+    T = 1, 2, 4, 8, 16 and 32 (4 to 128 query rows per KV head), each against the roofline of
     the bytes it must read.  The 419 MB cache exceeds L2.  Besides the algorithmic bytes,
     each point reports the tensor-core work per launch (the key- and value-side products
     of every row with every cached token)."""
     import torch
 
     import decode_attention_prefill_b200 as pm
-    Ts = [1, 2, 4, 8, 16]
+    Ts = [1, 2, 4, 8, 16, 32]
     Tmax = max(Ts)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)

@@ -311,6 +311,9 @@ cudaError_t launch_decode_ws(const Geometry& g, const uint16_t* q, const pnmix_c
                              float* out, DecodeWs ws, cudaStream_t s);
 cudaError_t launch_decode_tc(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                              float* out, DecodeWs ws, cudaStream_t s);
+// query rows per KV head the tcgen05 kernel takes (one per TMEM lane); the 8-row-warp
+// kernels stop at kMaxRows
+constexpr int kMaxTcRows = 128;
 cudaError_t launch_decode_rows(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax,
                                float* out, DecodeWs ws, cudaStream_t s);
 

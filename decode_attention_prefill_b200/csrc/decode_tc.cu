@@ -213,7 +213,8 @@ struct TcSmem {
   int bk;      // two buffers of fp16 [80 rows][128 positions] (zero row, hi, lo)
   int ap;      // fp16 [128 rows][32 tokens]
   int bv;      // two buffers of fp16 [144 rows][32 tokens] (zero rows, values)
-  int qnat;    // fp32 [64 rows][128], aliases the key tiles
+  int qnat;    // fp32 [64 or 128 rows][128] (segment setup only): the key tiles, then P and the
+               // value tiles
   int ring;    // [kTcSlots][R]
   int perm;    // 128 bytes
   int bars;    // uint64 full[kTcSlots], mma_k, mma_v, logits read; uint32 TMEM address
@@ -231,7 +232,7 @@ __host__ __device__ __forceinline__ TcSmem tc_smem(int R) {
   m.bk = m.aq + 128 * 128 * 2;
   m.ap = m.bk + 2 * kBkBuf;
   m.bv = m.ap + 128 * 32 * 2;
-  m.qnat = m.bk;   // 32 KB of the 40 KB of key tiles
+  m.qnat = m.bk;   // 32 or 64 KB from the key tiles on (bk, ap, bv: 66 KB)
   m.ring = m.bv + 2 * kVBuf;
   m.perm = m.ring + kTcSlots * ((R + 127) / 128 * 128);
   m.bars = m.perm + 128;
@@ -239,7 +240,9 @@ __host__ __device__ __forceinline__ TcSmem tc_smem(int R) {
   return m;
 }
 
-template <int BHI, int BLO, int NHS>
+// DUP: up to 64 rows, each row in TMEM lanes r and r + 64 (two halves of every group's
+// tokens); otherwise up to 128 rows, one per lane, each lane taking all 32 tokens.
+template <int BHI, int BLO, int NHS, bool DUP>
 __global__ void __launch_bounds__(kTcThreads, 2)
 decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, float* __restrict__ out, DecodeWs ws) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -293,10 +296,12 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
   constexpr uint32_t kIdescK = mma_idesc(kKRows), kIdescV = mma_idesc(kVRows);
   // operand descriptors of the first K step of each tile (a step further is a fixed offset)
   const uint64_t dq0 = tile_desc(aq), dk0 = tile_desc(bk), dp0 = tile_desc(ap), dv0 = tile_desc(smem + sm.bv);
-  // softmax thread tid (TMEM lane tid) holds query row rr = tid % 64 for the tokens
-  // [16 kc, 16 kc + 16) of every group: the two copies of a row are independent partials,
-  // merged at the segment's end
-  const int kc = (warp & 3) >> 1, rr = tid & 63;
+  // softmax thread tid (TMEM lane tid) holds query row rr for the tokens [tb, tb + kTok) of
+  // every group; with DUP rr = tid % 64, tb = 16 kc, and the two copies of a row are
+  // independent partials, merged at the segment's end
+  constexpr int kTok = DUP ? 16 : 32;
+  const int kc = DUP ? (warp & 3) >> 1 : 0, rr = DUP ? tid & 63 : tid & 127;
+  const int tb = kTok * kc;
   // records staged so far / taken so far (ring position); product commits and waits
   uint32_t nis = 0, ncons = 0, nk = 0, nv = 0, ck = 0, cv = 0, nl = 0;
   // bounded wait for phase `parity` of `bar`; gives up (error bit, CTA-wide stop) after
@@ -371,7 +376,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       for (int k = 0; k < kTcSlots; ++k) issue_next();
 
     // ---- query rows (fp32, natural order) and the position order; pruning as elsewhere
-    for (int i = tid; i < kMaxRows * (kHeadDim / 8); i += kTcThreads) {
+    for (int i = tid; i < (DUP ? kMaxRows : kMaxTcRows) * (kHeadDim / 8); i += kTcThreads) {
       const int hh = i >> 4;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (hh < G) v = __ldg(reinterpret_cast<const uint4*>(q + row_offset(g, b, h, hh)) + (i & 15));
@@ -398,7 +403,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     // A = Q (positions in order; bf16 -> fp16 is exact in fp16's normal range), one 16-byte
     // chunk of 8 positions per item; rows 64..127 repeat rows 0..63; rows >= G are zero
     for (int item = tid; item < 128 * 16; item += kTcThreads) {
-      const int r = item >> 4, c8 = item & 15, src = r & 63;
+      const int r = item >> 4, c8 = item & 15, src = DUP ? r & 63 : r;
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       if (src < G) {
 #pragma unroll
@@ -420,7 +425,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       reinterpret_cast<uint4*>(base)[j] = make_uint4(fill, fill, fill, fill);
     }
     // this lane's P row outside its tokens stays zero
-    if (!builder) {
+    if (DUP && !builder) {
 #pragma unroll
       for (int c8 = 0; c8 < 2; ++c8)
         *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * (1 - kc) + 8 * c8)) = make_uint4(0u, 0u, 0u, 0u);
@@ -566,34 +571,35 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         role_sync<1>();
         tc_fence_after();
         // ---- logits of this lane's row and tokens: hi + lo products (fp32), the zero term
-        float sv[16];
+        float sv[kTok];
         float zk;
-        {
+#pragma unroll
+        for (int h16 = 0; h16 < kTok / 16; ++h16) {
           uint32_t rh[16], rl[16], zraw;
-          tmem_ld16_nowait(t_row + kTmemKhi + 16 * kc, rh);
-          tmem_ld16_nowait(t_row + kTmemKlo + 16 * kc, rl);
+          tmem_ld16_nowait(t_row + kTmemKhi + tb + 16 * h16, rh);
+          tmem_ld16_nowait(t_row + kTmemKlo + tb + 16 * h16, rl);
           tmem_ld1_nowait(t_row + kTmemKz, zraw);
           tmem_wait_ld();
           zk = __uint_as_float(zraw);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) sv[t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
+          for (int t = 0; t < 16; ++t) sv[16 * h16 + t] = __uint_as_float(rh[t]) + __uint_as_float(rl[t]);
         }
         tc_fence_before();
         if (next) mbar_arrive(bar_l);   // this thread's logits are read
         if (tid == 0 && it > 0) wait_bar(bar_v, nv & 1u, kDecodeWaitLimit);   // value products of item i - 1
         role_sync<1>();   // P and the value accumulators are free
         tc_fence_after();
-        // tokens 16 kc + t of the group this row sees: t < nvis
+        // tokens tb + t of the group this row sees: t < nvis
         const int lim = row_query >= 0 ? vis_base + row_query : 0;
-        const int nvis = min(ntok, lim - tok0) - 16 * kc;
-        if (nvis < 16) {
+        const int nvis = min(ntok, lim - tok0) - tb;
+        if (nvis < kTok) {
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
+          for (int t = 0; t < kTok; ++t)
             if (t >= nvis) sv[t] = -INFINITY;
         }
         float mxr = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) mxr = fmaxf(mxr, sv[t]);
+        for (int t = 0; t < kTok; ++t) mxr = fmaxf(mxr, sv[t]);
         const float mx = (mxr + zk) * qscale;   // -inf when no token is visible
         // reference m of the row: the first visible logit's group maximum, moved up only when a
         // logit would give p above 2^kRefSlack (fp16 holds p up to 65504; the accumulators are
@@ -627,14 +633,14 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         // has seen none), 8 tokens per 16-byte store
         const float off = m_row == -INFINITY ? -INFINITY : zk * qscale - m_row;
 #pragma unroll
-        for (int c8 = 0; c8 < 2; ++c8) {
+        for (int c8 = 0; c8 < kTok / 8; ++c8) {
           uint32_t w[4];
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2) {
             const int t = 8 * c8 + 2 * k2;
             w[k2] = pack_f16(ex2(fmaf(sv[t], qscale, off)), ex2(fmaf(sv[t + 1], qscale, off)));
           }
-          *reinterpret_cast<uint4*>(ap + tile_off(128, tid, 16 * kc + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ap + tile_off(128, tid, tb + 8 * c8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       ++nk;
@@ -684,6 +690,42 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
         }
       }
     }
+    if constexpr (!DUP) {
+      // one lane per row: its partial (m, l = the ones-row product, O = the outputs plus the
+      // zero term of their channel group) goes to the slot directly
+      if (!builder) {
+        const bool live = out_live && !*fail;
+        float* o = partial_slot(ws, unit, G) + rr * kPartialStride;
+        float zv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zv[i] = 0.f;
+        if (out_live) {
+          uint32_t zr[8];
+          tmem_ld8_nowait(t_row + kTmemZv, zr);   // warp-collective
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) zv[i] = __uint_as_float(zr[i]);
+        }
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float v[32];
+          if (out_live) {
+            tmem_ld32(t_row + kTmemOut + 32 * c4, v);   // warp-collective
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          if (rr < G) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[2 + 32 * c4 + i] = live ? v[i] + zv[c4] : 0.f;
+          }
+        }
+        if (rr < G) {
+          o[0] = live ? m_row : -INFINITY;
+          o[1] = live ? zv[4] : 0.f;
+        }
+      }
+    } else
     // merge the two copies of each row (shared memory of the idle A and key tiles):
     // M = max(m0, m1), weights f = 2^(m - M), partial (M, f0 l0 + f1 l1, f0 O0 + f1 O1) with
     // O = the outputs plus the zero term of their channel group and l = the ones-row product
@@ -745,7 +787,7 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
     }
     tc_fence_before();
     // the combine's scratch: the A tile, idle until the next segment's setup
-    combine_segment<kMaxRows, true>(ws, seg, G, out, g, reinterpret_cast<CombineScratch<kMaxRows>*>(smem + sm.aq));
+    combine_segment<kMaxTcRows, true>(ws, seg, G, out, g, reinterpret_cast<CombineScratch<kMaxTcRows>*>(smem + sm.aq));
   });
   tc_fence_before();
   __syncthreads();
@@ -755,13 +797,13 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
 
 constexpr int kMaxDevices = 64;
 
-template <int BHI, int BLO, int NHS>
-cudaError_t launch_tc_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out, DecodeWs ws,
+template <int BHI, int BLO, int NHS, bool DUP>
+cudaError_t launch_tc_d(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out, DecodeWs ws,
                         cudaStream_t s) {
   static std::atomic<int> wave_cache[kMaxDevices];
   if (g.record_bytes != record_bytes_of<BHI, BLO, NHS>()) return cudaErrorInvalidValue;
   const TcSmem sm = tc_smem(g.record_bytes);
-  auto kern = decode_tc_kernel<BHI, BLO, NHS>;
+  auto kern = decode_tc_kernel<BHI, BLO, NHS, DUP>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -793,6 +835,14 @@ cudaError_t launch_tc_t(const Geometry& g, const uint16_t* q, const pnmix_cache&
   ws.N = wave < nmax ? wave : nmax;
   kern<<<ws.N, kTcThreads, sm.total, s>>>(g, q, c, out, ws);
   return cudaGetLastError();
+}
+
+template <int BHI, int BLO, int NHS>
+cudaError_t launch_tc_t(const Geometry& g, const uint16_t* q, const pnmix_cache& c, int nmax, float* out, DecodeWs ws,
+                        cudaStream_t s) {
+  if (g.rows > kMaxTcRows) return cudaErrorInvalidValue;
+  return g.rows <= kMaxRows ? launch_tc_d<BHI, BLO, NHS, true>(g, q, c, nmax, out, ws, s)
+                            : launch_tc_d<BHI, BLO, NHS, false>(g, q, c, nmax, out, ws, s);
 }
 
 template <int BHI, int BLO>

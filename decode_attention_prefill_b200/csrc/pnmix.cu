@@ -384,10 +384,16 @@ pnmix_status pnmix_debug_decode_stall(const pnmix_config* cfg, const uint16_t* q
   return cuda_status(launch_decode(g, q, *cache, max_context, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
+// Query rows per KV head a multi-query call may have: up to 128 on the tcgen05 kernel (the
+// automatic choice from 33 rows on, or forced), up to 64 on the others.
+static int max_query_rows(const Geometry& g) {
+  return g.kernel == PNMIX_DECODE_AUTO || g.kernel == PNMIX_DECODE_TC ? kMaxTcRows : kMaxRows;
+}
+
 size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch, int max_context, int n_queries) {
   Geometry g;
   if (batch <= 0 || n_queries < 1 || make_geometry(cfg, batch, 32, &g) != PNMIX_OK) return 0;
-  if (g.G * n_queries > kMaxRows) return 0;
+  if (g.G * n_queries > max_query_rows(g)) return 0;
   g.tq = n_queries;
   g.rows = g.G * n_queries;
   return decode_workspace_bytes(g, max_context);
@@ -402,7 +408,7 @@ pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_
   if (st != PNMIX_OK) return st;
   if ((st = check_cache(g, cache)) != PNMIX_OK) return st;
   if (!q || !out || !workspace || max_context < 0 || n_queries < 1) return PNMIX_ERR_INVALID_ARG;
-  if (g.G * n_queries > kMaxRows) return PNMIX_ERR_UNSUPPORTED;
+  if (g.G * n_queries > max_query_rows(g)) return PNMIX_ERR_UNSUPPORTED;
   if (g.kernel == PNMIX_DECODE_SIMT && n_queries > 1) return PNMIX_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return PNMIX_ERR_ALIGNMENT;
   g.tq = n_queries;

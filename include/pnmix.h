@@ -219,7 +219,7 @@ typedef struct {
  *   PNMIX_DECODE_PAIRS  tensor cores, a key-side and a value-side warp per group stream.
  *   PNMIX_DECODE_TC     5th-generation tensor cores (tcgen05, accumulators in TMEM): each
  *                       group's keys and values dequantized once into shared memory for all
- *                       of a unit's query rows (up to 64); its cost per group hardly depends
+ *                       of a unit's query rows (up to 128); its cost per group hardly depends
  *                       on the rows, so it is the multi-token kernel.  Keys and values whose
  *                       32-token group range exceeds 65504 are outside its domain (c * s must
  *                       be a finite fp16).
@@ -383,11 +383,13 @@ PNMIX_API size_t pnmix_workspace_bytes_multi(const pnmix_config* cfg, int batch,
  * Query j (0-based) of sequence b attends causally over the first len[b] - T + 1 + j
  * cached tokens: the cache before the step plus the new tokens up to its own.  The
  * pages have no such call; it is the multi-token neighbour of pnmix_decode_attention
- * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 64 (PNMIX_ERR_UNSUPPORTED
+ * (T = 1 gives the same result).  Requires 1 <= T and G * T <= 128 with the automatic
+ * choice or PNMIX_DECODE_TC, G * T <= 64 with the other kernels (PNMIX_ERR_UNSUPPORTED
  * otherwise; PNMIX_DECODE_SIMT takes T = 1 only).  Up to 8 query rows per KV head (G * T)
  * run on the single-query kernels; 9 to 32 rows on a kernel whose warps each hold 8 rows
  * and share one staging of the packed records, and from 33 rows on the tcgen05 kernel
- * (PNMIX_DECODE_TC), so the cache is read once for all T queries.  A query that sees no
+ * (PNMIX_DECODE_TC, one row per tensor-memory lane), so the cache is read once for all T
+ * queries.  A query that sees no
  * token gets zeros.  Workspace from pnmix_workspace_bytes_multi with the same T.
  */
 PNMIX_API pnmix_status pnmix_decode_attention_multi(const pnmix_config* cfg, const uint16_t* q,

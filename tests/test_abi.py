@@ -129,9 +129,13 @@ def test_multi_query_workspace_follows_the_rows():
     assert pm.workspace_bytes_multi(cfg, 2, 256, 1) == one
     assert pm.workspace_bytes_multi(cfg, 2, 256, 2) > one
     assert pm.workspace_bytes_multi(cfg, 2, 256, 3) > pm.workspace_bytes_multi(cfg, 2, 256, 2)   # 12 rows
-    assert pm.workspace_bytes_multi(cfg, 2, 256, 16) > 0       # 64 rows per KV head: the most
-    assert pm.workspace_bytes_multi(cfg, 2, 256, 17) == 0      # 68 rows: unsupported
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 16) > 0       # 64 rows per KV head
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 32) > 0       # 128 rows: the most (tcgen05 kernel)
+    assert pm.workspace_bytes_multi(cfg, 2, 256, 33) == 0      # 132 rows: unsupported
     assert pm.workspace_bytes_multi(cfg, 2, 256, 0) == 0
+    rows_kernel = pm.Config.make(8, 2, decode_kernel=pm.DECODE_MMA)   # forced: 8-row warps, up to 64
+    assert pm.workspace_bytes_multi(rows_kernel, 2, 256, 16) > 0
+    assert pm.workspace_bytes_multi(rows_kernel, 2, 256, 17) == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(),
@@ -142,8 +146,11 @@ def test_multi_query_entry_rejects_bad_arguments_before_launching():
     P = ctypes.c_void_p(1 << 41)
     L = pm._lib
     ws = pm.workspace_bytes_multi(cfg, 2, 256, 2)
-    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 17, ctypes.byref(c), 256, P, P, ws,
-                                          None) == pm.ERR_UNSUPPORTED      # 68 rows per KV head
+    assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 33, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_UNSUPPORTED      # 132 rows per KV head
+    forced = pm.Config.make(8, 2, decode_kernel=pm.DECODE_MMA)
+    assert L.pnmix_decode_attention_multi(ctypes.byref(forced), P, 17, ctypes.byref(c), 256, P, P, ws,
+                                          None) == pm.ERR_UNSUPPORTED      # 68 rows off the tcgen05 kernel
     assert L.pnmix_decode_attention_multi(ctypes.byref(cfg), P, 3, ctypes.byref(c), 256, P, P, ws,
                                           None) == pm.ERR_CAPACITY         # a 12-row workspace is larger
     simt = pm.Config.make(8, 2, decode_kernel=pm.DECODE_SIMT)

@@ -705,9 +705,12 @@ def test_fused_append_decode_on_a_full_cache_raises_the_error_bit():
     (2, 8, 1, 64, 3, 0),        # 24 rows, G = 8, the step starts a new group
     (2, 8, 2, 300, 6, 26),      # 24 rows with query-channel pruning
     (1, 16, 4, 2500, 5, 0),     # 20 rows, several split-K segments per unit
+    (1, 32, 8, 1000, 32, 0),    # 128 rows: the automatic choice only (tcgen05)
 ])
 @pytest.mark.parametrize("kernel", [None, "mma"])   # automatic (tcgen05 from 33 rows), 8-row warps
 def test_many_query_rows_per_kv_head_like_the_oracle(kernel, B, Hq, Hkv, L, T, n_prune):
+    if kernel == "mma" and Hq // Hkv * T > 64:
+        pytest.skip("more than 64 rows per KV head run on the tcgen05 kernel only")
     c = Case(B, Hq, Hkv, L, extra_tokens=T, seed=L + 5 * T, n_prune=n_prune, max_queries=T, kernel=kernel)
     c.prefill()
     for t in range(L, L + T):
@@ -781,6 +784,10 @@ def test_random_configurations_like_the_oracle(seed):
     (1, 16, 4, 2500, 8, 4, 2, 5, 26, 0),   # pair pruning, several segments per unit
     (2, 8, 2, 600, 8, 4, 2, 4, 0, 3),      # key-slice pruning
     (1, 32, 8, 8192, 8, 4, 2, 16, 0, 0),   # 64 rows at 8K: many groups and segments per CTA
+    (2, 8, 2, 900, 8, 4, 2, 24, 0, 0),     # 96 rows: one row per TMEM lane
+    (1, 16, 2, 1500, 8, 4, 2, 16, 0, 0),   # 128 rows (G = 8), several segments per unit
+    (1, 8, 2, 600, 16, 2, 1, 32, 26, 0),   # 128 rows (G = 4, T = 32), 1-bit block, pair pruning
+    (2, 8, 2, 700, 8, 4, 2, 20, 0, 3),     # 80 rows with key-slice pruning
 ])
 def test_tcgen05_decode_like_the_oracle(B, Hq, Hkv, L, k, bhi, blo, T, prune, slices):
     c = Case(B, Hq, Hkv, L, k, bhi, blo, extra_tokens=T, seed=L + T + prune, kernel="tc", max_queries=max(T, 2),
