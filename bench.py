@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one decode launch from the committed ncu capture (profiles/
 # decode_mma_stream32k.md): read + write bytes, the launch's algorithmic bytes, and a hash
 # of the decode sources it was taken on.  Reported only while the sources still match.
-DECODE_CAPTURE = {"sources_sha256_16": "68136e3acc70408e", "traffic_bytes": 425068032,
+DECODE_CAPTURE = {"sources_sha256_16": "f2df43601d39f9be", "traffic_bytes": 426606336,
                   "algorithmic_bytes": 420855808}
 DECODE_SOURCES = ["decode_attention_prefill_b200/csrc/decode_mma.cu",
                   "decode_attention_prefill_b200/csrc/decode_common.cuh",
