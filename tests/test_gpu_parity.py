@@ -788,6 +788,8 @@ def test_random_configurations_like_the_oracle(seed):
     (1, 16, 2, 1500, 8, 4, 2, 16, 0, 0),   # 128 rows (G = 8), several segments per unit
     (1, 8, 2, 600, 16, 2, 1, 32, 26, 0),   # 128 rows (G = 4, T = 32), 1-bit block, pair pruning
     (2, 8, 2, 700, 8, 4, 2, 20, 0, 3),     # 80 rows with key-slice pruning
+    (1, 16, 2, 400, 64, 4, 2, 16, 0, 0),   # 128 rows, k = 64 (the largest record)
+    (2, 8, 2, 500, 0, 2, 1, 32, 0, 0),     # 128 rows, 2/1 bits, k = 0
 ])
 def test_tcgen05_decode_like_the_oracle(B, Hq, Hkv, L, k, bhi, blo, T, prune, slices):
     c = Case(B, Hq, Hkv, L, k, bhi, blo, extra_tokens=T, seed=L + T + prune, kernel="tc", max_queries=max(T, 2),
