@@ -401,7 +401,8 @@ decode_tc_kernel(Geometry g, const uint16_t* __restrict__ q, pnmix_cache c, floa
       __syncthreads();
     }
     // A = Q (positions in order; bf16 -> fp16 is exact in fp16's normal range), one 16-byte
-    // chunk of 8 positions per item; rows 64..127 repeat rows 0..63; rows >= G are zero
+    // chunk of 8 positions per item; with DUP rows 64..127 repeat rows 0..63; rows >= G are
+    // zero
     for (int item = tid; item < 128 * 16; item += kTcThreads) {
       const int r = item >> 4, c8 = item & 15, src = DUP ? r & 63 : r;
       uint32_t w[4] = {0u, 0u, 0u, 0u};
